@@ -1,0 +1,35 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA device (B200, sm_100a) and the built library")
+
+
+def cuda_available() -> bool:
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.fixture(scope="session")
+def oracle():
+    import oracle as orc
+    return orc
+
+
+@pytest.fixture(scope="session")
+def lib():
+    """The CUDA library (C-ABI) -- loading it must succeed on a GPU machine."""
+    import decode_attention_kv_paged_b200 as attn
+    attn.load()
+    return attn

@@ -1,0 +1,404 @@
+"""Pins of the fp64 CPU oracle against what the pages and mathematics fix.
+
+Each test names the passage it follows.  Page shorthand used below:
+  HEADS  = xuesongtap "attention-head" article
+  MHAVS  = astro-blog "MHA vs MQA vs GQA vs MLA" article
+  EVOL   = toolsku "AI演算法注意力機制演進" article
+  LESSON = llmdeepdive lesson "MQA, GQA e MLA"
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as orc
+from workloads import BLOCK_SIZE, make_block_table
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _paged_from_dense(K, V, block_size=BLOCK_SIZE, perm_seed=None):
+    """Lay dense per-sequence caches [B][H_kv][T][d] into the paged format.
+
+    Returns (k_cache, v_cache, block_table).  With perm_seed, the physical
+    blocks are a random permutation; otherwise the identity.
+    """
+    B, H, T, d = K.shape
+    nb = (T + block_size - 1) // block_size
+    total = B * nb
+    ids = (np.random.default_rng(perm_seed).permutation(total)
+           if perm_seed is not None else np.arange(total))
+    kc = np.zeros((total, H, block_size, d), dtype=K.dtype)
+    vc = np.zeros_like(kc)
+    table = np.full((B, nb), -1, dtype=np.int32)
+    for b in range(B):
+        for i in range(nb):
+            phys = ids[b * nb + i]
+            table[b, i] = phys
+            n = min(block_size, T - i * block_size)
+            kc[phys, :, :n] = K[b, :, i * block_size:i * block_size + n]
+            vc[phys, :, :n] = V[b, :, i * block_size:i * block_size + n]
+    return kc, vc, table
+
+
+# ---------------------------------------------------------------- worked case
+def test_hand_computable_mha_case():
+    """MHAVS "small-matrix" MHA example setup (d_k=2, h=2, seq_len=4, 4x2
+    matrices; its numbers did not survive extraction), with a substitute whose
+    softmax has a closed form: keys e1, e2, e1+e2, 0."""
+    K = np.array([[1, 0], [0, 1], [1, 1], [0, 0]], dtype=np.float64)
+    V = np.array([[1, 2], [3, -1], [-2, 5], [7, 0]], dtype=np.float64)
+    q = np.array([[[1.0, 0.0], [0.0, 1.0]]])          # B=1, two heads
+    # head 0 uses K, V; head 1 uses its own (here: rows permuted) K, V.
+    K1 = K[[1, 0, 3, 2]]
+    V1 = V[[2, 3, 0, 1]]
+    Kd = np.stack([K, K1])[None]                       # [1][2][4][2]
+    Vd = np.stack([V, V1])[None]
+    kc, vc, table = _paged_from_dense(Kd, Vd, block_size=4)
+    scale = 1.0 / math.sqrt(2.0)
+    out, probs = orc.decode_gqa(q, kc, vc, np.array([4]), table, scale,
+                                return_probs=True)
+    e = math.exp(scale)
+    a, b = e / (2 * e + 2), 1.0 / (2 * e + 2)
+    # head 0: q=e1 -> scores [1,0,1,0]/sqrt2
+    p0 = np.array([a, b, a, b])
+    # head 1: q=e2 against rows [e2, e1, 0, e1+e2] -> scores [1,0,0,1]/sqrt2
+    p1 = np.array([a, b, b, a])
+    np.testing.assert_allclose(probs[0, 0], p0, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(probs[0, 1], p1, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(out[0, 0], p0 @ V, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out[0, 1], p1 @ V1, rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------- textbook special cases
+def _rand_problem(rng, B, H_q, H_kv, T, d, block_size=BLOCK_SIZE):
+    q = rng.standard_normal((B, H_q, d))
+    K = rng.standard_normal((B, H_kv, T, d))
+    V = rng.standard_normal((B, H_kv, T, d))
+    return q, K, V
+
+
+def test_single_token_returns_its_value_row():
+    """T=1: softmax over one key is 1, so out = v_0 (HEADS §1 equation)."""
+    rng = np.random.default_rng(1)
+    q, K, V = _rand_problem(rng, 2, 4, 2, 1, 16)
+    kc, vc, table = _paged_from_dense(K, V)
+    out = orc.decode_gqa(q, kc, vc, np.array([1, 1]), table, 0.25)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_array_equal(out[b, h], V[b, h // 2, 0])
+
+
+def test_identical_keys_give_mean_of_values():
+    """Identical keys -> equal scores -> uniform p -> mean of V (HEADS §1)."""
+    rng = np.random.default_rng(2)
+    T, d = 70, 8
+    K = np.broadcast_to(rng.standard_normal(d), (1, 1, T, d)).copy()
+    V = rng.standard_normal((1, 1, T, d))
+    q = rng.standard_normal((1, 1, d))
+    kc, vc, table = _paged_from_dense(K, V)
+    out, probs = orc.decode_gqa(q, kc, vc, np.array([T]), table, 0.3,
+                                return_probs=True)
+    np.testing.assert_allclose(probs[0, 0], np.full(T, 1.0 / T), atol=1e-16)
+    np.testing.assert_allclose(out[0, 0], V[0, 0].mean(axis=0), atol=1e-14)
+
+
+def test_dominant_score_selects_its_value_row():
+    """One score larger than the rest by 40 -> p concentrates on that key."""
+    rng = np.random.default_rng(3)
+    T, d = 100, 4
+    K = np.zeros((1, 1, T, d))
+    K[0, 0, 37, 0] = 40.0
+    V = rng.standard_normal((1, 1, T, d))
+    q = np.zeros((1, 1, d))
+    q[0, 0, 0] = 1.0
+    kc, vc, table = _paged_from_dense(K, V)
+    out = orc.decode_gqa(q, kc, vc, np.array([T]), table, 1.0)
+    np.testing.assert_allclose(out[0, 0], V[0, 0, 37], atol=1e-14)
+
+
+def test_rows_sum_to_one_and_match_library_softmax():
+    """Softmax is taken along key positions (HEADS §1): each row of p sums to
+    1 and equals scipy's softmax of the scaled dense scores; the output equals
+    p @ V computed densely (independent textbook formulation)."""
+    rng = np.random.default_rng(4)
+    B, H_q, H_kv, T, d = 3, 6, 3, 150, 32
+    q, K, V = _rand_problem(rng, B, H_q, H_kv, T, d)
+    lens = np.array([150, 1, 97])
+    kc, vc, table = _paged_from_dense(K, V, perm_seed=11)
+    scale = 1 / math.sqrt(d)
+    out, probs = orc.decode_gqa(q, kc, vc, lens, table, scale,
+                                return_probs=True)
+    G = H_q // H_kv
+    for b in range(B):
+        for h in range(H_q):
+            n = lens[b]
+            Kd, Vd = K[b, h // G, :n], V[b, h // G, :n]
+            p = scipy.special.softmax(scale * (Kd @ q[b, h]))
+            assert abs(probs[b, h, :n].sum() - 1.0) < 1e-14
+            np.testing.assert_allclose(probs[b, h, :n], p, rtol=1e-12,
+                                       atol=1e-16)
+            assert np.all(probs[b, h, n:] == 0)
+            np.testing.assert_allclose(out[b, h], p @ Vd, rtol=1e-12,
+                                       atol=1e-13)
+
+
+def test_empty_sequence_gives_zero_row():
+    rng = np.random.default_rng(5)
+    q, K, V = _rand_problem(rng, 2, 2, 1, 64, 16)
+    kc, vc, table = _paged_from_dense(K, V)
+    out = orc.decode_gqa(q, kc, vc, np.array([0, 64]), table, 0.25)
+    assert np.all(out[0] == 0)
+    assert np.any(out[1] != 0)
+
+
+# ------------------------------------------------------------- head sharing
+@pytest.mark.parametrize("case", _golden("head_groups.json")["cases"],
+                         ids=lambda c: f"{c['H_q']}q{c['H_kv']}kv")
+def test_group_mapping_matches_page(case):
+    """HEADS §2 figure and group rule; LESSON (24 over 4 in groups of 6).
+    Each KV head gets a distinct constant value row; the output of query head
+    h reveals which KV head it read."""
+    H_q, H_kv = case["H_q"], case["H_kv"]
+    T, d = 5, 4
+    K = np.zeros((1, H_kv, T, d))
+    V = np.zeros((1, H_kv, T, d))
+    for g in range(H_kv):
+        V[0, g, :, 0] = g
+    q = np.ones((1, H_q, d))
+    kc, vc, table = _paged_from_dense(K, V)
+    out = orc.decode_gqa(q, kc, vc, np.array([T]), table, 1.0)
+    got = [int(round(out[0, h, 0])) for h in range(H_q)]
+    assert got == case["kv_head_of_q_head"]
+
+
+def test_gqa_with_hkv_equal_hq_is_mha_head_by_head():
+    """H_kv = H_q is MHA (HEADS §2.2): each head equals a one-head problem."""
+    rng = np.random.default_rng(6)
+    B, H, T, d = 2, 5, 130, 16
+    q, K, V = _rand_problem(rng, B, H, H, T, d)
+    kc, vc, table = _paged_from_dense(K, V, perm_seed=3)
+    out = orc.decode_gqa(q, kc, vc, np.array([T, 77]), table, 0.25)
+    for h in range(H):
+        kc1, vc1, t1 = _paged_from_dense(K[:, h:h + 1], V[:, h:h + 1])
+        o1 = orc.decode_gqa(q[:, h:h + 1], kc1, vc1, np.array([T, 77]), t1,
+                            0.25)
+        np.testing.assert_array_equal(out[:, h], o1[:, 0])
+
+
+@pytest.mark.parametrize("H_q,H_kv", [(8, 1), (24, 4), (32, 8)])
+def test_shared_kv_equals_mha_with_replicated_kv(H_q, H_kv):
+    """MQA/GQA equal MHA whose K/V are replicated over each group
+    (EVOL repeat_kv expansion; HEADS §2.1, §2.2)."""
+    rng = np.random.default_rng(7)
+    B, T, d = 2, 90, 8
+    q, K, V = _rand_problem(rng, B, H_q, H_kv, T, d)
+    G = H_q // H_kv
+    Krep = np.repeat(K, G, axis=1)
+    Vrep = np.repeat(V, G, axis=1)
+    kc, vc, t = _paged_from_dense(K, V, perm_seed=5)
+    kr, vr, tr = _paged_from_dense(Krep, Vrep, perm_seed=6)
+    lens = np.array([T, 41])
+    a = orc.decode_gqa(q, kc, vc, lens, t, 0.35)
+    b = orc.decode_gqa(q, kr, vr, lens, tr, 0.35)
+    np.testing.assert_array_equal(a, b)
+    # sensitivity: the wrong (interleaved, h % H_kv) expansion differs
+    if H_kv > 1:
+        idx = [h % H_kv for h in range(H_q)]
+        kw, vw, tw = _paged_from_dense(K[:, idx], V[:, idx])
+        c = orc.decode_gqa(q, kw, vw, lens, tw, 0.35)
+        assert np.abs(a - c).max() > 1e-3
+
+
+# ----------------------------------------------------------- sliding window
+@pytest.mark.parametrize("case", _golden("window_membership.json")["cases"],
+                         ids=lambda c: f"w{c['window']}")
+def test_window_membership_matches_page_figure(case):
+    """HEADS §3 figure: row i=8, w=3 keeps {6,7,8}; full causal keeps 0..8."""
+    T, w = case["T"], case["window"]
+    lo, hi = orc.visible_range(T, w)
+    assert list(range(lo, hi)) == case["visible"]
+    rng = np.random.default_rng(8)
+    q, K, V = _rand_problem(rng, 1, 1, 1, T, 4)
+    kc, vc, table = _paged_from_dense(K, V)
+    _, probs = orc.decode_gqa(q, kc, vc, np.array([T]), table, 0.5, window=w,
+                              return_probs=True)
+    assert [j for j in range(T) if probs[0, 0, j] > 0] == case["visible"]
+
+
+def test_window_brute_force_membership():
+    """Brute force over small T and w: the visible set is exactly the w most
+    recent positions, the current one included (HEADS §3)."""
+    for T in range(0, 12):
+        for w in range(0, 14):
+            lo, hi = orc.visible_range(T, w)
+            expect = [j for j in range(T) if w <= 0 or T - 1 - j < w]
+            assert list(range(lo, hi)) == expect, (T, w)
+
+
+def test_window_at_least_T_equals_full_causal():
+    """A window w >= T drops nothing (BASELINE pin (d); HEADS §3)."""
+    rng = np.random.default_rng(9)
+    q, K, V = _rand_problem(rng, 2, 4, 2, 200, 16)
+    kc, vc, table = _paged_from_dense(K, V, perm_seed=1)
+    lens = np.array([200, 65])
+    full = orc.decode_gqa(q, kc, vc, lens, table, 0.25)
+    for w in (200, 201, 10_000):
+        np.testing.assert_array_equal(
+            orc.decode_gqa(q, kc, vc, lens, table, 0.25, window=w), full)
+    part = orc.decode_gqa(q, kc, vc, lens, table, 0.25, window=64)
+    assert np.abs(part - full).max() > 1e-3
+
+
+# ------------------------------------------------------------------- paging
+def test_permuted_block_table_equals_identity_table():
+    """The block table only relocates blocks: a random permutation gives the
+    bit-identical result of the identity layout (paging, Baidu article §4.3)."""
+    rng = np.random.default_rng(10)
+    q, K, V = _rand_problem(rng, 3, 8, 2, 333, 32)
+    lens = np.array([333, 64, 65])
+    kc0, vc0, t0 = _paged_from_dense(K, V)
+    a = orc.decode_gqa(q, kc0, vc0, lens, t0, 0.2)
+    kc, vc, t = _paged_from_dense(K, V, perm_seed=42)
+    b = orc.decode_gqa(q, kc, vc, lens, t, 0.2)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_slot_offset_follows_block_table():
+    table = np.array([[5, 2, 9], [0, 1, 3]], dtype=np.int32)
+    # position 130 of sequence 0 -> logical block 2 -> physical 9, slot 2
+    off = orc.slot_offset(table, 0, 130, 64, 4, 3, 16)
+    assert off == ((9 * 4 + 3) * 64 + 2) * 16
+
+
+# --------------------------------------------------------------- precision
+def test_bf16_inputs_widen_exactly():
+    """bf16 inputs are read as the exact fp64 value of the bf16 number."""
+    rng = np.random.default_rng(12)
+    qf, Kf, Vf = _rand_problem(rng, 1, 2, 1, 70, 16)
+    q16 = torch.from_numpy(qf).to(torch.bfloat16)
+    K16 = torch.from_numpy(Kf).to(torch.bfloat16)
+    V16 = torch.from_numpy(Vf).to(torch.bfloat16)
+    kc, vc, table = _paged_from_dense(K16.double().numpy(),
+                                      V16.double().numpy())
+    ref = orc.decode_gqa(q16.double().numpy(), kc, vc, np.array([70]), table,
+                         0.25)
+    kc16 = torch.from_numpy(kc).to(torch.bfloat16)
+    vc16 = torch.from_numpy(vc).to(torch.bfloat16)
+    got = orc.decode_gqa(q16, kc16, vc16, np.array([70]), table, 0.25)
+    np.testing.assert_array_equal(ref, got)
+
+
+# --------------------------------------------------------------------- MLA
+def _mla_problem(rng, B, H, d_c, d_r, d_h, d_v, T):
+    latent = rng.standard_normal((B, T, d_c + d_r)) / math.sqrt(d_c + d_r)
+    q_c = rng.standard_normal((B, H, d_h))
+    q_r = rng.standard_normal((B, H, d_r))
+    U_K = rng.standard_normal((H, d_c, d_h)) / math.sqrt(d_c)
+    U_V = rng.standard_normal((H, d_c, d_v)) / math.sqrt(d_c)
+    return latent, q_c, q_r, U_K, U_V
+
+
+def _paged_latent(latent, block_size=BLOCK_SIZE, perm_seed=None):
+    B, T, w = latent.shape
+    K = latent[:, None]                  # treat as one "head"
+    kc, _, table = _paged_from_dense(K, K, block_size, perm_seed)
+    return kc[:, 0], table
+
+
+@pytest.mark.parametrize("d_r", [0, 4])
+def test_mla_absorbed_equals_explicit(d_r):
+    """HEADS §5.2: q^C (U^K)^T c^T = q~ c^T and sum p (c U^V) = (sum p c) U^V
+    exactly; §5.3: one softmax over content + RoPE scores with scale
+    1/sqrt(d_c' + d_R).  Absorbed oracle (+ library matmuls for q~ and z U^V)
+    must equal the explicit per-head expansion to 1e-12."""
+    rng = np.random.default_rng(13)
+    B, H, d_c, d_h, d_v, T = 2, 3, 16, 8, 6, 75
+    latent, q_c, q_r, U_K, U_V = _mla_problem(rng, B, H, d_c, d_r, d_h, d_v, T)
+    cache, table = _paged_latent(latent, perm_seed=2)
+    lens = np.array([75, 13])
+    scale = 1.0 / math.sqrt(d_h + d_r)
+    o_explicit = orc.mla_explicit(q_c, q_r, cache, lens, table, U_K, U_V,
+                                  scale)
+    q_tilde = np.einsum("bhi,hci->bhc", q_c, U_K)     # q^C (U^K_h)^T
+    z = orc.decode_mla(q_tilde, q_r, cache, lens, table, scale)
+    o_absorbed = np.einsum("bhc,hcv->bhv", z, U_V)    # z U^V_h
+    np.testing.assert_allclose(o_absorbed, o_explicit, rtol=0, atol=1e-12)
+
+
+def test_mla_rope_branch_changes_scores():
+    """The decoupled RoPE branch contributes to the scores only (HEADS §5.3):
+    zeroing k^R changes the result, zeroing the rope columns of the output
+    is impossible since z is d_c wide."""
+    rng = np.random.default_rng(14)
+    B, H, d_c, d_r, T = 1, 2, 8, 4, 40
+    latent = rng.standard_normal((B, T, d_c + d_r))
+    cache, table = _paged_latent(latent)
+    q_l = rng.standard_normal((B, H, d_c))
+    q_r = rng.standard_normal((B, H, d_r)) * 3
+    z = orc.decode_mla(q_l, q_r, cache, np.array([T]), table, 0.3)
+    assert z.shape == (B, H, d_c)
+    cache0 = cache.copy()
+    cache0[..., d_c:] = 0
+    z0 = orc.decode_mla(q_l, q_r, cache0, np.array([T]), table, 0.3)
+    assert np.abs(z - z0).max() > 1e-3
+
+
+def test_mla_matches_dense_library_softmax():
+    rng = np.random.default_rng(15)
+    B, H, d_c, d_r, T = 2, 4, 32, 8, 130
+    latent = rng.standard_normal((B, T, d_c + d_r))
+    cache, table = _paged_latent(latent, perm_seed=9)
+    q_l = rng.standard_normal((B, H, d_c))
+    q_r = rng.standard_normal((B, H, d_r))
+    lens = np.array([130, 64])
+    z = orc.decode_mla(q_l, q_r, cache, lens, table, 0.1)
+    for b in range(B):
+        n = lens[b]
+        C, KR = latent[b, :n, :d_c], latent[b, :n, d_c:]
+        for h in range(H):
+            p = scipy.special.softmax(0.1 * (C @ q_l[b, h] + KR @ q_r[b, h]))
+            np.testing.assert_allclose(z[b, h], p @ C, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------- bytes model
+def test_cache_bytes_closed_form_matches_page_table():
+    g = _golden("cache_bytes.json")
+    MiB, GiB, KiB = 2.0 ** 20, 2.0 ** 30, 2.0 ** 10
+    for row in g["kv_per_layer_MiB"]:
+        got = orc.bytes_kv(row["B"], row["T"], row["H_kv"], row["d"], row["s"])
+        assert got == row["MiB"] * MiB
+    r = g["kv_32_layers_GiB"]
+    assert orc.bytes_kv(r["B"], r["T"], r["H_kv"], r["d"], r["s"]) * \
+        r["layers"] == r["GiB"] * GiB
+    m = g["mla"]
+    lat = orc.bytes_mla(m["B"], m["T"], m["r"], m["d_R"], m["s"])
+    assert lat / (m["B"] * m["T"] * m["s"]) == m["latent_elems_per_token"]
+    expanded = m["H"] * (m["d_c_head"] + m["d_R"] + m["d_v"])
+    assert expanded == m["expanded_elems_per_token"]
+    assert round(expanded / m["latent_elems_per_token"], 1) == m["ratio_approx"]
+    assert round(lat / MiB) == m["latent_MiB_approx"]
+    assert round(m["B"] * m["T"] * expanded * m["s"] / GiB, 1) == \
+        m["expanded_GiB_approx"]
+    for row in g["per_token_per_layer_KiB"]:
+        assert orc.bytes_kv(1, 1, row["H_kv"], row["d"], row["s"]) == \
+            row["KiB"] * KiB
+
+
+def test_workload_block_tables_are_permutations():
+    """The seeded generator's tables index every owned block exactly once."""
+    g = torch.Generator().manual_seed(0)
+    lens = [1, 64, 65, 1000]
+    table, nblk = make_block_table(lens, g)
+    ids = table[table >= 0].tolist()
+    assert sorted(ids) == list(range(nblk))
+    assert [(table[b] >= 0).sum().item() for b in range(4)] == [1, 1, 2, 16]
