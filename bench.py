@@ -1,0 +1,530 @@
+"""Benchmark: paged decode attention on B200 -- decode tokens/s and KV GB/s.
+
+One step = one decode-attention call of the whole hot path (split planning,
+paged block gather, K/V tile streaming, scores, online softmax, P V, split
+partials, log-sum-exp combine) over one batch of synthetic inputs resident in
+HBM.  Default workload: Llama-3-8B-shaped GQA (B=16, H_q=32, H_kv=8, d=128,
+T=4096, bf16, 64-token blocks, random-permutation block table).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl native|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU, each rank with its
+own batch (weak scaling; ranks share nothing on the data path -- the only
+collectives are the timing barrier and the max-over-ranks reduction).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = {
+    "gqa": ["decode_attention_kv_paged_b200/csrc/gqa_decode.cuh",
+            "decode_attention_kv_paged_b200/csrc/plan.cuh",
+            "decode_attention_kv_paged_b200/csrc/common.cuh"],
+    "mla": ["decode_attention_kv_paged_b200/csrc/mla_decode.cu",
+            "decode_attention_kv_paged_b200/csrc/plan.cuh",
+            "decode_attention_kv_paged_b200/csrc/common.cuh"],
+}
+
+WORKLOAD_ALIASES = {
+    "llama3_8b": W.LLAMA3_8B.name,
+    "tiny": W.TINY.name,
+    "ragged_full": W.RAGGED_FULL.name,
+    "ragged_window": W.RAGGED_WINDOW.name,
+    "mla": W.MLA_DSV2.name,
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="llama3_8b",
+                    help="llama3_8b | tiny | ragged_full | ragged_window | mla "
+                         "| a sweep name such as sweep_bf16_B8_Hq32_Hkv8_d128_T32768")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def workload(name):
+    return W.WORKLOADS[WORKLOAD_ALIASES.get(name, name)]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        return j, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_hash(kind):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kind, wl_name):
+    """dram bytes per launch from the committed ncu summary, if the kernel
+    source is unchanged since it was taken; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        j = json.load(f)
+    e = j.get(wl_name)
+    if not e or e.get("kernel_hash") != kernel_hash(kind):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+        return False
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for _, _, parts in rows:
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ distributed
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- helpers
+def algorithmic_bytes_gqa(inp):
+    """K+V bytes of visible keys (both caches) + q + out."""
+    cfg = inp.cfg
+    s = torch.finfo(cfg.dtype).bits // 8
+    vis = 0
+    for T in inp.seq_list:
+        lo = max(0, T - inp.window) if inp.window > 0 else 0
+        vis += max(0, T - lo)
+    kv = vis * cfg.H_kv * cfg.d * 2 * s
+    qo = 2 * cfg.B * cfg.H_q * cfg.d * s
+    return kv, kv + qo
+
+
+def tile_bytes_gqa(inp):
+    """Bytes the kernel reads in whole 64-token tiles (incl. edge over-read)."""
+    cfg = inp.cfg
+    s = torch.finfo(cfg.dtype).bits // 8
+    blocks = 0
+    for T in inp.seq_list:
+        if T <= 0:
+            continue
+        lo = max(0, T - inp.window) if inp.window > 0 else 0
+        blocks += (T - 1) // 64 - lo // 64 + 1
+    return blocks * 64 * cfg.H_kv * cfg.d * 2 * s
+
+
+def algorithmic_bytes_mla(inp):
+    cfg = inp.cfg
+    lat = sum(inp.seq_list) * (cfg.d_c + cfg.d_r) * 2
+    qo = cfg.B * cfg.H * (2 * cfg.d_c + cfg.d_r) * 2
+    return lat, lat + qo
+
+
+def mla_flops(inp):
+    cfg = inp.cfg
+    return sum(inp.seq_list) * cfg.H * 2 * (2 * cfg.d_c + cfg.d_r)
+
+
+# ------------------------------------------------------------ native arm
+def run_native(args, rank, world, local):
+    import decode_attention_kv_paged_b200 as attn
+    attn.load()
+    cfg = workload(args.workload)
+    is_mla = isinstance(cfg, W.MLAConfig)
+    dev = torch.device("cuda", local)
+    seed = cfg.seed + 1000 * rank
+    if is_mla:
+        base = W.make_mla_inputs(cfg, device=dev, seed=seed)
+        kv_bytes, alg_bytes = algorithmic_bytes_mla(base)
+        cache_bytes = base.latent_cache.numel() * 2
+    else:
+        base = W.make_gqa_inputs(cfg, device=dev, seed=seed)
+        kv_bytes, alg_bytes = algorithmic_bytes_gqa(base)
+        cache_bytes = (base.k_cache.numel() + base.v_cache.numel()) * \
+            base.k_cache.element_size()
+    # Rotate among enough cache replicas that consecutive steps never find
+    # the previous step's cache in the 126 MB L2.
+    reps = max(2, math.ceil(3 * L2_BYTES / max(cache_bytes, 1)))
+    reps = min(reps, 64)
+    inputs = [base]
+    for r in range(1, reps):
+        if is_mla:
+            inputs.append(W.make_mla_inputs(cfg, device=dev, seed=seed + r))
+        else:
+            inputs.append(W.make_gqa_inputs(cfg, device=dev, seed=seed + r))
+    outs = [torch.empty_like(i.q_lat if is_mla else i.q) for i in inputs]
+
+    def step(i):
+        x = inputs[i % reps]
+        if is_mla:
+            attn.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
+                            x.block_table, x.scale, out=outs[i % reps])
+        else:
+            attn.decode_gqa(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                            x.scale, window=x.window, out=outs[i % reps])
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    if attn.last_error() != attn.OK:
+        raise SystemExit("device error during warm-up")
+
+    K = args.steps
+    prof = attn.ProfileEvents(K)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        with prof:
+            ev0.record()
+            for i in range(K):
+                step(i)
+            ev1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    kern_ms = prof.times_ms(K)
+    if attn.last_error() != attn.OK:
+        raise SystemExit("device error during the timed region")
+    ms_max = max_over_ranks(ms, world)
+    kern_avg = max_over_ranks(sum(kern_ms) / K, world)
+
+    B = cfg.B
+    value = world * B * K / (ms_max / 1e3)            # tokens/s, whole job
+    kv_gbs = world * kv_bytes * K / (ms_max / 1e3) / 1e9
+    pk, pk_kind = peaks()
+    wl_name = cfg.name
+    kind = "mla" if is_mla else "gqa"
+    if is_mla:
+        flops = mla_flops(base)
+        t_hbm = alg_bytes / (pk["hbm_gbs"] * 1e9)
+        t_tc = flops / (pk.get("bf16_tflops", 1590.0) * 1e12)
+        if t_tc > t_hbm:
+            achieved = flops / (kern_avg / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved,
+                    "peak": pk.get("bf16_tflops"), "unit": "TFLOP/s"}
+        else:
+            achieved = alg_bytes / (kern_avg / 1e3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s"}
+    else:
+        achieved = alg_bytes / (kern_avg / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = pk_kind
+    roof["kernel"] = "mla_decode_kernel" if is_mla else "gqa_split_kernel"
+    roof["kernel_ms_avg"] = kern_avg
+    roof["algorithmic_bytes_per_launch"] = alg_bytes
+    roof["traffic"] = traffic_for(kind, wl_name)
+
+    line = {
+        "metric": "decode tokens/s and KV-cache read GB/s (% of B200 HBM peak), 1 GPU",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) q/K/V, random-permutation block table)",
+        "config": {"workload": wl_name, "global_batch": B * world,
+                   "seq_len": getattr(cfg, "T", None) or max(base.seq_list),
+                   "parallelism": f"dp{world} (independent batches, no collective)",
+                   "l2": f"inputs larger than L2, rotated among {reps} cache "
+                         f"replicas ({cache_bytes / 2**20:.0f} MiB each)"},
+        "kv_gbs": kv_gbs,
+        "kv_frac_of_peak": kv_gbs / world / pk["hbm_gbs"],
+        "kv_frac_of_8tbs_spec": kv_gbs / world / 8000.0,
+        "roofline": roof,
+        "gpu_launches": (1 if is_mla else 2) * K,
+        "clocks": clk.summary(),
+    }
+    if not is_mla:
+        line["tile_overread_bytes_per_step"] = tile_bytes_gqa(base) - kv_bytes
+    if not args.no_e2e:
+        line["e2e"] = e2e_native(attn, cfg, inputs[0], is_mla, K, world, dev)
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(cfg, is_mla, args.cpu_seconds)
+    return line
+
+
+def e2e_native(attn, cfg, x, is_mla, K, world, dev):
+    """The same metric through the public API with host buffers: each step
+    copies the new token's q (and K/V or latent row) from pinned host memory,
+    appends it to the paged cache at position T-1, runs decode attention and
+    reads the output back to the host."""
+    B = cfg.B
+    g = torch.Generator().manual_seed(7)
+    if is_mla:
+        width = cfg.d_c + cfg.d_r
+        h_q = W.randn((B, cfg.H, cfg.d_c), g, torch.bfloat16).pin_memory()
+        h_r = W.randn((B, cfg.H, cfg.d_r), g, torch.bfloat16).pin_memory()
+        h_lat = W.randn((B, width), g, torch.bfloat16).pin_memory()
+        h_out = torch.empty((B, cfg.H, cfg.d_c), dtype=torch.bfloat16).pin_memory()
+        d_q, d_r, d_lat = (torch.empty_like(t, device=dev) for t in (h_q, h_r, h_lat))
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_r, h_lat))
+    else:
+        h_q = W.randn((B, cfg.H_q, cfg.d), g, cfg.dtype).pin_memory()
+        h_k = W.randn((B, cfg.H_kv, cfg.d), g, cfg.dtype).pin_memory()
+        h_v = W.randn((B, cfg.H_kv, cfg.d), g, cfg.dtype).pin_memory()
+        h_out = torch.empty_like(h_q).pin_memory()
+        d_q, d_k, d_v = (torch.empty_like(t, device=dev) for t in (h_q, h_k, h_v))
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
+    d2h = h_out.numel() * h_out.element_size()
+    pos = (x.seq_lens - 1).clamp(min=0).contiguous()
+    d_out = torch.empty_like(h_out, device=dev)
+
+    def step():
+        d_q.copy_(h_q, non_blocking=True)
+        if is_mla:
+            d_r.copy_(h_r, non_blocking=True)
+            d_lat.copy_(h_lat, non_blocking=True)
+            attn.kv_append_mla(d_lat, x.latent_cache, pos, x.block_table)
+            attn.decode_mla(d_q, d_r, x.latent_cache, x.seq_lens, x.block_table,
+                            x.scale, out=d_out)
+        else:
+            d_k.copy_(h_k, non_blocking=True)
+            d_v.copy_(h_v, non_blocking=True)
+            attn.kv_append(d_k, d_v, x.k_cache, x.v_cache, pos, x.block_table)
+            attn.decode_gqa(d_q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                            x.scale, window=x.window, out=d_out)
+        h_out.copy_(d_out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"value": world * B * K / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / K,
+            "note": "cache stays resident (L2 not rotated); step = H2D of the new "
+                    "token's inputs + kv_append + decode + D2H of the output"}
+
+
+# ------------------------------------------------------------- oracle arm
+def _oracle_problem(cfg, is_mla, seqs, seed):
+    """Host-resident inputs of the first `seqs` sequences of the workload."""
+    if is_mla:
+        sub = W.MLAConfig(cfg.name, B=seqs, H=cfg.H, d_c=cfg.d_c, d_r=cfg.d_r,
+                          T=cfg.T, seed=seed)
+        return W.make_mla_inputs(sub)
+    lens = None
+    if cfg.ragged:
+        g = torch.Generator().manual_seed(cfg.seed)
+        lens = W.draw_seq_lens(cfg, g)[:seqs]
+    sub = W.GQAConfig(cfg.name, B=seqs, H_q=cfg.H_q, H_kv=cfg.H_kv, d=cfg.d,
+                      seq_lens=lens, T=cfg.T, dtype=cfg.dtype, window=cfg.window,
+                      contiguous=cfg.contiguous, seed=seed)
+    return W.make_gqa_inputs(sub)
+
+
+def _oracle_call(orc, x, is_mla):
+    if is_mla:
+        return orc.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
+                              x.block_table, x.scale)
+    return orc.decode_gqa(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                          x.scale, window=x.window)
+
+
+def _pick_sample(cfg, is_mla, orc, target_s):
+    """Sequences per oracle call sized to ~target_s of CPU time."""
+    x = _oracle_problem(cfg, is_mla, 1, cfg.seed)
+    t0 = time.perf_counter()
+    _oracle_call(orc, x, is_mla)
+    one = max(time.perf_counter() - t0, 1e-4)
+    return max(1, min(cfg.B, int(target_s / one))), one
+
+
+def cpu_baseline(cfg, is_mla, target_s):
+    import oracle as orc
+    cores = os.cpu_count() or 1
+    orc.set_threads(cores)
+    n, _ = _pick_sample(cfg, is_mla, orc, target_s)
+    x = _oracle_problem(cfg, is_mla, n, cfg.seed)
+    t0 = time.perf_counter()
+    _oracle_call(orc, x, is_mla)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": orc.get_threads(),
+            "kind": "oracle",
+            "sample": f"{n} of the workload's {cfg.B} sequences (fp64 C oracle, "
+                      f"OpenMP), one pass, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle as it stands, on the host cores."""
+    if rank != 0:
+        return None
+    import oracle as orc
+    cfg = workload(args.workload)
+    is_mla = isinstance(cfg, W.MLAConfig)
+    cores = os.cpu_count() or 1
+    orc.set_threads(cores)
+    # bound the whole run to a few minutes: each step ~ budget / (K + W)
+    per_step = max(0.2, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+    n, _ = _pick_sample(cfg, is_mla, orc, per_step)
+    x = _oracle_problem(cfg, is_mla, n, cfg.seed)
+    for _ in range(max(args.warmup, 3) if per_step < 1 else 1):
+        _oracle_call(orc, x, is_mla)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_call(orc, x, is_mla)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = (f"{n} of {cfg.B} sequences per step (fp64 C oracle, OpenMP over "
+              f"{orc.get_threads()} threads)")
+    return {
+        "impl": "reference",
+        "metric": "decode tokens/s and KV-cache read GB/s (% of B200 HBM peak), 1 GPU",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (same seeded recipe)",
+        "config": {"workload": cfg.name, "global_batch": cfg.B},
+        "cpu_baseline": {"value": value, "unit": "tokens/s",
+                         "cores": orc.get_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        line = run_native(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,348 @@
+// api.cu -- the C ABI of libattn_decode.so (declared in include/attn_decode.h):
+// argument validation, per-device state (split workspace, error word), launch
+// configuration, test and profiling hooks.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "attn_decode.h"
+#include "gqa_launch.cuh"
+#include "kv_append.cuh"
+#include "mla_launch.cuh"
+
+namespace attn {
+
+__device__ unsigned g_err_word;   // per-device error word (bits kErr*)
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned *err = nullptr;      // device address of g_err_word
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+};
+
+static std::mutex g_mu;
+static std::vector<DeviceState> g_dev;
+static thread_local int tl_num_ctas = 0;
+static thread_local int tl_gqa_path = -1;
+static std::atomic<int> g_force_timeout{0};
+static std::atomic<long long> g_force_timeout_ns{0};
+static const void *const *g_prof_start = nullptr;
+static const void *const *g_prof_stop = nullptr;
+static int g_prof_n = 0, g_prof_i = 0;
+
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
+
+// Per-device state of the current device (created on first use).
+static int device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
+    DeviceState &st = g_dev[dev];
+    if (!st.ready) {
+        if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess)
+            return ATTN_ERR_CUDA;
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&st.err), g_err_word) !=
+            cudaSuccess)
+            return ATTN_ERR_CUDA;
+        st.ready = true;
+    }
+    *out = &st;
+    return ATTN_OK;
+}
+
+// Grow the device's split workspace to at least `bytes`.  Never during
+// stream capture (a graph must not depend on an allocation made inside it).
+static int ensure_workspace(DeviceState *st, size_t bytes, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (st->ws_bytes >= bytes) return ATTN_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return ATTN_ERR_UNSUPPORTED;
+    size_t want = bytes < 2 * st->ws_bytes ? 2 * st->ws_bytes : bytes;
+    want = (want + (1u << 20) - 1) & ~(size_t)((1u << 20) - 1);
+    if (st->ws) {
+        cudaFree(st->ws);   // implicitly waits for work that may still use it
+        st->ws = nullptr;
+        st->ws_bytes = 0;
+    }
+    if (cudaMalloc(&st->ws, want) != cudaSuccess) return ATTN_ERR_CUDA;
+    st->ws_bytes = want;
+    return ATTN_OK;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static bool aligned16(const void *p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+static bool valid_head_dim(int d) {
+    return d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
+}
+
+// Query heads per CTA for a group of G: the largest instantiated divisor.
+static int heads_per_cta(int G) {
+    static const int options[] = {8, 6, 4, 3, 2, 1};
+    for (int hc : options)
+        if (G % hc == 0) return hc;
+    return 1;
+}
+
+static void take_profile_events(cudaEvent_t *start, cudaEvent_t *stop) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    *start = nullptr;
+    *stop = nullptr;
+    if (g_prof_n > 0 && g_prof_i < g_prof_n) {
+        *start = (cudaEvent_t)g_prof_start[g_prof_i];
+        *stop = (cudaEvent_t)g_prof_stop[g_prof_i];
+        ++g_prof_i;
+    }
+}
+
+static void take_force_timeout(int *flag, unsigned long long *ns) {
+    *flag = g_force_timeout.exchange(0);
+    long long t = g_force_timeout_ns.load();
+    *ns = (*flag && t > 0) ? (unsigned long long)t : kDefaultTimeoutNs;
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_version(void) { return 100; }
+
+const char *attn_status_string(int s) {
+    switch (s) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_ARG: return "ATTN_ERR_ARG";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+        case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+        case ATTN_ERR_BAD_BLOCK: return "ATTN_ERR_BAD_BLOCK";
+        case ATTN_ERR_BAD_SEQLEN: return "ATTN_ERR_BAD_SEQLEN";
+        default: return "ATTN_UNKNOWN_STATUS";
+    }
+}
+
+int attn_set_num_ctas(int n) {
+    if (n < 0) return ATTN_ERR_ARG;
+    tl_num_ctas = n;
+    return ATTN_OK;
+}
+
+int attn_set_gqa_path(int path) {
+    if (path < -1 || path > 1) return ATTN_ERR_ARG;
+    tl_gqa_path = path;
+    return ATTN_OK;
+}
+
+int attn_set_profile_events(void *const *start_events, void *const *stop_events,
+                            int n) {
+    if (n < 0 || (n > 0 && (!start_events || !stop_events))) return ATTN_ERR_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_prof_start = start_events;
+    g_prof_stop = stop_events;
+    g_prof_n = n;
+    g_prof_i = 0;
+    return ATTN_OK;
+}
+
+int attn_debug_force_timeout(int enable, long long timeout_ns) {
+    if (timeout_ns < 0) return ATTN_ERR_ARG;
+    g_force_timeout_ns.store(timeout_ns);
+    g_force_timeout.store(enable ? 1 : 0);
+    return ATTN_OK;
+}
+
+int attn_decode_last_error(void *stream) {
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    unsigned word = 0, zero = 0;
+    if (cudaMemcpy(&word, st->err, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (word && cudaMemcpy(st->err, &zero, sizeof zero, cudaMemcpyHostToDevice) !=
+                    cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (word & kErrTimeout) return ATTN_ERR_TIMEOUT;
+    if (word & kErrBadBlock) return ATTN_ERR_BAD_BLOCK;
+    if (word & kErrBadSeqLen) return ATTN_ERR_BAD_SEQLEN;
+    return ATTN_OK;
+}
+
+int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype, int *num_ctas,
+                           int *heads, int *path) {
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv || !valid_head_dim(d) ||
+        (dtype != ATTN_F32 && dtype != ATTN_BF16))
+        return ATTN_ERR_ARG;
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    if (num_ctas) *num_ctas = tl_num_ctas > 0 ? tl_num_ctas : st->num_sms;
+    if (heads) *heads = heads_per_cta(H_q / H_kv);
+    if (path) *path = 0;
+    return ATTN_OK;
+}
+
+int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seq_lens, const int32_t *block_table, void *out,
+                    int B, int H_q, int H_kv, int d, float scale, int window,
+                    void *stream, int max_blocks_per_seq, int num_blocks, int dtype) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !block_table || !out) return ATTN_ERR_ARG;
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return ATTN_ERR_ARG;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
+    if (dtype != ATTN_F32 && dtype != ATTN_BF16) return ATTN_ERR_ARG;
+    if (!std::isfinite(scale)) return ATTN_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return ATTN_ERR_ARG;
+    if (!valid_head_dim(d)) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_F32 && d > 128) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)max_blocks_per_seq * kBlockSize > (1ll << 30)) return ATTN_ERR_ARG;
+
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+
+    const int G = H_q / H_kv;
+    const int HC = heads_per_cta(G);
+    const int n_hc = G / HC;
+    const int P = tl_num_ctas > 0 ? tl_num_ctas : st->num_sms;
+    const long long units_total = (long long)B * H_kv * n_hc;
+    if (units_total > (1ll << 30)) return ATTN_ERR_ARG;
+    const long long slots = units_total + P;
+
+    const size_t o_bytes = align256((size_t)slots * HC * d * sizeof(float));
+    const size_t lse_bytes = align256((size_t)slots * HC * sizeof(float));
+    const size_t pre_bytes = align256((size_t)(B + 1) * sizeof(long long));
+    rc = ensure_workspace(st, o_bytes + lse_bytes + pre_bytes, s);
+    if (rc) return rc;
+    unsigned char *ws = static_cast<unsigned char *>(st->ws);
+
+    GqaLaunch L{};
+    GqaParams &kp = L.kp;
+    kp.q = q; kp.k_cache = k_cache; kp.v_cache = v_cache;
+    kp.seq_lens = seq_lens; kp.block_table = block_table;
+    kp.ws_o = reinterpret_cast<float *>(ws);
+    kp.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
+    kp.ws_prefix = reinterpret_cast<long long *>(ws + o_bytes + lse_bytes);
+    kp.err = st->err;
+    take_force_timeout(&kp.force_timeout, &kp.timeout_ns);
+    kp.scale_log2 = scale * 1.4426950408889634f;
+    kp.B = B; kp.H_q = H_q; kp.H_kv = H_kv; kp.group = G; kp.n_hc = n_hc;
+    kp.max_blocks = max_blocks_per_seq; kp.num_blocks = num_blocks;
+    kp.window = window > 0 ? window : 0;
+    kp.num_ctas = P;
+    CombineParams &cp = L.cp;
+    cp.seq_lens = seq_lens; cp.ws_prefix = kp.ws_prefix; cp.ws_o = kp.ws_o;
+    cp.ws_lse = kp.ws_lse; cp.out = out;
+    cp.B = B; cp.H_q = H_q; cp.H_kv = H_kv; cp.group = G; cp.n_hc = n_hc;
+    cp.max_blocks = max_blocks_per_seq; cp.window = kp.window; cp.num_ctas = P;
+    L.units_total = (int)units_total;
+    L.stream = s;
+    take_profile_events(&L.ev_start, &L.ev_stop);
+
+    const int bf16 = dtype == ATTN_BF16;
+    cudaError_t e;
+    switch (d) {
+        case 16: e = launch_gqa_d16(HC, bf16, L); break;
+        case 32: e = launch_gqa_d32(HC, bf16, L); break;
+        case 64: e = launch_gqa_d64(HC, bf16, L); break;
+        case 128: e = launch_gqa_d128(HC, bf16, L); break;
+        default: e = launch_gqa_d256(HC, bf16, L); break;
+    }
+    return cuda_status(e);
+}
+
+int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent_cache,
+                    const int32_t *seq_lens, const int32_t *block_table, void *out, int B,
+                    int H, int d_c, int d_r, float scale, void *stream,
+                    int max_blocks_per_seq, int num_blocks) {
+    if (!q_latent || !q_rope || !latent_cache || !seq_lens || !block_table || !out)
+        return ATTN_ERR_ARG;
+    if (B <= 0 || H <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
+    if (!std::isfinite(scale)) return ATTN_ERR_ARG;
+    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_cache) ||
+        !aligned16(out))
+        return ATTN_ERR_ARG;
+    if (d_c != 512 || d_r != 64) return ATTN_ERR_UNSUPPORTED;
+    if (H != 16 && H != 32 && H != 64 && H != 128) return ATTN_ERR_UNSUPPORTED;
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    return mla_decode_entry(q_latent, q_rope, latent_cache, seq_lens, block_table, out, B,
+                            H, scale, (cudaStream_t)stream, max_blocks_per_seq, num_blocks,
+                            st->num_sms, tl_num_ctas, st->err,
+                            [&](size_t bytes, void **ws) {
+                                int r = ensure_workspace(st, bytes, (cudaStream_t)stream);
+                                *ws = st->ws;
+                                return r;
+                            });
+}
+
+int kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+              const int32_t *positions, const int32_t *block_table, int B, int H_kv, int d,
+              int max_blocks_per_seq, int num_blocks, int dtype, void *stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !positions || !block_table)
+        return ATTN_ERR_ARG;
+    if (B <= 0 || H_kv <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
+    if (dtype != ATTN_F32 && dtype != ATTN_BF16) return ATTN_ERR_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return ATTN_ERR_ARG;
+    if (!valid_head_dim(d)) return ATTN_ERR_UNSUPPORTED;
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    KvAppendParams p{};
+    p.k_new = k_new; p.v_new = v_new; p.k_cache = k_cache; p.v_cache = v_cache;
+    p.positions = positions; p.block_table = block_table; p.err = st->err;
+    p.B = B; p.H_kv = H_kv;
+    p.chunks_per_row = d * (dtype == ATTN_BF16 ? 2 : 4) / 16;
+    p.max_blocks = max_blocks_per_seq; p.num_blocks = num_blocks;
+    return cuda_status(launch_kv_append(p, (cudaStream_t)stream));
+}
+
+int kv_append_mla(const void *latent_new, void *latent_cache, const int32_t *positions,
+                  const int32_t *block_table, int B, int d_c, int d_r,
+                  int max_blocks_per_seq, int num_blocks, void *stream) {
+    if (!latent_new || !latent_cache || !positions || !block_table) return ATTN_ERR_ARG;
+    if (B <= 0 || d_c <= 0 || d_r < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return ATTN_ERR_ARG;
+    if (((d_c + d_r) * 2) % 16 != 0) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(latent_new) || !aligned16(latent_cache)) return ATTN_ERR_ARG;
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    KvAppendParams p{};
+    p.k_new = latent_new; p.v_new = nullptr; p.k_cache = latent_cache; p.v_cache = nullptr;
+    p.positions = positions; p.block_table = block_table; p.err = st->err;
+    p.B = B; p.H_kv = 1; p.chunks_per_row = (d_c + d_r) * 2 / 16;
+    p.max_blocks = max_blocks_per_seq; p.num_blocks = num_blocks;
+    return cuda_status(launch_kv_append(p, (cudaStream_t)stream));
+}
+
+int attn_decode_plan(const int32_t *seq_lens, int B, int units_per_seq, int window,
+                     int max_blocks_per_seq, int num_ctas, int64_t *plan_out,
+                     void *stream) {
+    if (!seq_lens || !plan_out || B <= 0 || units_per_seq <= 0 || num_ctas <= 0 ||
+        max_blocks_per_seq <= 0)
+        return ATTN_ERR_ARG;
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    return cuda_status(launch_plan_kernel(seq_lens, B, units_per_seq, window > 0 ? window : 0,
+                                          max_blocks_per_seq, num_ctas,
+                                          reinterpret_cast<long long *>(plan_out), st->err,
+                                          (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,171 @@
+// common.cuh -- sm_100a helpers shared by the decode kernels: mbarriers,
+// bulk (TMA) copies, bounded waits, the device error word.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace attn {
+
+constexpr int kBlockSize = 64;              // tokens per paged cache block
+
+// Device error word bits (read and cleared by attn_decode_last_error).
+constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrBadBlock = 2u;
+constexpr unsigned kErrBadSeqLen = 4u;
+
+// Default bound of every spin-wait: 2 seconds of %globaltimer.
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+
+__device__ __forceinline__ void raise_error(unsigned *err, unsigned bits) {
+    atomicOr(err, bits);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(count)
+                 : "memory");
+}
+
+// Make mbarrier initialisation visible to the async proxy (bulk copies).
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    uint64_t state;
+    asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1];"
+                 : "=l"(state)
+                 : "r"(smem_u32(bar))
+                 : "memory");
+    (void)state;
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar,
+                                                      uint32_t bytes) {
+    uint64_t state;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 %0, [%1], %2;"
+                 : "=l"(state)
+                 : "r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+    (void)state;
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait for the phase of `bar` with the given parity to complete.
+// Returns false if it did not within timeout_ns (raising kErrTimeout), or as
+// soon as another warp of the CTA has set *abort (then without raising).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          unsigned long long timeout_ns,
+                                          unsigned *err,
+                                          volatile int *abort = nullptr) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (abort && *abort) return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            raise_error(err, kErrTimeout);
+            if (abort) *abort = 1;
+            return false;
+        }
+    }
+}
+
+// --------------------------------------------------------- bulk async copy
+// 1-D bulk copy global -> shared, completion counted on `bar` in bytes.
+// src and dst 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst_smem, const void *src,
+                                          uint32_t bytes, uint64_t *bar,
+                                          uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// L2 policy for data read exactly once (the streamed KV cache).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t policy;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;"
+                 : "=l"(policy));
+    return policy;
+}
+
+// ------------------------------------------------ programmatic dependent launch
+__device__ __forceinline__ void pdl_wait_primary() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------ conversions
+__device__ __forceinline__ float bf16lo(uint32_t w) {
+    return __uint_as_float(w << 16);
+}
+__device__ __forceinline__ float bf16hi(uint32_t w) {
+    return __uint_as_float(w & 0xffff0000u);
+}
+
+template <typename T> struct ElemTraits;
+template <> struct ElemTraits<float> {
+    static constexpr int kBytes = 4;
+    static __device__ __forceinline__ float to_float(float x) { return x; }
+    static __device__ __forceinline__ float from_float(float x) { return x; }
+};
+template <> struct ElemTraits<__nv_bfloat16> {
+    static constexpr int kBytes = 2;
+    static __device__ __forceinline__ float to_float(__nv_bfloat16 x) {
+        return __bfloat162float(x);
+    }
+    static __device__ __forceinline__ __nv_bfloat16 from_float(float x) {
+        return __float2bfloat16_rn(x);
+    }
+};
+
+// Unpack one 16-byte chunk into fp32 values (8 for bf16, 4 for fp32).
+template <typename T> struct Chunk;
+template <> struct Chunk<__nv_bfloat16> {
+    static constexpr int kElems = 8;
+    static __device__ __forceinline__ void unpack(const uint4 &v, float *f) {
+        f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
+        f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+        f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
+        f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+    }
+};
+template <> struct Chunk<float> {
+    static constexpr int kElems = 4;
+    static __device__ __forceinline__ void unpack(const uint4 &v, float *f) {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    }
+};
+
+}  // namespace attn

@@ -1,0 +1,89 @@
+// gqa_launch.cuh -- host-side launch of the CUDA-core split-KV kernel and the
+// combine kernel for one (head dim, heads-per-CTA, dtype) instantiation.
+#pragma once
+
+#include "gqa_decode.cuh"
+
+namespace attn {
+
+struct GqaLaunch {
+    GqaParams kp;
+    CombineParams cp;
+    int units_total;          // B * H_kv * n_hc
+    cudaStream_t stream;
+    cudaEvent_t ev_start;     // optional (profiling hook), may be null
+    cudaEvent_t ev_stop;
+};
+
+// Shared-memory bytes the split kernel of this instantiation needs.
+template <int D, int HC, typename T>
+int gqa_smem_bytes() { return GqaCfg<D, HC, T>::kSmemBytes; }
+
+template <int D, int HC, typename T>
+cudaError_t launch_gqa_impl(const GqaLaunch &L) {
+    using C = GqaCfg<D, HC, T>;
+    static bool configured = false;   // per-process; attribute is per function
+    cudaError_t e;
+    if (!configured) {
+        e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
+    gqa_split_kernel<D, HC, T>
+        <<<L.kp.num_ctas, kGqaThreads, C::kSmemBytes, L.stream>>>(L.kp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(L.units_total);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = L.ev_stop ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gqa_combine_kernel<D, HC, T>, L.cp);
+}
+
+// Dispatch over heads-per-CTA and dtype for one head dimension D.
+template <int D>
+cudaError_t launch_gqa_d(int HC, int dtype_bf16, const GqaLaunch &L) {
+#define ATTN_CASE(hc)                                                        \
+    case hc:                                                                 \
+        if (dtype_bf16) return launch_gqa_impl<D, hc, __nv_bfloat16>(L);     \
+        if constexpr (D <= 128) return launch_gqa_impl<D, hc, float>(L);     \
+        return cudaErrorNotSupported;
+    switch (HC) {
+        ATTN_CASE(1)
+        ATTN_CASE(2)
+        ATTN_CASE(3)
+        ATTN_CASE(4)
+        ATTN_CASE(6)
+        ATTN_CASE(8)
+        default: return cudaErrorInvalidValue;
+    }
+#undef ATTN_CASE
+}
+
+cudaError_t launch_gqa_d16(int HC, int bf16, const GqaLaunch &L);
+cudaError_t launch_gqa_d32(int HC, int bf16, const GqaLaunch &L);
+cudaError_t launch_gqa_d64(int HC, int bf16, const GqaLaunch &L);
+cudaError_t launch_gqa_d128(int HC, int bf16, const GqaLaunch &L);
+cudaError_t launch_gqa_d256(int HC, int bf16, const GqaLaunch &L);
+
+}  // namespace attn
+
+namespace attn {
+// Runs the split planner alone (one CTA per planned CTA) and writes the plan:
+// out[0] = W; out[1 + 4i .. 4 + 4i] = range start, range end, first sequence,
+// first unit of CTA i; then B + 1 exclusive work prefix sums.
+cudaError_t launch_plan_kernel(const int32_t *seq_lens, int B, int units_per_seq,
+                               int window, int max_blocks, int num_ctas,
+                               long long *out, unsigned *err, cudaStream_t stream);
+}  // namespace attn

@@ -1,0 +1,205 @@
+// plan.cuh -- split-KV work partition, computed on the device from seq_lens.
+//
+// The flattened work list orders sequences b, then the units of b (a unit is
+// one KV head, or one chunk of the query heads that share it), then the
+// visible 64-token blocks of b.  Only blocks that hold at least one visible
+// key are listed, so blocks wholly outside a sliding window are never read
+// (attention-head article, §3: the kernel must skip masked positions).
+// CTA i of P takes the contiguous block range [floor(i*W/P), floor((i+1)*W/P)).
+// A (unit, CTA) pair that meets writes one partial result; pair slots are
+// numbered unit + CTA, which is injective along the walk, so U + P slots
+// always suffice.
+#pragma once
+
+#include "common.cuh"
+
+namespace attn {
+
+// Visible blocks of a sequence with T cached tokens (current one included).
+// first_block receives the logical index of the first of them.
+__device__ __forceinline__ int visible_blocks(int T, int window, int max_blocks,
+                                              int *first_block, bool *bad) {
+    *first_block = 0;
+    if (T <= 0) {
+        *bad = (T < 0);
+        return 0;
+    }
+    if (T > max_blocks * kBlockSize) {
+        *bad = true;
+        return 0;
+    }
+    *bad = false;
+    const int lo = (window > 0 && T > window) ? T - window : 0;
+    *first_block = lo / kBlockSize;
+    return (T - 1) / kBlockSize - lo / kBlockSize + 1;
+}
+
+__device__ __forceinline__ long long cta_bound(long long i, long long W, int P) {
+    return (long long)(((unsigned long long)i * (unsigned long long)W) /
+                       (unsigned long long)P);
+}
+
+// The CTA whose range contains flattened block x (0 <= x < W).
+__device__ __forceinline__ int cta_of(long long x, long long W, int P) {
+    long long i = (long long)(((unsigned long long)x * (unsigned long long)P) /
+                              (unsigned long long)W);
+    while (i + 1 < P && cta_bound(i + 1, W, P) <= x) ++i;
+    while (i > 0 && cta_bound(i, W, P) > x) --i;
+    return (int)i;
+}
+
+struct PlanArgs {
+    const int32_t *seq_lens;
+    int B;
+    int units_per_seq;
+    int window;
+    int max_blocks;
+    int num_ctas;
+};
+
+struct PlanScratch {          // shared memory used by plan_locate
+    long long warp_sums[32];
+    long long total;
+    long long base;
+    int seq;
+    int bad;
+};
+
+// Block-wide: total work W, and the sequence holding flattened block
+// `target(W)` together with the work (blocks x units) before that sequence.
+// Every thread of the block must call it.  When prefix_out is non-null the
+// exclusive prefix sums of work per sequence (B + 1 values) are written.
+// `target_cta` selects target = cta_bound(target_cta, W, num_ctas).
+__device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_cta,
+                            PlanScratch *sh, long long *prefix_out,
+                            unsigned *err) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = (nt + 31) >> 5;
+    bool any_bad = false;
+
+    // Pass 1: W.
+    long long mine = 0;
+    for (int b = tid; b < a.B; b += nt) {
+        int fb;
+        bool bad;
+        mine += (long long)visible_blocks(a.seq_lens[b], a.window,
+                                          a.max_blocks, &fb, &bad) *
+                a.units_per_seq;
+        any_bad |= bad;
+    }
+    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    if (lane == 0) sh->warp_sums[warp] = mine;
+    if (tid == 0) { sh->seq = -1; sh->base = 0; sh->bad = 0; }
+    __syncthreads();
+    if (tid == 0) {
+        long long t = 0;
+        for (int w = 0; w < nwarps; ++w) t += sh->warp_sums[w];
+        sh->total = t;
+    }
+    if (any_bad) sh->bad = 1;
+    __syncthreads();
+    const long long W = sh->total;
+    const long long target =
+        (W > 0) ? cta_bound(target_cta, W, a.num_ctas) : 0;
+
+    // Pass 2: exclusive scan, locate target.
+    long long running = 0;
+    for (int c = 0; c < a.B; c += nt) {
+        const int b = c + tid;
+        long long w = 0;
+        if (b < a.B) {
+            int fb;
+            bool bad;
+            w = (long long)visible_blocks(a.seq_lens[b], a.window,
+                                          a.max_blocks, &fb, &bad) *
+                a.units_per_seq;
+        }
+        long long x = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        __syncthreads();
+        if (lane == 31) sh->warp_sums[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            long long s = (lane < nwarps) ? sh->warp_sums[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                long long y = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += y;
+            }
+            if (lane < nwarps) sh->warp_sums[lane] = s;
+        }
+        __syncthreads();
+        const long long excl =
+            running + (warp > 0 ? sh->warp_sums[warp - 1] : 0) + x - w;
+        if (b < a.B) {
+            if (prefix_out) prefix_out[b] = excl;
+            if (w > 0 && excl <= target && target < excl + w) {
+                sh->seq = b;
+                sh->base = excl;
+            }
+        }
+        running += sh->warp_sums[nwarps - 1];
+    }
+    if (tid == 0 && prefix_out) prefix_out[a.B] = running;
+    if (tid == 0 && sh->bad && err) raise_error(err, kErrBadSeqLen);
+    __syncthreads();
+}
+
+// Walks the segments of one CTA's block range.  A segment is the part of one
+// unit's visible blocks that lies in the range.
+struct SegmentWalker {
+    // fixed
+    const int32_t *seq_lens;
+    int B, units, window, max_blocks;
+    // state
+    long long pos, end;
+    int b, unit, blk_off, nb, first_blk, T;
+
+    __device__ void load_seq() {
+        bool bad;
+        T = seq_lens[b];
+        nb = visible_blocks(T, window, max_blocks, &first_blk, &bad);
+    }
+
+    __device__ void init(const PlanArgs &a, long long lo, long long hi,
+                         int seq, long long base) {
+        seq_lens = a.seq_lens; B = a.B; units = a.units_per_seq;
+        window = a.window; max_blocks = a.max_blocks;
+        pos = lo; end = hi; b = seq;
+        if (pos < end) {
+            load_seq();
+            const long long off = lo - base;
+            unit = (int)(off / nb);
+            blk_off = (int)(off % nb);
+        }
+    }
+
+    __device__ bool done() const { return pos >= end; }
+
+    // Length in blocks of the current segment.
+    __device__ int seg_len() const {
+        long long rem = end - pos;
+        int left = nb - blk_off;
+        return rem < left ? (int)rem : left;
+    }
+
+    __device__ void advance(int len) {
+        pos += len;
+        blk_off += len;
+        if (blk_off == nb) {
+            blk_off = 0;
+            if (++unit == units) {
+                unit = 0;
+                if (pos < end) {
+                    do { ++b; load_seq(); } while (nb == 0 && b + 1 < B);
+                }
+            }
+        }
+    }
+};
+
+}  // namespace attn

@@ -1,0 +1,214 @@
+/*
+ * attn_decode.h -- C ABI of libattn_decode.so: single-token decode attention
+ * over a paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (page title, section / equation):
+ *   [HEADS] xuesongtap "attention-head" article -- §1 Attention equation
+ *           softmax(q K^T / sqrt(d) + M) V with softmax along key positions;
+ *           §2 / §2.2 head sharing (MHA H_kv = H_q, GQA contiguous equal
+ *           groups of H_q / H_kv, MQA H_kv = 1); §3 causal sliding window
+ *           that covers the current position and the w-1 before it, and
+ *           whose masked part must be skipped, not computed and masked;
+ *           §5.2-§5.3 MLA with U^K absorbed into the query and U^V applied
+ *           after the latent-space weighted sum, one softmax over content +
+ *           RoPE scores.
+ *   [BAIDU] "大模型注意力机制对比：MLA与MQA该怎么选" -- §2 cache shapes
+ *           ([batch, heads, seq, head_dim]; MLA [batch, seq, latent + rope])
+ *           and §4.3 paged KV-cache management.
+ *   [EVOL]  toolsku "注意力機制演進" article -- FlashAttention tiling with
+ *           online softmax (the split-KV kernels use that technique).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or retains them past the call.  Calls are asynchronous and
+ *    ordered on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *  * Paged cache: 64-token blocks.  `block_table` is int32 row-major
+ *    [B][max_blocks_per_seq]; logical block i of sequence b is physical
+ *    block block_table[b * max_blocks_per_seq + i], 0 <= id < num_blocks.
+ *    A contiguous (unpaged) cache is the identity table.
+ *  * `seq_lens[b]` (int32, device) = T_b tokens cached for sequence b, the
+ *    current token included (its K/V is appended before attention); the
+ *    query sits at position T_b - 1 and sees keys [lo_b, T_b), where
+ *    lo_b = max(0, T_b - window) for window > 0 and 0 otherwise.
+ *    T_b = 0 yields a zero output row.
+ *  * Host-side validation returns a negative attn_status and launches
+ *    nothing.  Faults found on the device (a block id outside
+ *    [0, num_blocks), T_b outside [0, 64 * max_blocks_per_seq], a bounded
+ *    wait that ran out) never touch memory out of bounds: the offending
+ *    sequence/tile is skipped and a per-device error word is set, which
+ *    attn_decode_last_error() reports.
+ *  * All computation is on the GPU; there is no CPU fallback.
+ */
+#ifndef ATTN_DECODE_H
+#define ATTN_DECODE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_ARG = -1,          /* invalid argument (null, size, alignment) */
+    ATTN_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. head dim) */
+    ATTN_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
+    ATTN_ERR_TIMEOUT = -4,      /* device: a bounded wait ran out */
+    ATTN_ERR_BAD_BLOCK = -5,    /* device: block id outside [0, num_blocks) */
+    ATTN_ERR_BAD_SEQLEN = -6    /* device: T_b < 0 or > 64 * max_blocks */
+} attn_status;
+
+typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
+
+/* Tokens per cache block (fixed by the storage format). */
+#define ATTN_BLOCK_SIZE 64
+
+/*
+ * attn_decode_gqa -- decode attention for MHA / GQA / MQA ([HEADS] §1, §2).
+ *
+ *   out[b,h,:] = sum_{j in [lo_b, T_b)} softmax_j(scale * <q[b,h], K[b,g(h),j]>)
+ *                 * V[b,g(h),j,:],     g(h) = floor(h / (H_q / H_kv))
+ *
+ * q        [B][H_q][d]                   dtype, contiguous
+ * k_cache  [num_blocks][H_kv][64][d]     dtype; one (block, head) tile is
+ * v_cache  [num_blocks][H_kv][64][d]     64*d contiguous elements
+ * out      [B][H_q][d]                   dtype (rounded to nearest even)
+ * window   > 0: causal sliding window of that many positions, the current one
+ *          included ([HEADS] §3); <= 0: full causal.  Blocks wholly outside
+ *          the window are never read.
+ * dtype    ATTN_BF16 (any supported d) or ATTN_F32 (d <= 128); accumulation
+ *          is always fp32.
+ * Requirements: H_q % H_kv == 0; d in {16, 32, 64, 128, 256}; pointers
+ * 16-byte aligned; B >= 1; max_blocks_per_seq >= 1; num_blocks >= 1.
+ * Uses a library-owned per-device workspace for the split partials; it is
+ * grown (cudaMalloc) on first use outside stream capture.  Growing it while
+ * the stream is being captured returns ATTN_ERR_UNSUPPORTED.
+ */
+int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seq_lens, const int32_t *block_table,
+                    void *out, int B, int H_q, int H_kv, int d, float scale,
+                    int window, void *stream, int max_blocks_per_seq,
+                    int num_blocks, int dtype);
+
+/*
+ * attn_decode_mla -- absorbed MLA decode ([HEADS] §5.2, §5.3).
+ *
+ *   s_j     = scale * (<q_latent[b,h], c_j> + <q_rope[b,h], kR_j>)
+ *   out[b,h,:] = sum_{j < T_b} softmax_j(s) * c_j          (d_c wide)
+ *
+ * q_latent     [B][H][d_c]  bf16  absorbed query q^C (U^K_h)^T
+ * q_rope       [B][H][d_r]  bf16  rotated RoPE query
+ * latent_cache [num_blocks][64][d_c + d_r] bf16: row = c_j followed by the
+ *              already-rotated shared RoPE key kR_j
+ * out          [B][H][d_c]  bf16  latent-space output z (apply U^V_h after)
+ * Supported: d_c = 512, d_r = 64, H in {16, 32, 64, 128} (heads padded to a
+ * multiple of 64 inside the kernel); otherwise ATTN_ERR_UNSUPPORTED.
+ * Workspace as for attn_decode_gqa.
+ */
+int attn_decode_mla(const void *q_latent, const void *q_rope,
+                    const void *latent_cache, const int32_t *seq_lens,
+                    const int32_t *block_table, void *out, int B, int H,
+                    int d_c, int d_r, float scale, void *stream,
+                    int max_blocks_per_seq, int num_blocks);
+
+/*
+ * kv_append -- write the new token's K and V of every sequence into its
+ * paged slot ([BAIDU] §4.3 paging; [EVOL] cache concatenation before
+ * attention).  Position positions[b] (usually T_b - 1) lands in logical block
+ * positions[b] / 64, row positions[b] % 64, for every KV head.
+ * k_new, v_new [B][H_kv][d] dtype; caches as in attn_decode_gqa.
+ * Rows whose position or block id is out of range are skipped and flagged
+ * (ATTN_ERR_BAD_BLOCK).  Pointers 16-byte aligned; d as above.
+ */
+int kv_append(const void *k_new, const void *v_new, void *k_cache,
+              void *v_cache, const int32_t *positions,
+              const int32_t *block_table, int B, int H_kv, int d,
+              int max_blocks_per_seq, int num_blocks, int dtype,
+              void *stream);
+
+/*
+ * kv_append_mla -- write each sequence's new latent row (c followed by kR,
+ * d_c + d_r bf16 values) into latent_cache at positions[b].
+ * latent_new [B][d_c + d_r] bf16.  (d_c + d_r) * 2 must be a multiple of 16.
+ */
+int kv_append_mla(const void *latent_new, void *latent_cache,
+                  const int32_t *positions, const int32_t *block_table,
+                  int B, int d_c, int d_r, int max_blocks_per_seq,
+                  int num_blocks, void *stream);
+
+/*
+ * attn_decode_plan -- run the device split planner on its own and write the
+ * plan the decode kernels would follow (for bit-exact checks against a host
+ * model).  The flattened work list orders sequences b, then units
+ * (unit = a KV head, or a chunk of its query heads) of that sequence, then
+ * the visible 64-token blocks of the unit.  CTA i of num_ctas takes blocks
+ * [floor(i*W/num_ctas), floor((i+1)*W/num_ctas)) of the W in total.
+ * Output (int64, device) plan_out: [0] = W, then for every CTA i four
+ * values: range start, range end, sequence of the first block, unit of the
+ * first block (-1, -1 for an empty range); then B+1 exclusive prefix sums
+ * of blocks per sequence.  Size: 1 + 4*num_ctas + B + 1 int64.
+ * units_per_seq = H_kv * (query-head chunks per KV head).
+ */
+int attn_decode_plan(const int32_t *seq_lens, int B, int units_per_seq,
+                     int window, int max_blocks_per_seq, int num_ctas,
+                     int64_t *plan_out, void *stream);
+
+/*
+ * attn_decode_gqa_config -- the launch shape attn_decode_gqa uses for a
+ * problem: *num_ctas = CTAs of the split-KV kernel, *heads_per_cta = query
+ * heads a CTA processes per KV head (the group is split into
+ * H_q / H_kv / heads_per_cta chunks when it does not fit), *path = 0 for the
+ * CUDA-core kernel, 1 for the tensor-core (tcgen05) kernel.
+ */
+int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype,
+                           int *num_ctas, int *heads_per_cta, int *path);
+
+/*
+ * attn_set_num_ctas -- testing/tuning hook: force the number of split-KV CTAs
+ * used by later calls on this host thread's current device (0 = automatic).
+ */
+int attn_set_num_ctas(int num_ctas);
+
+/*
+ * attn_set_gqa_path -- testing/tuning hook: -1 = automatic, 0 = force the
+ * CUDA-core kernel, 1 = force the tensor-core kernel where it is supported.
+ */
+int attn_set_gqa_path(int path);
+
+/*
+ * attn_set_profile_events -- optional timing hook.  When n > 0, the next n
+ * decode calls record start_events[i] / stop_events[i] (cudaEvent_t handles
+ * owned by the caller) on their stream immediately around their main split-KV
+ * kernel; n = 0 disables.  The arrays must stay valid until disabled.
+ */
+int attn_set_profile_events(void *const *start_events,
+                            void *const *stop_events, int n);
+
+/*
+ * attn_debug_force_timeout -- fault-injection hook for tests: when enable is
+ * nonzero, the next decode launch waits on a barrier that is never signalled,
+ * bounded by timeout_ns, then sets ATTN_ERR_TIMEOUT and returns without
+ * hanging the device.  One-shot.
+ */
+int attn_debug_force_timeout(int enable, long long timeout_ns);
+
+/*
+ * attn_decode_last_error -- synchronise `stream`, then read and clear the
+ * current device's error word.  Returns ATTN_OK, or the first device-side
+ * status (ATTN_ERR_TIMEOUT, ATTN_ERR_BAD_BLOCK, ATTN_ERR_BAD_SEQLEN), or
+ * ATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+int attn_decode_last_error(void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *attn_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_DECODE_H */
