@@ -62,6 +62,8 @@ def parse():
                     help="llama3_8b | tiny | ragged_full | ragged_window | mla "
                          "| a sweep name such as sweep_bf16_B8_Hq32_Hkv8_d128_T32768")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true",
+                    help="skip the oracle CPU baseline (profiling runs)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -235,7 +237,7 @@ def mla_flops(inp):
 
 
 # ------------------------------------------------------------ native arm
-def run_native(args, rank, world, local):
+def run_native(args, rank, world, local):  # noqa: C901
     import decode_attention_kv_paged_b200 as attn
     attn.load()
     cfg = workload(args.workload)
@@ -351,7 +353,7 @@ def run_native(args, rank, world, local):
         line["tile_overread_bytes_per_step"] = tile_bytes_gqa(base) - kv_bytes
     if not args.no_e2e:
         line["e2e"] = e2e_native(attn, cfg, inputs[0], is_mla, K, world, dev)
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(cfg, is_mla, args.cpu_seconds)
     return line
 

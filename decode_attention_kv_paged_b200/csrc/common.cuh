@@ -126,11 +126,19 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 
 // ------------------------------------------------------------ conversions
+// bf16 -> fp32 widening of the low / high half of a packed pair.  A bf16 is
+// the top 16 bits of an fp32, so the widening is a shift or a mask; written
+// as integer PTX so it stays on the integer pipes (a conversion instruction
+// would run on the much narrower XU pipe).
 __device__ __forceinline__ float bf16lo(uint32_t w) {
-    return __uint_as_float(w << 16);
+    uint32_t r;
+    asm("shl.b32 %0, %1, 16;" : "=r"(r) : "r"(w));
+    return __uint_as_float(r);
 }
 __device__ __forceinline__ float bf16hi(uint32_t w) {
-    return __uint_as_float(w & 0xffff0000u);
+    uint32_t r;
+    asm("and.b32 %0, %1, 0xffff0000;" : "=r"(r) : "r"(w));
+    return __uint_as_float(r);
 }
 
 template <typename T> struct ElemTraits;

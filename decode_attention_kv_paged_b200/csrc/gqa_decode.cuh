@@ -281,6 +281,8 @@ gqa_split_kernel(const GqaParams p) {
     float *sc = s_scores + warp * C::kTPW * C::kHCP;   // [TPW][HCP]
     long long n_tile = 0;
     int n_seg = 0;
+    int c_stage = 0, p_stage = 0;          // stage of tile n_tile / n_tile - 1
+    uint32_t c_phase = 0, p_phase = 0;     // their use parity
 
     while (!*abort_flag && !walk.done()) {
         const int len = walk.seg_len();
@@ -314,9 +316,8 @@ gqa_split_kernel(const GqaParams p) {
 
         bool ok = true;
         for (int t = 0; t < len; ++t) {
-            const int stage = (int)(n_tile % C::kStages);
-            if (!mbar_wait(&full_bar[stage], (uint32_t)((n_tile / C::kStages) & 1),
-                           p.timeout_ns, p.err, abort_flag)) {
+            const int stage = c_stage;
+            if (!mbar_wait(&full_bar[stage], c_phase, p.timeout_ns, p.err, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -414,10 +415,8 @@ gqa_split_kernel(const GqaParams p) {
             // Refill the stage released one tile ago (one-tile lag keeps the
             // producer from waiting on the slowest warp's current tile).
             if (producer && n_tile >= 1 && issued < n_tiles) {
-                const long long prev = n_tile - 1;
-                const int ps = (int)(prev % C::kStages);
-                if (mbar_wait(&empty_bar[ps], (uint32_t)((prev / C::kStages) & 1),
-                              p.timeout_ns, p.err, abort_flag)) {
+                const int ps = p_stage;
+                if (mbar_wait(&empty_bar[ps], p_phase, p.timeout_ns, p.err, abort_flag)) {
                     issue_tile<D, T, C::kTileBytes>(p, prod, stage_base + ps * C::kStageBytes,
                                                     &full_bar[ps], pol);
                     prod.next();
@@ -426,12 +425,41 @@ gqa_split_kernel(const GqaParams p) {
                     ok = false;
                 }
             }
+            p_stage = c_stage;
+            p_phase = c_phase;
+            if (++c_stage == C::kStages) {
+                c_stage = 0;
+                c_phase ^= 1u;
+            }
             ++n_tile;
             if (!ok) break;
         }
         if (!ok) break;
 
         // ---- merge the 8 warps' states, write the segment's partial
+        // Row groups with a rotated chunk order hold chunk (c + shift) mod CPL
+        // in register slot c; put them back in the unrotated order first so
+        // the cross-row-group sums below add like columns.
+        if constexpr (C::kLPR < 8 && C::kCPL > 1) {
+            const int shift = rot / C::kLPR;
+#pragma unroll
+            for (int sh = 1; sh < 8 / C::kLPR; ++sh) {
+                if (shift == sh) {
+#pragma unroll
+                    for (int g = 0; g < HC; ++g) {
+                        float tmp[C::kEPL];
+#pragma unroll
+                        for (int c = 0; c < C::kCPL; ++c)
+#pragma unroll
+                            for (int e = 0; e < C::kLE; ++e)
+                                tmp[((c + sh) % C::kCPL) * C::kLE + e] =
+                                    o[g][c * C::kLE + e];
+#pragma unroll
+                        for (int e = 0; e < C::kEPL; ++e) o[g][e] = tmp[e];
+                    }
+                }
+            }
+        }
 #pragma unroll
         for (int m = C::kLPR; m < 32; m <<= 1)
 #pragma unroll
@@ -535,12 +563,18 @@ gqa_combine_kernel(const CombineParams p) {
         if (c0 == c1) {
             r = p.ws_o[(slot0 * HC + g) * D + k];
         } else {
+            // CTAs between c0 and c1 with an empty range wrote no partial.
             float L = kNegInf;
-            for (int c = c0; c <= c1; ++c)
-                L = fmaxf(L, p.ws_lse[(slot0 + (c - c0)) * HC + g]);
+            for (int c = c0; c <= c1; ++c) {
+                if (cta_bound(c, W, p.num_ctas) >= cta_bound(c + 1, W, p.num_ctas))
+                    continue;
+                L = fmaxf(L, p.ws_lse[((long long)u + c) * HC + g]);
+            }
             float num = 0.f, den = 0.f;
             for (int c = c0; c <= c1; ++c) {
-                const long long s = slot0 + (c - c0);
+                if (cta_bound(c, W, p.num_ctas) >= cta_bound(c + 1, W, p.num_ctas))
+                    continue;
+                const long long s = (long long)u + c;
                 const float w = exp2f(p.ws_lse[s * HC + g] - L);
                 num = fmaf(w, p.ws_o[(s * HC + g) * D + k], num);
                 den += w;

@@ -61,7 +61,8 @@ def cta_of(x, W, P):
 
 def splits_of_unit(seq_lens, units_per_seq, window, max_blocks, num_ctas, b,
                    unit):
-    """CTAs (in order) that hold a part of (sequence b, unit)."""
+    """CTAs (in order) that hold a part of (sequence b, unit).  CTAs whose
+    range is empty hold nothing and are left out."""
     p = plan(seq_lens, units_per_seq, window, max_blocks, num_ctas)
     W = p[0]
     prefix = p[1 + 4 * num_ctas:]
@@ -69,4 +70,5 @@ def splits_of_unit(seq_lens, units_per_seq, window, max_blocks, num_ctas, b,
     if nb == 0:
         return []
     s = prefix[b] + unit * nb
-    return list(range(cta_of(s, W, num_ctas), cta_of(s + nb - 1, W, num_ctas) + 1))
+    return [c for c in range(cta_of(s, W, num_ctas), cta_of(s + nb - 1, W, num_ctas) + 1)
+            if cta_bound(c, W, num_ctas) < cta_bound(c + 1, W, num_ctas)]
