@@ -7,13 +7,14 @@
 //
 // Design (B200):
 //   * One CTA per SM (persistent range of the flattened block list, see
-//     plan.cuh), 8 warps (two per SM sub-partition, so each thread may use up
-//     to 255 registers).  Thread 0 also streams each 64-token K tile and V
+//     plan.cuh) of 16 warps (4 per SM sub-partition, <= 128 registers each)
+//     or, for register-heavy shapes, 8 warps.  Thread 0 also streams each
+//     64-token K tile and V
 //     tile (64*d contiguous elements each in the paged layout) with 1-D bulk
 //     async copies (TMA engine) into a multi-stage shared-memory ring,
 //     completion tracked by mbarriers, L2 policy evict-first; it refills a
 //     stage one tile after the CTA has released it.
-//   * Every warp computes.  Each warp owns 8 of the 64 tokens of a tile and the
+//   * Every warp computes.  Each warp owns 64/NW tokens of a tile and the
 //     HC query heads of its unit, so a K/V tile is read from HBM once for the
 //     whole GQA group.  Lanes split the head dimension: each lane keeps its
 //     slice of the HC queries and of the HC output accumulators in fp32
@@ -32,8 +33,6 @@
 
 namespace attn {
 
-constexpr int kGqaConsumerWarps = 8;
-constexpr int kGqaThreads = kGqaConsumerWarps * 32;
 constexpr int kSmemBudget = 227 * 1024 - 1024;
 #define kNegInf (__int_as_float(0xff800000u))
 
@@ -43,12 +42,22 @@ constexpr int pow2_floor(int x) {
     return p;
 }
 
-// Elements of the head dimension each lane owns.  At most ~128 fp32
-// registers for the queries plus accumulators, at least 4 lanes per row (so a
-// warp covers at most the 8 tokens it owns per instruction), at most 32.
-constexpr int gqa_epl(int D, int HC) {
-    int e = pow2_floor(64 / HC);
-    if (e > D / 4) e = D / 4;
+// Warps per CTA.  Sixteen (four per SM sub-partition, so one warp's
+// dependency chain -- shuffle reductions, exp2, shared-memory round trips --
+// overlaps three others) whenever the per-thread state fits the 128
+// registers that allows; otherwise eight (up to 255 registers each).
+constexpr int gqa_warps(int D, int HC) {
+    return (D >= 64 && HC <= 4 && false) ? 16 : 8;
+}
+
+// Elements of the head dimension each lane owns: the queries plus the
+// accumulators take 2*HC*EPL fp32 registers (at most 64 with 16 warps, 128
+// with 8), a warp covers no more rows per instruction than the 64/NW tokens
+// it owns, and no fewer than one row per instruction.
+constexpr int gqa_epl(int D, int HC, int NW) {
+    int e = pow2_floor((NW == 16 ? 32 : 64) / HC);
+    const int tpw = 64 / NW;
+    if (e > D * tpw / 32) e = D * tpw / 32;
     if (e < D / 32) e = D / 32;
     return e;
 }
@@ -72,16 +81,18 @@ struct GqaParams {
 template <int D, int HC, typename T>
 struct GqaCfg {
     static constexpr int kS = (int)sizeof(T);
-    static constexpr int kNW = kGqaConsumerWarps;
-    static constexpr int kTPW = kBlockSize / kNW;                 // 8
-    static constexpr int kEPL = gqa_epl(D, HC);
+    static constexpr int kNW = gqa_warps(D, HC);
+    static constexpr int kThreads = kNW * 32;
+    static constexpr int kTPW = kBlockSize / kNW;                 // tokens/warp
+    static constexpr int kEPL = gqa_epl(D, HC, kNW);
     static constexpr int kLE = (16 / kS < kEPL) ? 16 / kS : kEPL; // per load
     static constexpr int kCPL = kEPL / kLE;                       // loads/lane/row
     static constexpr int kLPR = D / kEPL;                         // lanes per row
     static constexpr int kRPW = 32 / kLPR;                        // rows per instr.
     static constexpr int kIters = kTPW / kRPW;
     static constexpr int kCPR = D / kLE;                          // chunks per row
-    static constexpr int kPasses = (HC + 3) / 4;                  // softmax passes
+    static constexpr int kHPP = 32 / kTPW;                        // heads/pass
+    static constexpr int kPasses = (HC + kHPP - 1) / kHPP;        // softmax passes
     static constexpr int kHCP = (HC == 3) ? 4 : (HC > 4 ? 8 : HC);// padded heads
     static constexpr int kTileBytes = kBlockSize * D * kS;
     static constexpr int kStageBytes = 2 * kTileBytes;
@@ -94,6 +105,7 @@ struct GqaCfg {
         kScoreBytes + kMergeOBytes + kMergeMLBytes + kMiscBytes;
     static constexpr int kStagesRaw = (kSmemBudget - kOther) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+    static_assert(kTPW * kHPP == 32, "softmax lane map");
     static constexpr int kSmemBytes = kStages * kStageBytes + kOther;
     static_assert(kStages >= 2, "not enough shared memory for two stages");
     static_assert(kLPR >= 4 && kLPR <= 32 && (kLPR & (kLPR - 1)) == 0, "LPR");
@@ -116,6 +128,50 @@ __device__ __forceinline__ void load_widen(const T *p, float *f) {
         } else {
             f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
         }
+    }
+}
+
+// Load kLE consecutive elements and widen them to fp32 pairs (element 2j in
+// .x, 2j+1 in .y), ready for packed fp32x2 arithmetic.
+template <typename T, int LE>
+__device__ __forceinline__ void load_pairs(const T *p, float2 *f) {
+    if constexpr (sizeof(T) == 2) {
+        if constexpr (LE == 8) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(p);
+            f[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+            f[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+            f[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+            f[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+        } else {
+            static_assert(LE == 4, "load width");
+            const uint2 v = *reinterpret_cast<const uint2 *>(p);
+            f[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+            f[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+        }
+    } else {
+        static_assert(LE == 4, "load width");
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        f[0] = make_float2(v.x, v.y);
+        f[1] = make_float2(v.z, v.w);
+    }
+}
+
+// Read n consecutive fp32 from shared memory with the widest aligned loads
+// (rows of the score buffer are n floats, n in {1, 2, 4, 8}).
+template <int n>
+__device__ __forceinline__ void load_row(const float *p, float *v) {
+    if constexpr (n % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < n; i += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(p + i);
+            v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+        }
+    } else if constexpr (n == 2) {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x; v[1] = x.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < n; ++i) v[i] = p[i];
     }
 }
 
@@ -179,13 +235,50 @@ struct TileCursor {
     }
 };
 
-// Issue the bulk copies of the cursor's current tile into `stage`.
+// Producer of warp 0: walks the CTA's tiles and keeps the physical block ids
+// of the current segment in registers, 32 at a time (lane i holds tile
+// bt0 + i), fetched with one coalesced load and the next batch prefetched
+// half a batch early, so no bulk copy waits on a dependent global load.
+// All 32 lanes call it together; lane 0 issues the copies.
+struct Producer {
+    TileCursor cur;
+    int id_cur, id_nxt, bt0;
+    bool has_next;
+
+    __device__ int fetch(const GqaParams &p, int i, int lane) const {
+        const int j = i + lane;
+        if (j >= cur.len) return -1;
+        return __ldg(p.block_table + (size_t)cur.w.b * p.max_blocks + cur.w.first_blk +
+                     cur.w.blk_off + j);
+    }
+
+    // Physical block id of the current tile (warp-uniform call).
+    __device__ int block_id(const GqaParams &p, int lane) {
+        const int t = cur.t;
+        if (t == 0) {
+            bt0 = 0;
+            id_cur = fetch(p, 0, lane);
+            has_next = false;
+        } else if (t == bt0 + 32) {
+            bt0 += 32;
+            id_cur = has_next ? id_nxt : fetch(p, bt0, lane);
+            has_next = false;
+        }
+        if (!has_next && t == bt0 + 16 && bt0 + 32 < cur.len) {
+            id_nxt = fetch(p, bt0 + 32, lane);
+            has_next = true;
+        }
+        return __shfl_sync(0xffffffffu, id_cur, t - bt0);
+    }
+};
+
+// Issue the bulk copies of one tile (physical block `phys`, KV head of the
+// cursor's unit) into a stage.  Called by one lane.
 template <int D, typename T, int kTileBytes>
 __device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor &cur,
-                                          unsigned char *dst, uint64_t *full,
+                                          int phys, unsigned char *dst, uint64_t *full,
                                           uint64_t pol) {
     const int kvh = cur.w.unit / p.n_hc;
-    const int phys = p.block_table[(size_t)cur.w.b * p.max_blocks + cur.logical_block()];
     if (phys < 0 || phys >= p.num_blocks) {
         raise_error(p.err, kErrBadBlock);
         mbar_arrive(full);
@@ -199,7 +292,7 @@ __device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor 
 }
 
 template <int D, int HC, typename T>
-__global__ void __launch_bounds__(kGqaThreads, 1)
+__global__ void __launch_bounds__(GqaCfg<D, HC, T>::kThreads, 1)
 gqa_split_kernel(const GqaParams p) {
     using C = GqaCfg<D, HC, T>;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -245,19 +338,22 @@ gqa_split_kernel(const GqaParams p) {
     walk.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
 
     // ------------------------------------------------------------ producer
-    // Thread 0 streams the tiles; prologue fills every stage.
-    const bool producer = (tid == 0);
-    TileCursor prod;
+    // Warp 0 streams the tiles (lane 0 issues); the prologue fills every stage.
+    const bool producer = (warp == 0);
+    Producer prod;
     long long issued = 0;
     const long long n_tiles = hi - lo;
     uint64_t pol = 0;
     if (producer) {
         pol = l2_policy_evict_first();
-        prod.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
+        prod.cur.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
         while (issued < C::kStages && issued < n_tiles) {
-            issue_tile<D, T, C::kTileBytes>(p, prod, stage_base + issued * C::kStageBytes,
-                                            &full_bar[issued], pol);
-            prod.next();
+            const int phys = prod.block_id(p, lane);
+            if (lane == 0)
+                issue_tile<D, T, C::kTileBytes>(p, prod.cur, phys,
+                                                stage_base + issued * C::kStageBytes,
+                                                &full_bar[issued], pol);
+            prod.cur.next();
             ++issued;
         }
     }
@@ -292,24 +388,26 @@ gqa_split_kernel(const GqaParams p) {
         const int Tb = walk.T;
         const int lo_tok = (p.window > 0 && Tb > p.window) ? Tb - p.window : 0;
 
-        float qf[HC][C::kEPL];
+        constexpr int LP = C::kLE / 2;          // pairs per load
+        constexpr int EP = C::kEPL / 2;         // pairs per lane
+        float2 q2[HC][EP];
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
         for (int g = 0; g < HC; ++g) {
             const T *qrow = qg + ((size_t)b * p.H_q + head0 + g) * D;
 #pragma unroll
             for (int c = 0; c < C::kCPL; ++c) {
-                float f[C::kLE];
-                load_widen<T, C::kLE>(qrow + col[c], f);
+                float2 f[LP];
+                load_pairs<T, C::kLE>(qrow + col[c], f);
 #pragma unroll
-                for (int e = 0; e < C::kLE; ++e)
-                    qf[g][c * C::kLE + e] = f[e] * p.scale_log2;
+                for (int j = 0; j < LP; ++j) q2[g][c * LP + j] = __fmul2_rn(f[j], sc2);
             }
         }
-        float o[HC][C::kEPL];
+        float2 o2[HC][EP];
 #pragma unroll
         for (int g = 0; g < HC; ++g)
 #pragma unroll
-            for (int e = 0; e < C::kEPL; ++e) o[g][e] = 0.f;
+            for (int j = 0; j < EP; ++j) o2[g][j] = make_float2(0.f, 0.f);
         float m_run[C::kPasses], l_run[C::kPasses];
 #pragma unroll
         for (int ps = 0; ps < C::kPasses; ++ps) { m_run[ps] = -1e30f; l_run[ps] = 0.f; }
@@ -327,24 +425,27 @@ gqa_split_kernel(const GqaParams p) {
                              warp * C::kTPW;
 
             // ---- scores: partial dot products, then reduce over the row group
-            float part[C::kIters * HC];
+            float2 acc[C::kIters * HC];
 #pragma unroll
             for (int it = 0; it < C::kIters; ++it) {
                 const T *krow = Ks + (warp * C::kTPW + it * C::kRPW + rg) * D;
 #pragma unroll
-                for (int g = 0; g < HC; ++g) part[it * HC + g] = 0.f;
+                for (int g = 0; g < HC; ++g) acc[it * HC + g] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < C::kCPL; ++c) {
-                    float kf[C::kLE];
-                    load_widen<T, C::kLE>(krow + col[c], kf);
+                    float2 kp[LP];
+                    load_pairs<T, C::kLE>(krow + col[c], kp);
 #pragma unroll
                     for (int g = 0; g < HC; ++g)
 #pragma unroll
-                        for (int e = 0; e < C::kLE; ++e)
-                            part[it * HC + g] =
-                                fmaf(qf[g][c * C::kLE + e], kf[e], part[it * HC + g]);
+                        for (int j = 0; j < LP; ++j)
+                            acc[it * HC + g] =
+                                __ffma2_rn(q2[g][c * LP + j], kp[j], acc[it * HC + g]);
                 }
             }
+            float part[C::kIters * HC];
+#pragma unroll
+            for (int i = 0; i < C::kIters * HC; ++i) part[i] = acc[i].x + acc[i].y;
             using RR = RowReduce<C::kIters * HC, C::kLPR>;
             const int base = RR::run(part, lane);
 #pragma unroll
@@ -359,22 +460,22 @@ gqa_split_kernel(const GqaParams p) {
             float alpha_reg[C::kPasses];
 #pragma unroll
             for (int ps = 0; ps < C::kPasses; ++ps) {
-                const int gs = lane / 8 + 4 * ps;
-                const int tt = lane % 8;
+                const int gs = lane / C::kTPW + C::kHPP * ps;
+                const int tt = lane % C::kTPW;
                 const bool active = gs < HC;
                 const int pos = tok0 + tt;
                 const bool valid = active && pos >= lo_tok && pos < Tb;
                 float s = valid ? sc[tt * C::kHCP + gs] : kNegInf;
                 float mx = s;
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+#pragma unroll
+                for (int m = 1; m < C::kTPW; m <<= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
                 const float m_new = fmaxf(m_run[ps], mx);
                 const float pr = exp2f(s - m_new);
                 float sum = pr;
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+#pragma unroll
+                for (int m = 1; m < C::kTPW; m <<= 1)
+                    sum += __shfl_xor_sync(0xffffffffu, sum, m);
                 const float alpha = exp2f(m_run[ps] - m_new);
                 l_run[ps] = l_run[ps] * alpha + sum;
                 m_run[ps] = m_new;
@@ -384,10 +485,12 @@ gqa_split_kernel(const GqaParams p) {
             __syncwarp();
 #pragma unroll
             for (int g = 0; g < HC; ++g) {
-                const float a = __shfl_sync(0xffffffffu, alpha_reg[g / 4], (g % 4) * 8);
+                const float a = __shfl_sync(0xffffffffu, alpha_reg[g / C::kHPP],
+                                            (g % C::kHPP) * C::kTPW);
                 if (a != 1.f) {
+                    const float2 a2 = make_float2(a, a);
 #pragma unroll
-                    for (int e = 0; e < C::kEPL; ++e) o[g][e] *= a;
+                    for (int j = 0; j < EP; ++j) o2[g][j] = __fmul2_rn(o2[g][j], a2);
                 }
             }
 
@@ -396,18 +499,20 @@ gqa_split_kernel(const GqaParams p) {
             for (int it = 0; it < C::kIters; ++it) {
                 const int rl = it * C::kRPW + rg;
                 const T *vrow = Vs + (warp * C::kTPW + rl) * D;
-                float pg[HC];
+                float pg[C::kHCP];
+                load_row<C::kHCP>(sc + rl * C::kHCP, pg);
+                float2 pp[HC];
 #pragma unroll
-                for (int g = 0; g < HC; ++g) pg[g] = sc[rl * C::kHCP + g];
+                for (int g = 0; g < HC; ++g) pp[g] = make_float2(pg[g], pg[g]);
 #pragma unroll
                 for (int c = 0; c < C::kCPL; ++c) {
-                    float vf[C::kLE];
-                    load_widen<T, C::kLE>(vrow + col[c], vf);
+                    float2 vp[LP];
+                    load_pairs<T, C::kLE>(vrow + col[c], vp);
 #pragma unroll
                     for (int g = 0; g < HC; ++g)
 #pragma unroll
-                        for (int e = 0; e < C::kLE; ++e)
-                            o[g][c * C::kLE + e] = fmaf(pg[g], vf[e], o[g][c * C::kLE + e]);
+                        for (int j = 0; j < LP; ++j)
+                            o2[g][c * LP + j] = __ffma2_rn(pp[g], vp[j], o2[g][c * LP + j]);
                 }
             }
             __syncwarp();
@@ -416,10 +521,15 @@ gqa_split_kernel(const GqaParams p) {
             // producer from waiting on the slowest warp's current tile).
             if (producer && n_tile >= 1 && issued < n_tiles) {
                 const int ps = p_stage;
-                if (mbar_wait(&empty_bar[ps], p_phase, p.timeout_ns, p.err, abort_flag)) {
-                    issue_tile<D, T, C::kTileBytes>(p, prod, stage_base + ps * C::kStageBytes,
-                                                    &full_bar[ps], pol);
-                    prod.next();
+                const bool freed =
+                    mbar_wait(&empty_bar[ps], p_phase, p.timeout_ns, p.err, abort_flag);
+                if (__all_sync(0xffffffffu, freed)) {
+                    const int phys = prod.block_id(p, lane);
+                    if (lane == 0)
+                        issue_tile<D, T, C::kTileBytes>(p, prod.cur, phys,
+                                                        stage_base + ps * C::kStageBytes,
+                                                        &full_bar[ps], pol);
+                    prod.cur.next();
                     ++issued;
                 } else {
                     ok = false;
@@ -436,7 +546,7 @@ gqa_split_kernel(const GqaParams p) {
         }
         if (!ok) break;
 
-        // ---- merge the 8 warps' states, write the segment's partial
+        // ---- merge the warps' states, write the segment's partial
         // Row groups with a rotated chunk order hold chunk (c + shift) mod CPL
         // in register slot c; put them back in the unrotated order first so
         // the cross-row-group sums below add like columns.
@@ -447,15 +557,14 @@ gqa_split_kernel(const GqaParams p) {
                 if (shift == sh) {
 #pragma unroll
                     for (int g = 0; g < HC; ++g) {
-                        float tmp[C::kEPL];
+                        float2 tmp[EP];
 #pragma unroll
                         for (int c = 0; c < C::kCPL; ++c)
 #pragma unroll
-                            for (int e = 0; e < C::kLE; ++e)
-                                tmp[((c + sh) % C::kCPL) * C::kLE + e] =
-                                    o[g][c * C::kLE + e];
+                            for (int j = 0; j < LP; ++j)
+                                tmp[((c + sh) % C::kCPL) * LP + j] = o2[g][c * LP + j];
 #pragma unroll
-                        for (int e = 0; e < C::kEPL; ++e) o[g][e] = tmp[e];
+                        for (int j = 0; j < EP; ++j) o2[g][j] = tmp[j];
                     }
                 }
             }
@@ -465,21 +574,24 @@ gqa_split_kernel(const GqaParams p) {
 #pragma unroll
             for (int g = 0; g < HC; ++g)
 #pragma unroll
-                for (int e = 0; e < C::kEPL; ++e)
-                    o[g][e] += __shfl_xor_sync(0xffffffffu, o[g][e], m);
+                for (int j = 0; j < EP; ++j) {
+                    o2[g][j].x += __shfl_xor_sync(0xffffffffu, o2[g][j].x, m);
+                    o2[g][j].y += __shfl_xor_sync(0xffffffffu, o2[g][j].y, m);
+                }
         if (rg == 0) {
 #pragma unroll
             for (int g = 0; g < HC; ++g)
 #pragma unroll
                 for (int c = 0; c < C::kCPL; ++c)
 #pragma unroll
-                    for (int e = 0; e < C::kLE; ++e)
-                        s_mo[(warp * HC + g) * D + col[c] + e] = o[g][c * C::kLE + e];
+                    for (int j = 0; j < LP; ++j)
+                        *reinterpret_cast<float2 *>(&s_mo[(warp * HC + g) * D + col[c] + 2 * j]) =
+                            o2[g][c * LP + j];
         }
-        if ((lane & 7) == 0) {
+        if ((lane % C::kTPW) == 0) {
 #pragma unroll
             for (int ps = 0; ps < C::kPasses; ++ps) {
-                const int gs = lane / 8 + 4 * ps;
+                const int gs = lane / C::kTPW + C::kHPP * ps;
                 if (gs < HC) {
                     s_mm[warp * HC + gs] = m_run[ps];
                     s_ml[warp * HC + gs] = l_run[ps];
@@ -515,7 +627,7 @@ gqa_split_kernel(const GqaParams p) {
     }
 
     // Abort path: copies still in flight must land before the CTA exits.
-    if (producer) {
+    if (producer && lane == 0) {
         for (long long n = n_tile; n < issued; ++n)
             mbar_wait(&full_bar[n % C::kStages], (uint32_t)((n / C::kStages) & 1),
                       p.timeout_ns, p.err, nullptr);

@@ -33,7 +33,7 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     }
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
     gqa_split_kernel<D, HC, T>
-        <<<L.kp.num_ctas, kGqaThreads, C::kSmemBytes, L.stream>>>(L.kp);
+        <<<L.kp.num_ctas, C::kThreads, C::kSmemBytes, L.stream>>>(L.kp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
