@@ -27,7 +27,7 @@ C_SYMBOLS = (
     "attn_decode_plan", "attn_decode_gqa_config", "attn_set_num_ctas",
     "attn_set_gqa_path", "attn_set_profile_events",
     "attn_debug_force_timeout", "attn_decode_last_error",
-    "attn_status_string", "attn_version",
+    "attn_status_string", "attn_version", "attn_decode_gqa_noalloc",
 )
 
 _lib = None
@@ -54,6 +54,7 @@ def load():
     p, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.attn_decode_gqa.argtypes = [p] * 6 + [i] * 4 + [f, i, p, i, i, i]
     lib.attn_decode_mla.argtypes = [p] * 6 + [i] * 4 + [f, p, i, i]
+    lib.attn_decode_gqa_noalloc.argtypes = lib.attn_decode_gqa.argtypes
     lib.kv_append.argtypes = [p] * 6 + [i] * 6 + [p]
     lib.kv_append_mla.argtypes = [p] * 4 + [i] * 5 + [p]
     lib.attn_decode_plan.argtypes = [p, i, i, i, i, i, p, p]
@@ -125,6 +126,29 @@ def decode_gqa(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
         B, H_q, H_kv, d, float(scale), int(window), _stream_ptr(stream),
         block_table.shape[1], nblk, dt)
     _check(rc, "attn_decode_gqa")
+    return out
+
+
+def decode_gqa_noalloc(q, k_cache, v_cache, seq_lens, block_table, scale,
+                       window=0, out=None, stream=None):
+    """decode_gqa through attn_decode_gqa_noalloc: same result, but the split
+    scratch is the library's fixed device array, so the call never allocates
+    device memory (for callers that must not allocate while running).  Calls
+    share that array: keep them on one stream."""
+    B, H_q, d = q.shape
+    nblk, H_kv, bs, d2 = k_cache.shape
+    if bs != BLOCK_SIZE or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("cache must be [num_blocks][H_kv][64][d] for K and V")
+    dt = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = load().attn_decode_gqa_noalloc(
+        _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
+        _dev(v_cache, "v_cache", q.dtype), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(block_table, "block_table", torch.int32), _dev(out, "out", q.dtype),
+        B, H_q, H_kv, d, float(scale), int(window), _stream_ptr(stream),
+        block_table.shape[1], nblk, dt)
+    _check(rc, "attn_decode_gqa_noalloc")
     return out
 
 

@@ -111,6 +111,13 @@ static void take_force_timeout(int *flag, unsigned long long *ns) {
     *ns = (*flag && t > 0) ? (unsigned long long)t : kDefaultTimeoutNs;
 }
 
+// Device address of the current device's error word, for entry points
+// defined in other translation units (null on failure).
+unsigned *internal_error_word() {
+    DeviceState *st;
+    return device_state(&st) == ATTN_OK ? st->err : nullptr;
+}
+
 }  // namespace attn
 
 using namespace attn;

@@ -201,6 +201,39 @@ int attn_debug_force_timeout(int enable, long long timeout_ns);
  */
 int attn_decode_last_error(void *stream);
 
+/*
+ * attn_decode_gqa_noalloc -- attn_decode_gqa for callers that may not
+ * allocate device memory while they run.  (The source pages have no
+ * counterpart: this is a deployment variant of the same operation.)
+ *
+ * Some callers cannot call cudaMalloc/cudaFree after start-up: a serving
+ * process that gives all device memory to its own pool, or a latency-critical
+ * thread that cannot take the device-wide synchronisation cudaFree implies.
+ * This entry point computes exactly what attn_decode_gqa computes, with the
+ * same arguments and layouts, but keeps its split scratch in a fixed array
+ * of ATTN_NOALLOC_SCRATCH_BYTES compiled into the library (every GPU that
+ * loads the library holds that array until the process exits).  It never
+ * allocates.  The caller still passes all inputs and the output.
+ *
+ * Scratch needed: 4 * (B*H_q/hc + SMs) * hc * (d + 1) bytes plus 8*(B+1)
+ * (hc = query heads per CTA, see attn_decode_gqa_config; each term rounded
+ * up to 256 bytes); above the limit the call returns ATTN_ERR_UNSUPPORTED.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, on the current device); make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents (nothing in it needs to start at zero): calls that can
+ * overlap on the GPU -- on different streams, or from several threads -- race
+ * on it, so order them on one stream.  The attn_set_num_ctas, profiling and
+ * fault-injection hooks do not apply to this entry point.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *seq_lens,
+                            const int32_t *block_table, void *out, int B,
+                            int H_q, int H_kv, int d, float scale, int window,
+                            void *stream, int max_blocks_per_seq,
+                            int num_blocks, int dtype);
+
 /* Human-readable name of a status code (static storage). */
 const char *attn_status_string(int status);
 
