@@ -282,7 +282,7 @@ int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent
         !aligned16(out))
         return ATTN_ERR_ARG;
     if (d_c != 512 || d_r != 64) return ATTN_ERR_UNSUPPORTED;
-    if (H != 16 && H != 32 && H != 64 && H != 128) return ATTN_ERR_UNSUPPORTED;
+    if (H != 128) return ATTN_ERR_UNSUPPORTED;
     DeviceState *st;
     int rc = device_state(&st);
     if (rc) return rc;

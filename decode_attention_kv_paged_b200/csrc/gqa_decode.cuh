@@ -330,10 +330,10 @@ gqa_split_kernel(const GqaParams p) {
     plan_locate(pa, blockIdx.x, plan_sh, blockIdx.x == 0 ? p.ws_prefix : nullptr,
                 p.err);
     const long long W = plan_sh->total;
-    if (W <= 0) return;
-    const long long lo = cta_bound(blockIdx.x, W, p.num_ctas);
-    const long long hi = cta_bound(blockIdx.x + 1, W, p.num_ctas);
-    if (lo >= hi) return;
+    const int P = working_ctas(W, p.num_ctas);
+    if ((int)blockIdx.x >= P) return;
+    const long long lo = cta_bound(blockIdx.x, W, P);
+    const long long hi = cta_bound(blockIdx.x + 1, W, P);
     SegmentWalker walk;
     walk.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
 
@@ -641,60 +641,81 @@ struct CombineParams {
     const float *ws_lse;
     void *out;
     int B, H_q, H_kv, group, n_hc, max_blocks, window, num_ctas;
+    int D, HC;               // head dim, query heads per unit
+    int blocks_per_unit;     // CTAs of kCombineThreads per unit
 };
 
-// One CTA per unit: out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L) over
-// the unit's split partials in CTA order (fixed, deterministic).
-template <int D, int HC, typename T>
-__global__ void __launch_bounds__(128)
-gqa_combine_kernel(const CombineParams p) {
+constexpr int kCombineThreads = 256;
+
+// out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L) over the unit's split
+// partials, in CTA order (fixed, deterministic).  Each thread produces four
+// consecutive outputs of one head; a unit's HC*D outputs are spread over
+// blocks_per_unit CTAs.
+template <typename T>
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(const CombineParams p) {
+    __shared__ long long s_first_slot;
+    __shared__ int s_nsplit, s_nb;
     pdl_wait_primary();
     const int units = p.H_kv * p.n_hc;
-    const int u = blockIdx.x;
+    const int u = blockIdx.x / p.blocks_per_unit;
+    const int part = blockIdx.x % p.blocks_per_unit;
     const int b = u / units, rem = u % units;
-    const int kvh = rem / p.n_hc, hc = rem % p.n_hc;
-    const int head0 = kvh * p.group + hc * HC;
-    T *out = static_cast<T *>(p.out) + ((size_t)b * p.H_q + head0) * D;
-    int fb;
-    bool bad;
-    const int nb = visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad);
-    if (nb == 0) {
-        for (int i = threadIdx.x; i < HC * D; i += blockDim.x)
-            out[i] = ElemTraits<T>::from_float(0.f);
-        return;
+    if (threadIdx.x == 0) {
+        int fb;
+        bool bad;
+        const int nb = visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad);
+        s_nb = nb;
+        s_nsplit = 0;
+        s_first_slot = 0;
+        if (nb > 0) {
+            const long long W = p.ws_prefix[p.B];
+            const int P = working_ctas(W, p.num_ctas);
+            const long long s_u = p.ws_prefix[b] + (long long)rem * nb;
+            const int c0 = cta_of(s_u, W, P);
+            const int c1 = cta_of(s_u + nb - 1, W, P);
+            s_nsplit = c1 - c0 + 1;
+            s_first_slot = (long long)u + c0;
+        }
     }
-    const long long W = p.ws_prefix[p.B];
-    const long long s_u = p.ws_prefix[b] + (long long)rem * nb;
-    const long long e_u = s_u + nb;
-    const int c0 = cta_of(s_u, W, p.num_ctas);
-    const int c1 = cta_of(e_u - 1, W, p.num_ctas);
-    const long long slot0 = (long long)u + c0;
-    for (int i = threadIdx.x; i < HC * D; i += blockDim.x) {
-        const int g = i / D, k = i % D;
-        float r;
-        if (c0 == c1) {
-            r = p.ws_o[(slot0 * HC + g) * D + k];
+    __syncthreads();
+    const int e = (part * kCombineThreads + threadIdx.x) * 4;   // output index in unit
+    if (e >= p.HC * p.D) return;
+    const int g = e / p.D, k = e % p.D;
+    const int kvh = rem / p.n_hc, hc = rem % p.n_hc;
+    T *out = static_cast<T *>(p.out) +
+             ((size_t)b * p.H_q + kvh * p.group + hc * p.HC + g) * p.D + k;
+    float r[4];
+    const int ns = s_nsplit;
+    if (s_nb == 0) {
+        r[0] = r[1] = r[2] = r[3] = 0.f;
+    } else {
+        const long long s0 = s_first_slot;
+        if (ns == 1) {
+            const float4 v = *reinterpret_cast<const float4 *>(
+                p.ws_o + ((size_t)s0 * p.HC + g) * p.D + k);
+            r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
         } else {
-            // CTAs between c0 and c1 with an empty range wrote no partial.
             float L = kNegInf;
-            for (int c = c0; c <= c1; ++c) {
-                if (cta_bound(c, W, p.num_ctas) >= cta_bound(c + 1, W, p.num_ctas))
-                    continue;
-                L = fmaxf(L, p.ws_lse[((long long)u + c) * HC + g]);
-            }
-            float num = 0.f, den = 0.f;
-            for (int c = c0; c <= c1; ++c) {
-                if (cta_bound(c, W, p.num_ctas) >= cta_bound(c + 1, W, p.num_ctas))
-                    continue;
-                const long long s = (long long)u + c;
-                const float w = exp2f(p.ws_lse[s * HC + g] - L);
-                num = fmaf(w, p.ws_o[(s * HC + g) * D + k], num);
+            for (int i = 0; i < ns; ++i) L = fmaxf(L, p.ws_lse[(s0 + i) * p.HC + g]);
+            float den = 0.f;
+            r[0] = r[1] = r[2] = r[3] = 0.f;
+            for (int i = 0; i < ns; ++i) {
+                const float w = exp2f(p.ws_lse[(s0 + i) * p.HC + g] - L);
+                const float4 v = *reinterpret_cast<const float4 *>(
+                    p.ws_o + ((size_t)(s0 + i) * p.HC + g) * p.D + k);
+                r[0] = fmaf(w, v.x, r[0]);
+                r[1] = fmaf(w, v.y, r[1]);
+                r[2] = fmaf(w, v.z, r[2]);
+                r[3] = fmaf(w, v.w, r[3]);
                 den += w;
             }
-            r = num / den;
+            const float inv = 1.f / den;
+            r[0] *= inv; r[1] *= inv; r[2] *= inv; r[3] *= inv;
         }
-        out[i] = ElemTraits<T>::from_float(r);
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[j] = ElemTraits<T>::from_float(r[j]);
 }
 
 }  // namespace attn

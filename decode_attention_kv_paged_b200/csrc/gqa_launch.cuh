@@ -38,9 +38,13 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
 
+    CombineParams cp = L.cp;
+    cp.D = D;
+    cp.HC = HC;
+    cp.blocks_per_unit = (HC * D / 4 + kCombineThreads - 1) / kCombineThreads;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(L.units_total);
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3((unsigned)((long long)L.units_total * cp.blocks_per_unit));
+    cfg.blockDim = dim3(kCombineThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = L.stream;
     cudaLaunchAttribute attr[1];
@@ -48,7 +52,7 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     attr[0].val.programmaticStreamSerializationAllowed = L.ev_stop ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gqa_combine_kernel<D, HC, T>, L.cp);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<T>, cp);
 }
 
 // Dispatch over heads-per-CTA and dtype for one head dimension D.

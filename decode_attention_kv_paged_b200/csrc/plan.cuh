@@ -5,7 +5,9 @@
 // visible 64-token blocks of b.  Only blocks that hold at least one visible
 // key are listed, so blocks wholly outside a sliding window are never read
 // (attention-head article, §3: the kernel must skip masked positions).
-// CTA i of P takes the contiguous block range [floor(i*W/P), floor((i+1)*W/P)).
+// Only P' = min(P, W) CTAs take work, so every working CTA has a non-empty
+// range: CTA i < P' takes the contiguous block range
+// [floor(i*W/P'), floor((i+1)*W/P')); CTAs i >= P' have nothing to do.
 // A (unit, CTA) pair that meets writes one partial result; pair slots are
 // numbered unit + CTA, which is injective along the walk, so U + P slots
 // always suffice.
@@ -32,6 +34,11 @@ __device__ __forceinline__ int visible_blocks(int T, int window, int max_blocks,
     const int lo = (window > 0 && T > window) ? T - window : 0;
     *first_block = lo / kBlockSize;
     return (T - 1) / kBlockSize - lo / kBlockSize + 1;
+}
+
+// Number of CTAs that take work.
+__device__ __forceinline__ int working_ctas(long long W, int P) {
+    return W < (long long)P ? (int)W : P;
 }
 
 __device__ __forceinline__ long long cta_bound(long long i, long long W, int P) {
@@ -69,7 +76,8 @@ struct PlanScratch {          // shared memory used by plan_locate
 // `target(W)` together with the work (blocks x units) before that sequence.
 // Every thread of the block must call it.  When prefix_out is non-null the
 // exclusive prefix sums of work per sequence (B + 1 values) are written.
-// `target_cta` selects target = cta_bound(target_cta, W, num_ctas).
+// `target_cta` selects target = cta_bound(target_cta, W, P') (none if the
+// CTA has no work).
 __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_cta,
                             PlanScratch *sh, long long *prefix_out,
                             unsigned *err) {
@@ -99,8 +107,9 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
     if (any_bad) sh->bad = 1;
     __syncthreads();
     const long long W = sh->total;
+    const int P = working_ctas(W, a.num_ctas);
     const long long target =
-        (W > 0) ? cta_bound(target_cta, W, a.num_ctas) : 0;
+        (W > 0 && target_cta < P) ? cta_bound(target_cta, W, P) : W;
 
     // Pass 2: exclusive scan, locate target.
     long long running = 0;

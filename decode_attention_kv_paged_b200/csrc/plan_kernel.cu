@@ -14,8 +14,9 @@ __global__ void __launch_bounds__(256) plan_kernel(PlanArgs a, long long *out,
     const long long W = sh.total;
     long long *row = out + 1 + 4ll * blockIdx.x;
     if (blockIdx.x == 0) out[0] = W;
-    const long long lo = W > 0 ? cta_bound(blockIdx.x, W, a.num_ctas) : 0;
-    const long long hi = W > 0 ? cta_bound(blockIdx.x + 1, W, a.num_ctas) : 0;
+    const int P = working_ctas(W, a.num_ctas);
+    const long long lo = (int)blockIdx.x < P ? cta_bound(blockIdx.x, W, P) : W;
+    const long long hi = (int)blockIdx.x < P ? cta_bound(blockIdx.x + 1, W, P) : W;
     row[0] = lo;
     row[1] = hi;
     if (lo >= hi) {

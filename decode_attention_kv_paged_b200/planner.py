@@ -10,7 +10,8 @@ or one chunk of the query heads sharing it) in order; inside a unit the
 visible blocks [first_b, last_b] in order, where the visible key range is
 [lo_b, T_b) with lo_b = max(0, T_b - window) for window > 0, else 0, and only
 blocks holding a visible key are listed.  CTA i of P takes the block range
-[floor(i W / P), floor((i + 1) W / P)).
+[floor(i W / P'), floor((i + 1) W / P')) for i < P' = min(P, W); the other
+CTAs have no work.
 """
 BLOCK_SIZE = 64
 
@@ -22,6 +23,11 @@ def visible_blocks(T, window, max_blocks):
     lo = T - window if (window > 0 and T > window) else 0
     first = lo // BLOCK_SIZE
     return first, (T - 1) // BLOCK_SIZE - first + 1
+
+
+def working_ctas(W, P):
+    """CTAs that take work: min(P, W), so no working CTA has an empty range."""
+    return min(P, W)
 
 
 def cta_bound(i, W, P):
@@ -36,10 +42,11 @@ def plan(seq_lens, units_per_seq, window, max_blocks, num_ctas):
     for w in work:
         prefix.append(prefix[-1] + w)
     W = prefix[-1]
+    P = working_ctas(W, num_ctas)
     out = [W]
     for i in range(num_ctas):
-        lo = cta_bound(i, W, num_ctas) if W else 0
-        hi = cta_bound(i + 1, W, num_ctas) if W else 0
+        lo = cta_bound(i, W, P) if i < P else W
+        hi = cta_bound(i + 1, W, P) if i < P else W
         if lo >= hi:
             out += [lo, hi, -1, -1]
             continue
@@ -61,8 +68,7 @@ def cta_of(x, W, P):
 
 def splits_of_unit(seq_lens, units_per_seq, window, max_blocks, num_ctas, b,
                    unit):
-    """CTAs (in order) that hold a part of (sequence b, unit).  CTAs whose
-    range is empty hold nothing and are left out."""
+    """CTAs (in order) that hold a part of (sequence b, unit)."""
     p = plan(seq_lens, units_per_seq, window, max_blocks, num_ctas)
     W = p[0]
     prefix = p[1 + 4 * num_ctas:]
@@ -70,5 +76,5 @@ def splits_of_unit(seq_lens, units_per_seq, window, max_blocks, num_ctas, b,
     if nb == 0:
         return []
     s = prefix[b] + unit * nb
-    return [c for c in range(cta_of(s, W, num_ctas), cta_of(s + nb - 1, W, num_ctas) + 1)
-            if cta_bound(c, W, num_ctas) < cta_bound(c + 1, W, num_ctas)]
+    P = working_ctas(W, num_ctas)
+    return list(range(cta_of(s, W, P), cta_of(s + nb - 1, W, P) + 1))

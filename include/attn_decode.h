@@ -102,9 +102,9 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
  * latent_cache [num_blocks][64][d_c + d_r] bf16: row = c_j followed by the
  *              already-rotated shared RoPE key kR_j
  * out          [B][H][d_c]  bf16  latent-space output z (apply U^V_h after)
- * Supported: d_c = 512, d_r = 64, H in {16, 32, 64, 128} (heads padded to a
- * multiple of 64 inside the kernel); otherwise ATTN_ERR_UNSUPPORTED.
- * Workspace as for attn_decode_gqa.
+ * Supported: d_c = 512, d_r = 64, H = 128 (the tensor-core tile is 128
+ * heads); otherwise ATTN_ERR_UNSUPPORTED.  Workspace as for attn_decode_gqa.
+ * Runs as clusters of two CTAs; uses 512 TMEM columns per CTA.
  */
 int attn_decode_mla(const void *q_latent, const void *q_rope,
                     const void *latent_cache, const int32_t *seq_lens,
