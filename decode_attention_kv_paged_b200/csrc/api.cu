@@ -286,6 +286,8 @@ int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent
     DeviceState *st;
     int rc = device_state(&st);
     if (rc) return rc;
+    cudaEvent_t ev_start, ev_stop;
+    take_profile_events(&ev_start, &ev_stop);
     return mla_decode_entry(q_latent, q_rope, latent_cache, seq_lens, block_table, out, B,
                             H, scale, (cudaStream_t)stream, max_blocks_per_seq, num_blocks,
                             st->num_sms, tl_num_ctas, st->err,
@@ -293,7 +295,8 @@ int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent
                                 int r = ensure_workspace(st, bytes, (cudaStream_t)stream);
                                 *ws = st->ws;
                                 return r;
-                            });
+                            },
+                            ev_start, ev_stop);
 }
 
 int kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -78,19 +78,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // Returns false if it did not within timeout_ns (raising kErrTimeout), or as
 // soon as another warp of the CTA has set *abort (then without raising).
+// The clock is read only every 64 failed polls: reading %globaltimer is not
+// free, and a tight loop of it starves other warps of the same pipe.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           unsigned long long timeout_ns,
                                           unsigned *err,
                                           volatile int *abort = nullptr) {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
-    while (true) {
+    unsigned long long t0 = 0;
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort && *abort) return false;
-        if (global_timer_ns() - t0 > timeout_ns) {
-            raise_error(err, kErrTimeout);
-            if (abort) *abort = 1;
-            return false;
+        if ((it & 63u) == 0) {
+            const unsigned long long now = global_timer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > timeout_ns) {
+                raise_error(err, kErrTimeout);
+                if (abort) *abort = 1;
+                return false;
+            }
         }
     }
 }

@@ -10,22 +10,34 @@
 // (sequence, 64-token block) list.  The latent columns are split between
 // them -- rank 0 owns columns [0, 256), rank 1 owns [256, 512) plus the RoPE
 // columns [512, 576) -- so each CTA streams only its slice of every block
-// with 2-D TMA (128-byte swizzle), and no cache byte is read twice.
-//   * S = Q C^T is a 128 x 64 (heads x tokens) tcgen05 MMA with K = 256 or
-//     320 per CTA, accumulated in TMEM; the two partial S are exchanged
-//     through distributed shared memory and summed identically in both CTAs.
-//   * Softmax runs one thread per head row directly on the TMEM rows (no
-//     cross-thread reductions); the running max is only raised when it grows
-//     by more than 2^8, so O is rescaled rarely (the result is exact either
-//     way: numerator and denominator use the same max).
+// with 2-D TMA (128-byte swizzle, 3-stage ring), and no cache byte is read
+// twice.
+//   * The query slice lives in tensor memory (row = head = TMEM lane, bf16
+//     pairs per 32-bit column), written once per sequence by the softmax
+//     threads; S = Q C^T is a 128 x 64 (heads x tokens) tcgen05 MMA with A in
+//     TMEM and B = the C tile in shared memory, accumulated in TMEM.
+//   * The two partial S are exchanged between the CTAs of the cluster: each
+//     thread stages its half-row in local shared memory and one thread moves
+//     the 32 KiB to the peer with a single bulk copy (shared::cta ->
+//     shared::cluster, completion on the peer's barrier); both CTAs sum the
+//     halves identically.  The softmax loop is software-pipelined: in
+//     iteration i a CTA first consumes the peer's S(i), then stages and sends
+//     its own S(i+1), then does the softmax of tile i, which hides the
+//     transfer.
+//   * Softmax runs one thread per head row on the TMEM rows (no cross-thread
+//     reductions); the running max is only raised when it grows by more than
+//     2^8, so O is rescaled rarely (the result is exact either way: numerator
+//     and denominator use the same max).
 //   * P is split into two bf16 halves, P = P_hi + P_lo (P_lo = the rounding
 //     remainder), so the weights keep ~16 significant bits instead of bf16's
 //     8; both halves (128 x 64, swizzled like a TMA tile) are A operands of
 //     O += P_hi C + P_lo C, 128 x 256 MMAs whose B operand is the same C tile
 //     read MN-major.  Each CTA keeps its 256 output columns in TMEM.
-//   * Warp 0 issues TMA, warp 1 issues MMAs, warps 4-7 do softmax and the
-//     epilogue.  Every wait is bounded; TMEM is always freed; the final
-//     cluster handshake is a bounded mbarrier exchange.
+//   * Warp 0 issues TMA; one thread of warp 1 issues MMAs, polling the S and
+//     P V dependencies and issuing whichever is ready (no head-of-line
+//     blocking); warps 4-7 load Q, run the softmax and the epilogue.  Every
+//     wait is bounded; TMEM is always freed; the final cluster handshake is a
+//     bounded mbarrier exchange.
 // Each (sequence, cluster) segment writes an fp32 partial (O/l and log2-sum-
 // exp) that the combine kernel reduces in cluster order.
 #include <mutex>
@@ -40,29 +52,33 @@ namespace attn {
 
 constexpr int kMlaH = 128;                 // heads = MMA M
 constexpr int kMlaDc = 512, kMlaDr = 64, kMlaWidth = 576;
-constexpr int kMlaQBox = 128 * 128;        // [128 heads][64 cols] bf16
 constexpr int kMlaCBox = 64 * 128;         // [64 tokens][64 cols] bf16
 constexpr int kMlaMaxBoxes = 5;
-constexpr int kMlaStages = 2;
-constexpr int kMlaThreads = 256;
-constexpr int kOffQ = 0;
-constexpr int kOffC = kOffQ + kMlaMaxBoxes * kMlaQBox;
-constexpr int kOffP = kOffC + kMlaStages * kMlaMaxBoxes * kMlaCBox;
+constexpr int kMlaStages = 3;
+constexpr int kMlaStageBytes = kMlaMaxBoxes * kMlaCBox;
+constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA, 4-11 softmax
+constexpr int kSoftThreads = 256;
 constexpr int kPBytes = kMlaH * 128;       // one P half: [128 heads][64 tokens] bf16
-constexpr int kOffX = kOffP + 2 * kPBytes;
-constexpr int kOffBar = kOffX + kMlaH * 64 * 4;
-constexpr int kMlaSmemUsed = kOffBar + 512;
+constexpr int kXBytes = kMlaH * 64 * 4;    // exchange buffer: 16 chunks x [128 rows] x 16 B
+constexpr int kOffC = 0;
+constexpr int kOffP = kOffC + kMlaStages * kMlaStageBytes;
+constexpr int kOffX = kOffP + 2 * kPBytes;   // receives the peer's partial S
+constexpr int kOffStg = kOffX + kXBytes;     // stages this CTA's partial S
+constexpr int kOffBar = kOffStg + kXBytes;
+constexpr int kOffRed = kOffBar + 512;     // [2][2][128] row-max halves + [2][2][128] sums
+constexpr int kMlaSmemUsed = kOffRed + 2 * 2 * 2 * 128 * 4;
 constexpr int kMlaSmem = kMlaSmemUsed + 1024;       // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0, kTmemS = 256;       // S buffers at 256, 320
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320;   // Q: 32 columns per box
 constexpr float kRescaleThreshold = 8.0f;           // log2 units
 
 struct MlaBars {
     uint64_t q_full, q_empty;
     uint64_t c_full[kMlaStages], c_empty[kMlaStages];
-    uint64_t s_full[2], s_free[2];
+    uint64_t s_full, s_free;
     uint64_t p_full, pv_done, o_free;
-    uint64_t x_full, x_free;
+    uint64_t x_full, x_free, stg_full;
+    uint64_t red_bar, sum_bar;
     uint64_t end_bar, mma_final;
     uint32_t tmem_base;
     int abort;
@@ -70,8 +86,11 @@ struct MlaBars {
 };
 static_assert(sizeof(MlaBars) <= 512, "barrier block");
 static_assert(kMlaSmem <= 227 * 1024, "shared memory per CTA");
+static_assert(kTmemQ + 32 * kMlaMaxBoxes <= kTmemCols, "TMEM columns");
 
 struct MlaParams {
+    const __nv_bfloat16 *q_lat;    // [B][128][512]
+    const __nv_bfloat16 *q_rope;   // [B][128][64]
     const int32_t *seq_lens;
     const int32_t *block_table;
     float *ws_o;          // [slots][128][512]
@@ -84,13 +103,10 @@ struct MlaParams {
 };
 
 __global__ void __launch_bounds__(kMlaThreads, 1)
-mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_qr,
-                  const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
+mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    unsigned char *sQ = smem + kOffQ;
     unsigned char *sC = smem + kOffC;
     unsigned char *sP = smem + kOffP;
     unsigned char *sX = smem + kOffX;
@@ -119,21 +135,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     // ---- set-up: barriers, TMEM, cluster handshake
     if (tid == 0) {
-        mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_full, kSoftThreads);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMlaStages; ++s) {
             mbar_init(&bars->c_full[s], 1);
             mbar_init(&bars->c_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars->s_full[s], 1);
-            mbar_init(&bars->s_free[s], 128);
-        }
-        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_free, kSoftThreads);
+        mbar_init(&bars->p_full, kSoftThreads);
         mbar_init(&bars->pv_done, 1);
-        mbar_init(&bars->o_free, 128);
-        mbar_init(&bars->x_full, 128);
-        mbar_init(&bars->x_free, 128);
+        mbar_init(&bars->o_free, kSoftThreads);
+        mbar_init(&bars->x_full, 1);               // peer's arrive.expect_tx + bulk copy
+        mbar_init(&bars->x_free, kSoftThreads);    // peer's threads consumed my data
+        mbar_init(&bars->stg_full, kSoftThreads);  // my threads staged their halves
+        mbar_init(&bars->red_bar, kSoftThreads);
+        mbar_init(&bars->sum_bar, kSoftThreads);
         mbar_init(&bars->end_bar, 1);
         mbar_init(&bars->mma_final, 1);
         bars->abort = 0;
@@ -151,43 +168,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
             tma_prefetch_map(&tm_c);
-            tma_prefetch_map(&tm_q);
             TileCursor cur;
             cur.init(pa, lo, hi, first_seq, first_base);
-            int seg = 0, tile = 0, q_issued = 0;
-            bool ok = true;
-            while (ok && !cur.done()) {
-                if (cur.t == 0) {
-                    if (seg > 0 && !mbar_wait(&bars->q_empty, (uint32_t)((seg - 1) & 1),
-                                              p.timeout_ns, p.err, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const int row = cur.w.b * kMlaH;
-                    mbar_arrive_expect_tx(&bars->q_full, nbox * kMlaQBox);
-                    for (int i = 0; i < nbox; ++i) {
-                        if (rank == 1 && i == 4)
-                            tma_load_2d(sQ + i * kMlaQBox, &tm_qr, 0, row, &bars->q_full, pol);
-                        else
-                            tma_load_2d(sQ + i * kMlaQBox, &tm_q, col0 + i * 64, row,
-                                        &bars->q_full, pol);
-                    }
-                    ++seg;
-                    q_issued = seg;
-                }
+            int tile = 0;
+            while (!cur.done()) {
                 const int st = tile % kMlaStages;
                 if (tile >= kMlaStages &&
-                    !mbar_wait(&bars->c_empty[st], (uint32_t)(((tile - kMlaStages) / kMlaStages) & 1),
-                               p.timeout_ns, p.err, abort_flag)) {
-                    ok = false;
+                    !mbar_wait(&bars->c_empty[st],
+                               (uint32_t)(((tile - kMlaStages) / kMlaStages) & 1),
+                               p.timeout_ns, p.err, abort_flag))
                     break;
-                }
                 int phys = p.block_table[(size_t)cur.w.b * p.max_blocks + cur.logical_block()];
                 if (phys < 0 || phys >= p.num_blocks) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;            // wholly out of bounds: zero fill
                 }
-                unsigned char *dst = sC + st * (kMlaMaxBoxes * kMlaCBox);
+                unsigned char *dst = sC + st * kMlaStageBytes;
                 mbar_arrive_expect_tx(&bars->c_full[st], nbox * kMlaCBox);
                 for (int i = 0; i < nbox; ++i)
                     tma_load_2d(dst + i * kMlaCBox, &tm_c, col0 + i * 64, phys * 64,
@@ -199,9 +195,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int t = tile - kMlaStages < 0 ? 0 : tile - kMlaStages; t < tile; ++t)
                 mbar_wait(&bars->c_full[t % kMlaStages], (uint32_t)((t / kMlaStages) & 1),
                           p.timeout_ns, p.err, nullptr);
-            if (q_issued > 0)
-                mbar_wait(&bars->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns, p.err,
-                          nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -209,72 +202,82 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 256, 0, 1);
-            const uint32_t q_base = smem_u32(sQ), c_base = smem_u32(sC), p_base = smem_u32(sP);
-            TileCursor cs, cv;           // S runs one tile ahead of P V
+            const uint32_t c_base = smem_u32(sC), p_base = smem_u32(sP);
+            TileCursor cs, cv;           // next tile to issue S for / P V for
             cs.init(pa, lo, hi, first_seq, first_base);
             cv.init(pa, lo, hi, first_seq, first_base);
-            int seg_s = 0, seg_v = 0;
-            bool ok = true;
-
-            auto issue_s = [&](int i) -> bool {
-                const bool first = cs.t == 0, last = cs.t == cs.len - 1;
-                if (first) {
-                    if (!mbar_wait(&bars->q_full, (uint32_t)(seg_s & 1), p.timeout_ns, p.err,
-                                   abort_flag))
-                        return false;
-                }
-                const int st = i % kMlaStages, sb = i & 1;
-                if (!mbar_wait(&bars->c_full[st], (uint32_t)((i / kMlaStages) & 1),
-                               p.timeout_ns, p.err, abort_flag))
-                    return false;
-                if (i >= 2 && !mbar_wait(&bars->s_free[sb], (uint32_t)(((i - 2) / 2) & 1),
-                                         p.timeout_ns, p.err, abort_flag))
-                    return false;
-                tc_fence_after();
-                const uint32_t cst = c_base + st * (kMlaMaxBoxes * kMlaCBox);
-                for (int bx = 0; bx < nbox; ++bx)
+            int next_s = 0, next_pv = 0, seg_s = 0, seg_v = 0;
+            unsigned long long idle_since = 0;
+            uint32_t idle_polls = 0;
+            while (next_pv < n_tiles) {
+                bool did = false;
+                if (next_s < n_tiles) {
+                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
+                    const int st = next_s % kMlaStages;
+                    const bool ready =
+                        (!first || mbar_test(&bars->q_full, (uint32_t)(seg_s & 1))) &&
+                        mbar_test(&bars->c_full[st], (uint32_t)((next_s / kMlaStages) & 1)) &&
+                        (next_s == 0 || mbar_test(&bars->s_free, (uint32_t)((next_s - 1) & 1)));
+                    if (ready) {
+                        tc_fence_after();
+                        const uint32_t cst = c_base + st * kMlaStageBytes;
+                        for (int bx = 0; bx < nbox; ++bx)
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t a = umma_desc_sw128(q_base + bx * kMlaQBox + k * 32, 16, 1024);
-                        const uint64_t b = umma_desc_sw128(cst + bx * kMlaCBox + k * 32, 16, 1024);
-                        umma_bf16(tmem + kTmemS + 64 * sb, a, b, idesc_s, (bx | k) != 0);
+                            for (int k = 0; k < 4; ++k) {
+                                const uint64_t b =
+                                    umma_desc_sw128(cst + bx * kMlaCBox + k * 32, 16, 1024);
+                                umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 32 * bx + 8 * k, b,
+                                             idesc_s, (bx | k) != 0);
+                            }
+                        umma_commit(&bars->s_full);
+                        if (last) umma_commit(&bars->q_empty);
+                        if (first) ++seg_s;
+                        cs.next();
+                        ++next_s;
+                        did = true;
                     }
-                umma_commit(&bars->s_full[sb]);
-                if (last) umma_commit(&bars->q_empty);
-                if (first) ++seg_s;
-                cs.next();
-                return true;
-            };
-            auto issue_pv = [&](int i) -> bool {
-                const bool first = cv.t == 0;
-                if (!mbar_wait(&bars->p_full, (uint32_t)(i & 1), p.timeout_ns, p.err, abort_flag))
-                    return false;
-                if (first && seg_v > 0 &&
-                    !mbar_wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1), p.timeout_ns, p.err,
-                               abort_flag))
-                    return false;
-                tc_fence_after();
-                const int st = i % kMlaStages;
-                const uint32_t cst = c_base + st * (kMlaMaxBoxes * kMlaCBox);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t b = umma_desc_sw128(cst + k * 2048, kMlaCBox, 1024);
-                    const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
-                    const uint64_t a_lo = umma_desc_sw128(p_base + kPBytes + k * 32, 16, 1024);
-                    umma_bf16(tmem + kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
-                    umma_bf16(tmem + kTmemO, a_lo, b, idesc_pv, 1);
                 }
-                umma_commit(&bars->c_empty[st]);
-                umma_commit(&bars->pv_done);
-                if (first) ++seg_v;
-                cv.next();
-                return true;
-            };
-
-            ok = issue_s(0);
-            for (int i = 0; ok && i < n_tiles; ++i) {
-                if (i + 1 < n_tiles && !issue_s(i + 1)) { ok = false; break; }
-                if (!issue_pv(i)) { ok = false; break; }
+                if (next_pv < next_s) {
+                    const bool first = cv.t == 0;
+                    const bool ready =
+                        mbar_test(&bars->p_full, (uint32_t)(next_pv & 1)) &&
+                        (!first || seg_v == 0 ||
+                         mbar_test(&bars->o_free, (uint32_t)((seg_v - 1) & 1)));
+                    if (ready) {
+                        tc_fence_after();
+                        const int st = next_pv % kMlaStages;
+                        const uint32_t cst = c_base + st * kMlaStageBytes;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t b = umma_desc_sw128(cst + k * 2048, kMlaCBox, 1024);
+                            const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
+                            const uint64_t a_lo =
+                                umma_desc_sw128(p_base + kPBytes + k * 32, 16, 1024);
+                            umma_bf16(tmem + kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
+                            umma_bf16(tmem + kTmemO, a_lo, b, idesc_pv, 1);
+                        }
+                        umma_commit(&bars->c_empty[st]);
+                        umma_commit(&bars->pv_done);
+                        if (first) ++seg_v;
+                        cv.next();
+                        ++next_pv;
+                        did = true;
+                    }
+                }
+                if (did) {
+                    idle_since = 0;
+                    idle_polls = 0;
+                } else if ((++idle_polls & 7u) == 0 && (__nanosleep(32), (idle_polls & 63u) == 0)) {
+                    // the clock is read only every 64 idle polls
+                    const unsigned long long now = global_timer_ns();
+                    if (idle_since == 0) idle_since = now;
+                    if (*abort_flag) break;
+                    if (now - idle_since > p.timeout_ns) {
+                        raise_error(p.err, kErrTimeout);
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
             }
             // All MMAs issued so far complete before TMEM is released.
             umma_commit(&bars->mma_final);
@@ -282,111 +285,197 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ===================================================== softmax
-        const int row = tid - 128;                       // head = TMEM lane
-        const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        // ============================================ Q load, softmax, epilogue
+        // Two threads per head row: warps w and w + 4 share TMEM lanes
+        // 32*(w%4) .. +31; half h takes tokens [32h, 32h+32) of each tile and
+        // output columns [128h, 128h+128) of this CTA's 256.
+        const int q4 = warp & 3, h = (warp - 4) >> 2;
+        const int row = 32 * q4 + lane;                      // head = TMEM lane
+        const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
         const uint32_t x_peer = map_to_rank(sX, peer);
         const uint32_t x_full_peer = map_to_rank(&bars->x_full, peer);
         const uint32_t x_free_peer = map_to_rank(&bars->x_free, peer);
-        float *xrow = reinterpret_cast<float *>(sX) + row * 64;
+        unsigned char *sStg = smem + kOffStg;
+        const bool sender = (warp == 4 && lane == 0);
         unsigned char *prow = sP + row * 128;
-        // Every wait outcome is made warp-uniform: the TMEM loads and stores
-        // below are warp-collective and must never run in a partial warp.
+        float *red = reinterpret_cast<float *>(smem + kOffRed);   // [2][2][128] then sums
+        // Wait outcomes are made warp-uniform: the TMEM loads and stores are
+        // warp-collective and must never run in a partial warp.
         auto all = [](bool v) { return __all_sync(0xffffffffu, v); };
-        TileCursor cur;
-        cur.init(pa, lo, hi, first_seq, first_base);
-        float m_run = -1e30f, l_run = 0.f;
-        float s[64];
-        for (int i = 0; i < n_tiles; ++i) {
-            const bool first = cur.t == 0, last = cur.t == cur.len - 1;
-            const int b = cur.w.b, T = cur.w.T;
-            const int tok0 = cur.logical_block() * 64;
-            const int sb = i & 1;
-            if (!all(mbar_wait(&bars->s_full[sb], (uint32_t)((i >> 1) & 1), p.timeout_ns,
-                               p.err, abort_flag)))
-                break;
-            tc_fence_after();
-            tmem_ld64(trow + kTmemS + 64 * sb, s);
-            tc_fence_before();
-            mbar_arrive(&bars->s_free[sb]);
+        const int box_lo = h == 0 ? 0 : (nbox + 1) / 2;
+        const int box_hi = h == 0 ? (nbox + 1) / 2 : nbox;
 
-            // exchange the partial scores with the other CTA of the cluster
+        // Write this head's query slice (this half's boxes) into TMEM.
+        auto load_q = [&](int b, int q_seg) -> bool {
+            if (q_seg > 0 && !all(mbar_wait(&bars->q_empty, (uint32_t)((q_seg - 1) & 1),
+                                            p.timeout_ns, p.err, abort_flag)))
+                return false;
+            tc_fence_after();
+            for (int bx = box_lo; bx < box_hi; ++bx) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    (rank == 1 && bx == 4)
+                        ? p.q_rope + ((size_t)b * kMlaH + row) * kMlaDr
+                        : p.q_lat + ((size_t)b * kMlaH + row) * kMlaDc + col0 + 64 * bx);
+                uint32_t r[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 v = __ldg(src + j);
+                    r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+                }
+                tmem_st32(trow + kTmemQ + 32 * bx, r);
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->q_full);
+            return true;
+        };
+        // Read this half of the CTA's partial S(i) from TMEM, free it, stage it
+        // and (one thread) send the whole staged tile to the peer.  The peer
+        // must have consumed the previous tile (x_free) before the staging
+        // buffer and its receive buffer are reused.
+        auto fetch_s = [&](int i, float *dst) -> bool {
+            if (!all(mbar_wait(&bars->s_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                return false;
+            tc_fence_after();
+            tmem_ld32(trow + kTmemS + 32 * h, dst);
+            tc_fence_before();
+            mbar_arrive(&bars->s_free);
             if (i >= 1 && !all(mbar_wait_cluster(&bars->x_free, (uint32_t)((i - 1) & 1),
                                                  p.timeout_ns, p.err, abort_flag)))
-                break;
+                return false;
+            unsigned char *stg = sStg + row * 16;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                st_cluster_v4(x_peer + (uint32_t)(row * 256 + ((c ^ (row & 15)) * 16)),
-                              s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-            mbar_arrive_remote(x_full_peer);
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<float4 *>(stg + (8 * h + c) * (kMlaH * 16)) =
+                    make_float4(dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3]);
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->stg_full);
+            bool sent = true;
+            if (sender) {
+                sent = mbar_wait(&bars->stg_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
+                                 abort_flag);
+                if (sent) {
+                    mbar_arrive_expect_tx_remote(x_full_peer, kXBytes);
+                    bulk_copy_to_peer(x_peer, sStg, kXBytes, x_full_peer);
+                }
+            }
+            return all(sent);
+        };
+
+        TileCursor cur, nxt;
+        cur.init(pa, lo, hi, first_seq, first_base);
+        nxt.init(pa, lo, hi, first_seq, first_base);
+        int q_seg = 0, n_seg = 0;
+        float m_run = -1e30f, l_run = 0.f;                // l_run: this half's sum
+        float s_nxt[32];
+        bool ok = load_q(nxt.w.b, q_seg++) && fetch_s(0, s_nxt);
+        for (int i = 0; ok && i < n_tiles; ++i) {
+            float s[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] = s_nxt[j];
+            const bool first = cur.t == 0, last = cur.t == cur.len - 1;
+            const int b = cur.w.b, T = cur.w.T;
+            const int nvalid = T - (cur.logical_block() * 64 + 32 * h);   // valid in this half
+
+            // add the peer's partial scores of tile i, scale to log2 units
             if (!all(mbar_wait_cluster(&bars->x_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
                                        abort_flag)))
                 break;
+            const unsigned char *xrow = sX + row * 16;
+            const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float4 v = *reinterpret_cast<const float4 *>(
-                    reinterpret_cast<const unsigned char *>(xrow) + ((c ^ (row & 15)) * 16));
-                s[4 * c] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
+            for (int c = 0; c < 8; ++c) {
+                const float4 v =
+                    *reinterpret_cast<const float4 *>(xrow + (8 * h + c) * (kMlaH * 16));
+                float2 a = __fadd2_rn(make_float2(s[4 * c], s[4 * c + 1]), make_float2(v.x, v.y));
+                float2 bb = __fadd2_rn(make_float2(s[4 * c + 2], s[4 * c + 3]), make_float2(v.z, v.w));
+                a = __fmul2_rn(a, sl2);
+                bb = __fmul2_rn(bb, sl2);
+                s[4 * c] = a.x; s[4 * c + 1] = a.y; s[4 * c + 2] = bb.x; s[4 * c + 3] = bb.y;
             }
             mbar_arrive_remote(x_free_peer);
 
-            // online softmax (log2 domain), lazy rescale
-            const int nvalid = T - tok0 < 64 ? T - tok0 : 64;
-            float mx = kNegInf;
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                s[j] = j < nvalid ? s[j] * p.scale_log2 : kNegInf;
-                mx = fmaxf(mx, s[j]);
+            // prefetch: next tile's query (new sequence) and partial scores
+            nxt.next();
+            if (i + 1 < n_tiles) {
+                if (nxt.t == 0 && !load_q(nxt.w.b, q_seg++)) break;
+                if (!fetch_s(i + 1, s_nxt)) break;
             }
+
+            if (nvalid < 32) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j >= nvalid) s[j] = kNegInf;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int j = 1; j < 32; ++j) mx = fmaxf(mx, s[j]);
+            // row max across the two halves (double-buffered by tile parity)
+            float *rb = red + (i & 1) * 256;
+            rb[h * 128 + row] = mx;
+            mbar_arrive(&bars->red_bar);
+            if (!all(mbar_wait(&bars->red_bar, (uint32_t)(i & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                break;
+            mx = fmaxf(mx, rb[(h ^ 1) * 128 + row]);
+
+            // online softmax (log2 domain), lazy rescale -- same decision in
+            // both halves and both CTAs (same scores)
             bool rescale = false;
             float alpha = 1.f;
             if (first) {
                 m_run = mx;
                 l_run = 0.f;
             } else if (mx > m_run + kRescaleThreshold) {
-                alpha = exp2f(m_run - mx);
+                alpha = exp2_approx(m_run - mx);
                 m_run = mx;
                 l_run *= alpha;
                 rescale = true;
             }
-            float sum = 0.f;
+            float2 sum2 = make_float2(0.f, 0.f);
+            const float2 m2 = make_float2(-m_run, -m_run);
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                s[j] = exp2f(s[j] - m_run);
-                sum += s[j];
+            for (int j = 0; j < 32; j += 2) {
+                const float2 d = __fadd2_rn(make_float2(s[j], s[j + 1]), m2);
+                s[j] = exp2_approx(d.x);
+                s[j + 1] = exp2_approx(d.y);
+                sum2 = __fadd2_rn(sum2, make_float2(s[j], s[j + 1]));
             }
-            l_run += sum;
+            l_run += sum2.x + sum2.y;
 
             // P and O may be touched once the previous P V has completed
             if (i >= 1 && !all(mbar_wait(&bars->pv_done, (uint32_t)((i - 1) & 1),
                                          p.timeout_ns, p.err, abort_flag)))
                 break;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t hi[4], lo[4];
+            for (int c = 0; c < 4; ++c) {          // 8 tokens per 16-byte chunk
+                uint32_t hi_w[4], lo_w[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const float a = s[8 * c + 2 * k], b = s[8 * c + 2 * k + 1];
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-                    const float2 hf = __bfloat1622float2(h);
-                    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
-                    hi[k] = *reinterpret_cast<const uint32_t *>(&h);
-                    lo[k] = *reinterpret_cast<const uint32_t *>(&l);
+                    const float a = s[8 * c + 2 * k], bb = s[8 * c + 2 * k + 1];
+                    hi_w[k] = pack_bf16x2(a, bb);
+                    const float2 r = __fadd2_rn(
+                        make_float2(a, bb),
+                        make_float2(-__uint_as_float(hi_w[k] << 16),
+                                    -__uint_as_float(hi_w[k] & 0xFFFF0000u)));
+                    lo_w[k] = pack_bf16x2(r.x, r.y);
                 }
-                const int off = (c ^ (row & 7)) * 16;
-                *reinterpret_cast<uint4 *>(prow + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                const int off = ((4 * h + c) ^ (row & 7)) * 16;
+                *reinterpret_cast<uint4 *>(prow + off) =
+                    make_uint4(hi_w[0], hi_w[1], hi_w[2], hi_w[3]);
                 *reinterpret_cast<uint4 *>(prow + kPBytes + off) =
-                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    make_uint4(lo_w[0], lo_w[1], lo_w[2], lo_w[3]);
             }
             tc_fence_after();
             if (__any_sync(0xffffffffu, rescale)) {   // rows without a new max use alpha = 1
-                float o[64];
+                float o[32];
 #pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
-                    tmem_ld64(trow + kTmemO + 64 * ch, o);
+                    tmem_ld32(trow + kTmemO + 128 * h + 32 * ch, o);
+                    uint32_t r[32];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) o[j] *= alpha;
-                    tmem_st64(trow + kTmemO + 64 * ch, o);
+                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(o[j] * alpha);
+                    tmem_st32(trow + kTmemO + 128 * h + 32 * ch, r);
                 }
             }
             fence_proxy_async_smem();
@@ -394,24 +483,32 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_arrive(&bars->p_full);
 
             if (last) {
+                float *sb = red + 512 + (n_seg & 1) * 256;
+                sb[h * 128 + row] = l_run;
+                mbar_arrive(&bars->sum_bar);
+                if (!all(mbar_wait(&bars->sum_bar, (uint32_t)(n_seg & 1), p.timeout_ns, p.err,
+                                   abort_flag)))
+                    break;
+                const float l_tot = l_run + sb[(h ^ 1) * 128 + row];
+                ++n_seg;
                 if (!all(mbar_wait(&bars->pv_done, (uint32_t)(i & 1), p.timeout_ns, p.err,
                                    abort_flag)))
                     break;
                 tc_fence_after();
                 const long long slot = (long long)b + cluster;
-                float *dst = p.ws_o + ((size_t)slot * kMlaH + row) * kMlaDc + col0;
-                const float inv = 1.f / l_run;
-                float o[64];
+                float *dst = p.ws_o + ((size_t)slot * kMlaH + row) * kMlaDc + col0 + 128 * h;
+                const float inv = 1.f / l_tot;
+                float o[32];
 #pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
-                    tmem_ld64(trow + kTmemO + 64 * ch, o);
+                    tmem_ld32(trow + kTmemO + 128 * h + 32 * ch, o);
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4)
-                        *reinterpret_cast<float4 *>(dst + 64 * ch + j) =
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(dst + 32 * ch + j) =
                             make_float4(o[j] * inv, o[j + 1] * inv, o[j + 2] * inv,
                                         o[j + 3] * inv);
                 }
-                if (rank == 0) p.ws_lse[slot * kMlaH + row] = m_run + log2f(l_run);
+                if (rank == 0 && h == 0) p.ws_lse[slot * kMlaH + row] = m_run + log2f(l_tot);
                 tc_fence_before();
                 mbar_arrive(&bars->o_free);
             }
@@ -508,7 +605,8 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
                      const int32_t *seq_lens, const int32_t *block_table, void *out, int B,
                      int H, float scale, cudaStream_t stream, int max_blocks, int num_blocks,
                      int num_sms, int forced_ctas, unsigned *err,
-                     const WorkspaceFn &workspace) {
+                     const WorkspaceFn &workspace, cudaEvent_t ev_start,
+                     cudaEvent_t ev_stop) {
     if (H != kMlaH) return ATTN_ERR_UNSUPPORTED;
     if ((long long)num_blocks * 64 > (1ll << 31) - 64 || (long long)B * kMlaH > (1ll << 31))
         return ATTN_ERR_ARG;
@@ -530,13 +628,13 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     if (rc) return rc;
     unsigned char *w = static_cast<unsigned char *>(ws);
 
-    CUtensorMap tq, tr, tc;
-    if (!make_map(&tq, q_latent, kMlaDc, (uint64_t)B * kMlaH, kMlaDc * 2, 128) ||
-        !make_map(&tr, q_rope, kMlaDr, (uint64_t)B * kMlaH, kMlaDr * 2, 128) ||
-        !make_map(&tc, latent_cache, kMlaWidth, (uint64_t)num_blocks * 64, kMlaWidth * 2, 64))
+    CUtensorMap tc;
+    if (!make_map(&tc, latent_cache, kMlaWidth, (uint64_t)num_blocks * 64, kMlaWidth * 2, 64))
         return ATTN_ERR_CUDA;
 
     MlaParams mp{};
+    mp.q_lat = static_cast<const __nv_bfloat16 *>(q_latent);
+    mp.q_rope = static_cast<const __nv_bfloat16 *>(q_rope);
     mp.seq_lens = seq_lens;
     mp.block_table = block_table;
     mp.ws_o = reinterpret_cast<float *>(w);
@@ -562,8 +660,10 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mla_decode_kernel, tq, tr, tc, mp) != cudaSuccess)
+    if (ev_start) cudaEventRecord(ev_start, stream);
+    if (cudaLaunchKernelEx(&cfg, mla_decode_kernel, tc, mp) != cudaSuccess)
         return ATTN_ERR_CUDA;
+    if (ev_stop) cudaEventRecord(ev_stop, stream);
 
     CombineParams cp{};
     cp.seq_lens = seq_lens;

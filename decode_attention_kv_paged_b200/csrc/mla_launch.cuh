@@ -16,6 +16,7 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
                      const int32_t *seq_lens, const int32_t *block_table, void *out,
                      int B, int H, float scale, cudaStream_t stream, int max_blocks,
                      int num_blocks, int num_sms, int forced_ctas, unsigned *err,
-                     const WorkspaceFn &workspace);
+                     const WorkspaceFn &workspace, cudaEvent_t ev_start = nullptr,
+                     cudaEvent_t ev_stop = nullptr);
 
 }  // namespace attn

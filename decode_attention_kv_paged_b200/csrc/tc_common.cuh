@@ -140,6 +140,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x with the hardware approximation (MUFU); flushes denormal results.
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Two fp32 -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Round an fp32 (finite) to the nearest bf16, ties to even, with integer
+// operations only; returns the 16-bit pattern.
+__device__ __forceinline__ uint32_t bf16_rne_bits(float x) {
+    const uint32_t u = __float_as_uint(x);
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+}
+
+// Split x into bf16 hi + lo (hi = RNE(x), lo = RNE(x - hi)); both returned as
+// 16-bit patterns.  hi + lo carries ~16 significant bits of x.
+__device__ __forceinline__ void bf16_split(float x, uint32_t &hi, uint32_t &lo) {
+    hi = bf16_rne_bits(x);
+    lo = bf16_rne_bits(x - __uint_as_float(hi << 16));
+}
+
 // ------------------------------------------------------------ UMMA (MMA)
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile.
 // start: byte address in shared memory; lbo/sbo: leading/stride byte offsets.
@@ -258,16 +286,44 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
                                                   unsigned long long timeout_ns,
                                                   unsigned *err, volatile int *abort) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
-    while (true) {
+    unsigned long long t0 = 0;
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if (abort && *abort) return false;
-        if (global_timer_ns() - t0 > timeout_ns) {
-            raise_error(err, kErrTimeout);
-            if (abort) *abort = 1;
-            return false;
+        if ((it & 63u) == 0) {
+            const unsigned long long now = global_timer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > timeout_ns) {
+                raise_error(err, kErrTimeout);
+                if (abort) *abort = 1;
+                return false;
+            }
         }
     }
+}
+
+// Arrive on a barrier of another CTA of the cluster and raise its expected
+// transaction count by `bytes` (paired with a bulk copy into that CTA).
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar,
+                                                             uint32_t bytes) {
+    asm volatile(
+        "mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+            remote_bar),
+        "r"(bytes)
+        : "memory");
+}
+
+// Bulk copy from this CTA's shared memory into another CTA's shared memory
+// (cluster), completion counted in bytes on that CTA's barrier.  16-byte
+// aligned addresses, size a multiple of 16.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const void *src,
+                                                  uint32_t bytes, uint32_t remote_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes "
+        "[%0], [%1], %2, [%3];" ::"r"(dst_cluster),
+        "r"(smem_u32(src)), "r"(bytes), "r"(remote_bar)
+        : "memory");
 }
 
 // Named barrier among `count` threads (multiple of 32), id 1..15.
