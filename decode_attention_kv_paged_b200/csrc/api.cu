@@ -9,6 +9,7 @@
 
 #include "attn_decode.h"
 #include "gqa_launch.cuh"
+#include "gqa_tc.cuh"
 #include "kv_append.cuh"
 #include "mla_launch.cuh"
 
@@ -84,6 +85,16 @@ static bool aligned16(const void *p) {
 
 static bool valid_head_dim(int d) {
     return d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
+}
+
+// Whether attn_decode_gqa runs the tensor-core kernel for this problem: by
+// default for groups of kTcMinGroup heads or more (there every K/V element
+// feeds enough heads to make the products dense), or when forced.
+static bool use_tc_path(int G, int d, int dtype) {
+    const bool ok = gqa_tc_supported(d, dtype == ATTN_BF16, G);
+    if (tl_gqa_path == 0) return false;
+    if (tl_gqa_path == 1) return ok;
+    return ok && G >= kTcMinGroup;
 }
 
 // Query heads per CTA for a group of G: the largest instantiated divisor.
@@ -194,9 +205,11 @@ int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype, int *num_
     DeviceState *st;
     int rc = device_state(&st);
     if (rc) return rc;
+    const int G = H_q / H_kv;
+    const bool tc = use_tc_path(G, d, dtype);
     if (num_ctas) *num_ctas = tl_num_ctas > 0 ? tl_num_ctas : st->num_sms;
-    if (heads) *heads = heads_per_cta(H_q / H_kv);
-    if (path) *path = 0;
+    if (heads) *heads = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
+    if (path) *path = tc ? 1 : 0;
     return ATTN_OK;
 }
 
@@ -221,10 +234,14 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     cudaStream_t s = (cudaStream_t)stream;
 
     const int G = H_q / H_kv;
-    const int HC = heads_per_cta(G);
+    const bool tc = use_tc_path(G, d, dtype);
+    const int HC = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
     const int n_hc = G / HC;
-    const int P = tl_num_ctas > 0 ? tl_num_ctas : st->num_sms;
     const long long units_total = (long long)B * H_kv * n_hc;
+    // No more CTAs than the work could possibly fill (units x table width).
+    const long long work_bound = units_total * max_blocks_per_seq;
+    const int P = tl_num_ctas > 0 ? tl_num_ctas
+                                  : (int)(work_bound < st->num_sms ? work_bound : st->num_sms);
     if (units_total > (1ll << 30)) return ATTN_ERR_ARG;
     const long long slots = units_total + P;
 
@@ -260,6 +277,10 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
 
     const int bf16 = dtype == ATTN_BF16;
     cudaError_t e;
+    if (tc) {
+        e = launch_gqa_tc(L, d, HC);
+        return cuda_status(e);
+    }
     switch (d) {
         case 16: e = launch_gqa_d16(HC, bf16, L); break;
         case 32: e = launch_gqa_d32(HC, bf16, L); break;

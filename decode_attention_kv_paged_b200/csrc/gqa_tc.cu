@@ -1,0 +1,507 @@
+// gqa_tc.cu -- decode attention for large query groups (MQA / wide GQA) on
+// the tcgen05 tensor cores.
+//
+// Computes the same as the CUDA-core kernel (attention-head article, §1
+// Attention equation, §2 group rule), for one KV head and up to 64 of the
+// query heads that share it at a time:
+//     S = Q K^T   (heads x 64 tokens)      O += P V   (heads x d)
+// With a large group every K/V element feeds many heads, so the two products
+// are real dense contractions and belong on the tensor cores; the CUDA-core
+// path would need ~G flops per loaded byte.
+//
+// Design (B200):
+//   * One CTA per SM over the split-KV partition (plan.cuh).  Warp 0 issues
+//     2-D TMA loads (128-byte swizzle) of each 64-token K and V tile of the
+//     paged cache into a multi-stage ring and of the unit's query rows; one
+//     thread of warp 1 issues tcgen05 MMAs as their inputs become ready;
+//     warps 4-7 run the softmax and the epilogue.
+//   * S: M = 64 query rows (heads, zero-padded), N = 64 tokens, K = d, both
+//     operands in shared memory, fp32 accumulator in TMEM (double-buffered).
+//     The M = 64 accumulator puts row r in TMEM lane (r % 16) + 32 (r / 16),
+//     so each head row is read by one thread: the softmax needs no
+//     cross-thread reductions.  The running max is only raised when it grows
+//     by more than 2^8 (lazy rescale, exact either way).
+//   * P is split into bf16 P_hi + P_lo (the rounding remainder) so the
+//     weights keep ~16 significant bits; O += P_hi V + P_lo V with V read
+//     MN-major from the same swizzled tile; O stays in TMEM for the segment.
+//   * Every wait is bounded; TMEM is always freed.
+#include <mutex>
+#include <vector>
+
+#include "attn_decode.h"
+#include "gqa_decode.cuh"
+#include "gqa_tc.cuh"
+#include "tc_common.cuh"
+
+namespace attn {
+
+constexpr int kTcM = 64;                    // MMA M: query rows per CTA pass
+constexpr int kTcThreads = 256;
+constexpr int kTcBox = 64 * 128;            // [64 rows][64 cols] bf16, swizzled
+constexpr int kTcPBytes = kTcM * 128;       // one P half: [64 heads][64 tokens]
+constexpr float kTcRescaleThreshold = 8.0f;
+
+template <int D>
+struct TcCfg {
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kQBytes = kBoxes * kTcBox;
+    static constexpr int kStageBytes = 2 * kBoxes * kTcBox;     // K then V
+    static constexpr int kFixed = kQBytes + 2 * kTcPBytes + 1024 /*bars*/ + 1024 /*align*/;
+    static constexpr int kStagesRaw = (227 * 1024 - kFixed) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffC = kOffQ + kQBytes;
+    static constexpr int kOffP = kOffC + kStages * kStageBytes;
+    static constexpr int kOffBar = kOffP + 2 * kTcPBytes;
+    static constexpr int kSmem = kOffBar + 1024 + 1024;
+    static constexpr uint32_t kTmemO = 0, kTmemS = D;            // S buffers at D, D + 64
+    static constexpr uint32_t kTmemCols = D + 128 <= 256 ? 256 : 512;
+    static_assert(kStages >= 2, "at least two stages");
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+struct TcBars {
+    uint64_t q_full, q_empty;
+    uint64_t c_full[6], c_empty[6];
+    uint64_t s_full[2], s_free[2];
+    uint64_t p_full, pv_done, o_free, mma_final;
+    uint32_t tmem_base;
+    int abort;
+    PlanScratch plan;
+};
+static_assert(sizeof(TcBars) <= 1024, "barrier block");
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const GqaParams p, int HC) {
+    using C = TcCfg<D>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    unsigned char *sQ = smem + C::kOffQ;
+    unsigned char *sC = smem + C::kOffC;
+    unsigned char *sP = smem + C::kOffP;
+    TcBars *bars = reinterpret_cast<TcBars *>(smem + C::kOffBar);
+    volatile int *abort_flag = &bars->abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int units = p.H_kv * p.n_hc;
+    PlanArgs pa{p.seq_lens, p.B, units, p.window, p.max_blocks, p.num_ctas};
+    plan_locate(pa, blockIdx.x, &bars->plan, blockIdx.x == 0 ? p.ws_prefix : nullptr, p.err);
+    const long long W = bars->plan.total;
+    const int P = working_ctas(W, p.num_ctas);
+    if ((int)blockIdx.x >= P) return;
+    const long long lo = cta_bound(blockIdx.x, W, P);
+    const long long hi = cta_bound(blockIdx.x + 1, W, P);
+    const int first_seq = bars->plan.seq;
+    const long long first_base = bars->plan.base;
+    const int n_tiles = (int)(hi - lo);
+
+    // Zero Q (rows beyond the group stay zero) and P (rows beyond the group
+    // are never written), then make the zeros visible to the tensor cores.
+    for (int i = tid; i < (C::kQBytes + 2 * kTcPBytes) / 16; i += kTcThreads) {
+        const int off = i * 16;
+        uint4 *dst = reinterpret_cast<uint4 *>(off < C::kQBytes ? sQ + off
+                                                                : sP + (off - C::kQBytes));
+        *dst = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    if (tid == 0) {
+        mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&bars->c_full[s], 1);
+            mbar_init(&bars->c_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->s_full[s], 1);
+            mbar_init(&bars->s_free[s], 128);
+        }
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->pv_done, 1);
+        mbar_init(&bars->o_free, 128);
+        mbar_init(&bars->mma_final, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(&bars->tmem_base, C::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ============================================================ TMA
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            tma_prefetch_map(&tm_k);
+            tma_prefetch_map(&tm_v);
+            TileCursor cur;
+            cur.init(pa, lo, hi, first_seq, first_base);
+            int tile = 0, seg = 0;
+            while (!cur.done()) {
+                const int kvh = cur.w.unit / p.n_hc, hc = cur.w.unit % p.n_hc;
+                if (cur.t == 0) {
+                    if (seg > 0 && !mbar_wait(&bars->q_empty, (uint32_t)((seg - 1) & 1),
+                                              p.timeout_ns, p.err, abort_flag))
+                        break;
+                    const int qrow = cur.w.b * p.H_q + kvh * p.group + hc * HC;
+                    mbar_arrive_expect_tx(&bars->q_full, C::kBoxes * HC * 128);
+                    for (int j = 0; j < C::kBoxes; ++j)
+                        tma_load_2d(sQ + j * kTcBox, &tm_q, 64 * j, qrow, &bars->q_full, pol);
+                    ++seg;
+                }
+                const int st = tile % C::kStages;
+                if (tile >= C::kStages &&
+                    !mbar_wait(&bars->c_empty[st], (uint32_t)(((tile - C::kStages) / C::kStages) & 1),
+                               p.timeout_ns, p.err, abort_flag))
+                    break;
+                int phys = p.block_table[(size_t)cur.w.b * p.max_blocks + cur.logical_block()];
+                if (phys < 0 || phys >= p.num_blocks) {
+                    raise_error(p.err, kErrBadBlock);
+                    phys = p.num_blocks;                 // wholly out of bounds: zero fill
+                }
+                const int row = (phys * p.H_kv + kvh) * 64;
+                unsigned char *dst = sC + st * C::kStageBytes;
+                mbar_arrive_expect_tx(&bars->c_full[st], C::kStageBytes);
+                for (int j = 0; j < C::kBoxes; ++j) {
+                    tma_load_2d(dst + j * kTcBox, &tm_k, 64 * j, row, &bars->c_full[st], pol);
+                    tma_load_2d(dst + (C::kBoxes + j) * kTcBox, &tm_v, 64 * j, row,
+                                &bars->c_full[st], pol);
+                }
+                cur.next();
+                ++tile;
+            }
+            for (int t = tile - C::kStages < 0 ? 0 : tile - C::kStages; t < tile; ++t)
+                mbar_wait(&bars->c_full[t % C::kStages], (uint32_t)((t / C::kStages) & 1),
+                          p.timeout_ns, p.err, nullptr);
+            if (seg > 0)
+                mbar_wait(&bars->q_full, (uint32_t)((seg - 1) & 1), p.timeout_ns, p.err, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ============================================================ MMA
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16(kTcM, 64, 0, 0);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, 0, 1);
+            const uint32_t q_base = smem_u32(sQ), c_base = smem_u32(sC), p_base = smem_u32(sP);
+            TileCursor cs, cv;
+            cs.init(pa, lo, hi, first_seq, first_base);
+            cv.init(pa, lo, hi, first_seq, first_base);
+            int next_s = 0, next_pv = 0, seg_s = 0, seg_v = 0;
+            unsigned long long idle_since = 0;
+            uint32_t idle_polls = 0;
+            while (next_pv < n_tiles) {
+                bool did = false;
+                if (next_s < n_tiles && next_s < next_pv + 2) {
+                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
+                    const int st = next_s % C::kStages, sb = next_s & 1;
+                    const bool ready =
+                        (!first || mbar_test(&bars->q_full, (uint32_t)(seg_s & 1))) &&
+                        mbar_test(&bars->c_full[st], (uint32_t)((next_s / C::kStages) & 1)) &&
+                        (next_s < 2 ||
+                         mbar_test(&bars->s_free[sb], (uint32_t)(((next_s - 2) >> 1) & 1)));
+                    if (ready) {
+                        tc_fence_after();
+                        const uint32_t kst = c_base + st * C::kStageBytes;
+                        for (int j = 0; j < C::kBoxes; ++j)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint64_t a =
+                                    umma_desc_sw128(q_base + j * kTcBox + k * 32, 16, 1024);
+                                const uint64_t b =
+                                    umma_desc_sw128(kst + j * kTcBox + k * 32, 16, 1024);
+                                umma_bf16(tmem + C::kTmemS + 64 * sb, a, b, idesc_s, (j | k) != 0);
+                            }
+                        umma_commit(&bars->s_full[sb]);
+                        if (last) umma_commit(&bars->q_empty);
+                        if (first) ++seg_s;
+                        cs.next();
+                        ++next_s;
+                        did = true;
+                    }
+                }
+                if (next_pv < next_s) {
+                    const bool first = cv.t == 0;
+                    const bool ready =
+                        mbar_test(&bars->p_full, (uint32_t)(next_pv & 1)) &&
+                        (!first || seg_v == 0 ||
+                         mbar_test(&bars->o_free, (uint32_t)((seg_v - 1) & 1)));
+                    if (ready) {
+                        tc_fence_after();
+                        const int st = next_pv % C::kStages;
+                        const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kTcBox;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t b = umma_desc_sw128(vst + k * 2048, kTcBox, 1024);
+                            const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
+                            const uint64_t a_lo =
+                                umma_desc_sw128(p_base + kTcPBytes + k * 32, 16, 1024);
+                            umma_bf16(tmem + C::kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
+                            umma_bf16(tmem + C::kTmemO, a_lo, b, idesc_pv, 1);
+                        }
+                        umma_commit(&bars->c_empty[st]);
+                        umma_commit(&bars->pv_done);
+                        if (first) ++seg_v;
+                        cv.next();
+                        ++next_pv;
+                        did = true;
+                    }
+                }
+                if (did) {
+                    idle_since = 0;
+                    idle_polls = 0;
+                } else if ((++idle_polls & 7u) == 0 && (__nanosleep(32), (idle_polls & 63u) == 0)) {
+                    const unsigned long long now = global_timer_ns();
+                    if (idle_since == 0) idle_since = now;
+                    if (*abort_flag) break;
+                    if (now - idle_since > p.timeout_ns) {
+                        raise_error(p.err, kErrTimeout);
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+            }
+            umma_commit(&bars->mma_final);
+            mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ================================================ softmax, epilogue
+        // M = 64 accumulator: row r lives in TMEM lane (r % 16) + 32 (r / 16);
+        // warp 4 + q owns rows 16q .. 16q + 15 in its lanes 0..15.
+        const int q4 = warp & 3;
+        const int row = 16 * q4 + lane;
+        const bool active = lane < 16 && row < HC;
+        const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
+        unsigned char *prow = sP + (row < kTcM ? row : 0) * 128;
+        auto all = [](bool v) { return __all_sync(0xffffffffu, v); };
+        TileCursor cur;
+        cur.init(pa, lo, hi, first_seq, first_base);
+        float m_run = -1e30f, l_run = 0.f;
+        int n_seg = 0;
+        for (int i = 0; i < n_tiles; ++i) {
+            const bool first = cur.t == 0, last = cur.t == cur.len - 1;
+            const int b = cur.w.b, T = cur.w.T;
+            const int lo_tok = (p.window > 0 && T > p.window) ? T - p.window : 0;
+            const int tok0 = cur.logical_block() * 64;
+            const int sb = i & 1;
+            if (!all(mbar_wait(&bars->s_full[sb], (uint32_t)((i >> 1) & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                break;
+            tc_fence_after();
+            float s[64];
+            tmem_ld64(trow + C::kTmemS + 64 * sb, s);
+            tc_fence_before();
+            mbar_arrive(&bars->s_free[sb]);
+
+            // scale to log2 units, mask keys outside [lo_tok, T)
+            const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+                const float2 v = __fmul2_rn(make_float2(s[j], s[j + 1]), sl2);
+                s[j] = v.x;
+                s[j + 1] = v.y;
+            }
+            if (tok0 < lo_tok || tok0 + 64 > T) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const int pos = tok0 + j;
+                    if (pos < lo_tok || pos >= T) s[j] = kNegInf;
+                }
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int j = 1; j < 64; ++j) mx = fmaxf(mx, s[j]);
+            bool rescale = false;
+            float alpha = 1.f;
+            if (first) {
+                m_run = mx;
+                l_run = 0.f;
+            } else if (mx > m_run + kTcRescaleThreshold) {
+                alpha = exp2_approx(m_run - mx);
+                m_run = mx;
+                l_run *= alpha;
+                rescale = true;
+            }
+            float2 sum2 = make_float2(0.f, 0.f);
+            const float2 m2 = make_float2(-m_run, -m_run);
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+                const float2 d = __fadd2_rn(make_float2(s[j], s[j + 1]), m2);
+                s[j] = exp2_approx(d.x);
+                s[j + 1] = exp2_approx(d.y);
+                sum2 = __fadd2_rn(sum2, make_float2(s[j], s[j + 1]));
+            }
+            l_run += sum2.x + sum2.y;
+
+            if (i >= 1 && !all(mbar_wait(&bars->pv_done, (uint32_t)((i - 1) & 1), p.timeout_ns,
+                                         p.err, abort_flag)))
+                break;
+            if (active) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t hi_w[4], lo_w[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float a = s[8 * c + 2 * k], bb = s[8 * c + 2 * k + 1];
+                        hi_w[k] = pack_bf16x2(a, bb);
+                        const float2 r = __fadd2_rn(
+                            make_float2(a, bb),
+                            make_float2(-__uint_as_float(hi_w[k] << 16),
+                                        -__uint_as_float(hi_w[k] & 0xFFFF0000u)));
+                        lo_w[k] = pack_bf16x2(r.x, r.y);
+                    }
+                    const int off = (c ^ (row & 7)) * 16;
+                    *reinterpret_cast<uint4 *>(prow + off) =
+                        make_uint4(hi_w[0], hi_w[1], hi_w[2], hi_w[3]);
+                    *reinterpret_cast<uint4 *>(prow + kTcPBytes + off) =
+                        make_uint4(lo_w[0], lo_w[1], lo_w[2], lo_w[3]);
+                }
+            }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, active && rescale)) {
+                const float a = (active && rescale) ? alpha : 1.f;
+                float o[32];
+#pragma unroll 1
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    tmem_ld32(trow + C::kTmemO + 32 * ch, o);
+                    uint32_t r[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(o[j] * a);
+                    tmem_st32(trow + C::kTmemO + 32 * ch, r);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+
+            if (last) {
+                if (!all(mbar_wait(&bars->pv_done, (uint32_t)(i & 1), p.timeout_ns, p.err,
+                                   abort_flag)))
+                    break;
+                tc_fence_after();
+                const long long slot = (long long)b * units + cur.w.unit + blockIdx.x;
+                const float inv = 1.f / l_run;
+                float *dst = p.ws_o + ((size_t)slot * HC + (active ? row : 0)) * D;
+                float o[32];
+#pragma unroll 1
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    tmem_ld32(trow + C::kTmemO + 32 * ch, o);
+                    if (active) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4 *>(dst + 32 * ch + j) =
+                                make_float4(o[j] * inv, o[j + 1] * inv, o[j + 2] * inv,
+                                            o[j + 3] * inv);
+                    }
+                }
+                if (active) p.ws_lse[slot * HC + row] = m_run + log2f(l_run);
+                tc_fence_before();
+                mbar_arrive(&bars->o_free);
+                ++n_seg;
+            }
+            cur.next();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// -------------------------------------------------------------- host side
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tc_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+bool tc_make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                 uint32_t box_rows) {
+    EncodeTiledFn fn = tc_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc(const GqaLaunch &L, int HC) {
+    using C = TcCfg<D>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gqa_tc_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const GqaParams &kp = L.kp;
+    CUtensorMap tq, tk, tv;
+    if (!tc_make_map(&tq, kp.q, D, (uint64_t)kp.B * kp.H_q, (uint32_t)HC) ||
+        !tc_make_map(&tk, kp.k_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64) ||
+        !tc_make_map(&tv, kp.v_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64))
+        return cudaErrorInvalidValue;
+    if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
+    gqa_tc_kernel<D><<<kp.num_ctas, kTcThreads, C::kSmem, L.stream>>>(tq, tk, tv, kp, HC);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
+
+    CombineParams cp = L.cp;
+    cp.D = D;
+    cp.HC = HC;
+    cp.blocks_per_unit = (HC * D / 4 + kCombineThreads - 1) / kCombineThreads;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((long long)L.units_total * cp.blocks_per_unit));
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = L.ev_stop ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel<__nv_bfloat16>, cp);
+}
+
+}  // namespace
+
+bool gqa_tc_supported(int d, int dtype_bf16, int G) {
+    return dtype_bf16 && (d == 64 || d == 128 || d == 256) && (G <= kTcM || G % kTcM == 0);
+}
+
+int gqa_tc_heads_per_cta(int G) { return G <= kTcM ? G : kTcM; }
+
+cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC) {
+    switch (d) {
+        case 64: return launch_tc<64>(L, HC);
+        case 128: return launch_tc<128>(L, HC);
+        case 256: return launch_tc<256>(L, HC);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace attn

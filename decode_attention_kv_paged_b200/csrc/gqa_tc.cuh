@@ -1,0 +1,17 @@
+// gqa_tc.cuh -- host entry of the tensor-core (tcgen05) GQA/MQA decode path.
+#pragma once
+
+#include "gqa_launch.cuh"
+
+namespace attn {
+
+// The tensor-core kernel handles bf16, d in {64, 128, 256}, and groups of up
+// to 64 query heads per pass (larger groups in multiples of 64).
+bool gqa_tc_supported(int d, int dtype_bf16, int G);
+int gqa_tc_heads_per_cta(int G);
+// Group size from which the tensor-core path is the default.
+constexpr int kTcMinGroup = 8;
+
+cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC);
+
+}  // namespace attn

@@ -294,3 +294,37 @@ def test_ragged_qwen_shape_sampled(lib, cfg):
         assert_parity(got[b], ref[b], torch.bfloat16, f"{cfg.name} b={b}")
     # every output row is a convex combination of V rows: finite and bounded
     assert np.isfinite(got).all()
+
+
+# ------------------------------------------- both kernels, forced per case
+PATH_CASES = [
+    # (H_q, H_kv, d, lens, window)
+    (8, 8, 128, [300, 65], 0),            # MHA
+    (8, 4, 64, [129, 1000], 0),           # G=2
+    (16, 4, 128, [700, 64, 1], 0),        # G=4
+    (24, 4, 256, [999, 4097], 700),       # G=6 + window
+    (32, 4, 128, [2000, 130], 0),         # G=8
+    (32, 1, 128, [1500, 63, 64], 0),      # MQA G=32
+    (64, 1, 64, [800, 257], 100),         # G=64 + window
+    (128, 1, 128, [520, 77], 0),          # G=128: two 64-head passes
+]
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["cuda_core", "tcgen05"])
+@pytest.mark.parametrize("H_q,H_kv,d,lens,window", PATH_CASES,
+                         ids=[f"q{c[0]}_kv{c[1]}_d{c[2]}_w{c[4]}" for c in PATH_CASES])
+def test_each_kernel_matches_oracle(lib, path, H_q, H_kv, d, lens, window):
+    """The CUDA-core and the tensor-core (tcgen05) kernels each reproduce the
+    oracle for every group size, whichever one the library would pick."""
+    cfg = GQAConfig("paths", B=len(lens), H_q=H_q, H_kv=H_kv, d=d, seq_lens=lens,
+                    window=window, seed=4000 + H_q + d)
+    inp = make_gqa_inputs(cfg)
+    ref = full_oracle(inp)
+    lib.set_gqa_path(path)
+    try:
+        n, hc, used = lib.gqa_config(len(lens), H_q, H_kv, d)
+        assert used == path
+        got = run_gpu(lib, inp).float().cpu().numpy()
+    finally:
+        lib.set_gqa_path(-1)
+    assert_parity(got, ref, torch.bfloat16, f"path {path}")
