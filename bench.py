@@ -34,13 +34,20 @@ import workloads as W  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+# Sources of each main kernel: a committed DRAM-traffic figure is used only
+# while the hash of these files matches the one recorded with it.
 KERNEL_SOURCES = {
-    "gqa": ["decode_attention_kv_paged_b200/csrc/gqa_decode.cuh",
-            "decode_attention_kv_paged_b200/csrc/plan.cuh",
-            "decode_attention_kv_paged_b200/csrc/common.cuh"],
-    "mla": ["decode_attention_kv_paged_b200/csrc/mla_decode.cu",
-            "decode_attention_kv_paged_b200/csrc/plan.cuh",
-            "decode_attention_kv_paged_b200/csrc/common.cuh"],
+    "gqa_split_kernel": ["decode_attention_kv_paged_b200/csrc/gqa_decode.cuh",
+                         "decode_attention_kv_paged_b200/csrc/plan.cuh",
+                         "decode_attention_kv_paged_b200/csrc/common.cuh"],
+    "gqa_tc_kernel": ["decode_attention_kv_paged_b200/csrc/gqa_tc.cu",
+                      "decode_attention_kv_paged_b200/csrc/tc_common.cuh",
+                      "decode_attention_kv_paged_b200/csrc/plan.cuh",
+                      "decode_attention_kv_paged_b200/csrc/common.cuh"],
+    "mla_decode_kernel": ["decode_attention_kv_paged_b200/csrc/mla_decode.cu",
+                          "decode_attention_kv_paged_b200/csrc/tc_common.cuh",
+                          "decode_attention_kv_paged_b200/csrc/plan.cuh",
+                          "decode_attention_kv_paged_b200/csrc/common.cuh"],
 }
 
 WORKLOAD_ALIASES = {
@@ -90,15 +97,17 @@ def kernel_hash(kind):
     return h.hexdigest()[:16]
 
 
-def traffic_for(kind, wl_name):
-    """dram bytes per launch from the committed ncu summary, if the kernel
-    source is unchanged since it was taken; else None."""
+def traffic_for(kernel, wl_name):
+    """dram bytes per launch of `kernel` on `wl_name` from the committed ncu
+    summary, if the kernel's sources are unchanged since it was taken; else
+    None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         j = json.load(f)
     e = j.get(wl_name)
-    if not e or e.get("kernel_hash") != kernel_hash(kind):
+    if (not e or e.get("kernel") != kernel
+            or e.get("kernel_hash") != kernel_hash(kernel)):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -189,12 +198,26 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank scalar over all ranks (timing only; NCCL on GPUs,
+    gloo on CPU)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(cfg_seed, rank):
+    """Each rank draws its own batch (weak scaling: per-GPU work is fixed)."""
+    return cfg_seed + 1000 * rank
+
+
+def whole_job_tokens_per_s(world, batch, steps, ms_max):
+    """Decode tokens/s of the whole job: all ranks' sequences over the
+    slowest rank's time."""
+    return world * batch * steps / (ms_max / 1e3)
 
 
 # --------------------------------------------------------------- helpers
@@ -243,7 +266,7 @@ def run_native(args, rank, world, local):  # noqa: C901
     cfg = workload(args.workload)
     is_mla = isinstance(cfg, W.MLAConfig)
     dev = torch.device("cuda", local)
-    seed = cfg.seed + 1000 * rank
+    seed = rank_seed(cfg.seed, rank)
     if is_mla:
         base = W.make_mla_inputs(cfg, device=dev, seed=seed)
         kv_bytes, alg_bytes = algorithmic_bytes_mla(base)
@@ -302,11 +325,15 @@ def run_native(args, rank, world, local):  # noqa: C901
     kern_avg = max_over_ranks(sum(kern_ms) / K, world)
 
     B = cfg.B
-    value = world * B * K / (ms_max / 1e3)            # tokens/s, whole job
+    value = whole_job_tokens_per_s(world, B, K, ms_max)
     kv_gbs = world * kv_bytes * K / (ms_max / 1e3) / 1e9
     pk, pk_kind = peaks()
     wl_name = cfg.name
-    kind = "mla" if is_mla else "gqa"
+    if is_mla:
+        kernel = "mla_decode_kernel"
+    else:
+        _, _, path = attn.gqa_config(cfg.B, cfg.H_q, cfg.H_kv, cfg.d, cfg.dtype)
+        kernel = "gqa_tc_kernel" if path == 1 else "gqa_split_kernel"
     if is_mla:
         flops = mla_flops(base)
         t_hbm = alg_bytes / (pk["hbm_gbs"] * 1e9)
@@ -325,10 +352,10 @@ def run_native(args, rank, world, local):  # noqa: C901
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = pk_kind
-    roof["kernel"] = "mla_decode_kernel" if is_mla else "gqa_split_kernel"
+    roof["kernel"] = kernel
     roof["kernel_ms_avg"] = kern_avg
     roof["algorithmic_bytes_per_launch"] = alg_bytes
-    roof["traffic"] = traffic_for(kind, wl_name)
+    roof["traffic"] = traffic_for(kernel, wl_name)
 
     line = {
         "metric": "decode tokens/s and KV-cache read GB/s (% of B200 HBM peak), 1 GPU",
