@@ -42,24 +42,26 @@ constexpr int pow2_floor(int x) {
     return p;
 }
 
-// Warps per CTA.  Sixteen (four per SM sub-partition, so one warp's
-// dependency chain -- shuffle reductions, exp2, shared-memory round trips --
-// overlaps three others) whenever the per-thread state fits the 128
-// registers that allows; otherwise eight (up to 255 registers each).
-constexpr int gqa_warps(int D, int HC) {
-    return (D >= 64 && HC <= 4 && false) ? 16 : 8;
-}
-
-// Elements of the head dimension each lane owns: the queries plus the
-// accumulators take 2*HC*EPL fp32 registers (at most 64 with 16 warps, 128
-// with 8), a warp covers no more rows per instruction than the 64/NW tokens
-// it owns, and no fewer than one row per instruction.
-constexpr int gqa_epl(int D, int HC, int NW) {
-    int e = pow2_floor((NW == 16 ? 32 : 64) / HC);
-    const int tpw = 64 / NW;
+// Elements of the head dimension each lane owns.  The queries plus the
+// accumulators take 2*HC*EPL fp32 registers (at most 128), a warp covers no
+// more rows per instruction than the `tpw` tokens it owns, a row is split
+// over 4 to 32 lanes.
+constexpr int gqa_epl(int D, int HC, int tpw) {
+    int e = pow2_floor(64 / HC);
     if (e > D * tpw / 32) e = D * tpw / 32;
+    if (e > D / 4) e = D / 4;
     if (e < D / 32) e = D / 32;
     return e;
+}
+
+// Row-iterations whose partial dot products are reduced together: the
+// largest divisor of `iters` with at most 16 (iteration, head) sums.
+constexpr int gqa_chunk(int iters, int HC) {
+    int c = 16 / HC;
+    if (c < 1) c = 1;
+    if (c > iters) c = iters;
+    while (iters % c != 0) --c;
+    return c;
 }
 
 struct GqaParams {
@@ -81,20 +83,43 @@ struct GqaParams {
 template <int D, int HC, typename T>
 struct GqaCfg {
     static constexpr int kS = (int)sizeof(T);
-    static constexpr int kNW = gqa_warps(D, HC);
-    static constexpr int kThreads = kNW * 32;
-    static constexpr int kTPW = kBlockSize / kNW;                 // tokens/warp
-    static constexpr int kEPL = gqa_epl(D, HC, kNW);
+    // Warp specialisation: warpgroup 0 is the producer (its warp 0 streams
+    // the tiles; the other three exit at once), warpgroups 1 and 2 are the
+    // kNW compute warps.  setmaxnreg moves the producer group's registers to
+    // the compute groups; the shares add up to the launch's 384 x 168.
+    static constexpr int kNW = 8;                                 // compute warps
+    static constexpr int kThreads = 32 * (4 + kNW);
+    static constexpr int kProducerRegs = 40;
+    static constexpr int kConsumerRegs = 232;
+    static constexpr int kLaunchRegs = 168;
+    static_assert(4 * 32 * kProducerRegs + kNW * 32 * kConsumerRegs <=
+                      kThreads * kLaunchRegs, "register split exceeds the launch");
+    // A staged tile is a whole 64-token block, or half of one when a block's
+    // K and V would take more than 32 KiB (d = 256 bf16, fp32 d = 128).
+    static constexpr int kTileTok =
+        (kBlockSize * D * kS * 2 > 32768) ? 32768 / (2 * D * kS) : kBlockSize;
+    static constexpr int kSub = kBlockSize / kTileTok;            // tiles/block
+    // The warps form kNG groups; group g consumes the CTA's tiles n with
+    // n % kNG == g, so kNG tiles are in work at once and each warp owns
+    // kTPW rows of its group's tiles.
+    static constexpr int kNG = 2;
+    static constexpr int kWPG = kNW / kNG;                        // warps/group
+    static constexpr int kTPW = kTileTok / kWPG;                  // tokens/warp
+    static constexpr int kEPL = gqa_epl(D, HC, kTPW);
     static constexpr int kLE = (16 / kS < kEPL) ? 16 / kS : kEPL; // per load
     static constexpr int kCPL = kEPL / kLE;                       // loads/lane/row
     static constexpr int kLPR = D / kEPL;                         // lanes per row
     static constexpr int kRPW = 32 / kLPR;                        // rows per instr.
     static constexpr int kIters = kTPW / kRPW;
+    // Score rows are reduced kChunk row-iterations at a time (bounds the
+    // live partial sums to 16 fp32x2 registers).
+    static constexpr int kChunk = gqa_chunk(kIters, HC);
+    static constexpr int kChunks = (kIters + kChunk - 1) / kChunk;
     static constexpr int kCPR = D / kLE;                          // chunks per row
     static constexpr int kHPP = 32 / kTPW;                        // heads/pass
     static constexpr int kPasses = (HC + kHPP - 1) / kHPP;        // softmax passes
     static constexpr int kHCP = (HC == 3) ? 4 : (HC > 4 ? 8 : HC);// padded heads
-    static constexpr int kTileBytes = kBlockSize * D * kS;
+    static constexpr int kTileBytes = kTileTok * D * kS;
     static constexpr int kStageBytes = 2 * kTileBytes;
     // shared memory carve-up (bytes)
     static constexpr int kScoreBytes = kNW * kTPW * kHCP * 4;
@@ -104,12 +129,13 @@ struct GqaCfg {
     static constexpr int kOther =
         kScoreBytes + kMergeOBytes + kMergeMLBytes + kMiscBytes;
     static constexpr int kStagesRaw = (kSmemBudget - kOther) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static_assert(kTPW * kHPP == 32, "softmax lane map");
     static constexpr int kSmemBytes = kStages * kStageBytes + kOther;
-    static_assert(kStages >= 2, "not enough shared memory for two stages");
+    static_assert(kStages >= kNG + 2, "not enough shared memory for the ring");
     static_assert(kLPR >= 4 && kLPR <= 32 && (kLPR & (kLPR - 1)) == 0, "LPR");
     static_assert(kIters >= 1 && kIters * kRPW == kTPW, "rows per warp");
+    static_assert(kChunks * kChunk == kIters, "score chunks");
     static_assert(kTileBytes % 16 == 0, "bulk copy size");
 };
 
@@ -272,50 +298,94 @@ struct Producer {
     }
 };
 
-// Issue the bulk copies of one tile (physical block `phys`, KV head of the
-// cursor's unit) into a stage.  Called by one lane.
-template <int D, typename T, int kTileBytes>
+// Issue the bulk copies of one tile -- tile `sub` (kTileTok tokens) of the
+// physical block `phys`, KV head of the cursor's unit -- into a stage.
+// Called by one lane.
+template <int D, typename T, int kTileTok>
 __device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor &cur,
-                                          int phys, unsigned char *dst, uint64_t *full,
-                                          uint64_t pol) {
+                                          int phys, int sub, unsigned char *dst,
+                                          uint64_t *full, uint64_t pol) {
+    constexpr uint32_t kTileBytes = kTileTok * D * sizeof(T);
     const int kvh = cur.w.unit / p.n_hc;
     if (phys < 0 || phys >= p.num_blocks) {
         raise_error(p.err, kErrBadBlock);
         mbar_arrive(full);
         return;
     }
-    const size_t off = ((size_t)phys * p.H_kv + kvh) * kBlockSize * D;
+    const size_t off = (((size_t)phys * p.H_kv + kvh) * kBlockSize + (size_t)sub * kTileTok) * D;
     mbar_arrive_expect_tx(full, 2 * kTileBytes);
     bulk_load(dst, static_cast<const T *>(p.k_cache) + off, kTileBytes, full, pol);
     bulk_load(dst + kTileBytes, static_cast<const T *>(p.v_cache) + off, kTileBytes,
               full, pol);
 }
 
+// The producer warp: streams the CTA's tiles, numbered n = 0, 1, ... over
+// its range (kSub per block), into stage n % S once tile n - S has been
+// released by the compute warps; then waits for the copies still in flight
+// (the last S issued) so none lands after the CTA exits.  All 32 lanes run
+// it; lane 0 issues the copies.
+template <int D, typename T, int S, int kTileTok, int kSub>
+__device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long lo,
+                              long long hi, int seq, long long base,
+                              unsigned char *stage_base, uint64_t *full_bar,
+                              uint64_t *empty_bar, int lane, volatile int *abort_flag) {
+    constexpr int kStageBytes = 2 * kTileTok * D * (int)sizeof(T);
+    const uint64_t pol = l2_policy_evict_first();
+    Producer prod;
+    prod.cur.init(pa, lo, hi, seq, base);
+    const long long n_tiles = (hi - lo) * kSub;
+    int sub = 0, phys = -1;
+    long long m = 0;
+    for (; m < n_tiles; ++m) {
+        const int s = (int)(m % S);
+        if (m >= S) {
+            const bool fr = mbar_wait(&empty_bar[s], (uint32_t)(((m / S) - 1) & 1),
+                                      p.timeout_ns, p.err, abort_flag);
+            if (!__all_sync(0xffffffffu, fr)) break;
+        }
+        if (sub == 0) phys = prod.block_id(p, lane);
+        if (lane == 0)
+            issue_tile<D, T, kTileTok>(p, prod.cur, phys, sub,
+                                       stage_base + (size_t)s * kStageBytes, &full_bar[s],
+                                       pol);
+        if (++sub == kSub) {
+            sub = 0;
+            prod.cur.next();
+        }
+    }
+    if (lane == 0) {
+        for (long long k = m > S ? m - S : 0; k < m; ++k)
+            mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1), p.timeout_ns, p.err,
+                      nullptr);
+    }
+}
+
 template <int D, int HC, typename T>
 __global__ void __launch_bounds__(GqaCfg<D, HC, T>::kThreads, 1)
 gqa_split_kernel(const GqaParams p) {
     using C = GqaCfg<D, HC, T>;
+    constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *stage_base = smem;
-    float *s_scores = reinterpret_cast<float *>(smem + C::kStages * C::kStageBytes);
+    float *s_scores = reinterpret_cast<float *>(smem + S * C::kStageBytes);
     float *s_mo = s_scores + C::kScoreBytes / 4;
     float *s_mm = s_mo + C::kMergeOBytes / 4;
     float *s_ml = s_mm + C::kNW * HC;
     unsigned char *misc = reinterpret_cast<unsigned char *>(s_ml + C::kNW * HC);
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(misc);
-    uint64_t *empty_bar = full_bar + C::kStages;
-    uint64_t *merge_bar = empty_bar + C::kStages;       // [2]
+    uint64_t *empty_bar = full_bar + S;
+    uint64_t *merge_bar = empty_bar + S;                // [2]
     uint64_t *never_bar = merge_bar + 2;                // fault injection
     PlanScratch *plan_sh = reinterpret_cast<PlanScratch *>(never_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(plan_sh + 1);
 
     const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
+    const int lane = tid & 31;
 
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], C::kNW);
+            mbar_init(&empty_bar[s], C::kWPG);
         }
         mbar_init(&merge_bar[0], C::kNW * 32);
         mbar_init(&merge_bar[1], C::kNW * 32);
@@ -338,27 +408,21 @@ gqa_split_kernel(const GqaParams p) {
     walk.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
 
     // ------------------------------------------------------------ producer
-    // Warp 0 streams the tiles (lane 0 issues); the prologue fills every stage.
-    const bool producer = (warp == 0);
-    Producer prod;
-    long long issued = 0;
-    const long long n_tiles = hi - lo;
-    uint64_t pol = 0;
-    if (producer) {
-        pol = l2_policy_evict_first();
-        prod.cur.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
-        while (issued < C::kStages && issued < n_tiles) {
-            const int phys = prod.block_id(p, lane);
-            if (lane == 0)
-                issue_tile<D, T, C::kTileBytes>(p, prod.cur, phys,
-                                                stage_base + issued * C::kStageBytes,
-                                                &full_bar[issued], pol);
-            prod.cur.next();
-            ++issued;
-        }
+    if (tid < 128) {
+        regs_decrease<C::kProducerRegs>();
+        if (tid < 32)
+            produce_tiles<D, T, S, C::kTileTok, C::kSub>(p, pa, lo, hi, plan_sh->seq,
+                                                         plan_sh->base, stage_base, full_bar,
+                                                         empty_bar, lane, abort_flag);
+        return;
     }
 
     // ------------------------------------------------------------ consumers
+    regs_increase<C::kConsumerRegs>();
+    const int ctid = tid - 128;             // thread among the compute warps
+    const int warp = ctid >> 5;             // compute warp 0 .. kNW-1
+    const int grp = warp / C::kWPG;         // tile group of this warp
+    const int wig = warp % C::kWPG;         // warp within its group
     if (p.force_timeout) {
         // Fault injection: wait on a barrier nobody signals; bounded.
         mbar_wait(never_bar, 0, p.timeout_ns, p.err, abort_flag);
@@ -375,18 +439,18 @@ gqa_split_kernel(const GqaParams p) {
 
     const T *qg = static_cast<const T *>(p.q);
     float *sc = s_scores + warp * C::kTPW * C::kHCP;   // [TPW][HCP]
-    long long n_tile = 0;
+    long long seg_t0 = 0;                  // first tile of the current segment
     int n_seg = 0;
-    int c_stage = 0, p_stage = 0;          // stage of tile n_tile / n_tile - 1
-    uint32_t c_phase = 0, p_phase = 0;     // their use parity
 
     while (!*abort_flag && !walk.done()) {
         const int len = walk.seg_len();
+        const long long seg_t1 = seg_t0 + (long long)len * C::kSub;
         const int b = walk.b, unit = walk.unit;
         const int kvh = unit / p.n_hc, hc = unit % p.n_hc;
         const int head0 = kvh * p.group + hc * HC;
         const int Tb = walk.T;
         const int lo_tok = (p.window > 0 && Tb > p.window) ? Tb - p.window : 0;
+        const int blk0 = walk.first_blk + walk.blk_off;
 
         constexpr int LP = C::kLE / 2;          // pairs per load
         constexpr int EP = C::kEPL / 2;         // pairs per lane
@@ -413,50 +477,59 @@ gqa_split_kernel(const GqaParams p) {
         for (int ps = 0; ps < C::kPasses; ++ps) { m_run[ps] = -1e30f; l_run[ps] = 0.f; }
 
         bool ok = true;
-        for (int t = 0; t < len; ++t) {
-            const int stage = c_stage;
-            if (!mbar_wait(&full_bar[stage], c_phase, p.timeout_ns, p.err, abort_flag)) {
+        // This group's first tile of the segment.
+        long long n = seg_t0 + (long long)(((grp - (int)(seg_t0 % C::kNG)) % C::kNG + C::kNG) % C::kNG);
+        for (; n < seg_t1; n += C::kNG) {
+            const int stage = (int)(n % S);
+            if (!mbar_wait(&full_bar[stage], (uint32_t)((n / S) & 1), p.timeout_ns, p.err,
+                           abort_flag)) {
                 ok = false;
                 break;
             }
             const T *Ks = reinterpret_cast<const T *>(stage_base + stage * C::kStageBytes);
-            const T *Vs = Ks + kBlockSize * D;
-            const int tok0 = (walk.first_blk + walk.blk_off + t) * kBlockSize +
-                             warp * C::kTPW;
+            const T *Vs = Ks + C::kTileTok * D;
+            const int tl = (int)(n - seg_t0);
+            const int tok0 = (blk0 + tl / C::kSub) * kBlockSize +
+                             (tl % C::kSub) * C::kTileTok + wig * C::kTPW;
+            const int row0 = wig * C::kTPW;
 
-            // ---- scores: partial dot products, then reduce over the row group
-            float2 acc[C::kIters * HC];
+            // ---- scores: partial dot products, reduced over the row group
 #pragma unroll
-            for (int it = 0; it < C::kIters; ++it) {
-                const T *krow = Ks + (warp * C::kTPW + it * C::kRPW + rg) * D;
+            for (int ch = 0; ch < C::kChunks; ++ch) {
+                float2 acc[C::kChunk * HC];
 #pragma unroll
-                for (int g = 0; g < HC; ++g) acc[it * HC + g] = make_float2(0.f, 0.f);
+                for (int i = 0; i < C::kChunk; ++i) {
+                    const int it = ch * C::kChunk + i;
+                    const T *krow = Ks + (row0 + it * C::kRPW + rg) * D;
 #pragma unroll
-                for (int c = 0; c < C::kCPL; ++c) {
-                    float2 kp[LP];
-                    load_pairs<T, C::kLE>(krow + col[c], kp);
+                    for (int g = 0; g < HC; ++g) acc[i * HC + g] = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int g = 0; g < HC; ++g)
+                    for (int c = 0; c < C::kCPL; ++c) {
+                        float2 kp[LP];
+                        load_pairs<T, C::kLE>(krow + col[c], kp);
 #pragma unroll
-                        for (int j = 0; j < LP; ++j)
-                            acc[it * HC + g] =
-                                __ffma2_rn(q2[g][c * LP + j], kp[j], acc[it * HC + g]);
+                        for (int g = 0; g < HC; ++g)
+#pragma unroll
+                            for (int j = 0; j < LP; ++j)
+                                acc[i * HC + g] =
+                                    __ffma2_rn(q2[g][c * LP + j], kp[j], acc[i * HC + g]);
+                    }
                 }
-            }
-            float part[C::kIters * HC];
+                float part[C::kChunk * HC];
 #pragma unroll
-            for (int i = 0; i < C::kIters * HC; ++i) part[i] = acc[i].x + acc[i].y;
-            using RR = RowReduce<C::kIters * HC, C::kLPR>;
-            const int base = RR::run(part, lane);
+                for (int i = 0; i < C::kChunk * HC; ++i) part[i] = acc[i].x + acc[i].y;
+                using RR = RowReduce<C::kChunk * HC, C::kLPR>;
+                const int base = RR::run(part, lane);
 #pragma unroll
-            for (int i = 0; i < RR::final_count(); ++i) {
-                const int v = base + i;
-                const int it = v / HC, g = v % HC;
-                sc[(it * C::kRPW + rg) * C::kHCP + g] = part[i];
+                for (int i = 0; i < RR::final_count(); ++i) {
+                    const int v = base + i;
+                    const int it = ch * C::kChunk + v / HC, g = v % HC;
+                    sc[(it * C::kRPW + rg) * C::kHCP + g] = part[i];
+                }
             }
             __syncwarp();
 
-            // ---- online softmax over this warp's 8 tokens (log2 domain)
+            // ---- online softmax over this warp's rows (log2 domain)
             float alpha_reg[C::kPasses];
 #pragma unroll
             for (int ps = 0; ps < C::kPasses; ++ps) {
@@ -498,7 +571,7 @@ gqa_split_kernel(const GqaParams p) {
 #pragma unroll
             for (int it = 0; it < C::kIters; ++it) {
                 const int rl = it * C::kRPW + rg;
-                const T *vrow = Vs + (warp * C::kTPW + rl) * D;
+                const T *vrow = Vs + (row0 + rl) * D;
                 float pg[C::kHCP];
                 load_row<C::kHCP>(sc + rl * C::kHCP, pg);
                 float2 pp[HC];
@@ -517,32 +590,6 @@ gqa_split_kernel(const GqaParams p) {
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[stage]);
-            // Refill the stage released one tile ago (one-tile lag keeps the
-            // producer from waiting on the slowest warp's current tile).
-            if (producer && n_tile >= 1 && issued < n_tiles) {
-                const int ps = p_stage;
-                const bool freed =
-                    mbar_wait(&empty_bar[ps], p_phase, p.timeout_ns, p.err, abort_flag);
-                if (__all_sync(0xffffffffu, freed)) {
-                    const int phys = prod.block_id(p, lane);
-                    if (lane == 0)
-                        issue_tile<D, T, C::kTileBytes>(p, prod.cur, phys,
-                                                        stage_base + ps * C::kStageBytes,
-                                                        &full_bar[ps], pol);
-                    prod.cur.next();
-                    ++issued;
-                } else {
-                    ok = false;
-                }
-            }
-            p_stage = c_stage;
-            p_phase = c_phase;
-            if (++c_stage == C::kStages) {
-                c_stage = 0;
-                c_phase ^= 1u;
-            }
-            ++n_tile;
-            if (!ok) break;
         }
         if (!ok) break;
 
@@ -603,7 +650,7 @@ gqa_split_kernel(const GqaParams p) {
                        abort_flag))
             break;
         const long long slot = (long long)b * units + unit + blockIdx.x;
-        for (int idx = tid; idx < HC * D; idx += C::kNW * 32) {
+        for (int idx = ctid; idx < HC * D; idx += C::kNW * 32) {
             const int g = idx / D, k = idx % D;
             float M = -1e30f;
 #pragma unroll
@@ -623,15 +670,10 @@ gqa_split_kernel(const GqaParams p) {
                        abort_flag))
             break;
         ++n_seg;
+        seg_t0 = seg_t1;
         walk.advance(len);
     }
 
-    // Abort path: copies still in flight must land before the CTA exits.
-    if (producer && lane == 0) {
-        for (long long n = n_tile; n < issued; ++n)
-            mbar_wait(&full_bar[n % C::kStages], (uint32_t)((n / C::kStages) & 1),
-                      p.timeout_ns, p.err, nullptr);
-    }
 }
 
 struct CombineParams {

@@ -25,6 +25,14 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     static bool configured = false;   // per-process; attribute is per function
     cudaError_t e;
     if (!configured) {
+        // The warpgroups' setmaxnreg shares must fit in the registers the
+        // kernel is launched with, or the increase would never be granted.
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs * C::kThreads <
+            4 * 32 * C::kProducerRegs + C::kNW * 32 * C::kConsumerRegs)
+            return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes);
