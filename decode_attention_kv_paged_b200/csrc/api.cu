@@ -23,6 +23,8 @@ struct DeviceState {
     unsigned *err = nullptr;      // device address of g_err_word
     void *ws = nullptr;
     size_t ws_bytes = 0;
+    unsigned *cnt = nullptr;      // split arrival counters (zero between launches)
+    size_t cnt_elems = 0;
 };
 
 static std::mutex g_mu;
@@ -74,6 +76,29 @@ static int ensure_workspace(DeviceState *st, size_t bytes, cudaStream_t stream) 
     }
     if (cudaMalloc(&st->ws, want) != cudaSuccess) return ATTN_ERR_CUDA;
     st->ws_bytes = want;
+    return ATTN_OK;
+}
+
+// Grow the device's split arrival counters to at least `n` (zeroed when
+// allocated; every launch leaves them at zero).  Never during capture.
+static int ensure_counters(DeviceState *st, size_t n, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (st->cnt_elems >= n) return ATTN_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return ATTN_ERR_UNSUPPORTED;
+    size_t want = n < 2 * st->cnt_elems ? 2 * st->cnt_elems : n;
+    want = (want + 4095) & ~(size_t)4095;
+    if (st->cnt) {
+        cudaFree(st->cnt);
+        st->cnt = nullptr;
+        st->cnt_elems = 0;
+    }
+    if (cudaMalloc(&st->cnt, want * sizeof(unsigned)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (cudaMemset(st->cnt, 0, want * sizeof(unsigned)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    st->cnt_elems = want;
     return ATTN_OK;
 }
 
@@ -129,6 +154,7 @@ unsigned *internal_error_word() {
     return device_state(&st) == ATTN_OK ? st->err : nullptr;
 }
 
+
 }  // namespace attn
 
 using namespace attn;
@@ -151,7 +177,7 @@ const char *attn_status_string(int s) {
 }
 
 int attn_set_num_ctas(int n) {
-    if (n < 0) return ATTN_ERR_ARG;
+    if (n < 0 || n > 65535) return ATTN_ERR_ARG;
     tl_num_ctas = n;
     return ATTN_OK;
 }
@@ -260,6 +286,12 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     kp.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
     kp.ws_prefix = reinterpret_cast<long long *>(ws + o_bytes + lse_bytes);
     kp.err = st->err;
+    kp.out = out;
+    if (!tc) {
+        rc = ensure_counters(st, (size_t)units_total, s);
+        if (rc) return rc;
+        kp.ws_cnt = st->cnt;
+    }
     take_force_timeout(&kp.force_timeout, &kp.timeout_ns);
     kp.scale_log2 = scale * 1.4426950408889634f;
     kp.B = B; kp.H_q = H_q; kp.H_kv = H_kv; kp.group = G; kp.n_hc = n_hc;

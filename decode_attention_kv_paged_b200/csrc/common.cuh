@@ -63,14 +63,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar,
     (void)state;
 }
 
+// Waits for the phase for at most about kSuspendNs (the thread sleeps until
+// the phase completes or the hint expires), then reports whether it did.
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
         : "memory");
     return done != 0;
 }
@@ -115,6 +118,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
+// Named barrier among `count` threads (multiple of 32), id 1..15.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------ register split
 // Per-warpgroup register budget (all threads of the warpgroup execute it).
 template <uint32_t N>
@@ -136,6 +144,16 @@ __device__ __forceinline__ void bulk_load(void *dst_smem, const void *src,
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
         ".L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst_smem)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// The same without a cache hint.
+__device__ __forceinline__ void bulk_load(void *dst_smem, const void *src,
+                                          uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 

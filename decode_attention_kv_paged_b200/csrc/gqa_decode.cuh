@@ -34,6 +34,8 @@
 namespace attn {
 
 constexpr int kSmemBudget = 227 * 1024 - 1024;
+// Headroom of the lazy softmax rescale, log2 units: probabilities <= 2^8.
+constexpr float kRescaleLog2 = 8.0f;
 #define kNegInf (__int_as_float(0xff800000u))
 
 constexpr int pow2_floor(int x) {
@@ -70,9 +72,11 @@ struct GqaParams {
     const void *v_cache;
     const int32_t *seq_lens;
     const int32_t *block_table;
+    void *out;            // [B][H_q][D]
     float *ws_o;          // [slots][HC][D]
     float *ws_lse;        // [slots][HC]  log2-sum-exp of the scaled scores
     long long *ws_prefix; // [B + 1]
+    unsigned *ws_cnt;     // [B * units] split arrival counters, zero between launches
     unsigned *err;
     unsigned long long timeout_ns;
     float scale_log2;     // scale * log2(e)
@@ -125,9 +129,11 @@ struct GqaCfg {
     static constexpr int kScoreBytes = kNW * kTPW * kHCP * 4;
     static constexpr int kMergeOBytes = kNW * HC * D * 4;
     static constexpr int kMergeMLBytes = 2 * kNW * HC * 4;
+    static constexpr int kQBytes = HC * D * kS;                   // one unit's queries
+    static constexpr int kQRingBytes = 2 * ((kQBytes + 127) / 128 * 128);
     static constexpr int kMiscBytes = 1024;  // barriers + plan scratch + flags
     static constexpr int kOther =
-        kScoreBytes + kMergeOBytes + kMergeMLBytes + kMiscBytes;
+        kQRingBytes + kScoreBytes + kMergeOBytes + kMergeMLBytes + kMiscBytes;
     static constexpr int kStagesRaw = (kSmemBudget - kOther) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static_assert(kTPW * kHPP == 32, "softmax lane map");
@@ -319,24 +325,56 @@ __device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor 
               full, pol);
 }
 
+// Arrival of one split of a unit: true for the last of its `ns` splits,
+// which also puts the counter back to zero for the next launch.
+__device__ __forceinline__ bool unit_arrive(unsigned *cnt, int ns) {
+    const unsigned old = atomicAdd(cnt, 1u);
+    const bool last = old + 1 == (unsigned)ns;
+    if (last) *cnt = 0u;
+    return last;
+}
+
 // The producer warp: streams the CTA's tiles, numbered n = 0, 1, ... over
 // its range (kSub per block), into stage n % S once tile n - S has been
 // released by the compute warps; then waits for the copies still in flight
 // (the last S issued) so none lands after the CTA exits.  All 32 lanes run
 // it; lane 0 issues the copies.
-template <int D, typename T, int S, int kTileTok, int kSub>
+template <int D, int HC, typename T, int S, int kTileTok, int kSub>
 __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long lo,
                               long long hi, int seq, long long base,
                               unsigned char *stage_base, uint64_t *full_bar,
-                              uint64_t *empty_bar, int lane, volatile int *abort_flag) {
+                              uint64_t *empty_bar, unsigned char *q_ring, int q_slot_bytes,
+                              uint64_t *q_full, uint64_t *q_empty, int lane,
+                              volatile int *abort_flag) {
     constexpr int kStageBytes = 2 * kTileTok * D * (int)sizeof(T);
+    constexpr uint32_t kQBytes = HC * D * sizeof(T);
     const uint64_t pol = l2_policy_evict_first();
     Producer prod;
     prod.cur.init(pa, lo, hi, seq, base);
     const long long n_tiles = (hi - lo) * kSub;
-    int sub = 0, phys = -1;
+    int sub = 0, phys = -1, seg = 0;
     long long m = 0;
     for (; m < n_tiles; ++m) {
+        if (sub == 0 && prod.cur.t == 0) {
+            // First tile of a segment: its unit's queries go first, into
+            // slot seg % 2 once segment seg - 2 has read that slot.
+            const int qs = seg & 1;
+            if (seg >= 2) {
+                const bool fr = mbar_wait(&q_empty[qs], (uint32_t)(((seg >> 1) - 1) & 1),
+                                          p.timeout_ns, p.err, abort_flag);
+                if (!__all_sync(0xffffffffu, fr)) break;
+            }
+            if (lane == 0) {
+                const int u = prod.cur.w.unit;
+                const int head0 = (u / p.n_hc) * p.group + (u % p.n_hc) * HC;
+                mbar_arrive_expect_tx(&q_full[qs], kQBytes);
+                bulk_load(q_ring + qs * q_slot_bytes,
+                          static_cast<const T *>(p.q) +
+                              ((size_t)prod.cur.w.b * p.H_q + head0) * D,
+                          kQBytes, &q_full[qs]);
+            }
+            ++seg;
+        }
         const int s = (int)(m % S);
         if (m >= S) {
             const bool fr = mbar_wait(&empty_bar[s], (uint32_t)(((m / S) - 1) & 1),
@@ -357,6 +395,9 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
         for (long long k = m > S ? m - S : 0; k < m; ++k)
             mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1), p.timeout_ns, p.err,
                       nullptr);
+        for (int j = seg > 2 ? seg - 2 : 0; j < seg; ++j)
+            mbar_wait(&q_full[j & 1], (uint32_t)((j >> 1) & 1), p.timeout_ns, p.err,
+                      nullptr);
     }
 }
 
@@ -367,7 +408,9 @@ gqa_split_kernel(const GqaParams p) {
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *stage_base = smem;
-    float *s_scores = reinterpret_cast<float *>(smem + S * C::kStageBytes);
+    unsigned char *q_ring = smem + S * C::kStageBytes;          // [2][HC][D]
+    constexpr int kQSlot = C::kQRingBytes / 2;
+    float *s_scores = reinterpret_cast<float *>(q_ring + C::kQRingBytes);
     float *s_mo = s_scores + C::kScoreBytes / 4;
     float *s_mm = s_mo + C::kMergeOBytes / 4;
     float *s_ml = s_mm + C::kNW * HC;
@@ -375,9 +418,12 @@ gqa_split_kernel(const GqaParams p) {
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(misc);
     uint64_t *empty_bar = full_bar + S;
     uint64_t *merge_bar = empty_bar + S;                // [2]
-    uint64_t *never_bar = merge_bar + 2;                // fault injection
+    uint64_t *q_full = merge_bar + 2;                   // [2]
+    uint64_t *q_empty = q_full + 2;                     // [2]
+    uint64_t *never_bar = q_empty + 2;                  // fault injection
     PlanScratch *plan_sh = reinterpret_cast<PlanScratch *>(never_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(plan_sh + 1);
+    volatile int *last_flag = abort_flag + 1;
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -389,11 +435,20 @@ gqa_split_kernel(const GqaParams p) {
         }
         mbar_init(&merge_bar[0], C::kNW * 32);
         mbar_init(&merge_bar[1], C::kNW * 32);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], C::kNW);
+        }
         mbar_init(never_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     __syncthreads();
+
+    // Programmatic dependent launch: everything above overlaps the previous
+    // kernel on the stream; inputs are read only after it has completed.
+    pdl_wait_primary();
+    pdl_launch_dependents();
 
     const int units = p.H_kv * p.n_hc;
     PlanArgs pa{p.seq_lens, p.B, units, p.window, p.max_blocks, p.num_ctas};
@@ -410,10 +465,23 @@ gqa_split_kernel(const GqaParams p) {
     // ------------------------------------------------------------ producer
     if (tid < 128) {
         regs_decrease<C::kProducerRegs>();
-        if (tid < 32)
-            produce_tiles<D, T, S, C::kTileTok, C::kSub>(p, pa, lo, hi, plan_sh->seq,
-                                                         plan_sh->base, stage_base, full_bar,
-                                                         empty_bar, lane, abort_flag);
+        if (tid < 32) {
+            produce_tiles<D, HC, T, S, C::kTileTok, C::kSub>(
+                p, pa, lo, hi, plan_sh->seq, plan_sh->base, stage_base, full_bar, empty_bar,
+                q_ring, kQSlot, q_full, q_empty, lane, abort_flag);
+        } else {
+            // A sequence without a visible block (empty) has a zero output
+            // and no split works on it; the idle producer warps write it.
+            for (int b = blockIdx.x; b < p.B; b += P) {
+                int fb;
+                bool bad;
+                if (visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad) == 0) {
+                    T *o = static_cast<T *>(p.out) + (size_t)b * p.H_q * D;
+                    for (int i = tid - 32; i < p.H_q * D; i += 96)
+                        o[i] = ElemTraits<T>::from_float(0.f);
+                }
+            }
+        }
         return;
     }
 
@@ -437,10 +505,12 @@ gqa_split_kernel(const GqaParams p) {
     for (int c = 0; c < C::kCPL; ++c)
         col[c] = ((lr + rot + c * C::kLPR) % C::kCPR) * C::kLE;
 
-    const T *qg = static_cast<const T *>(p.q);
     float *sc = s_scores + warp * C::kTPW * C::kHCP;   // [TPW][HCP]
     long long seg_t0 = 0;                  // first tile of the current segment
     int n_seg = 0;
+
+    constexpr int LP = C::kLE / 2;          // pairs per load
+    constexpr int EP = C::kEPL / 2;         // pairs per lane
 
     while (!*abort_flag && !walk.done()) {
         const int len = walk.seg_len();
@@ -452,21 +522,25 @@ gqa_split_kernel(const GqaParams p) {
         const int lo_tok = (p.window > 0 && Tb > p.window) ? Tb - p.window : 0;
         const int blk0 = walk.first_blk + walk.blk_off;
 
-        constexpr int LP = C::kLE / 2;          // pairs per load
-        constexpr int EP = C::kEPL / 2;         // pairs per lane
+        // The unit's queries, staged in shared memory by the producer.
+        if (!mbar_wait(&q_full[n_seg & 1], (uint32_t)((n_seg >> 1) & 1), p.timeout_ns, p.err,
+                       abort_flag))
+            break;
+        const T *qs = reinterpret_cast<const T *>(q_ring + (n_seg & 1) * kQSlot);
         float2 q2[HC][EP];
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
         for (int g = 0; g < HC; ++g) {
-            const T *qrow = qg + ((size_t)b * p.H_q + head0 + g) * D;
 #pragma unroll
             for (int c = 0; c < C::kCPL; ++c) {
                 float2 f[LP];
-                load_pairs<T, C::kLE>(qrow + col[c], f);
+                load_pairs<T, C::kLE>(qs + g * D + col[c], f);
 #pragma unroll
                 for (int j = 0; j < LP; ++j) q2[g][c * LP + j] = __fmul2_rn(f[j], sc2);
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_empty[n_seg & 1]);
         float2 o2[HC][EP];
 #pragma unroll
         for (int g = 0; g < HC; ++g)
@@ -529,8 +603,12 @@ gqa_split_kernel(const GqaParams p) {
             }
             __syncwarp();
 
-            // ---- online softmax over this warp's rows (log2 domain)
-            float alpha_reg[C::kPasses];
+            // ---- online softmax over this warp's rows (log2 domain), lazy:
+            // probabilities are taken against the running max m_run, which
+            // (with O and the partial sums) is raised only when a score
+            // exceeds it by more than kRescaleLog2 -- every probability stays
+            // below 2^kRescaleLog2.  Each lane keeps the partial sum of its
+            // own (token slot, head); they are added up at the merge.
 #pragma unroll
             for (int ps = 0; ps < C::kPasses; ++ps) {
                 const int gs = lane / C::kTPW + C::kHPP * ps;
@@ -538,34 +616,32 @@ gqa_split_kernel(const GqaParams p) {
                 const bool active = gs < HC;
                 const int pos = tok0 + tt;
                 const bool valid = active && pos >= lo_tok && pos < Tb;
-                float s = valid ? sc[tt * C::kHCP + gs] : kNegInf;
-                float mx = s;
+                const float s = valid ? sc[tt * C::kHCP + gs] : kNegInf;
+                if (__any_sync(0xffffffffu, s > m_run[ps] + kRescaleLog2)) {
+                    float mx = s;
 #pragma unroll
-                for (int m = 1; m < C::kTPW; m <<= 1)
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-                const float m_new = fmaxf(m_run[ps], mx);
-                const float pr = exp2f(s - m_new);
-                float sum = pr;
+                    for (int m = 1; m < C::kTPW; m <<= 1)
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+                    const float m_new = fmaxf(m_run[ps], mx);
+                    const float alpha = exp2f(m_run[ps] - m_new);
+                    l_run[ps] *= alpha;
+                    m_run[ps] = m_new;
 #pragma unroll
-                for (int m = 1; m < C::kTPW; m <<= 1)
-                    sum += __shfl_xor_sync(0xffffffffu, sum, m);
-                const float alpha = exp2f(m_run[ps] - m_new);
-                l_run[ps] = l_run[ps] * alpha + sum;
-                m_run[ps] = m_new;
-                alpha_reg[ps] = alpha;
+                    for (int j = 0; j < C::kHPP; ++j) {
+                        const int g = C::kHPP * ps + j;
+                        if (g < HC) {
+                            const float a = __shfl_sync(0xffffffffu, alpha, j * C::kTPW);
+                            const float2 a2 = make_float2(a, a);
+#pragma unroll
+                            for (int e = 0; e < EP; ++e) o2[g][e] = __fmul2_rn(o2[g][e], a2);
+                        }
+                    }
+                }
+                const float pr = exp2f(s - m_run[ps]);
+                l_run[ps] += pr;
                 if (active) sc[tt * C::kHCP + gs] = pr;
             }
             __syncwarp();
-#pragma unroll
-            for (int g = 0; g < HC; ++g) {
-                const float a = __shfl_sync(0xffffffffu, alpha_reg[g / C::kHPP],
-                                            (g % C::kHPP) * C::kTPW);
-                if (a != 1.f) {
-                    const float2 a2 = make_float2(a, a);
-#pragma unroll
-                    for (int j = 0; j < EP; ++j) o2[g][j] = __fmul2_rn(o2[g][j], a2);
-                }
-            }
 
             // ---- P V
 #pragma unroll
@@ -592,6 +668,9 @@ gqa_split_kernel(const GqaParams p) {
             if (lane == 0) mbar_arrive(&empty_bar[stage]);
         }
         if (!ok) break;
+
+        SegmentWalker next = walk;
+        next.advance(len);
 
         // ---- merge the warps' states, write the segment's partial
         // Row groups with a rotated chunk order hold chunk (c + shift) mod CPL
@@ -635,6 +714,11 @@ gqa_split_kernel(const GqaParams p) {
                         *reinterpret_cast<float2 *>(&s_mo[(warp * HC + g) * D + col[c] + 2 * j]) =
                             o2[g][c * LP + j];
         }
+#pragma unroll
+        for (int ps = 0; ps < C::kPasses; ++ps)
+#pragma unroll
+            for (int m = 1; m < C::kTPW; m <<= 1)
+                l_run[ps] += __shfl_xor_sync(0xffffffffu, l_run[ps], m);
         if ((lane % C::kTPW) == 0) {
 #pragma unroll
             for (int ps = 0; ps < C::kPasses; ++ps) {
@@ -649,7 +733,13 @@ gqa_split_kernel(const GqaParams p) {
         if (!mbar_wait(&merge_bar[0], (uint32_t)(n_seg & 1), p.timeout_ns, p.err,
                        abort_flag))
             break;
-        const long long slot = (long long)b * units + unit + blockIdx.x;
+        // Splits of this unit: the CTAs whose ranges meet its blocks.
+        const long long u = (long long)b * units + unit;
+        const long long s_u = walk.pos - walk.blk_off;     // the unit's first block
+        const int c0 = cta_of(s_u, W, P);
+        const int ns = cta_of(s_u + walk.nb - 1, W, P) - c0 + 1;
+        T *out_u = static_cast<T *>(p.out) + ((size_t)b * p.H_q + head0) * D;
+        const long long slot = u + blockIdx.x;
         for (int idx = ctid; idx < HC * D; idx += C::kNW * 32) {
             const int g = idx / D, k = idx % D;
             float M = -1e30f;
@@ -662,18 +752,126 @@ gqa_split_kernel(const GqaParams p) {
                 num = fmaf(wt, s_mo[(w * HC + g) * D + k], num);
                 den = fmaf(wt, s_ml[w * HC + g], den);
             }
-            p.ws_o[(slot * HC + g) * D + k] = num / den;
-            if (k == 0) p.ws_lse[slot * HC + g] = M + log2f(den);
+            if (ns == 1) {
+                out_u[idx] = ElemTraits<T>::from_float(num / den);
+            } else {
+                p.ws_o[(slot * HC + g) * D + k] = num / den;
+                if (k == 0) p.ws_lse[slot * HC + g] = M + log2f(den);
+            }
         }
         mbar_arrive(&merge_bar[1]);
         if (!mbar_wait(&merge_bar[1], (uint32_t)(n_seg & 1), p.timeout_ns, p.err,
                        abort_flag))
             break;
+        if (ns > 1) {
+            // The last split to arrive combines the unit's partials, in CTA
+            // order (fixed, deterministic):
+            //   out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L).
+            // The CTA barrier above orders every thread's partial before
+            // thread 0's fence; the fence publishes them, cumulatively,
+            // before the arrival (and orders the last arrival's reads).
+            if (ctid == 0) {
+                __threadfence();
+                const bool last = unit_arrive(p.ws_cnt + u, ns);
+                if (last) __threadfence();
+                *last_flag = last ? 1 : 0;
+            }
+            named_barrier(1, C::kNW * 32);
+            if (*last_flag) {
+                const long long slot0 = u + c0;
+                T *dst = out_u;
+                if (ns <= C::kNW * D) {
+                    // Split weights 2^(lse - L) in shared memory (the merge
+                    // buffers are free here), one warp per head reduces them.
+                    float *wts = s_mo;             // [ns][HC]
+                    float *inv = s_mm;             // [HC]
+                    for (int i = ctid; i < ns * HC; i += C::kNW * 32)
+                        wts[i] = __ldcg(p.ws_lse + slot0 * HC + i);
+                    named_barrier(1, C::kNW * 32);
+                    if (warp < HC) {
+                        float L = kNegInf;
+                        for (int i = lane; i < ns; i += 32) L = fmaxf(L, wts[i * HC + warp]);
+#pragma unroll
+                        for (int m = 16; m >= 1; m >>= 1)
+                            L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, m));
+                        float den = 0.f;
+                        for (int i = lane; i < ns; i += 32) {
+                            const float w = exp2f(wts[i * HC + warp] - L);
+                            wts[i * HC + warp] = w;
+                            den += w;
+                        }
+#pragma unroll
+                        for (int m = 16; m >= 1; m >>= 1)
+                            den += __shfl_xor_sync(0xffffffffu, den, m);
+                        if (lane == 0) inv[warp] = 1.f / den;
+                    }
+                    named_barrier(1, C::kNW * 32);
+                    for (int e = ctid * 4; e < HC * D; e += C::kNW * 32 * 4) {
+                        const int g = e / D, k = e % D;
+                        const float *src = p.ws_o + (slot0 * HC + g) * D + k;
+                        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll 4
+                        for (int i = 0; i < ns; ++i) {
+                            const float w = wts[i * HC + g];
+                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                src + (size_t)i * HC * D));
+                            r0 = fmaf(w, v.x, r0);
+                            r1 = fmaf(w, v.y, r1);
+                            r2 = fmaf(w, v.z, r2);
+                            r3 = fmaf(w, v.w, r3);
+                        }
+                        const float iv = inv[g];
+                        dst[e] = ElemTraits<T>::from_float(r0 * iv);
+                        dst[e + 1] = ElemTraits<T>::from_float(r1 * iv);
+                        dst[e + 2] = ElemTraits<T>::from_float(r2 * iv);
+                        dst[e + 3] = ElemTraits<T>::from_float(r3 * iv);
+                    }
+                    // The next segment's merge rewrites these buffers.
+                    named_barrier(1, C::kNW * 32);
+                } else {
+                    for (int e = ctid * 4; e < HC * D; e += C::kNW * 32 * 4) {
+                        const int g = e / D, k = e % D;
+                        float L = kNegInf;
+                        for (int i = 0; i < ns; ++i)
+                            L = fmaxf(L, __ldcg(p.ws_lse + (slot0 + i) * HC + g));
+                        float den = 0.f, r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+                        for (int i = 0; i < ns; ++i) {
+                            const float w =
+                                exp2f(__ldcg(p.ws_lse + (slot0 + i) * HC + g) - L);
+                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                p.ws_o + ((slot0 + i) * HC + g) * D + k));
+                            r0 = fmaf(w, v.x, r0);
+                            r1 = fmaf(w, v.y, r1);
+                            r2 = fmaf(w, v.z, r2);
+                            r3 = fmaf(w, v.w, r3);
+                            den += w;
+                        }
+                        const float iv = 1.f / den;
+                        dst[e] = ElemTraits<T>::from_float(r0 * iv);
+                        dst[e + 1] = ElemTraits<T>::from_float(r1 * iv);
+                        dst[e + 2] = ElemTraits<T>::from_float(r2 * iv);
+                        dst[e + 3] = ElemTraits<T>::from_float(r3 * iv);
+                    }
+                }
+            }
+        }
         ++n_seg;
         seg_t0 = seg_t1;
-        walk.advance(len);
+        walk = next;
     }
 
+    // After an abort the CTA still arrives on every unit it had not
+    // finished, so each unit's counter is back at zero when the launch ends
+    // (the outputs of those units are not valid; the error word says so).
+    if (ctid == 0) {
+        while (!walk.done()) {
+            const int len = walk.seg_len();
+            const long long s_u = walk.pos - walk.blk_off;
+            const int ns = cta_of(s_u + walk.nb - 1, W, P) - cta_of(s_u, W, P) + 1;
+            if (ns > 1) unit_arrive(p.ws_cnt + (long long)walk.b * units + walk.unit, ns);
+            walk.advance(len);
+        }
+    }
 }
 
 struct CombineParams {

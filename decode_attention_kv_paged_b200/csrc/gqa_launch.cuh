@@ -1,5 +1,6 @@
-// gqa_launch.cuh -- host-side launch of the CUDA-core split-KV kernel and the
-// combine kernel for one (head dim, heads-per-CTA, dtype) instantiation.
+// gqa_launch.cuh -- host-side launch of the CUDA-core split-KV kernel (which
+// also combines its split partials) for one (head dim, heads-per-CTA, dtype)
+// instantiation.
 #pragma once
 
 #include "gqa_decode.cuh"
@@ -8,7 +9,7 @@ namespace attn {
 
 struct GqaLaunch {
     GqaParams kp;
-    CombineParams cp;
+    CombineParams cp;         // combine launch of the tensor-core path
     int units_total;          // B * H_kv * n_hc
     cudaStream_t stream;
     cudaEvent_t ev_start;     // optional (profiling hook), may be null
@@ -40,27 +41,22 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
         configured = true;
     }
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
-    gqa_split_kernel<D, HC, T>
-        <<<L.kp.num_ctas, C::kThreads, C::kSmemBytes, L.stream>>>(L.kp);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
-
-    CombineParams cp = L.cp;
-    cp.D = D;
-    cp.HC = HC;
-    cp.blocks_per_unit = (HC * D / 4 + kCombineThreads - 1) / kCombineThreads;
+    // The split partials are combined inside the kernel (by the last split
+    // of each unit), so this is the call's only launch.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((long long)L.units_total * cp.blocks_per_unit));
-    cfg.blockDim = dim3(kCombineThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.gridDim = dim3((unsigned)L.kp.num_ctas);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = L.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = L.ev_stop ? 0 : 1;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, combine_kernel<T>, cp);
+    e = cudaLaunchKernelEx(&cfg, gqa_split_kernel<D, HC, T>, L.kp);
+    if (e != cudaSuccess) return e;
+    if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
+    return cudaSuccess;
 }
 
 // Dispatch over heads-per-CTA and dtype for one head dimension D.

@@ -26,10 +26,13 @@ unsigned *internal_error_word();   // api.cu
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+// Split arrival counters: zero when the library loads, zero after every call.
+static __device__ __align__(256) unsigned g_noalloc_cnt[ATTN_NOALLOC_MAX_UNITS];
 
 struct NoAllocDevice {
     bool ready = false;
     void *scratch = nullptr;   // device address of g_noalloc_scratch
+    unsigned *cnt = nullptr;   // device address of g_noalloc_cnt
     int num_sms = 0;
 };
 
@@ -45,9 +48,12 @@ int noalloc_setup(NoAllocDevice **out) {
     if ((int)g_noalloc_dev.size() <= dev) g_noalloc_dev.resize(dev + 1);
     NoAllocDevice &d = g_noalloc_dev[dev];
     if (!d.ready) {
-        void *ptr = nullptr;
+        void *ptr = nullptr, *cptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
             return ATTN_ERR_CUDA;
+        if (cudaGetSymbolAddress(&cptr, g_noalloc_cnt) != cudaSuccess || !cptr)
+            return ATTN_ERR_CUDA;
+        d.cnt = static_cast<unsigned *>(cptr);
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return ATTN_ERR_CUDA;
@@ -106,13 +112,15 @@ extern "C" int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
     const size_t o_bytes = round256((size_t)slots * HC * d * sizeof(float));
     const size_t lse_bytes = round256((size_t)slots * HC * sizeof(float));
     const size_t pre_bytes = round256((size_t)(B + 1) * sizeof(long long));
-    if (units_total > (1ll << 30) ||
+    if (units_total > ATTN_NOALLOC_MAX_UNITS ||
         o_bytes + lse_bytes + pre_bytes > (size_t)ATTN_NOALLOC_SCRATCH_BYTES)
         return ATTN_ERR_UNSUPPORTED;   // scratch would exceed the fixed array
     unsigned char *ws = static_cast<unsigned char *>(dev->scratch);
 
     // Nothing in the scratch has to start at zero: every partial, log-sum-exp
     // and prefix value a call reads was written earlier in the same call.
+    // The arrival counters are a separate array that each call leaves at
+    // zero (an aborted split still arrives).
     GqaLaunch L{};
     GqaParams &kp = L.kp;
     kp.q = q; kp.k_cache = k_cache; kp.v_cache = v_cache;
@@ -121,6 +129,8 @@ extern "C" int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
     kp.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
     kp.ws_prefix = reinterpret_cast<long long *>(ws + o_bytes + lse_bytes);
     kp.err = err;
+    kp.out = out;
+    kp.ws_cnt = dev->cnt;
     kp.force_timeout = 0;
     kp.timeout_ns = kDefaultTimeoutNs;
     kp.scale_log2 = scale * 1.4426950408889634f;

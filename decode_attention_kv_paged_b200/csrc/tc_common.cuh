@@ -313,9 +313,5 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const vo
         : "memory");
 }
 
-// Named barrier among `count` threads (multiple of 32), id 1..15.
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 }  // namespace attn

@@ -217,16 +217,20 @@ int attn_decode_last_error(void *stream);
  *
  * Scratch needed: 4 * (B*H_q/hc + SMs) * hc * (d + 1) bytes plus 8*(B+1)
  * (hc = query heads per CTA, see attn_decode_gqa_config; each term rounded
- * up to 256 bytes); above the limit the call returns ATTN_ERR_UNSUPPORTED.
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, on the current device); make that first call
- * before any stream capture.  All calls share the one array and it keeps the
- * last call's contents (nothing in it needs to start at zero): calls that can
- * overlap on the GPU -- on different streams, or from several threads -- race
- * on it, so order them on one stream.  The attn_set_num_ctas, profiling and
+ * up to 256 bytes), and at most ATTN_NOALLOC_MAX_UNITS (sequence, KV head,
+ * head chunk) units, B*H_q/hc; above either limit the call returns
+ * ATTN_ERR_UNSUPPORTED.  A second fixed array holds one split-arrival
+ * counter per unit: zero when the library loads, zero again after every
+ * call.  The first call on each device looks up the arrays' device
+ * addresses (cudaGetSymbolAddress, on the current device); make that first
+ * call before any stream capture.  All calls share the arrays and the
+ * scratch keeps the last call's contents (nothing in it needs to start at
+ * zero): calls that can overlap on the GPU -- on different streams, or from
+ * several threads -- race on them, so order them on one stream.  The attn_set_num_ctas, profiling and
  * fault-injection hooks do not apply to this entry point.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define ATTN_NOALLOC_MAX_UNITS 65536
 int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
                             const void *v_cache, const int32_t *seq_lens,
                             const int32_t *block_table, void *out, int B,
