@@ -271,8 +271,10 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     if (units_total > (1ll << 30)) return ATTN_ERR_ARG;
     const long long slots = units_total + P;
 
-    const size_t o_bytes = align256((size_t)slots * HC * d * sizeof(float));
-    const size_t lse_bytes = align256((size_t)slots * HC * sizeof(float));
+    // The tensor-core kernel writes gqa_tc_copies(HC) partials per slot.
+    const int copies = tc ? gqa_tc_copies(HC) : 1;
+    const size_t o_bytes = align256((size_t)slots * copies * HC * d * sizeof(float));
+    const size_t lse_bytes = align256((size_t)slots * copies * HC * sizeof(float));
     const size_t pre_bytes = align256((size_t)(B + 1) * sizeof(long long));
     rc = ensure_workspace(st, o_bytes + lse_bytes + pre_bytes, s);
     if (rc) return rc;
@@ -303,6 +305,7 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     cp.ws_lse = kp.ws_lse; cp.out = out;
     cp.B = B; cp.H_q = H_q; cp.H_kv = H_kv; cp.group = G; cp.n_hc = n_hc;
     cp.max_blocks = max_blocks_per_seq; cp.window = kp.window; cp.num_ctas = P;
+    cp.copies = copies;
     L.units_total = (int)units_total;
     L.stream = s;
     take_profile_events(&L.ev_start, &L.ev_stop);

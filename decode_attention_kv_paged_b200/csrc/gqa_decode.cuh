@@ -129,11 +129,13 @@ struct GqaCfg {
     static constexpr int kScoreBytes = kNW * kTPW * kHCP * 4;
     static constexpr int kMergeOBytes = kNW * HC * D * 4;
     static constexpr int kMergeMLBytes = 2 * kNW * HC * 4;
+    static constexpr int kEpiBytes = (kNW + 2) * HC * 4;         // merge weights
+    static constexpr int kEpiThreads = 96;                        // producer WG warps 1-3
     static constexpr int kQBytes = HC * D * kS;                   // one unit's queries
     static constexpr int kQRingBytes = 2 * ((kQBytes + 127) / 128 * 128);
     static constexpr int kMiscBytes = 1024;  // barriers + plan scratch + flags
     static constexpr int kOther =
-        kQRingBytes + kScoreBytes + kMergeOBytes + kMergeMLBytes + kMiscBytes;
+        kQRingBytes + kScoreBytes + kMergeOBytes + kMergeMLBytes + kEpiBytes + kMiscBytes;
     static constexpr int kStagesRaw = (kSmemBudget - kOther) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static_assert(kTPW * kHPP == 32, "softmax lane map");
@@ -401,6 +403,136 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
     }
 }
 
+// Segment epilogue, run by the kEpiThreads epilogue threads (et = 0 ..) on the
+// compute warps' stashed states: s_mo [NW][HC][D] partial outputs, s_mm /
+// s_ml [NW][HC] running max / sum of each warp.  Merges them, then writes the
+// unit's output (one split) or its fp32 partial; the last split of a unit to
+// arrive combines the unit's partials in CTA order (fixed, deterministic):
+//     out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L).
+template <int D, int HC, typename T, int NW, int NT>
+__device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0, int ns,
+                                 long long slot, T *out_u, float *s_mo, const float *s_mm,
+                                 const float *s_ml, float *s_w, volatile int *last_flag) {
+    float *s_inv = s_w + NW * HC;          // [HC]
+    float *s_lse = s_inv + HC;             // [HC]
+    // Per head: the common max, each warp's weight, the normaliser.
+    if (et < HC) {
+        const int g = et;
+        float M = -1e30f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, s_mm[w * HC + g]);
+        float den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float wt = exp2f(s_mm[w * HC + g] - M);
+            s_w[w * HC + g] = wt;
+            den = fmaf(wt, s_ml[w * HC + g], den);
+        }
+        s_inv[g] = 1.f / den;
+        s_lse[g] = M + log2f(den);
+    }
+    named_barrier(1, NT);
+    for (int e = et * 4; e < HC * D; e += NT * 4) {
+        const int g = e / D;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float wt = s_w[w * HC + g];
+            const float4 v = *reinterpret_cast<const float4 *>(s_mo + (size_t)w * HC * D + e);
+            acc.x = fmaf(wt, v.x, acc.x);
+            acc.y = fmaf(wt, v.y, acc.y);
+            acc.z = fmaf(wt, v.z, acc.z);
+            acc.w = fmaf(wt, v.w, acc.w);
+        }
+        const float iv = s_inv[g];
+        acc.x *= iv; acc.y *= iv; acc.z *= iv; acc.w *= iv;
+        if (ns == 1) {
+            out_u[e] = ElemTraits<T>::from_float(acc.x);
+            out_u[e + 1] = ElemTraits<T>::from_float(acc.y);
+            out_u[e + 2] = ElemTraits<T>::from_float(acc.z);
+            out_u[e + 3] = ElemTraits<T>::from_float(acc.w);
+        } else {
+            *reinterpret_cast<float4 *>(p.ws_o + slot * HC * D + e) = acc;
+        }
+    }
+    if (ns == 1) return;
+    if (et < HC) p.ws_lse[slot * HC + et] = s_lse[et];
+    // The barrier orders every thread's partial before thread 0's fence,
+    // which publishes them, cumulatively, before the arrival (and orders the
+    // last arrival's reads after the other splits' partials).
+    named_barrier(1, NT);
+    if (et == 0) {
+        __threadfence();
+        const bool last = unit_arrive(p.ws_cnt + u, ns);
+        if (last) __threadfence();
+        *last_flag = last ? 1 : 0;
+    }
+    named_barrier(1, NT);
+    if (!*last_flag) return;
+    const long long slot0 = u + c0;
+    if (ns <= NW * D) {
+        // Split weights 2^(lse - L) in shared memory (the stash is no longer
+        // needed), then each output is one weighted sum.
+        float *wts = s_mo;                 // [ns][HC]
+        for (int i = et; i < ns * HC; i += NT) wts[i] = __ldcg(p.ws_lse + slot0 * HC + i);
+        named_barrier(1, NT);
+        if (et < HC) {
+            const int g = et;
+            float L = kNegInf;
+            for (int i = 0; i < ns; ++i) L = fmaxf(L, wts[i * HC + g]);
+            float den = 0.f;
+            for (int i = 0; i < ns; ++i) {
+                const float w = exp2f(wts[i * HC + g] - L);
+                wts[i * HC + g] = w;
+                den += w;
+            }
+            s_inv[g] = 1.f / den;
+        }
+        named_barrier(1, NT);
+        for (int e = et * 4; e < HC * D; e += NT * 4) {
+            const int g = e / D;
+            const float *src = p.ws_o + slot0 * HC * D + e;
+            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < ns; ++i) {
+                const float w = wts[i * HC + g];
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)i * HC * D));
+                r0 = fmaf(w, v.x, r0);
+                r1 = fmaf(w, v.y, r1);
+                r2 = fmaf(w, v.z, r2);
+                r3 = fmaf(w, v.w, r3);
+            }
+            const float iv = s_inv[g];
+            out_u[e] = ElemTraits<T>::from_float(r0 * iv);
+            out_u[e + 1] = ElemTraits<T>::from_float(r1 * iv);
+            out_u[e + 2] = ElemTraits<T>::from_float(r2 * iv);
+            out_u[e + 3] = ElemTraits<T>::from_float(r3 * iv);
+        }
+    } else {
+        for (int e = et * 4; e < HC * D; e += NT * 4) {
+            const int g = e / D, k = e % D;
+            float L = kNegInf;
+            for (int i = 0; i < ns; ++i) L = fmaxf(L, __ldcg(p.ws_lse + (slot0 + i) * HC + g));
+            float den = 0.f, r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+            for (int i = 0; i < ns; ++i) {
+                const float w = exp2f(__ldcg(p.ws_lse + (slot0 + i) * HC + g) - L);
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                    p.ws_o + ((slot0 + i) * HC + g) * D + k));
+                r0 = fmaf(w, v.x, r0);
+                r1 = fmaf(w, v.y, r1);
+                r2 = fmaf(w, v.z, r2);
+                r3 = fmaf(w, v.w, r3);
+                den += w;
+            }
+            const float iv = 1.f / den;
+            out_u[e] = ElemTraits<T>::from_float(r0 * iv);
+            out_u[e + 1] = ElemTraits<T>::from_float(r1 * iv);
+            out_u[e + 2] = ElemTraits<T>::from_float(r2 * iv);
+            out_u[e + 3] = ElemTraits<T>::from_float(r3 * iv);
+        }
+    }
+}
+
 template <int D, int HC, typename T>
 __global__ void __launch_bounds__(GqaCfg<D, HC, T>::kThreads, 1)
 gqa_split_kernel(const GqaParams p) {
@@ -414,13 +546,15 @@ gqa_split_kernel(const GqaParams p) {
     float *s_mo = s_scores + C::kScoreBytes / 4;
     float *s_mm = s_mo + C::kMergeOBytes / 4;
     float *s_ml = s_mm + C::kNW * HC;
-    unsigned char *misc = reinterpret_cast<unsigned char *>(s_ml + C::kNW * HC);
+    float *s_w = s_ml + C::kNW * HC;                    // epilogue scratch
+    unsigned char *misc = reinterpret_cast<unsigned char *>(s_w + C::kEpiBytes / 4);
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(misc);
     uint64_t *empty_bar = full_bar + S;
-    uint64_t *merge_bar = empty_bar + S;                // [2]
-    uint64_t *q_full = merge_bar + 2;                   // [2]
+    uint64_t *q_full = empty_bar + S;                   // [2]
     uint64_t *q_empty = q_full + 2;                     // [2]
-    uint64_t *never_bar = q_empty + 2;                  // fault injection
+    uint64_t *epi_full = q_empty + 2;                   // stash written
+    uint64_t *epi_empty = epi_full + 1;                 // stash consumed
+    uint64_t *never_bar = epi_empty + 1;                // fault injection
     PlanScratch *plan_sh = reinterpret_cast<PlanScratch *>(never_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(plan_sh + 1);
     volatile int *last_flag = abort_flag + 1;
@@ -433,8 +567,8 @@ gqa_split_kernel(const GqaParams p) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], C::kWPG);
         }
-        mbar_init(&merge_bar[0], C::kNW * 32);
-        mbar_init(&merge_bar[1], C::kNW * 32);
+        mbar_init(epi_full, C::kNW * 32);
+        mbar_init(epi_empty, C::kEpiThreads);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1);
             mbar_init(&q_empty[i], C::kNW);
@@ -470,15 +604,47 @@ gqa_split_kernel(const GqaParams p) {
                 p, pa, lo, hi, plan_sh->seq, plan_sh->base, stage_base, full_bar, empty_bar,
                 q_ring, kQSlot, q_full, q_empty, lane, abort_flag);
         } else {
+            const int et = tid - 32;
             // A sequence without a visible block (empty) has a zero output
-            // and no split works on it; the idle producer warps write it.
+            // and no split works on it.
             for (int b = blockIdx.x; b < p.B; b += P) {
                 int fb;
                 bool bad;
                 if (visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad) == 0) {
                     T *o = static_cast<T *>(p.out) + (size_t)b * p.H_q * D;
-                    for (int i = tid - 32; i < p.H_q * D; i += 96)
+                    for (int i = et; i < p.H_q * D; i += C::kEpiThreads)
                         o[i] = ElemTraits<T>::from_float(0.f);
+                }
+            }
+            // The epilogue of every segment, while the compute warps go on
+            // with the next one.
+            SegmentWalker ew;
+            ew.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
+            for (int es = 0; !ew.done(); ++es) {
+                if (!mbar_wait(epi_full, (uint32_t)(es & 1), p.timeout_ns, p.err, abort_flag))
+                    break;
+                const int len = ew.seg_len();
+                const long long u = (long long)ew.b * units + ew.unit;
+                const long long s_u = ew.pos - ew.blk_off;     // the unit's first block
+                const int c0 = cta_of(s_u, W, P);
+                const int ns = cta_of(s_u + ew.nb - 1, W, P) - c0 + 1;
+                const int head0 = (ew.unit / p.n_hc) * p.group + (ew.unit % p.n_hc) * HC;
+                T *out_u = static_cast<T *>(p.out) + ((size_t)ew.b * p.H_q + head0) * D;
+                segment_epilogue<D, HC, T, C::kNW, C::kEpiThreads>(
+                    p, et, u, c0, ns, u + blockIdx.x, out_u, s_mo, s_mm, s_ml, s_w, last_flag);
+                mbar_arrive(epi_empty);
+                ew.advance(len);
+            }
+            // After an abort the CTA still arrives on every unit it had not
+            // finished, so each unit's counter is back at zero when the
+            // launch ends (those outputs are not valid; the error word says so).
+            if (et == 0) {
+                while (!ew.done()) {
+                    const int len = ew.seg_len();
+                    const long long s_u = ew.pos - ew.blk_off;
+                    const int ns = cta_of(s_u + ew.nb - 1, W, P) - cta_of(s_u, W, P) + 1;
+                    if (ns > 1) unit_arrive(p.ws_cnt + (long long)ew.b * units + ew.unit, ns);
+                    ew.advance(len);
                 }
             }
         }
@@ -515,9 +681,6 @@ gqa_split_kernel(const GqaParams p) {
     while (!*abort_flag && !walk.done()) {
         const int len = walk.seg_len();
         const long long seg_t1 = seg_t0 + (long long)len * C::kSub;
-        const int b = walk.b, unit = walk.unit;
-        const int kvh = unit / p.n_hc, hc = unit % p.n_hc;
-        const int head0 = kvh * p.group + hc * HC;
         const int Tb = walk.T;
         const int lo_tok = (p.window > 0 && Tb > p.window) ? Tb - p.window : 0;
         const int blk0 = walk.first_blk + walk.blk_off;
@@ -672,7 +835,7 @@ gqa_split_kernel(const GqaParams p) {
         SegmentWalker next = walk;
         next.advance(len);
 
-        // ---- merge the warps' states, write the segment's partial
+        // ---- stash this warp's state for the epilogue warps
         // Row groups with a rotated chunk order hold chunk (c + shift) mod CPL
         // in register slot c; put them back in the unrotated order first so
         // the cross-row-group sums below add like columns.
@@ -704,6 +867,15 @@ gqa_split_kernel(const GqaParams p) {
                     o2[g][j].x += __shfl_xor_sync(0xffffffffu, o2[g][j].x, m);
                     o2[g][j].y += __shfl_xor_sync(0xffffffffu, o2[g][j].y, m);
                 }
+#pragma unroll
+        for (int ps = 0; ps < C::kPasses; ++ps)
+#pragma unroll
+            for (int m = 1; m < C::kTPW; m <<= 1)
+                l_run[ps] += __shfl_xor_sync(0xffffffffu, l_run[ps], m);
+        // The epilogue of the previous segment must be done with the stash.
+        if (n_seg > 0 && !mbar_wait(epi_empty, (uint32_t)((n_seg - 1) & 1), p.timeout_ns,
+                                    p.err, abort_flag))
+            break;
         if (rg == 0) {
 #pragma unroll
             for (int g = 0; g < HC; ++g)
@@ -714,11 +886,6 @@ gqa_split_kernel(const GqaParams p) {
                         *reinterpret_cast<float2 *>(&s_mo[(warp * HC + g) * D + col[c] + 2 * j]) =
                             o2[g][c * LP + j];
         }
-#pragma unroll
-        for (int ps = 0; ps < C::kPasses; ++ps)
-#pragma unroll
-            for (int m = 1; m < C::kTPW; m <<= 1)
-                l_run[ps] += __shfl_xor_sync(0xffffffffu, l_run[ps], m);
         if ((lane % C::kTPW) == 0) {
 #pragma unroll
             for (int ps = 0; ps < C::kPasses; ++ps) {
@@ -729,148 +896,10 @@ gqa_split_kernel(const GqaParams p) {
                 }
             }
         }
-        mbar_arrive(&merge_bar[0]);
-        if (!mbar_wait(&merge_bar[0], (uint32_t)(n_seg & 1), p.timeout_ns, p.err,
-                       abort_flag))
-            break;
-        // Splits of this unit: the CTAs whose ranges meet its blocks.
-        const long long u = (long long)b * units + unit;
-        const long long s_u = walk.pos - walk.blk_off;     // the unit's first block
-        const int c0 = cta_of(s_u, W, P);
-        const int ns = cta_of(s_u + walk.nb - 1, W, P) - c0 + 1;
-        T *out_u = static_cast<T *>(p.out) + ((size_t)b * p.H_q + head0) * D;
-        const long long slot = u + blockIdx.x;
-        for (int idx = ctid; idx < HC * D; idx += C::kNW * 32) {
-            const int g = idx / D, k = idx % D;
-            float M = -1e30f;
-#pragma unroll
-            for (int w = 0; w < C::kNW; ++w) M = fmaxf(M, s_mm[w * HC + g]);
-            float num = 0.f, den = 0.f;
-#pragma unroll
-            for (int w = 0; w < C::kNW; ++w) {
-                const float wt = exp2f(s_mm[w * HC + g] - M);
-                num = fmaf(wt, s_mo[(w * HC + g) * D + k], num);
-                den = fmaf(wt, s_ml[w * HC + g], den);
-            }
-            if (ns == 1) {
-                out_u[idx] = ElemTraits<T>::from_float(num / den);
-            } else {
-                p.ws_o[(slot * HC + g) * D + k] = num / den;
-                if (k == 0) p.ws_lse[slot * HC + g] = M + log2f(den);
-            }
-        }
-        mbar_arrive(&merge_bar[1]);
-        if (!mbar_wait(&merge_bar[1], (uint32_t)(n_seg & 1), p.timeout_ns, p.err,
-                       abort_flag))
-            break;
-        if (ns > 1) {
-            // The last split to arrive combines the unit's partials, in CTA
-            // order (fixed, deterministic):
-            //   out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L).
-            // The CTA barrier above orders every thread's partial before
-            // thread 0's fence; the fence publishes them, cumulatively,
-            // before the arrival (and orders the last arrival's reads).
-            if (ctid == 0) {
-                __threadfence();
-                const bool last = unit_arrive(p.ws_cnt + u, ns);
-                if (last) __threadfence();
-                *last_flag = last ? 1 : 0;
-            }
-            named_barrier(1, C::kNW * 32);
-            if (*last_flag) {
-                const long long slot0 = u + c0;
-                T *dst = out_u;
-                if (ns <= C::kNW * D) {
-                    // Split weights 2^(lse - L) in shared memory (the merge
-                    // buffers are free here), one warp per head reduces them.
-                    float *wts = s_mo;             // [ns][HC]
-                    float *inv = s_mm;             // [HC]
-                    for (int i = ctid; i < ns * HC; i += C::kNW * 32)
-                        wts[i] = __ldcg(p.ws_lse + slot0 * HC + i);
-                    named_barrier(1, C::kNW * 32);
-                    if (warp < HC) {
-                        float L = kNegInf;
-                        for (int i = lane; i < ns; i += 32) L = fmaxf(L, wts[i * HC + warp]);
-#pragma unroll
-                        for (int m = 16; m >= 1; m >>= 1)
-                            L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, m));
-                        float den = 0.f;
-                        for (int i = lane; i < ns; i += 32) {
-                            const float w = exp2f(wts[i * HC + warp] - L);
-                            wts[i * HC + warp] = w;
-                            den += w;
-                        }
-#pragma unroll
-                        for (int m = 16; m >= 1; m >>= 1)
-                            den += __shfl_xor_sync(0xffffffffu, den, m);
-                        if (lane == 0) inv[warp] = 1.f / den;
-                    }
-                    named_barrier(1, C::kNW * 32);
-                    for (int e = ctid * 4; e < HC * D; e += C::kNW * 32 * 4) {
-                        const int g = e / D, k = e % D;
-                        const float *src = p.ws_o + (slot0 * HC + g) * D + k;
-                        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
-#pragma unroll 4
-                        for (int i = 0; i < ns; ++i) {
-                            const float w = wts[i * HC + g];
-                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(
-                                src + (size_t)i * HC * D));
-                            r0 = fmaf(w, v.x, r0);
-                            r1 = fmaf(w, v.y, r1);
-                            r2 = fmaf(w, v.z, r2);
-                            r3 = fmaf(w, v.w, r3);
-                        }
-                        const float iv = inv[g];
-                        dst[e] = ElemTraits<T>::from_float(r0 * iv);
-                        dst[e + 1] = ElemTraits<T>::from_float(r1 * iv);
-                        dst[e + 2] = ElemTraits<T>::from_float(r2 * iv);
-                        dst[e + 3] = ElemTraits<T>::from_float(r3 * iv);
-                    }
-                    // The next segment's merge rewrites these buffers.
-                    named_barrier(1, C::kNW * 32);
-                } else {
-                    for (int e = ctid * 4; e < HC * D; e += C::kNW * 32 * 4) {
-                        const int g = e / D, k = e % D;
-                        float L = kNegInf;
-                        for (int i = 0; i < ns; ++i)
-                            L = fmaxf(L, __ldcg(p.ws_lse + (slot0 + i) * HC + g));
-                        float den = 0.f, r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
-                        for (int i = 0; i < ns; ++i) {
-                            const float w =
-                                exp2f(__ldcg(p.ws_lse + (slot0 + i) * HC + g) - L);
-                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(
-                                p.ws_o + ((slot0 + i) * HC + g) * D + k));
-                            r0 = fmaf(w, v.x, r0);
-                            r1 = fmaf(w, v.y, r1);
-                            r2 = fmaf(w, v.z, r2);
-                            r3 = fmaf(w, v.w, r3);
-                            den += w;
-                        }
-                        const float iv = 1.f / den;
-                        dst[e] = ElemTraits<T>::from_float(r0 * iv);
-                        dst[e + 1] = ElemTraits<T>::from_float(r1 * iv);
-                        dst[e + 2] = ElemTraits<T>::from_float(r2 * iv);
-                        dst[e + 3] = ElemTraits<T>::from_float(r3 * iv);
-                    }
-                }
-            }
-        }
+        mbar_arrive(epi_full);
         ++n_seg;
         seg_t0 = seg_t1;
         walk = next;
-    }
-
-    // After an abort the CTA still arrives on every unit it had not
-    // finished, so each unit's counter is back at zero when the launch ends
-    // (the outputs of those units are not valid; the error word says so).
-    if (ctid == 0) {
-        while (!walk.done()) {
-            const int len = walk.seg_len();
-            const long long s_u = walk.pos - walk.blk_off;
-            const int ns = cta_of(s_u + walk.nb - 1, W, P) - cta_of(s_u, W, P) + 1;
-            if (ns > 1) unit_arrive(p.ws_cnt + (long long)walk.b * units + walk.unit, ns);
-            walk.advance(len);
-        }
     }
 }
 
@@ -882,13 +911,15 @@ struct CombineParams {
     void *out;
     int B, H_q, H_kv, group, n_hc, max_blocks, window, num_ctas;
     int D, HC;               // head dim, query heads per unit
+    int copies;              // partials per (unit, CTA) slot (>= 1)
     int blocks_per_unit;     // CTAs of kCombineThreads per unit
 };
 
 constexpr int kCombineThreads = 256;
 
 // out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L) over the unit's split
-// partials, in CTA order (fixed, deterministic).  Each thread produces four
+// partials (`copies` per slot, slot-major), in CTA order (fixed,
+// deterministic).  A partial with lse = -inf has weight zero.  Each thread produces four
 // consecutive outputs of one head; a unit's HC*D outputs are spread over
 // blocks_per_unit CTAs.
 template <typename T>
@@ -914,8 +945,8 @@ combine_kernel(const CombineParams p) {
             const long long s_u = p.ws_prefix[b] + (long long)rem * nb;
             const int c0 = cta_of(s_u, W, P);
             const int c1 = cta_of(s_u + nb - 1, W, P);
-            s_nsplit = c1 - c0 + 1;
-            s_first_slot = (long long)u + c0;
+            s_nsplit = (c1 - c0 + 1) * p.copies;
+            s_first_slot = ((long long)u + c0) * p.copies;
         }
     }
     __syncthreads();

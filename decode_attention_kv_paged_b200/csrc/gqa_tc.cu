@@ -15,12 +15,17 @@
 //     paged cache into a multi-stage ring and of the unit's query rows; one
 //     thread of warp 1 issues tcgen05 MMAs as their inputs become ready;
 //     warps 4-7 run the softmax and the epilogue.
-//   * S: M = 64 query rows (heads, zero-padded), N = 64 tokens, K = d, both
-//     operands in shared memory, fp32 accumulator in TMEM (double-buffered).
-//     The M = 64 accumulator puts row r in TMEM lane (r % 16) + 32 (r / 16),
-//     so each head row is read by one thread: the softmax needs no
-//     cross-thread reductions.  The running max is only raised when it grows
-//     by more than 2^8 (lazy rescale, exact either way).
+//   * S: M = 64 query rows, N = 64 tokens, K = d, both operands in shared
+//     memory, fp32 accumulator in TMEM (double-buffered).  The M = 64
+//     accumulator puts row r in TMEM lane (r % 16) + 32 (r / 16), so each
+//     row is read by one thread: the softmax needs no cross-thread
+//     reductions.  A group of HC <= 32 heads (padded to HCP = 16 or 32) is
+//     loaded 64 / HCP times into the 64 rows; copy c of the heads takes only
+//     the token slice [c TPC, (c + 1) TPC) of every tile (TPC = HCP), so all
+//     four softmax warps work and each thread handles TPC tokens.  Every
+//     copy keeps its own (m, l, O) and writes its own partial, merged with
+//     the split partials by the log-sum-exp combine.  The running max is only
+//     raised when it grows by more than 2^8 (lazy rescale, exact either way).
 //   * P is split into bf16 P_hi + P_lo (the rounding remainder) so the
 //     weights keep ~16 significant bits; O += P_hi V + P_lo V with V read
 //     MN-major from the same swizzled tile; O stays in TMEM for the segment.
@@ -46,13 +51,16 @@ struct TcCfg {
     static constexpr int kBoxes = D / 64;
     static constexpr int kQBytes = kBoxes * kTcBox;
     static constexpr int kStageBytes = 2 * kBoxes * kTcBox;     // K then V
-    static constexpr int kFixed = kQBytes + 2 * kTcPBytes + 1024 /*bars*/ + 1024 /*align*/;
+    // P is double-buffered (hi and lo halves each): the softmax of tile i + 1
+    // writes while the P V of tile i reads.
+    static constexpr int kPBytes = 4 * kTcPBytes;
+    static constexpr int kFixed = kQBytes + kPBytes + 1024 /*bars*/ + 1024 /*align*/;
     static constexpr int kStagesRaw = (227 * 1024 - kFixed) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
     static constexpr int kOffQ = 0;
     static constexpr int kOffC = kOffQ + kQBytes;
     static constexpr int kOffP = kOffC + kStages * kStageBytes;
-    static constexpr int kOffBar = kOffP + 2 * kTcPBytes;
+    static constexpr int kOffBar = kOffP + kPBytes;
     static constexpr int kSmem = kOffBar + 1024 + 1024;
     static constexpr uint32_t kTmemO = 0, kTmemS = D;            // S buffers at D, D + 64
     static constexpr uint32_t kTmemCols = D + 128 <= 256 ? 256 : 512;
@@ -64,18 +72,23 @@ struct TcBars {
     uint64_t q_full, q_empty;
     uint64_t c_full[6], c_empty[6];
     uint64_t s_full[2], s_free[2];
-    uint64_t p_full, pv_done, o_free, mma_final;
+    // One P-ready and one P V-done barrier per P buffer: the softmax can
+    // finish two tiles before the MMA thread tests the first, which a single
+    // barrier could not tell apart.
+    uint64_t p_full[2], pv_done[2], o_free, mma_final;
     uint32_t tmem_base;
     int abort;
     PlanScratch plan;
 };
 static_assert(sizeof(TcBars) <= 1024, "barrier block");
 
-template <int D>
+template <int D, int TPC>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const GqaParams p, int HC) {
     using C = TcCfg<D>;
+    constexpr int kCopies = kTcM / TPC;     // copies of the head group in the 64 rows
+    constexpr int kHCP = TPC;               // rows per copy (heads, padded)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -100,7 +113,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     // Zero Q (rows beyond the group stay zero) and P (rows beyond the group
     // are never written), then make the zeros visible to the tensor cores.
-    for (int i = tid; i < (C::kQBytes + 2 * kTcPBytes) / 16; i += kTcThreads) {
+    for (int i = tid; i < (C::kQBytes + C::kPBytes) / 16; i += kTcThreads) {
         const int off = i * 16;
         uint4 *dst = reinterpret_cast<uint4 *>(off < C::kQBytes ? sQ + off
                                                                 : sP + (off - C::kQBytes));
@@ -118,8 +131,10 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&bars->s_full[s], 1);
             mbar_init(&bars->s_free[s], 128);
         }
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->pv_done, 1);
+        mbar_init(&bars->p_full[0], 128);
+        mbar_init(&bars->p_full[1], 128);
+        mbar_init(&bars->pv_done[0], 1);
+        mbar_init(&bars->pv_done[1], 1);
         mbar_init(&bars->o_free, 128);
         mbar_init(&bars->mma_final, 1);
         bars->abort = 0;
@@ -147,9 +162,11 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                               p.timeout_ns, p.err, abort_flag))
                         break;
                     const int qrow = cur.w.b * p.H_q + kvh * p.group + hc * HC;
-                    mbar_arrive_expect_tx(&bars->q_full, C::kBoxes * HC * 128);
-                    for (int j = 0; j < C::kBoxes; ++j)
-                        tma_load_2d(sQ + j * kTcBox, &tm_q, 64 * j, qrow, &bars->q_full, pol);
+                    mbar_arrive_expect_tx(&bars->q_full, kCopies * C::kBoxes * HC * 128);
+                    for (int c = 0; c < kCopies; ++c)
+                        for (int j = 0; j < C::kBoxes; ++j)
+                            tma_load_2d(sQ + j * kTcBox + c * kHCP * 128, &tm_q, 64 * j, qrow,
+                                        &bars->q_full, pol);
                     ++seg;
                 }
                 const int st = tile % C::kStages;
@@ -182,6 +199,9 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         __syncwarp();
     } else if (warp == 1) {
         // ============================================================ MMA
+        // One thread issues in a fixed order -- S(0), S(1), then S(i + 2) and
+        // P V(i) for each tile i -- polling each barrier it needs (a sleeping
+        // wait wakes up too late for this chain).
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16(kTcM, 64, 0, 0);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, 0, 1);
@@ -189,79 +209,77 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             TileCursor cs, cv;
             cs.init(pa, lo, hi, first_seq, first_base);
             cv.init(pa, lo, hi, first_seq, first_base);
-            int next_s = 0, next_pv = 0, seg_s = 0, seg_v = 0;
-            unsigned long long idle_since = 0;
-            uint32_t idle_polls = 0;
-            while (next_pv < n_tiles) {
-                bool did = false;
-                if (next_s < n_tiles && next_s < next_pv + 2) {
-                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
-                    const int st = next_s % C::kStages, sb = next_s & 1;
-                    const bool ready =
-                        (!first || mbar_test(&bars->q_full, (uint32_t)(seg_s & 1))) &&
-                        mbar_test(&bars->c_full[st], (uint32_t)((next_s / C::kStages) & 1)) &&
-                        (next_s < 2 ||
-                         mbar_test(&bars->s_free[sb], (uint32_t)(((next_s - 2) >> 1) & 1)));
-                    if (ready) {
-                        tc_fence_after();
-                        const uint32_t kst = c_base + st * C::kStageBytes;
-                        for (int j = 0; j < C::kBoxes; ++j)
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const uint64_t a =
-                                    umma_desc_sw128(q_base + j * kTcBox + k * 32, 16, 1024);
-                                const uint64_t b =
-                                    umma_desc_sw128(kst + j * kTcBox + k * 32, 16, 1024);
-                                umma_bf16(tmem + C::kTmemS + 64 * sb, a, b, idesc_s, (j | k) != 0);
-                            }
-                        umma_commit(&bars->s_full[sb]);
-                        if (last) umma_commit(&bars->q_empty);
-                        if (first) ++seg_s;
-                        cs.next();
-                        ++next_s;
-                        did = true;
+            int seg_s = 0, seg_v = 0;
+            auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+                unsigned long long t0 = 0;
+                for (uint32_t it = 0;; ++it) {
+                    if (mbar_test(bar, parity)) return true;
+                    if ((it & 15u) == 15u) {
+                        if (*abort_flag) return false;
+                        __nanosleep(20);
                     }
-                }
-                if (next_pv < next_s) {
-                    const bool first = cv.t == 0;
-                    const bool ready =
-                        mbar_test(&bars->p_full, (uint32_t)(next_pv & 1)) &&
-                        (!first || seg_v == 0 ||
-                         mbar_test(&bars->o_free, (uint32_t)((seg_v - 1) & 1)));
-                    if (ready) {
-                        tc_fence_after();
-                        const int st = next_pv % C::kStages;
-                        const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kTcBox;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint64_t b = umma_desc_sw128(vst + k * 2048, kTcBox, 1024);
-                            const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
-                            const uint64_t a_lo =
-                                umma_desc_sw128(p_base + kTcPBytes + k * 32, 16, 1024);
-                            umma_bf16(tmem + C::kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
-                            umma_bf16(tmem + C::kTmemO, a_lo, b, idesc_pv, 1);
+                    if ((it & 1023u) == 1023u) {
+                        const unsigned long long now = global_timer_ns();
+                        if (t0 == 0) {
+                            t0 = now;
+                        } else if (now - t0 > p.timeout_ns) {
+                            raise_error(p.err, kErrTimeout);
+                            *abort_flag = 1;
+                            return false;
                         }
-                        umma_commit(&bars->c_empty[st]);
-                        umma_commit(&bars->pv_done);
-                        if (first) ++seg_v;
-                        cv.next();
-                        ++next_pv;
-                        did = true;
                     }
                 }
-                if (did) {
-                    idle_since = 0;
-                    idle_polls = 0;
-                } else if ((++idle_polls & 7u) == 0 && (__nanosleep(32), (idle_polls & 63u) == 0)) {
-                    const unsigned long long now = global_timer_ns();
-                    if (idle_since == 0) idle_since = now;
-                    if (*abort_flag) break;
-                    if (now - idle_since > p.timeout_ns) {
-                        raise_error(p.err, kErrTimeout);
-                        *abort_flag = 1;
-                        break;
+            };
+            // S(n) = Q K(n)^T into S buffer n % 2.
+            auto issue_s = [&](int n) -> bool {
+                const bool first = cs.t == 0, last = cs.t == cs.len - 1;
+                const int st = n % C::kStages, sb = n & 1;
+                if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) return false;
+                if (!wait(&bars->c_full[st], (uint32_t)((n / C::kStages) & 1))) return false;
+                if (n >= 2 && !wait(&bars->s_free[sb], (uint32_t)(((n - 2) >> 1) & 1)))
+                    return false;
+                tc_fence_after();
+                const uint32_t kst = c_base + st * C::kStageBytes;
+                for (int j = 0; j < C::kBoxes; ++j)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t a = umma_desc_sw128(q_base + j * kTcBox + k * 32, 16, 1024);
+                        const uint64_t b = umma_desc_sw128(kst + j * kTcBox + k * 32, 16, 1024);
+                        umma_bf16(tmem + C::kTmemS + 64 * sb, a, b, idesc_s, (j | k) != 0);
                     }
+                umma_commit(&bars->s_full[sb]);
+                if (last) umma_commit(&bars->q_empty);
+                if (first) ++seg_s;
+                cs.next();
+                return true;
+            };
+            bool ok = true;
+            for (int n = 0; ok && n < 2 && n < n_tiles; ++n) ok = issue_s(n);
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                if (i + 2 < n_tiles && !issue_s(i + 2)) break;
+                // O += P(i) V(i), P from buffer i % 2 (hi and lo halves).
+                const bool first = cv.t == 0;
+                if (!wait(&bars->p_full[i & 1], (uint32_t)((i >> 1) & 1)) ||
+                    (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const int st = i % C::kStages;
+                const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kTcBox;
+                const uint32_t pb = p_base + (i & 1) * 2 * kTcPBytes;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t b = umma_desc_sw128(vst + k * 2048, kTcBox, 1024);
+                    const uint64_t a_hi = umma_desc_sw128(pb + k * 32, 16, 1024);
+                    const uint64_t a_lo = umma_desc_sw128(pb + kTcPBytes + k * 32, 16, 1024);
+                    umma_bf16(tmem + C::kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
+                    umma_bf16(tmem + C::kTmemO, a_lo, b, idesc_pv, 1);
+                }
+                umma_commit(&bars->c_empty[st]);
+                umma_commit(&bars->pv_done[i & 1]);
+                if (first) ++seg_v;
+                cv.next();
             }
             umma_commit(&bars->mma_final);
             mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
@@ -270,65 +288,86 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     } else if (warp >= 4) {
         // ================================================ softmax, epilogue
         // M = 64 accumulator: row r lives in TMEM lane (r % 16) + 32 (r / 16);
-        // warp 4 + q owns rows 16q .. 16q + 15 in its lanes 0..15.
+        // warp 4 + q owns rows 16q .. 16q + 15 in its lanes 0..15, which are
+        // head rows of copy c (warp-uniform) for the token slice c * TPC.
         const int q4 = warp & 3;
         const int row = 16 * q4 + lane;
-        const bool active = lane < 16 && row < HC;
+        const int copy = (16 * q4) / kHCP;
+        const int head = row - copy * kHCP;
+        const bool active = lane < 16 && head < HC;
         const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
-        unsigned char *prow = sP + (row < kTcM ? row : 0) * 128;
+        unsigned char *prow0 = sP + (lane < 16 ? row : 0) * 128;
         auto all = [](bool v) { return __all_sync(0xffffffffu, v); };
         TileCursor cur;
         cur.init(pa, lo, hi, first_seq, first_base);
-        float m_run = -1e30f, l_run = 0.f;
-        int n_seg = 0;
+        float m_run = kNegInf, l_run = 0.f;
         for (int i = 0; i < n_tiles; ++i) {
             const bool first = cur.t == 0, last = cur.t == cur.len - 1;
             const int b = cur.w.b, T = cur.w.T;
             const int lo_tok = (p.window > 0 && T > p.window) ? T - p.window : 0;
-            const int tok0 = cur.logical_block() * 64;
+            const int tok0 = cur.logical_block() * 64 + copy * TPC;
             const int sb = i & 1;
             if (!all(mbar_wait(&bars->s_full[sb], (uint32_t)((i >> 1) & 1), p.timeout_ns, p.err,
                                abort_flag)))
                 break;
             tc_fence_after();
-            float s[64];
-            tmem_ld64(trow + C::kTmemS + 64 * sb, s);
+            float s[TPC];
+            const uint32_t saddr = trow + C::kTmemS + 64 * sb + copy * TPC;
+            if constexpr (TPC == 64) tmem_ld64(saddr, s);
+            else if constexpr (TPC == 32) tmem_ld32(saddr, s);
+            else tmem_ld16(saddr, s);
             tc_fence_before();
             mbar_arrive(&bars->s_free[sb]);
 
             // scale to log2 units, mask keys outside [lo_tok, T)
             const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-            for (int j = 0; j < 64; j += 2) {
+            for (int j = 0; j < TPC; j += 2) {
                 const float2 v = __fmul2_rn(make_float2(s[j], s[j + 1]), sl2);
                 s[j] = v.x;
                 s[j + 1] = v.y;
             }
-            if (tok0 < lo_tok || tok0 + 64 > T) {
+            if (tok0 < lo_tok || tok0 + TPC > T) {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
+                for (int j = 0; j < TPC; ++j) {
                     const int pos = tok0 + j;
                     if (pos < lo_tok || pos >= T) s[j] = kNegInf;
                 }
             }
-            float mx = s[0];
+            float mx;
+            {
+                float t[8];
 #pragma unroll
-            for (int j = 1; j < 64; ++j) mx = fmaxf(mx, s[j]);
+                for (int j = 0; j < 8; ++j) {
+                    t[j] = s[j];
+#pragma unroll
+                    for (int k = j + 8; k < TPC; k += 8) t[j] = fmaxf(t[j], s[k]);
+                }
+#pragma unroll
+                for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+                mx = t[0];
+            }
+            // Raise the running max on the segment's first tile, or when a
+            // score exceeds it by more than the headroom.  A slice with no
+            // visible key so far keeps m_run = -inf (its probabilities are 0).
             bool rescale = false;
             float alpha = 1.f;
             if (first) {
                 m_run = mx;
                 l_run = 0.f;
             } else if (mx > m_run + kTcRescaleThreshold) {
-                alpha = exp2_approx(m_run - mx);
+                alpha = m_run == kNegInf ? 0.f : exp2_approx(m_run - mx);
                 m_run = mx;
                 l_run *= alpha;
                 rescale = true;
             }
+            const float mref = m_run == kNegInf ? 0.f : m_run;
             float2 sum2 = make_float2(0.f, 0.f);
-            const float2 m2 = make_float2(-m_run, -m_run);
+            const float2 m2 = make_float2(-mref, -mref);
 #pragma unroll
-            for (int j = 0; j < 64; j += 2) {
+            for (int j = 0; j < TPC; j += 2) {
                 const float2 d = __fadd2_rn(make_float2(s[j], s[j + 1]), m2);
                 s[j] = exp2_approx(d.x);
                 s[j + 1] = exp2_approx(d.y);
@@ -336,16 +375,20 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             l_run += sum2.x + sum2.y;
 
-            if (i >= 1 && !all(mbar_wait(&bars->pv_done, (uint32_t)((i - 1) & 1), p.timeout_ns,
-                                         p.err, abort_flag)))
+            // P buffer i % 2 was last read by P V(i - 2).
+            if (i >= 2 && !all(mbar_wait(&bars->pv_done[i & 1], (uint32_t)(((i >> 1) - 1) & 1),
+                                         p.timeout_ns, p.err, abort_flag)))
                 break;
+            unsigned char *prow = prow0 + (i & 1) * 2 * kTcPBytes;
             if (active) {
+                // This row's 16-byte chunks (8 tokens each) of its slice; the
+                // rest of the row stays zero.
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int cc = 0; cc < TPC / 8; ++cc) {
                     uint32_t hi_w[4], lo_w[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float a = s[8 * c + 2 * k], bb = s[8 * c + 2 * k + 1];
+                        const float a = s[8 * cc + 2 * k], bb = s[8 * cc + 2 * k + 1];
                         hi_w[k] = pack_bf16x2(a, bb);
                         const float2 r = __fadd2_rn(
                             make_float2(a, bb),
@@ -353,7 +396,8 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                         -__uint_as_float(hi_w[k] & 0xFFFF0000u)));
                         lo_w[k] = pack_bf16x2(r.x, r.y);
                     }
-                    const int off = (c ^ (row & 7)) * 16;
+                    const int chunk = copy * (TPC / 8) + cc;
+                    const int off = (chunk ^ (row & 7)) * 16;
                     *reinterpret_cast<uint4 *>(prow + off) =
                         make_uint4(hi_w[0], hi_w[1], hi_w[2], hi_w[3]);
                     *reinterpret_cast<uint4 *>(prow + kTcPBytes + off) =
@@ -361,6 +405,11 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             tc_fence_after();
+            // O may be rescaled only once P V(i - 1) has completed.
+            if (__any_sync(0xffffffffu, active && rescale) && i >= 1 &&
+                !all(mbar_wait(&bars->pv_done[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1),
+                               p.timeout_ns, p.err, abort_flag)))
+                break;
             if (__any_sync(0xffffffffu, active && rescale)) {
                 const float a = (active && rescale) ? alpha : 1.f;
                 float o[32];
@@ -375,16 +424,20 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive(&bars->p_full[i & 1]);
 
             if (last) {
-                if (!all(mbar_wait(&bars->pv_done, (uint32_t)(i & 1), p.timeout_ns, p.err,
-                                   abort_flag)))
+                if (!all(mbar_wait(&bars->pv_done[i & 1], (uint32_t)((i >> 1) & 1), p.timeout_ns,
+                                   p.err, abort_flag)))
                     break;
                 tc_fence_after();
+                // Partial of copy `copy` of this (unit, CTA) slot; a copy
+                // that saw no visible key writes zero weight (lse = -inf).
                 const long long slot = (long long)b * units + cur.w.unit + blockIdx.x;
-                const float inv = 1.f / l_run;
-                float *dst = p.ws_o + ((size_t)slot * HC + (active ? row : 0)) * D;
+                const long long part = (slot * kCopies + copy) * HC + (active ? head : 0);
+                const bool empty = l_run == 0.f;
+                const float inv = empty ? 0.f : 1.f / l_run;
+                float *dst = p.ws_o + (size_t)part * D;
                 float o[32];
 #pragma unroll 1
                 for (int ch = 0; ch < D / 32; ++ch) {
@@ -397,10 +450,9 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                             o[j + 3] * inv);
                     }
                 }
-                if (active) p.ws_lse[slot * HC + row] = m_run + log2f(l_run);
+                if (active) p.ws_lse[part] = empty ? kNegInf : m_run + log2f(l_run);
                 tc_fence_before();
                 mbar_arrive(&bars->o_free);
-                ++n_seg;
             }
             cur.next();
         }
@@ -449,12 +501,12 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int TPC>
 cudaError_t launch_tc(const GqaLaunch &L, int HC) {
     using C = TcCfg<D>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_tc_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(gqa_tc_kernel<D, TPC>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -466,7 +518,7 @@ cudaError_t launch_tc(const GqaLaunch &L, int HC) {
         !tc_make_map(&tv, kp.v_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64))
         return cudaErrorInvalidValue;
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
-    gqa_tc_kernel<D><<<kp.num_ctas, kTcThreads, C::kSmem, L.stream>>>(tq, tk, tv, kp, HC);
+    gqa_tc_kernel<D, TPC><<<kp.num_ctas, kTcThreads, C::kSmem, L.stream>>>(tq, tk, tv, kp, HC);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
@@ -474,6 +526,7 @@ cudaError_t launch_tc(const GqaLaunch &L, int HC) {
     CombineParams cp = L.cp;
     cp.D = D;
     cp.HC = HC;
+    cp.copies = kTcM / TPC;
     cp.blocks_per_unit = (HC * D / 4 + kCombineThreads - 1) / kCombineThreads;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((long long)L.units_total * cp.blocks_per_unit));
@@ -495,11 +548,22 @@ bool gqa_tc_supported(int d, int dtype_bf16, int G) {
 
 int gqa_tc_heads_per_cta(int G) { return G <= kTcM ? G : kTcM; }
 
+int gqa_tc_copies(int HC) { return HC <= 16 ? 4 : (HC <= 32 ? 2 : 1); }
+
+template <int D>
+cudaError_t launch_tc_d(const GqaLaunch &L, int HC) {
+    switch (gqa_tc_copies(HC)) {
+        case 4: return launch_tc<D, 16>(L, HC);
+        case 2: return launch_tc<D, 32>(L, HC);
+        default: return launch_tc<D, 64>(L, HC);
+    }
+}
+
 cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC) {
     switch (d) {
-        case 64: return launch_tc<64>(L, HC);
-        case 128: return launch_tc<128>(L, HC);
-        case 256: return launch_tc<256>(L, HC);
+        case 64: return launch_tc_d<64>(L, HC);
+        case 128: return launch_tc_d<128>(L, HC);
+        case 256: return launch_tc_d<256>(L, HC);
         default: return cudaErrorNotSupported;
     }
 }

@@ -9,6 +9,9 @@ namespace attn {
 // to 64 query heads per pass (larger groups in multiples of 64).
 bool gqa_tc_supported(int d, int dtype_bf16, int G);
 int gqa_tc_heads_per_cta(int G);
+// Copies of a group of HC heads in the 64 MMA rows (each takes a token
+// slice); the kernel writes this many partials per (unit, CTA) slot.
+int gqa_tc_copies(int HC);
 // Group size from which the tensor-core path is the default.
 constexpr int kTcMinGroup = 8;
 

@@ -681,6 +681,7 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     cp.num_ctas = clusters;
     cp.D = kMlaDc;
     cp.HC = kMlaH;
+    cp.copies = 1;
     cp.blocks_per_unit = kMlaH * kMlaDc / 4 / kCombineThreads;
     combine_kernel<__nv_bfloat16><<<B * cp.blocks_per_unit, kCombineThreads, 0, stream>>>(cp);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

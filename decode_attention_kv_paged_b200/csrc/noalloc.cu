@@ -143,6 +143,7 @@ extern "C" int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
     cp.ws_lse = kp.ws_lse; cp.out = out;
     cp.B = B; cp.H_q = H_q; cp.H_kv = H_kv; cp.group = G; cp.n_hc = n_hc;
     cp.max_blocks = max_blocks_per_seq; cp.window = kp.window; cp.num_ctas = P;
+    cp.copies = 1;
     L.units_total = (int)units_total;
     L.stream = (cudaStream_t)stream;
     L.ev_start = nullptr;

@@ -305,6 +305,9 @@ PATH_CASES = [
     (24, 4, 256, [999, 4097], 700),       # G=6 + window
     (32, 4, 128, [2000, 130], 0),         # G=8
     (32, 1, 128, [1500, 63, 64], 0),      # MQA G=32
+    (16, 1, 128, [333, 2050, 17], 50),    # G=16: four head copies, window
+    (24, 1, 128, [1200, 40], 0),          # G=24: two copies, padded rows
+    (48, 1, 64, [900, 129], 0),           # G=48: one copy, padded rows
     (64, 1, 64, [800, 257], 100),         # G=64 + window
     (128, 1, 128, [520, 77], 0),          # G=128: two 64-head passes
 ]
