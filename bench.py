@@ -373,7 +373,9 @@ def run_native(args, rank, world, local):  # noqa: C901
         "kv_frac_of_peak": kv_gbs / world / pk["hbm_gbs"],
         "kv_frac_of_8tbs_spec": kv_gbs / world / 8000.0,
         "roofline": roof,
-        "gpu_launches": (1 if is_mla else 2) * K,
+        # main kernel per step, plus the combine kernel on the tensor-core
+        # paths (the CUDA-core GQA kernel combines its splits itself)
+        "gpu_launches": (1 if kernel == "gqa_split_kernel" else 2) * K,
         "clocks": clk.summary(),
     }
     if not is_mla:

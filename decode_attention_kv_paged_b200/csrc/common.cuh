@@ -157,6 +157,12 @@ __device__ __forceinline__ void bulk_load(void *dst_smem, const void *src,
         : "memory");
 }
 
+// Prefetch `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes)
+                 : "memory");
+}
+
 // L2 policy for data read exactly once (the streamed KV cache).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t policy;

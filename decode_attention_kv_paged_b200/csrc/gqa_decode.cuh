@@ -912,69 +912,90 @@ struct CombineParams {
     int B, H_q, H_kv, group, n_hc, max_blocks, window, num_ctas;
     int D, HC;               // head dim, query heads per unit
     int copies;              // partials per (unit, CTA) slot (>= 1)
-    int blocks_per_unit;     // CTAs of kCombineThreads per unit
+    int lanes;               // threads per float4 of output: 1, 4 or 8
+    int blocks_per_unit;     // CTAs per unit: combine_blocks_per_unit(HC, D, lanes)
 };
 
 constexpr int kCombineThreads = 256;
+constexpr int kCombineMaxW = 4096;       // (head, partial) weights held in shared memory
+
+// Threads that share one float4 of output in the combine: more when a unit
+// has many partials (each takes every lanes-th partial), one when it has few.
+__host__ __device__ constexpr int combine_lanes(int expected_partials) {
+    return expected_partials >= 32 ? 8 : (expected_partials >= 8 ? 4 : 1);
+}
+// CTAs of the combine kernel per unit.
+__host__ __device__ constexpr int combine_blocks_per_unit(int HC, int D, int lanes) {
+    return (HC * D + 4 * (kCombineThreads / lanes) - 1) / (4 * (kCombineThreads / lanes));
+}
 
 // out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L) over the unit's split
 // partials (`copies` per slot, slot-major), in CTA order (fixed,
-// deterministic).  A partial with lse = -inf has weight zero.  Each thread produces four
-// consecutive outputs of one head; a unit's HC*D outputs are spread over
-// blocks_per_unit CTAs.
+// deterministic).  A partial with lse = -inf has weight zero.  A CTA makes
+// 4 * kCombineThreads / lanes consecutive outputs of one unit: the split
+// weights of the heads it spans are computed once, in shared memory (one
+// warp per head), then each float4 of output is accumulated by `lanes`
+// threads that take every lanes-th partial, summed with shuffles in a fixed
+// order (deterministic).
 template <typename T>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const CombineParams p) {
-    __shared__ long long s_first_slot;
-    __shared__ int s_nsplit, s_nb;
+    __shared__ long long s_first;
+    __shared__ int s_n, s_nb;
+    __shared__ float s_w[kCombineMaxW];
+    __shared__ float s_inv[kCombineThreads / 4];
     pdl_wait_primary();
     const int units = p.H_kv * p.n_hc;
     const int u = blockIdx.x / p.blocks_per_unit;
     const int part = blockIdx.x % p.blocks_per_unit;
     const int b = u / units, rem = u % units;
-    if (threadIdx.x == 0) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
         int fb;
         bool bad;
         const int nb = visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad);
         s_nb = nb;
-        s_nsplit = 0;
-        s_first_slot = 0;
+        s_n = 0;
+        s_first = 0;
         if (nb > 0) {
             const long long W = p.ws_prefix[p.B];
             const int P = working_ctas(W, p.num_ctas);
             const long long s_u = p.ws_prefix[b] + (long long)rem * nb;
             const int c0 = cta_of(s_u, W, P);
             const int c1 = cta_of(s_u + nb - 1, W, P);
-            s_nsplit = (c1 - c0 + 1) * p.copies;
-            s_first_slot = ((long long)u + c0) * p.copies;
+            s_n = (c1 - c0 + 1) * p.copies;
+            s_first = ((long long)u + c0) * p.copies;
         }
     }
     __syncthreads();
-    const int e = (part * kCombineThreads + threadIdx.x) * 4;   // output index in unit
-    if (e >= p.HC * p.D) return;
-    const int g = e / p.D, k = e % p.D;
+    const int lanes = p.lanes;
+    const int outs = 4 * (kCombineThreads / lanes);      // outputs of this CTA
+    const int total = p.HC * p.D;
+    const int e0 = part * outs;
+    const int g0 = e0 / p.D;
+    const int e_last = (e0 + outs < total ? e0 + outs : total) - 1;
+    const int nh = e_last / p.D - g0 + 1;                // heads spanned
     const int kvh = rem / p.n_hc, hc = rem % p.n_hc;
     T *out = static_cast<T *>(p.out) +
-             ((size_t)b * p.H_q + kvh * p.group + hc * p.HC + g) * p.D + k;
-    float r[4];
-    const int ns = s_nsplit;
-    if (s_nb == 0) {
-        r[0] = r[1] = r[2] = r[3] = 0.f;
-    } else {
-        const long long s0 = s_first_slot;
-        if (ns == 1) {
-            const float4 v = *reinterpret_cast<const float4 *>(
-                p.ws_o + ((size_t)s0 * p.HC + g) * p.D + k);
-            r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
-        } else {
+             ((size_t)b * p.H_q + kvh * p.group + hc * p.HC) * p.D;
+    const int n = s_n;
+    const long long s0 = s_first;
+    const int o = tid / lanes, j = tid % lanes;
+    const int e = e0 + 4 * o;                            // this thread's float4
+    const bool has = e < total;
+    const int g = has ? e / p.D : g0;
+    if (s_nb == 0 || nh * n > kCombineMaxW || nh > kCombineThreads / 4) {
+        // Empty sequence: zeros.  More weights than fit: plain two-pass loop.
+        if (!has || j != 0) return;
+        float r[4] = {0.f, 0.f, 0.f, 0.f};
+        if (s_nb > 0) {
             float L = kNegInf;
-            for (int i = 0; i < ns; ++i) L = fmaxf(L, p.ws_lse[(s0 + i) * p.HC + g]);
+            for (int i = 0; i < n; ++i) L = fmaxf(L, p.ws_lse[(s0 + i) * p.HC + g]);
             float den = 0.f;
-            r[0] = r[1] = r[2] = r[3] = 0.f;
-            for (int i = 0; i < ns; ++i) {
+            for (int i = 0; i < n; ++i) {
                 const float w = exp2f(p.ws_lse[(s0 + i) * p.HC + g] - L);
                 const float4 v = *reinterpret_cast<const float4 *>(
-                    p.ws_o + ((size_t)(s0 + i) * p.HC + g) * p.D + k);
+                    p.ws_o + ((s0 + i) * p.HC + g) * p.D + (e % p.D));
                 r[0] = fmaf(w, v.x, r[0]);
                 r[1] = fmaf(w, v.y, r[1]);
                 r[2] = fmaf(w, v.z, r[2]);
@@ -982,11 +1003,65 @@ combine_kernel(const CombineParams p) {
                 den += w;
             }
             const float inv = 1.f / den;
-            r[0] *= inv; r[1] *= inv; r[2] *= inv; r[3] *= inv;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) r[q] *= inv;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) out[e + q] = ElemTraits<T>::from_float(r[q]);
+        return;
+    }
+    // Split weights of heads g0 .. g0 + nh - 1 ([head][partial]), one warp
+    // per head.
+    for (int hh = warp; hh < nh; hh += kCombineThreads / 32) {
+        const int gh = g0 + hh;
+        float *w_h = s_w + hh * n;
+        float L = kNegInf;
+        for (int i = lane; i < n; i += 32) {
+            const float v = p.ws_lse[(s0 + i) * p.HC + gh];
+            w_h[i] = v;
+            L = fmaxf(L, v);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, m));
+        float den = 0.f;
+        for (int i = lane; i < n; i += 32) {
+            const float w = exp2f(w_h[i] - L);
+            w_h[i] = w;
+            den += w;
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
+        if (lane == 0) s_inv[hh] = 1.f / den;
+    }
+    __syncthreads();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (has) {
+        const float *wts = s_w + (g - g0) * n;
+        const float *src = p.ws_o + (s0 * p.HC + g) * p.D + (e % p.D);
+        const size_t stride = (size_t)p.HC * p.D;
+#pragma unroll 4
+        for (int i = j; i < n; i += lanes) {
+            const float w = wts[i];
+            const float4 v = *reinterpret_cast<const float4 *>(src + (size_t)i * stride);
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
         }
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) out[j] = ElemTraits<T>::from_float(r[j]);
+    for (int m = lanes / 2; m >= 1; m >>= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+    }
+    if (has && j == 0) {
+        const float inv = s_inv[g - g0];
+        out[e] = ElemTraits<T>::from_float(acc.x * inv);
+        out[e + 1] = ElemTraits<T>::from_float(acc.y * inv);
+        out[e + 2] = ElemTraits<T>::from_float(acc.z * inv);
+        out[e + 3] = ElemTraits<T>::from_float(acc.w * inv);
+    }
 }
 
 }  // namespace attn

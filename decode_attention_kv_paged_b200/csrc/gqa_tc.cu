@@ -527,7 +527,10 @@ cudaError_t launch_tc(const GqaLaunch &L, int HC) {
     cp.D = D;
     cp.HC = HC;
     cp.copies = kTcM / TPC;
-    cp.blocks_per_unit = (HC * D / 4 + kCombineThreads - 1) / kCombineThreads;
+    // Partials per unit: about (CTAs / units + 1) splits, times the copies.
+    cp.lanes = combine_lanes((int)((kp.num_ctas / (L.units_total > 0 ? L.units_total : 1) + 1) *
+                                   cp.copies));
+    cp.blocks_per_unit = combine_blocks_per_unit(HC, D, cp.lanes);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((long long)L.units_total * cp.blocks_per_unit));
     cfg.blockDim = dim3(kCombineThreads);

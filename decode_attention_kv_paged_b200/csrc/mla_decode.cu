@@ -55,6 +55,7 @@ constexpr int kMlaDc = 512, kMlaDr = 64, kMlaWidth = 576;
 constexpr int kMlaCBox = 64 * 128;         // [64 tokens][64 cols] bf16
 constexpr int kMlaMaxBoxes = 5;
 constexpr int kMlaStages = 3;
+constexpr int kMlaPrefetch = 4;            // blocks pulled into L2 ahead of the ring
 constexpr int kMlaStageBytes = kMlaMaxBoxes * kMlaCBox;
 constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA, 4-11 softmax
 constexpr int kSoftThreads = 256;
@@ -91,6 +92,7 @@ static_assert(kTmemQ + 32 * kMlaMaxBoxes <= kTmemCols, "TMEM columns");
 struct MlaParams {
     const __nv_bfloat16 *q_lat;    // [B][128][512]
     const __nv_bfloat16 *q_rope;   // [B][128][64]
+    const __nv_bfloat16 *latent;   // [num_blocks][64][576]
     const int32_t *seq_lens;
     const int32_t *block_table;
     float *ws_o;          // [slots][128][512]
@@ -170,8 +172,23 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             tma_prefetch_map(&tm_c);
             TileCursor cur;
             cur.init(pa, lo, hi, first_seq, first_base);
+            // Rank 0 also pulls whole blocks (all 576 columns, contiguous)
+            // into L2 kMlaPrefetch tiles ahead, so the ring's loads of both
+            // CTAs are served from L2 rather than waiting on HBM.
+            TileCursor pf;
+            pf.init(pa, lo, hi, first_seq, first_base);
+            auto prefetch_next = [&]() {
+                if (rank != 0 || pf.done()) return;
+                const int pb = p.block_table[(size_t)pf.w.b * p.max_blocks + pf.logical_block()];
+                if (pb >= 0 && pb < p.num_blocks)
+                    bulk_prefetch_l2(p.latent + (size_t)pb * 64 * kMlaWidth,
+                                     64 * kMlaWidth * (uint32_t)sizeof(__nv_bfloat16));
+                pf.next();
+            };
+            for (int k = 0; k < kMlaPrefetch; ++k) prefetch_next();
             int tile = 0;
             while (!cur.done()) {
+                prefetch_next();
                 const int st = tile % kMlaStages;
                 if (tile >= kMlaStages &&
                     !mbar_wait(&bars->c_empty[st],
@@ -635,6 +652,7 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     MlaParams mp{};
     mp.q_lat = static_cast<const __nv_bfloat16 *>(q_latent);
     mp.q_rope = static_cast<const __nv_bfloat16 *>(q_rope);
+    mp.latent = static_cast<const __nv_bfloat16 *>(latent_cache);
     mp.seq_lens = seq_lens;
     mp.block_table = block_table;
     mp.ws_o = reinterpret_cast<float *>(w);
@@ -682,7 +700,8 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     cp.D = kMlaDc;
     cp.HC = kMlaH;
     cp.copies = 1;
-    cp.blocks_per_unit = kMlaH * kMlaDc / 4 / kCombineThreads;
+    cp.lanes = combine_lanes(clusters / B + 1);
+    cp.blocks_per_unit = combine_blocks_per_unit(kMlaH, kMlaDc, cp.lanes);
     combine_kernel<__nv_bfloat16><<<B * cp.blocks_per_unit, kCombineThreads, 0, stream>>>(cp);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
