@@ -40,6 +40,10 @@ KERNEL_SOURCES = {
     "gqa_split_kernel": ["decode_attention_kv_paged_b200/csrc/gqa_decode.cuh",
                          "decode_attention_kv_paged_b200/csrc/plan.cuh",
                          "decode_attention_kv_paged_b200/csrc/common.cuh"],
+    "gqa_tc128_kernel": ["decode_attention_kv_paged_b200/csrc/gqa_tc128.cu",
+                         "decode_attention_kv_paged_b200/csrc/tc_common.cuh",
+                         "decode_attention_kv_paged_b200/csrc/plan.cuh",
+                         "decode_attention_kv_paged_b200/csrc/common.cuh"],
     "gqa_tc_kernel": ["decode_attention_kv_paged_b200/csrc/gqa_tc.cu",
                       "decode_attention_kv_paged_b200/csrc/tc_common.cuh",
                       "decode_attention_kv_paged_b200/csrc/plan.cuh",
@@ -333,7 +337,7 @@ def run_native(args, rank, world, local):  # noqa: C901
         kernel = "mla_decode_kernel"
     else:
         _, _, path = attn.gqa_config(cfg.B, cfg.H_q, cfg.H_kv, cfg.d, cfg.dtype)
-        kernel = "gqa_tc_kernel" if path == 1 else "gqa_split_kernel"
+        kernel = {0: "gqa_split_kernel", 1: "gqa_tc128_kernel", 2: "gqa_tc_kernel"}[path]
     if is_mla:
         flops = mla_flops(base)
         t_hbm = alg_bytes / (pk["hbm_gbs"] * 1e9)

@@ -219,7 +219,9 @@ def plan(seq_lens, units_per_seq, window, max_blocks, num_ctas, stream=None):
 
 
 def gqa_config(B, H_q, H_kv, d, dtype=torch.bfloat16):
-    """(num_ctas, heads_per_cta, path) the GQA call uses for this problem."""
+    """(num_ctas, heads_per_cta, path) the GQA call uses for this problem;
+    path 0 = CUDA-core kernel, 1 = M=128 tensor-core kernel, 2 = M=64
+    tensor-core kernel."""
     n, h, pth = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     rc = load().attn_decode_gqa_config(B, H_q, H_kv, d, _dtype_code(dtype),
                                        ctypes.byref(n), ctypes.byref(h),
@@ -233,6 +235,8 @@ def set_num_ctas(n):
 
 
 def set_gqa_path(path):
+    """-1 automatic, 0 CUDA cores, 1 tensor cores (best kernel), 2 the M=64
+    tensor-core kernel (testing/tuning hook)."""
     _check(load().attn_set_gqa_path(int(path)), "attn_set_gqa_path")
 
 

@@ -118,8 +118,15 @@ static bool valid_head_dim(int d) {
 static bool use_tc_path(int G, int d, int dtype) {
     const bool ok = gqa_tc_supported(d, dtype == ATTN_BF16, G);
     if (tl_gqa_path == 0) return false;
-    if (tl_gqa_path == 1) return ok;
+    if (tl_gqa_path >= 1) return ok;
     return ok && G >= kTcMinGroup;
+}
+
+// Which tensor-core kernel runs a unit of HC heads: the M = 128 one (Q and P
+// in tensor memory) where it applies, else the M = 64 one; the testing hook
+// path 2 forces the M = 64 kernel.
+static bool use_tc128(int d, int HC) {
+    return tl_gqa_path != 2 && gqa_tc128_supported(d, HC);
 }
 
 // Query heads per CTA for a group of G: the largest instantiated divisor.
@@ -183,7 +190,7 @@ int attn_set_num_ctas(int n) {
 }
 
 int attn_set_gqa_path(int path) {
-    if (path < -1 || path > 1) return ATTN_ERR_ARG;
+    if (path < -1 || path > 2) return ATTN_ERR_ARG;
     tl_gqa_path = path;
     return ATTN_OK;
 }
@@ -234,8 +241,9 @@ int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype, int *num_
     const int G = H_q / H_kv;
     const bool tc = use_tc_path(G, d, dtype);
     if (num_ctas) *num_ctas = tl_num_ctas > 0 ? tl_num_ctas : st->num_sms;
-    if (heads) *heads = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
-    if (path) *path = tc ? 1 : 0;
+    const int hc = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
+    if (heads) *heads = hc;
+    if (path) *path = tc ? (use_tc128(d, hc) ? 1 : 2) : 0;
     return ATTN_OK;
 }
 
@@ -271,8 +279,9 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     if (units_total > (1ll << 30)) return ATTN_ERR_ARG;
     const long long slots = units_total + P;
 
-    // The tensor-core kernel writes gqa_tc_copies(HC) partials per slot.
-    const int copies = tc ? gqa_tc_copies(HC) : 1;
+    // The tensor-core kernels write one partial per head-group copy per slot.
+    const bool tc128 = tc && use_tc128(d, HC);
+    const int copies = tc ? (tc128 ? gqa_tc128_copies(HC) : gqa_tc_copies(HC)) : 1;
     const size_t o_bytes = align256((size_t)slots * copies * HC * d * sizeof(float));
     const size_t lse_bytes = align256((size_t)slots * copies * HC * sizeof(float));
     const size_t pre_bytes = align256((size_t)(B + 1) * sizeof(long long));
@@ -313,7 +322,7 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     const int bf16 = dtype == ATTN_BF16;
     cudaError_t e;
     if (tc) {
-        e = launch_gqa_tc(L, d, HC);
+        e = tc128 ? launch_gqa_tc128(L, d, HC) : launch_gqa_tc(L, d, HC);
         return cuda_status(e);
     }
     switch (d) {

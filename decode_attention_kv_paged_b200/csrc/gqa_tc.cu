@@ -465,8 +465,6 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 // -------------------------------------------------------------- host side
-namespace {
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave,
@@ -500,6 +498,8 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int D, int TPC>
 cudaError_t launch_tc(const GqaLaunch &L, int HC) {

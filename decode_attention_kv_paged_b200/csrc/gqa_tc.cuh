@@ -1,6 +1,8 @@
 // gqa_tc.cuh -- host entry of the tensor-core (tcgen05) GQA/MQA decode path.
 #pragma once
 
+#include <cuda.h>
+
 #include "gqa_launch.cuh"
 
 namespace attn {
@@ -16,5 +18,17 @@ int gqa_tc_copies(int HC);
 constexpr int kTcMinGroup = 8;
 
 cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC);
+
+// The M = 128 tensor-core kernel (query and P in tensor memory): d in
+// {64, 128} and units of at most 32 heads; it writes gqa_tc128_copies(HC)
+// partials per (unit, CTA) slot.
+bool gqa_tc128_supported(int d, int HC);
+int gqa_tc128_copies(int HC);
+cudaError_t launch_gqa_tc128(const GqaLaunch &L, int d, int HC);
+
+// 2-D tensor map over a row-major bf16 matrix [rows][cols] with 64-column,
+// box_rows-row boxes and 128-byte swizzle.
+bool tc_make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                 uint32_t box_rows);
 
 }  // namespace attn

@@ -159,7 +159,8 @@ int attn_decode_plan(const int32_t *seq_lens, int B, int units_per_seq,
  * problem: *num_ctas = CTAs of the split-KV kernel, *heads_per_cta = query
  * heads a CTA processes per KV head (the group is split into
  * H_q / H_kv / heads_per_cta chunks when it does not fit), *path = 0 for the
- * CUDA-core kernel, 1 for the tensor-core (tcgen05) kernel.
+ * CUDA-core kernel, 1 for the M = 128 tensor-core (tcgen05) kernel, 2 for
+ * the M = 64 tensor-core kernel.
  */
 int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype,
                            int *num_ctas, int *heads_per_cta, int *path);
@@ -172,7 +173,9 @@ int attn_set_num_ctas(int num_ctas);
 
 /*
  * attn_set_gqa_path -- testing/tuning hook: -1 = automatic, 0 = force the
- * CUDA-core kernel, 1 = force the tensor-core kernel where it is supported.
+ * CUDA-core kernel, 1 = force the tensor-core path where it is supported (the
+ * M = 128 kernel for d <= 128 and units of <= 32 heads, else the M = 64
+ * kernel), 2 = force the M = 64 tensor-core kernel.
  */
 int attn_set_gqa_path(int path);
 
