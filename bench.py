@@ -384,11 +384,40 @@ def run_native(args, rank, world, local):  # noqa: C901
     }
     if not is_mla:
         line["tile_overread_bytes_per_step"] = tile_bytes_gqa(base) - kv_bytes
+    if is_mla:
+        line["mla_absorb"] = mla_absorb_timing(attn, cfg, dev, rank_seed(cfg.seed, rank))
     if not args.no_e2e:
         line["e2e"] = e2e_native(attn, cfg, inputs[0], is_mla, K, world, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(cfg, is_mla, args.cpu_seconds)
     return line
+
+
+def mla_absorb_timing(attn, cfg, dev, seed, iters=20):
+    """Device time of the products either side of the absorbed decode at this
+    shape (q_c (U^K)^T before, z U^V after), per call; they stream the
+    per-head weights (H x d_c x 128 bf16 each) once per call."""
+    w = W.make_mla_absorb_inputs(cfg, device=dev, seed=seed)
+    z = torch.empty((cfg.B, cfg.H, cfg.d_c), dtype=torch.bfloat16, device=dev).normal_()
+    out = {}
+    for name, fn in (("absorb_q", lambda: attn.mla_absorb_q(w.q_c, w.U_K)),
+                     ("project_out", lambda: attn.mla_project_out(z, w.U_V))):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name + "_us"] = e0.elapsed_time(e1) * 1e3 / iters
+    wbytes = cfg.H * cfg.d_c * 128 * 2
+    out["weight_bytes_each"] = wbytes
+    out["absorb_q_gbs"] = wbytes / (out["absorb_q_us"] * 1e-6) / 1e9
+    out["project_out_gbs"] = wbytes / (out["project_out_us"] * 1e-6) / 1e9
+    return out
 
 
 def e2e_native(attn, cfg, x, is_mla, K, world, dev):

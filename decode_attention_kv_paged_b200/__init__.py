@@ -28,6 +28,7 @@ C_SYMBOLS = (
     "attn_set_gqa_path", "attn_set_profile_events",
     "attn_debug_force_timeout", "attn_decode_last_error",
     "attn_status_string", "attn_version", "attn_decode_gqa_noalloc",
+    "attn_mla_absorb_q", "attn_mla_project_out",
 )
 
 _lib = None
@@ -55,6 +56,8 @@ def load():
     lib.attn_decode_gqa.argtypes = [p] * 6 + [i] * 4 + [f, i, p, i, i, i]
     lib.attn_decode_mla.argtypes = [p] * 6 + [i] * 4 + [f, p, i, i]
     lib.attn_decode_gqa_noalloc.argtypes = lib.attn_decode_gqa.argtypes
+    lib.attn_mla_absorb_q.argtypes = [p] * 3 + [i] * 4 + [p]
+    lib.attn_mla_project_out.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.kv_append.argtypes = [p] * 6 + [i] * 6 + [p]
     lib.kv_append_mla.argtypes = [p] * 4 + [i] * 5 + [p]
     lib.attn_decode_plan.argtypes = [p, i, i, i, i, i, p, p]
@@ -175,6 +178,38 @@ def decode_mla(q_latent, q_rope, latent_cache, seq_lens, block_table, scale,
         B, H, d_c, d_r, float(scale), _stream_ptr(stream), block_table.shape[1],
         nblk)
     _check(rc, "attn_decode_mla")
+    return out
+
+
+def mla_absorb_q(q_c, u_k, out=None, stream=None):
+    """q_latent [B][H][d_c] = q_c (U^K_h)^T per head (bf16).
+
+    q_c [B][H][d_h]; u_k [H][d_c][d_h]."""
+    B, H, d_h = q_c.shape
+    d_c = u_k.shape[1]
+    if tuple(u_k.shape) != (H, d_c, d_h):
+        raise ValueError("u_k must be [H][d_c][d_h]")
+    bf = torch.bfloat16
+    if out is None:
+        out = torch.empty((B, H, d_c), dtype=bf, device=q_c.device)
+    _check(load().attn_mla_absorb_q(_dev(q_c, "q_c", bf), _dev(u_k, "u_k", bf),
+                                    _dev(out, "out", bf), B, H, d_c, d_h,
+                                    _stream_ptr(stream)), "attn_mla_absorb_q")
+    return out
+
+
+def mla_project_out(z, u_v, out=None, stream=None):
+    """o [B][H][d_v] = z U^V_h per head (bf16).  z [B][H][d_c]; u_v [H][d_c][d_v]."""
+    B, H, d_c = z.shape
+    d_v = u_v.shape[2]
+    if tuple(u_v.shape) != (H, d_c, d_v):
+        raise ValueError("u_v must be [H][d_c][d_v]")
+    bf = torch.bfloat16
+    if out is None:
+        out = torch.empty((B, H, d_v), dtype=bf, device=z.device)
+    _check(load().attn_mla_project_out(_dev(z, "z", bf), _dev(u_v, "u_v", bf),
+                                       _dev(out, "out", bf), B, H, d_c, d_v,
+                                       _stream_ptr(stream)), "attn_mla_project_out")
     return out
 
 

@@ -241,6 +241,32 @@ int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
                             void *stream, int max_blocks_per_seq,
                             int num_blocks, int dtype);
 
+/*
+ * attn_mla_absorb_q -- the key up-projection folded into the query, before
+ * the absorbed MLA decode (attention-head §5.2): per sequence b and head h,
+ *     q_latent[b][h][:] = sum_i q_c[b][h][i] * u_k[h][:][i]
+ * i.e. q_c (U^K_h)^T with k^C_j = c_j U^K_h.  q_c [B][H][d_h], u_k
+ * [H][d_c][d_h], q_latent [B][H][d_c] (the q_latent input of
+ * attn_decode_mla); all bf16, device, 16-byte aligned, row-major; fp32
+ * accumulation, result rounded to bf16.  d_c and d_h multiples of 8
+ * (ATTN_ERR_UNSUPPORTED otherwise).  Stream-ordered; a plain batched GEMM
+ * over the heads (cuBLAS).
+ */
+int attn_mla_absorb_q(const void *q_c, const void *u_k, void *q_latent, int B, int H,
+                      int d_c, int d_h, void *stream);
+
+/*
+ * attn_mla_project_out -- the value up-projection after the absorbed MLA
+ * decode (attention-head §5.2): per sequence b and head h,
+ *     o[b][h][:] = sum_c z[b][h][c] * u_v[h][c][:]
+ * i.e. z U^V_h with v_j = c_j U^V_h.  z [B][H][d_c] (the output of
+ * attn_decode_mla), u_v [H][d_c][d_v], o [B][H][d_v]; bf16, device, 16-byte
+ * aligned, row-major; fp32 accumulation, result rounded to bf16.  d_c and
+ * d_v multiples of 8.  Stream-ordered; a plain batched GEMM (cuBLAS).
+ */
+int attn_mla_project_out(const void *z, const void *u_v, void *o, int B, int H, int d_c,
+                         int d_v, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *attn_status_string(int status);
 

@@ -173,6 +173,30 @@ def mla_explicit(q_c, q_rope, latent_cache, seq_lens, block_table, U_K, U_V,
     return out
 
 
+def mla_absorb_q(q_c, U_K):
+    """q_latent [B][H][d_c] (fp64) = q^C_h (U^K_h)^T per head: the key
+    up-projection folded into the query (attention-head §5.2, absorption).
+
+    q_c [B][H][d_h]; U_K [H][d_c][d_h] (k^C_j = c_j U^K_h).  A plain batched
+    product; pinned by the absorbed == explicit invariant.
+    """
+    q_c = np.asarray(q_c, dtype=np.float64)
+    U_K = np.asarray(U_K, dtype=np.float64)
+    return np.einsum("bhi,hci->bhc", q_c, U_K)
+
+
+def mla_project_out(z, U_V):
+    """o [B][H][d_v] (fp64) = z_h U^V_h per head: the value up-projection
+    applied after the attention in latent space (attention-head §5.2).
+
+    z [B][H][d_c]; U_V [H][d_c][d_v].  A plain batched product; pinned by the
+    absorbed == explicit invariant.
+    """
+    z = np.asarray(z, dtype=np.float64)
+    U_V = np.asarray(U_V, dtype=np.float64)
+    return np.einsum("bhc,hcv->bhv", z, U_V)
+
+
 def bytes_kv(B, T, H_kv, d, s):
     return _load().orc_bytes_kv(float(B), float(T), float(H_kv), float(d),
                                 float(s))

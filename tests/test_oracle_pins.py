@@ -329,9 +329,9 @@ def test_mla_absorbed_equals_explicit(d_r):
     scale = 1.0 / math.sqrt(d_h + d_r)
     o_explicit = orc.mla_explicit(q_c, q_r, cache, lens, table, U_K, U_V,
                                   scale)
-    q_tilde = np.einsum("bhi,hci->bhc", q_c, U_K)     # q^C (U^K_h)^T
+    q_tilde = orc.mla_absorb_q(q_c, U_K)              # q^C (U^K_h)^T
     z = orc.decode_mla(q_tilde, q_r, cache, lens, table, scale)
-    o_absorbed = np.einsum("bhc,hcv->bhv", z, U_V)    # z U^V_h
+    o_absorbed = orc.mla_project_out(z, U_V)          # z U^V_h
     np.testing.assert_allclose(o_absorbed, o_explicit, rtol=0, atol=1e-12)
 
 

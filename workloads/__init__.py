@@ -215,3 +215,27 @@ def make_mla_inputs(cfg: MLAConfig, device="cpu", seed: Optional[int] = None,
     sl = torch.tensor(seq, dtype=torch.int32, device=g.device)
     return MLAInputs(cfg, q_lat, q_rope, cache, sl, table, nblk, cfg.scale,
                      seq)
+
+
+@dataclass
+class MLAAbsorbInputs:
+    q_c: torch.Tensor     # [B][H][d_h] per-head content query (before absorption)
+    U_K: torch.Tensor     # [H][d_c][d_h] key up-projection, k^C_j = c_j U^K_h
+    U_V: torch.Tensor     # [H][d_c][d_v] value up-projection, v_j = c_j U^V_h
+
+    def to(self, device):
+        return MLAAbsorbInputs(self.q_c.to(device), self.U_K.to(device), self.U_V.to(device))
+
+
+def make_mla_absorb_inputs(cfg: MLAConfig, d_h=128, d_v=128, device="cpu",
+                           seed: Optional[int] = None) -> MLAAbsorbInputs:
+    """Random stand-ins for the per-head projections on either side of the
+    absorbed decode (no trained weights exist here): q_c ~ N(0,1), U^K ~
+    N(0,1)/(2 sqrt(d_h)) (q_c (U^K)^T has standard deviation 1/2, so even its
+    extremes over a full batch stay below ~2.5, where bf16 storage keeps the
+    1e-2 max-abs bar), U^V ~ N(0,1)/sqrt(d_c); bf16 like the cache."""
+    g = _generator((cfg.seed if seed is None else seed) + 7919, device)
+    q_c = randn((cfg.B, cfg.H, d_h), g, cfg.dtype, 1.0)
+    U_K = randn((cfg.H, cfg.d_c, d_h), g, cfg.dtype, 0.5 / math.sqrt(d_h))
+    U_V = randn((cfg.H, cfg.d_c, d_v), g, cfg.dtype, 1.0 / math.sqrt(cfg.d_c))
+    return MLAAbsorbInputs(q_c, U_K, U_V)
