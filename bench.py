@@ -59,6 +59,8 @@ WORKLOAD_ALIASES = {
     "tiny": W.TINY.name,
     "ragged_full": W.RAGGED_FULL.name,
     "ragged_window": W.RAGGED_WINDOW.name,
+    "ragged_window_sink": W.RAGGED_WINDOW_SINK.name,
+    "ragged_window_ring": W.RAGGED_WINDOW_RING.name,
     "mla": W.MLA_DSV2.name,
 }
 
@@ -70,7 +72,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="llama3_8b",
-                    help="llama3_8b | tiny | ragged_full | ragged_window | mla "
+                    help="llama3_8b | tiny | ragged_full | ragged_window | "
+                         "ragged_window_sink | ragged_window_ring | mla "
                          "| a sweep name such as sweep_bf16_B8_Hq32_Hkv8_d128_T32768")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true",
@@ -225,14 +228,32 @@ def whole_job_tokens_per_s(world, batch, steps, ms_max):
 
 
 # --------------------------------------------------------------- helpers
+def visible_keys(T, window, sink):
+    """Keys a decode query of a sequence with T cached tokens sees: the window
+    [T - window, T) (all of [0, T) without one) plus the first `sink`."""
+    if T <= 0:
+        return 0
+    lo = max(0, T - window) if window > 0 else 0
+    return T - lo + min(sink, lo)
+
+
+def visible_tiles(T, window, sink):
+    """64-token blocks holding at least one visible key."""
+    if T <= 0:
+        return 0
+    lo = max(0, T - window) if window > 0 else 0
+    w0, w1 = lo // 64, (T - 1) // 64 + 1
+    a = min((sink + 63) // 64, w1)
+    return w1 if a >= w0 else a + w1 - w0
+
+
 def algorithmic_bytes_gqa(inp):
     """K+V bytes of visible keys (both caches) + q + out."""
     cfg = inp.cfg
     s = torch.finfo(cfg.dtype).bits // 8
     vis = 0
     for T in inp.seq_list:
-        lo = max(0, T - inp.window) if inp.window > 0 else 0
-        vis += max(0, T - lo)
+        vis += visible_keys(T, inp.window, cfg.sink)
     kv = vis * cfg.H_kv * cfg.d * 2 * s
     qo = 2 * cfg.B * cfg.H_q * cfg.d * s
     return kv, kv + qo
@@ -244,10 +265,7 @@ def tile_bytes_gqa(inp):
     s = torch.finfo(cfg.dtype).bits // 8
     blocks = 0
     for T in inp.seq_list:
-        if T <= 0:
-            continue
-        lo = max(0, T - inp.window) if inp.window > 0 else 0
-        blocks += (T - 1) // 64 - lo // 64 + 1
+        blocks += visible_tiles(T, inp.window, cfg.sink)
     return blocks * 64 * cfg.H_kv * cfg.d * 2 * s
 
 
@@ -298,8 +316,9 @@ def run_native(args, rank, world, local):  # noqa: C901
             attn.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
                             x.block_table, x.scale, out=outs[i % reps])
         else:
-            attn.decode_gqa(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                            x.scale, window=x.window, out=outs[i % reps])
+            attn.decode_gqa_ext(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                                x.scale, window=x.window, sink_tokens=cfg.sink,
+                                ring_blocks=cfg.ring, out=outs[i % reps])
 
     for i in range(max(args.warmup, 3)):
         step(i)
@@ -457,9 +476,11 @@ def e2e_native(attn, cfg, x, is_mla, K, world, dev):
         else:
             d_k.copy_(h_k, non_blocking=True)
             d_v.copy_(h_v, non_blocking=True)
-            attn.kv_append(d_k, d_v, x.k_cache, x.v_cache, pos, x.block_table)
-            attn.decode_gqa(d_q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                            x.scale, window=x.window, out=d_out)
+            attn.kv_append_ext(d_k, d_v, x.k_cache, x.v_cache, pos, x.block_table,
+                               window=x.window, sink_tokens=cfg.sink, ring_blocks=cfg.ring)
+            attn.decode_gqa_ext(d_q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                                x.scale, window=x.window, sink_tokens=cfg.sink,
+                                ring_blocks=cfg.ring, out=d_out)
         h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(3):
@@ -496,7 +517,7 @@ def _oracle_problem(cfg, is_mla, seqs, seed):
         lens = W.draw_seq_lens(cfg, g)[:seqs]
     sub = W.GQAConfig(cfg.name, B=seqs, H_q=cfg.H_q, H_kv=cfg.H_kv, d=cfg.d,
                       seq_lens=lens, T=cfg.T, dtype=cfg.dtype, window=cfg.window,
-                      contiguous=cfg.contiguous, seed=seed)
+                      sink=cfg.sink, ring=cfg.ring, contiguous=cfg.contiguous, seed=seed)
     return W.make_gqa_inputs(sub)
 
 
@@ -504,8 +525,8 @@ def _oracle_call(orc, x, is_mla):
     if is_mla:
         return orc.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
                               x.block_table, x.scale)
-    return orc.decode_gqa(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                          x.scale, window=x.window)
+    return orc.decode_gqa_vis(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                              x.scale, window=x.window, sink=x.cfg.sink, ring=x.cfg.ring)
 
 
 def _pick_sample(cfg, is_mla, orc, target_s):

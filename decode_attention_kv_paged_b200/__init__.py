@@ -28,8 +28,14 @@ C_SYMBOLS = (
     "attn_set_gqa_path", "attn_set_profile_events",
     "attn_debug_force_timeout", "attn_decode_last_error",
     "attn_status_string", "attn_version", "attn_decode_gqa_noalloc",
-    "attn_mla_absorb_q", "attn_mla_project_out",
+    "attn_mla_absorb_q", "attn_mla_project_out", "attn_decode_gqa_ext", "kv_append_ext",
 )
+
+
+class Visibility(ctypes.Structure):
+    """attn_visibility: window, global (sink) tokens, ring table (blocks)."""
+    _fields_ = [("window", ctypes.c_int), ("sink_tokens", ctypes.c_int),
+                ("ring_blocks", ctypes.c_int)]
 
 _lib = None
 
@@ -56,6 +62,9 @@ def load():
     lib.attn_decode_gqa.argtypes = [p] * 6 + [i] * 4 + [f, i, p, i, i, i]
     lib.attn_decode_mla.argtypes = [p] * 6 + [i] * 4 + [f, p, i, i]
     lib.attn_decode_gqa_noalloc.argtypes = lib.attn_decode_gqa.argtypes
+    lib.attn_decode_gqa_ext.argtypes = ([p] * 6 + [i] * 4 +
+                                        [f, ctypes.POINTER(Visibility), p, i, i, i])
+    lib.kv_append_ext.argtypes = [p] * 6 + [i] * 6 + [ctypes.POINTER(Visibility), p]
     lib.attn_mla_absorb_q.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.attn_mla_project_out.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.kv_append.argtypes = [p] * 6 + [i] * 6 + [p]
@@ -129,6 +138,30 @@ def decode_gqa(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
         B, H_q, H_kv, d, float(scale), int(window), _stream_ptr(stream),
         block_table.shape[1], nblk, dt)
     _check(rc, "attn_decode_gqa")
+    return out
+
+
+def decode_gqa_ext(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
+                   sink_tokens=0, ring_blocks=0, out=None, stream=None):
+    """decode_gqa with global (sink) tokens and a ring-buffer block table:
+    key j < T is visible when window <= 0, j >= T - window or j < sink_tokens;
+    with ring_blocks > 0 logical block i lives in table slot i for the sink
+    blocks and in slot A + i % ring_blocks after them (A = ceil(sink / 64))."""
+    B, H_q, d = q.shape
+    nblk, H_kv, bs, d2 = k_cache.shape
+    if bs != BLOCK_SIZE or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("cache must be [num_blocks][H_kv][64][d] for K and V")
+    dt = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    rc = load().attn_decode_gqa_ext(
+        _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
+        _dev(v_cache, "v_cache", q.dtype), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(block_table, "block_table", torch.int32), _dev(out, "out", q.dtype),
+        B, H_q, H_kv, d, float(scale), ctypes.byref(vis), _stream_ptr(stream),
+        block_table.shape[1], nblk, dt)
+    _check(rc, "attn_decode_gqa_ext")
     return out
 
 
@@ -211,6 +244,23 @@ def mla_project_out(z, u_v, out=None, stream=None):
                                        _dev(out, "out", bf), B, H, d_c, d_v,
                                        _stream_ptr(stream)), "attn_mla_project_out")
     return out
+
+
+def kv_append_ext(k_new, v_new, k_cache, v_cache, positions, block_table,
+                  window=0, sink_tokens=0, ring_blocks=0, stream=None):
+    """kv_append through the table mapping of a visibility record (sink slots,
+    then the ring): with a ring, writing past the window overwrites the block
+    that left it."""
+    B, H_kv, d = k_new.shape
+    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    rc = load().kv_append_ext(
+        _dev(k_new, "k_new"), _dev(v_new, "v_new", k_new.dtype),
+        _dev(k_cache, "k_cache", k_new.dtype), _dev(v_cache, "v_cache", k_new.dtype),
+        _dev(positions, "positions", torch.int32),
+        _dev(block_table, "block_table", torch.int32), B, H_kv, d,
+        block_table.shape[1], k_cache.shape[0], _dtype_code(k_new.dtype),
+        ctypes.byref(vis), _stream_ptr(stream))
+    _check(rc, "kv_append_ext")
 
 
 def kv_append(k_new, v_new, k_cache, v_cache, positions, block_table,

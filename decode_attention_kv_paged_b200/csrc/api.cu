@@ -247,10 +247,11 @@ int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype, int *num_
     return ATTN_OK;
 }
 
-int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
-                    const int32_t *seq_lens, const int32_t *block_table, void *out,
-                    int B, int H_q, int H_kv, int d, float scale, int window,
-                    void *stream, int max_blocks_per_seq, int num_blocks, int dtype) {
+// Shared body of attn_decode_gqa and attn_decode_gqa_ext.
+static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *seq_lens, const int32_t *block_table, void *out,
+                           int B, int H_q, int H_kv, int d, float scale, Visibility vis,
+                           void *stream, int max_blocks_per_seq, int num_blocks, int dtype) {
     if (!q || !k_cache || !v_cache || !seq_lens || !block_table || !out) return ATTN_ERR_ARG;
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return ATTN_ERR_ARG;
     if (max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
@@ -307,13 +308,13 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
     kp.scale_log2 = scale * 1.4426950408889634f;
     kp.B = B; kp.H_q = H_q; kp.H_kv = H_kv; kp.group = G; kp.n_hc = n_hc;
     kp.max_blocks = max_blocks_per_seq; kp.num_blocks = num_blocks;
-    kp.window = window > 0 ? window : 0;
+    kp.vis = vis;
     kp.num_ctas = P;
     CombineParams &cp = L.cp;
     cp.seq_lens = seq_lens; cp.ws_prefix = kp.ws_prefix; cp.ws_o = kp.ws_o;
     cp.ws_lse = kp.ws_lse; cp.out = out;
     cp.B = B; cp.H_q = H_q; cp.H_kv = H_kv; cp.group = G; cp.n_hc = n_hc;
-    cp.max_blocks = max_blocks_per_seq; cp.window = kp.window; cp.num_ctas = P;
+    cp.max_blocks = max_blocks_per_seq; cp.vis = vis; cp.num_ctas = P;
     cp.copies = copies;
     L.units_total = (int)units_total;
     L.stream = s;
@@ -333,6 +334,44 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
         default: e = launch_gqa_d256(HC, bf16, L); break;
     }
     return cuda_status(e);
+}
+
+int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seq_lens, const int32_t *block_table, void *out,
+                    int B, int H_q, int H_kv, int d, float scale, int window,
+                    void *stream, int max_blocks_per_seq, int num_blocks, int dtype) {
+    return decode_gqa_impl(q, k_cache, v_cache, seq_lens, block_table, out, B, H_q, H_kv, d,
+                           scale, Visibility{window > 0 ? window : 0, 0, 0}, stream,
+                           max_blocks_per_seq, num_blocks, dtype);
+}
+
+// Validates a visibility record against the table width; fills `out`.
+static int check_visibility(const attn_visibility *v, int max_blocks_per_seq, Visibility *out) {
+    if (!v) return ATTN_ERR_ARG;
+    if (v->sink_tokens < 0 || v->ring_blocks < 0) return ATTN_ERR_ARG;
+    Visibility vis{v->window > 0 ? v->window : 0, v->sink_tokens, v->ring_blocks};
+    if (vis.ring > 0) {
+        // The ring must hold every block a window can reach, after the sink
+        // blocks, inside the table row.
+        if (vis.window <= 0) return ATTN_ERR_ARG;
+        if ((long long)vis.ring * kBlockSize < (long long)vis.window + kBlockSize - 1)
+            return ATTN_ERR_ARG;
+        if ((long long)sink_blocks(vis) + vis.ring > max_blocks_per_seq) return ATTN_ERR_ARG;
+    }
+    *out = vis;
+    return ATTN_OK;
+}
+
+int attn_decode_gqa_ext(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *seq_lens, const int32_t *block_table, void *out,
+                        int B, int H_q, int H_kv, int d, float scale,
+                        const attn_visibility *visibility, void *stream,
+                        int max_blocks_per_seq, int num_blocks, int dtype) {
+    Visibility vis;
+    const int rc = check_visibility(visibility, max_blocks_per_seq, &vis);
+    if (rc) return rc;
+    return decode_gqa_impl(q, k_cache, v_cache, seq_lens, block_table, out, B, H_q, H_kv, d,
+                           scale, vis, stream, max_blocks_per_seq, num_blocks, dtype);
 }
 
 int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent_cache,
@@ -364,9 +403,10 @@ int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent
                             ev_start, ev_stop);
 }
 
-int kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-              const int32_t *positions, const int32_t *block_table, int B, int H_kv, int d,
-              int max_blocks_per_seq, int num_blocks, int dtype, void *stream) {
+static int kv_append_impl(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                          const int32_t *positions, const int32_t *block_table, int B,
+                          int H_kv, int d, int max_blocks_per_seq, int num_blocks, int dtype,
+                          Visibility vis, void *stream) {
     if (!k_new || !v_new || !k_cache || !v_cache || !positions || !block_table)
         return ATTN_ERR_ARG;
     if (B <= 0 || H_kv <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
@@ -383,7 +423,26 @@ int kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache
     p.B = B; p.H_kv = H_kv;
     p.chunks_per_row = d * (dtype == ATTN_BF16 ? 2 : 4) / 16;
     p.max_blocks = max_blocks_per_seq; p.num_blocks = num_blocks;
+    p.vis = vis;
     return cuda_status(launch_kv_append(p, (cudaStream_t)stream));
+}
+
+int kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+              const int32_t *positions, const int32_t *block_table, int B, int H_kv, int d,
+              int max_blocks_per_seq, int num_blocks, int dtype, void *stream) {
+    return kv_append_impl(k_new, v_new, k_cache, v_cache, positions, block_table, B, H_kv, d,
+                          max_blocks_per_seq, num_blocks, dtype, Visibility{0, 0, 0}, stream);
+}
+
+int kv_append_ext(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                  const int32_t *positions, const int32_t *block_table, int B, int H_kv, int d,
+                  int max_blocks_per_seq, int num_blocks, int dtype,
+                  const attn_visibility *visibility, void *stream) {
+    Visibility vis;
+    const int rc = check_visibility(visibility, max_blocks_per_seq, &vis);
+    if (rc) return rc;
+    return kv_append_impl(k_new, v_new, k_cache, v_cache, positions, block_table, B, H_kv, d,
+                          max_blocks_per_seq, num_blocks, dtype, vis, stream);
 }
 
 int kv_append_mla(const void *latent_new, void *latent_cache, const int32_t *positions,
@@ -414,7 +473,8 @@ int attn_decode_plan(const int32_t *seq_lens, int B, int units_per_seq, int wind
     DeviceState *st;
     int rc = device_state(&st);
     if (rc) return rc;
-    return cuda_status(launch_plan_kernel(seq_lens, B, units_per_seq, window > 0 ? window : 0,
+    return cuda_status(launch_plan_kernel(seq_lens, B, units_per_seq,
+                                          Visibility{window > 0 ? window : 0, 0, 0},
                                           max_blocks_per_seq, num_ctas,
                                           reinterpret_cast<long long *>(plan_out), st->err,
                                           (cudaStream_t)stream));

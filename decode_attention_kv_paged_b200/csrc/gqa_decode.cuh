@@ -80,7 +80,8 @@ struct GqaParams {
     unsigned *err;
     unsigned long long timeout_ns;
     float scale_log2;     // scale * log2(e)
-    int B, H_q, H_kv, group, n_hc, max_blocks, num_blocks, window, num_ctas;
+    int B, H_q, H_kv, group, n_hc, max_blocks, num_blocks, num_ctas;
+    Visibility vis;       // window, sink (global) tokens, ring table
     int force_timeout;
 };
 
@@ -259,7 +260,7 @@ struct TileCursor {
         len = w.done() ? 0 : w.seg_len();
     }
     __device__ bool done() const { return w.done(); }
-    __device__ int logical_block() const { return w.first_blk + w.blk_off + t; }
+    __device__ int logical_block() const { return w.logical(w.blk_off + t); }
     __device__ void next() {
         if (++t == len) {
             w.advance(len);
@@ -282,8 +283,8 @@ struct Producer {
     __device__ int fetch(const GqaParams &p, int i, int lane) const {
         const int j = i + lane;
         if (j >= cur.len) return -1;
-        return __ldg(p.block_table + (size_t)cur.w.b * p.max_blocks + cur.w.first_blk +
-                     cur.w.blk_off + j);
+        return __ldg(p.block_table + (size_t)cur.w.b * p.max_blocks +
+                     table_slot(p.vis, cur.w.logical(cur.w.blk_off + j)));
     }
 
     // Physical block id of the current tile (warp-uniform call).
@@ -585,7 +586,7 @@ gqa_split_kernel(const GqaParams p) {
     pdl_launch_dependents();
 
     const int units = p.H_kv * p.n_hc;
-    PlanArgs pa{p.seq_lens, p.B, units, p.window, p.max_blocks, p.num_ctas};
+    PlanArgs pa{p.seq_lens, p.B, units, p.vis, p.max_blocks, p.num_ctas};
     plan_locate(pa, blockIdx.x, plan_sh, blockIdx.x == 0 ? p.ws_prefix : nullptr,
                 p.err);
     const long long W = plan_sh->total;
@@ -608,9 +609,9 @@ gqa_split_kernel(const GqaParams p) {
             // A sequence without a visible block (empty) has a zero output
             // and no split works on it.
             for (int b = blockIdx.x; b < p.B; b += P) {
-                int fb;
+                int fb, sb;
                 bool bad;
-                if (visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad) == 0) {
+                if (visible_blocks(p.seq_lens[b], p.vis, p.max_blocks, &fb, &sb, &bad) == 0) {
                     T *o = static_cast<T *>(p.out) + (size_t)b * p.H_q * D;
                     for (int i = et; i < p.H_q * D; i += C::kEpiThreads)
                         o[i] = ElemTraits<T>::from_float(0.f);
@@ -682,8 +683,8 @@ gqa_split_kernel(const GqaParams p) {
         const int len = walk.seg_len();
         const long long seg_t1 = seg_t0 + (long long)len * C::kSub;
         const int Tb = walk.T;
-        const int lo_tok = (p.window > 0 && Tb > p.window) ? Tb - p.window : 0;
-        const int blk0 = walk.first_blk + walk.blk_off;
+        const int lo_tok = window_lo(p.vis, Tb);
+        const int sink = p.vis.sink;
 
         // The unit's queries, staged in shared memory by the producer.
         if (!mbar_wait(&q_full[n_seg & 1], (uint32_t)((n_seg >> 1) & 1), p.timeout_ns, p.err,
@@ -726,7 +727,7 @@ gqa_split_kernel(const GqaParams p) {
             const T *Ks = reinterpret_cast<const T *>(stage_base + stage * C::kStageBytes);
             const T *Vs = Ks + C::kTileTok * D;
             const int tl = (int)(n - seg_t0);
-            const int tok0 = (blk0 + tl / C::kSub) * kBlockSize +
+            const int tok0 = walk.logical(walk.blk_off + tl / C::kSub) * kBlockSize +
                              (tl % C::kSub) * C::kTileTok + wig * C::kTPW;
             const int row0 = wig * C::kTPW;
 
@@ -778,7 +779,7 @@ gqa_split_kernel(const GqaParams p) {
                 const int tt = lane % C::kTPW;
                 const bool active = gs < HC;
                 const int pos = tok0 + tt;
-                const bool valid = active && pos >= lo_tok && pos < Tb;
+                const bool valid = active && pos < Tb && (pos >= lo_tok || pos < sink);
                 const float s = valid ? sc[tt * C::kHCP + gs] : kNegInf;
                 if (__any_sync(0xffffffffu, s > m_run[ps] + kRescaleLog2)) {
                     float mx = s;
@@ -909,7 +910,8 @@ struct CombineParams {
     const float *ws_o;
     const float *ws_lse;
     void *out;
-    int B, H_q, H_kv, group, n_hc, max_blocks, window, num_ctas;
+    int B, H_q, H_kv, group, n_hc, max_blocks, num_ctas;
+    Visibility vis;
     int D, HC;               // head dim, query heads per unit
     int copies;              // partials per (unit, CTA) slot (>= 1)
     int lanes;               // threads per float4 of output: 1, 4 or 8
@@ -951,9 +953,9 @@ combine_kernel(const CombineParams p) {
     const int b = u / units, rem = u % units;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        int fb;
+        int fb, sb;
         bool bad;
-        const int nb = visible_blocks(p.seq_lens[b], p.window, p.max_blocks, &fb, &bad);
+        const int nb = visible_blocks(p.seq_lens[b], p.vis, p.max_blocks, &fb, &sb, &bad);
         s_nb = nb;
         s_n = 0;
         s_first = 0;

@@ -92,6 +92,6 @@ namespace attn {
 // out[0] = W; out[1 + 4i .. 4 + 4i] = range start, range end, first sequence,
 // first unit of CTA i; then B + 1 exclusive work prefix sums.
 cudaError_t launch_plan_kernel(const int32_t *seq_lens, int B, int units_per_seq,
-                               int window, int max_blocks, int num_ctas,
+                               Visibility vis, int max_blocks, int num_ctas,
                                long long *out, unsigned *err, cudaStream_t stream);
 }  // namespace attn

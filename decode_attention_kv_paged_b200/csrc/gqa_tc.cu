@@ -100,7 +100,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int units = p.H_kv * p.n_hc;
-    PlanArgs pa{p.seq_lens, p.B, units, p.window, p.max_blocks, p.num_ctas};
+    PlanArgs pa{p.seq_lens, p.B, units, p.vis, p.max_blocks, p.num_ctas};
     plan_locate(pa, blockIdx.x, &bars->plan, blockIdx.x == 0 ? p.ws_prefix : nullptr, p.err);
     const long long W = bars->plan.total;
     const int P = working_ctas(W, p.num_ctas);
@@ -174,7 +174,8 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     !mbar_wait(&bars->c_empty[st], (uint32_t)(((tile - C::kStages) / C::kStages) & 1),
                                p.timeout_ns, p.err, abort_flag))
                     break;
-                int phys = p.block_table[(size_t)cur.w.b * p.max_blocks + cur.logical_block()];
+                int phys = p.block_table[(size_t)cur.w.b * p.max_blocks +
+                                         table_slot(p.vis, cur.logical_block())];
                 if (phys < 0 || phys >= p.num_blocks) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;                 // wholly out of bounds: zero fill
@@ -304,7 +305,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int i = 0; i < n_tiles; ++i) {
             const bool first = cur.t == 0, last = cur.t == cur.len - 1;
             const int b = cur.w.b, T = cur.w.T;
-            const int lo_tok = (p.window > 0 && T > p.window) ? T - p.window : 0;
+            const int lo_tok = window_lo(p.vis, T), sink = p.vis.sink;
             const int tok0 = cur.logical_block() * 64 + copy * TPC;
             const int sb = i & 1;
             if (!all(mbar_wait(&bars->s_full[sb], (uint32_t)((i >> 1) & 1), p.timeout_ns, p.err,
@@ -319,7 +320,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_before();
             mbar_arrive(&bars->s_free[sb]);
 
-            // scale to log2 units, mask keys outside [lo_tok, T)
+            // scale to log2 units, mask keys that are not visible
             const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
             for (int j = 0; j < TPC; j += 2) {
@@ -327,11 +328,11 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 s[j] = v.x;
                 s[j + 1] = v.y;
             }
-            if (tok0 < lo_tok || tok0 + TPC > T) {
+            if (tok0 + TPC > T || (tok0 < lo_tok && tok0 + TPC > sink)) {
 #pragma unroll
                 for (int j = 0; j < TPC; ++j) {
                     const int pos = tok0 + j;
-                    if (pos < lo_tok || pos >= T) s[j] = kNegInf;
+                    if (pos >= T || (pos < lo_tok && pos >= sink)) s[j] = kNegInf;
                 }
             }
             float mx;

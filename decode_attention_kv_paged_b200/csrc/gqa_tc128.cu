@@ -85,7 +85,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int units = p.H_kv * p.n_hc;
-    PlanArgs pa{p.seq_lens, p.B, units, p.window, p.max_blocks, p.num_ctas};
+    PlanArgs pa{p.seq_lens, p.B, units, p.vis, p.max_blocks, p.num_ctas};
     plan_locate(pa, blockIdx.x, &bars->plan, blockIdx.x == 0 ? p.ws_prefix : nullptr, p.err);
     const long long W = bars->plan.total;
     const int P = working_ctas(W, p.num_ctas);
@@ -136,7 +136,8 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     !mbar_wait(&bars->c_empty[st], (uint32_t)(((tile - C::kStages) / C::kStages) & 1),
                                p.timeout_ns, p.err, abort_flag))
                     break;
-                int phys = p.block_table[(size_t)cur.w.b * p.max_blocks + cur.logical_block()];
+                int phys = p.block_table[(size_t)cur.w.b * p.max_blocks +
+                                         table_slot(p.vis, cur.logical_block())];
                 if (phys < 0 || phys >= p.num_blocks) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;                 // wholly out of bounds: zero fill
@@ -280,7 +281,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         for (int i = 0; i < n_tiles; ++i) {
             const bool first = cur.t == 0, last = cur.t == cur.len - 1;
             const int b = cur.w.b, T = cur.w.T;
-            const int lo_tok = (p.window > 0 && T > p.window) ? T - p.window : 0;
+            const int lo_tok = window_lo(p.vis, T), sink = p.vis.sink;
             if (first) {
                 // This segment's queries into TMEM (rows beyond the group: 0),
                 // once the previous segment's last S has read the old ones.
@@ -325,11 +326,11 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if constexpr (kTPC == 8) v = half ? w16[8 + j] : w16[j];
                 s[j] = v * p.scale_log2;
             }
-            if (tok0 < lo_tok || tok0 + kTPC > T) {
+            if (tok0 + kTPC > T || (tok0 < lo_tok && tok0 + kTPC > sink)) {
 #pragma unroll
                 for (int j = 0; j < kTPC; ++j) {
                     const int pos = tok0 + j;
-                    if (pos < lo_tok || pos >= T) s[j] = kNegInf;
+                    if (pos >= T || (pos < lo_tok && pos >= sink)) s[j] = kNegInf;
                 }
             }
             float mx = s[0];

@@ -16,11 +16,12 @@ __global__ void kv_append_kernel(const KvAppendParams p) {
         const int h = (int)(bh % p.H_kv);
         const int b = (int)(bh / p.H_kv);
         const int pos = p.positions[b];
-        if (pos < 0 || pos >= p.max_blocks * kBlockSize) {
+        const int slot = pos < 0 ? -1 : table_slot(p.vis, pos / kBlockSize);
+        if (slot < 0 || slot >= p.max_blocks) {
             if (c == 0 && h == 0) raise_error(p.err, kErrBadBlock);
             continue;
         }
-        const int phys = p.block_table[(size_t)b * p.max_blocks + pos / kBlockSize];
+        const int phys = p.block_table[(size_t)b * p.max_blocks + slot];
         if (phys < 0 || phys >= p.num_blocks) {
             if (c == 0 && h == 0) raise_error(p.err, kErrBadBlock);
             continue;

@@ -1,7 +1,7 @@
 // kv_append.cuh -- parameters of the paged-cache append kernel.
 #pragma once
 
-#include "common.cuh"
+#include "plan.cuh"
 
 namespace attn {
 
@@ -14,6 +14,7 @@ struct KvAppendParams {
     const int32_t *block_table;
     unsigned *err;
     int B, H_kv, chunks_per_row, max_blocks, num_blocks;
+    Visibility vis;          // sink / ring: where logical block pos / 64 lives
 };
 
 cudaError_t launch_kv_append(const KvAppendParams &p, cudaStream_t stream);

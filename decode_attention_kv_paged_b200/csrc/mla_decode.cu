@@ -123,7 +123,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
     const int col0 = rank == 0 ? 0 : 256;
 
     // ---- plan (both CTAs of the cluster compute the same range)
-    PlanArgs pa{p.seq_lens, p.B, 1, 0, p.max_blocks, p.num_clusters};
+    PlanArgs pa{p.seq_lens, p.B, 1, Visibility{0, 0, 0}, p.max_blocks, p.num_clusters};
     plan_locate(pa, cluster, &bars->plan,
                 (cluster == 0 && rank == 0) ? p.ws_prefix : nullptr, p.err);
     const long long W = bars->plan.total;
@@ -695,7 +695,7 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     cp.group = kMlaH;
     cp.n_hc = 1;
     cp.max_blocks = max_blocks;
-    cp.window = 0;
+    cp.vis = Visibility{0, 0, 0};
     cp.num_ctas = clusters;
     cp.D = kMlaDc;
     cp.HC = kMlaH;

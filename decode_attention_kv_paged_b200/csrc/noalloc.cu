@@ -136,13 +136,13 @@ extern "C" int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
     kp.scale_log2 = scale * 1.4426950408889634f;
     kp.B = B; kp.H_q = H_q; kp.H_kv = H_kv; kp.group = G; kp.n_hc = n_hc;
     kp.max_blocks = max_blocks_per_seq; kp.num_blocks = num_blocks;
-    kp.window = window > 0 ? window : 0;
+    kp.vis = Visibility{window > 0 ? window : 0, 0, 0};
     kp.num_ctas = P;
     CombineParams &cp = L.cp;
     cp.seq_lens = seq_lens; cp.ws_prefix = kp.ws_prefix; cp.ws_o = kp.ws_o;
     cp.ws_lse = kp.ws_lse; cp.out = out;
     cp.B = B; cp.H_q = H_q; cp.H_kv = H_kv; cp.group = G; cp.n_hc = n_hc;
-    cp.max_blocks = max_blocks_per_seq; cp.window = kp.window; cp.num_ctas = P;
+    cp.max_blocks = max_blocks_per_seq; cp.vis = kp.vis; cp.num_ctas = P;
     cp.copies = 1;
     L.units_total = (int)units_total;
     L.stream = (cudaStream_t)stream;

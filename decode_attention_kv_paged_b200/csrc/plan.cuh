@@ -17,23 +17,64 @@
 
 namespace attn {
 
-// Visible blocks of a sequence with T cached tokens (current one included).
-// first_block receives the logical index of the first of them.
-__device__ __forceinline__ int visible_blocks(int T, int window, int max_blocks,
-                                              int *first_block, bool *bad) {
+// Which cached keys a query sees, and where the block table keeps them
+// (attention-head article, §3: sliding window, and window plus global
+// tokens).  Key j of a sequence with T cached tokens is visible when j < T
+// and (no window, or j >= T - window, or j < sink).  With ring > 0 the table
+// row is a ring: the blocks holding the sink keys keep slots [0, A)
+// (A = ceil(sink / 64)); logical block i >= A lives in slot A + i % ring, so
+// a window layer stores only the blocks its window can reach.
+struct Visibility {
+    int window;   // > 0: sliding window of the last `window` keys
+    int sink;     // > 0: the first `sink` keys stay visible (global tokens)
+    int ring;     // > 0: ring of this many table slots after the sink blocks
+};
+
+__host__ __device__ __forceinline__ int sink_blocks(const Visibility &v) {
+    return v.sink > 0 ? (v.sink + kBlockSize - 1) / kBlockSize : 0;
+}
+
+// Table slot of logical block i.
+__host__ __device__ __forceinline__ int table_slot(const Visibility &v, int i) {
+    if (v.ring <= 0) return i;
+    const int a = sink_blocks(v);
+    return i < a ? i : a + i % v.ring;
+}
+
+// First visible key of the window part (0 without a window).
+__host__ __device__ __forceinline__ int window_lo(const Visibility &v, int T) {
+    return (v.window > 0 && T > v.window) ? T - v.window : 0;
+}
+
+__host__ __device__ __forceinline__ bool key_visible(const Visibility &v, int j, int T) {
+    return j < T && (j >= window_lo(v, T) || j < v.sink);
+}
+
+// Visible blocks of a sequence with T cached tokens (current one included):
+// blocks holding at least one visible key, in order.  They are the first
+// *sink_blks logical blocks (the sink part) followed by a run starting at
+// logical block *first_block; visible block v is logical block
+// v < sink_blks ? v : first_block + v - sink_blks.
+__device__ __forceinline__ int visible_blocks(int T, const Visibility &v, int max_blocks,
+                                              int *first_block, int *sink_blks, bool *bad) {
     *first_block = 0;
+    *sink_blks = 0;
     if (T <= 0) {
         *bad = (T < 0);
         return 0;
     }
-    if (T > max_blocks * kBlockSize) {
+    if (v.ring <= 0 && T > max_blocks * kBlockSize) {
         *bad = true;
         return 0;
     }
     *bad = false;
-    const int lo = (window > 0 && T > window) ? T - window : 0;
-    *first_block = lo / kBlockSize;
-    return (T - 1) / kBlockSize - lo / kBlockSize + 1;
+    const int w0 = window_lo(v, T) / kBlockSize;        // first window block
+    const int w1 = (T - 1) / kBlockSize + 1;             // one past the last block
+    const int a = sink_blocks(v) < w1 ? sink_blocks(v) : w1;
+    if (a >= w0) return w1;                               // one run [0, w1)
+    *sink_blks = a;
+    *first_block = w0;
+    return a + (w1 - w0);
 }
 
 // Number of CTAs that take work.
@@ -59,7 +100,7 @@ struct PlanArgs {
     const int32_t *seq_lens;
     int B;
     int units_per_seq;
-    int window;
+    Visibility vis;
     int max_blocks;
     int num_ctas;
 };
@@ -88,10 +129,9 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
     // Pass 1: W.
     long long mine = 0;
     for (int b = tid; b < a.B; b += nt) {
-        int fb;
+        int fb, sb;
         bool bad;
-        mine += (long long)visible_blocks(a.seq_lens[b], a.window,
-                                          a.max_blocks, &fb, &bad) *
+        mine += (long long)visible_blocks(a.seq_lens[b], a.vis, a.max_blocks, &fb, &sb, &bad) *
                 a.units_per_seq;
         any_bad |= bad;
     }
@@ -117,10 +157,9 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
         const int b = c + tid;
         long long w = 0;
         if (b < a.B) {
-            int fb;
+            int fb, sb;
             bool bad;
-            w = (long long)visible_blocks(a.seq_lens[b], a.window,
-                                          a.max_blocks, &fb, &bad) *
+            w = (long long)visible_blocks(a.seq_lens[b], a.vis, a.max_blocks, &fb, &sb, &bad) *
                 a.units_per_seq;
         }
         long long x = w;
@@ -163,21 +202,27 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
 struct SegmentWalker {
     // fixed
     const int32_t *seq_lens;
-    int B, units, window, max_blocks;
+    Visibility vis;
+    int B, units, max_blocks;
     // state
     long long pos, end;
-    int b, unit, blk_off, nb, first_blk, T;
+    int b, unit, blk_off, nb, first_blk, sink_blks, T;
 
     __device__ void load_seq() {
         bool bad;
         T = seq_lens[b];
-        nb = visible_blocks(T, window, max_blocks, &first_blk, &bad);
+        nb = visible_blocks(T, vis, max_blocks, &first_blk, &sink_blks, &bad);
+    }
+
+    // Logical block of visible block v of the current sequence.
+    __device__ int logical(int v) const {
+        return v < sink_blks ? v : first_blk + (v - sink_blks);
     }
 
     __device__ void init(const PlanArgs &a, long long lo, long long hi,
                          int seq, long long base) {
         seq_lens = a.seq_lens; B = a.B; units = a.units_per_seq;
-        window = a.window; max_blocks = a.max_blocks;
+        vis = a.vis; max_blocks = a.max_blocks;
         pos = lo; end = hi; b = seq;
         if (pos < end) {
             load_seq();

@@ -31,9 +31,9 @@ __global__ void __launch_bounds__(256) plan_kernel(PlanArgs a, long long *out,
 }
 
 cudaError_t launch_plan_kernel(const int32_t *seq_lens, int B, int units_per_seq,
-                               int window, int max_blocks, int num_ctas,
+                               Visibility vis, int max_blocks, int num_ctas,
                                long long *out, unsigned *err, cudaStream_t stream) {
-    PlanArgs a{seq_lens, B, units_per_seq, window, max_blocks, num_ctas};
+    PlanArgs a{seq_lens, B, units_per_seq, vis, max_blocks, num_ctas};
     plan_kernel<<<num_ctas, 256, 0, stream>>>(a, out, err);
     return cudaGetLastError();
 }

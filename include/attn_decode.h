@@ -138,6 +138,52 @@ int kv_append_mla(const void *latent_new, void *latent_cache,
                   int num_blocks, void *stream);
 
 /*
+ * attn_visibility -- which cached keys each query sees, and how the block
+ * table row maps them (attention-head article, §3 sliding window; window plus
+ * global tokens).  Key j of a sequence with T = seq_lens[b] cached tokens is
+ * visible when j < T and (window <= 0, or j >= T - window, or j < sink_tokens).
+ * ring_blocks > 0 makes the table row a ring for window layers: the blocks
+ * holding the sink keys keep slots [0, A) with A = ceil(sink_tokens / 64),
+ * and logical block i >= A lives in slot A + (i mod ring_blocks), so a
+ * sequence stores only the blocks its window can reach; kv_append_ext
+ * writing token T-1 then overwrites (evicts) the block that left the
+ * window.  ring_blocks > 0 requires window > 0, ring_blocks * 64 >=
+ * window + 63 (the ring holds every block a window can touch) and
+ * A + ring_blocks <= max_blocks_per_seq; T is then not limited by the table
+ * width.  All zero: full causal attention, identity table (attn_decode_gqa).
+ */
+typedef struct attn_visibility {
+    int window;
+    int sink_tokens;
+    int ring_blocks;
+} attn_visibility;
+
+/*
+ * attn_decode_gqa_ext -- attn_decode_gqa with global (sink) tokens and a
+ * ring-buffer table (see attn_visibility; visibility must be non-null, host
+ * memory, read during the call).  Blocks holding no visible key are never
+ * read.  Same arguments, layouts, workspace and errors as attn_decode_gqa,
+ * plus ATTN_ERR_ARG for an invalid visibility record.
+ */
+int attn_decode_gqa_ext(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *seq_lens, const int32_t *block_table, void *out,
+                        int B, int H_q, int H_kv, int d, float scale,
+                        const attn_visibility *visibility, void *stream,
+                        int max_blocks_per_seq, int num_blocks, int dtype);
+
+/*
+ * kv_append_ext -- kv_append through the table mapping of `visibility`
+ * (sink slots, then the ring): token positions[b] goes to offset
+ * positions[b] % 64 of the block in slot table_slot(positions[b] / 64).
+ * A slot outside the table row or a block id outside the pool sets the
+ * bad-block error bit and skips that row.
+ */
+int kv_append_ext(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                  const int32_t *positions, const int32_t *block_table, int B, int H_kv,
+                  int d, int max_blocks_per_seq, int num_blocks, int dtype,
+                  const attn_visibility *visibility, void *stream);
+
+/*
  * attn_decode_plan -- run the device split planner on its own and write the
  * plan the decode kernels would follow (for bit-exact checks against a host
  * model).  The flattened work list orders sequences b, then units

@@ -104,6 +104,91 @@ static size_t orc_row_offset(const int32_t *block_table, int max_blocks, int b,
  * seq_lens[b] = T_b tokens cached, the current one included; T_b = 0 gives
  * a zero output row.
  */
+/*
+ * Decode attention with global (sink) tokens and a ring-buffer table
+ * (attention-head article, §3: sliding window; window plus global tokens).
+ * Key j of sequence b (T = seq_lens[b]) is visible when j < T and
+ * (window <= 0 or j >= T - window or j < sink).  The row of key j sits in
+ * the block of table slot slot(j / block_size): with ring > 0, logical block
+ * i < A = ceil(sink / block_size) keeps slot i and i >= A goes to slot
+ * A + i % ring; without ring, slot i = i.  Softmax over the visible keys only.
+ * Same arrays and dtypes as orc_decode_gqa; probs (optional) [B][H_q][max_T].
+ */
+static int orc_slot(int i, int sink, int ring, int block_size) {
+    if (ring <= 0) return i;
+    const int a = sink > 0 ? (sink + block_size - 1) / block_size : 0;
+    return i < a ? i : a + i % ring;
+}
+
+int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seq_lens, const int32_t *block_table,
+                       double *out, double *probs, int max_T, int B, int H_q,
+                       int H_kv, int d, int block_size, int max_blocks,
+                       double scale, int window, int sink, int ring, int dtype) {
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || d <= 0 || block_size <= 0 ||
+        H_q % H_kv != 0 || sink < 0 || ring < 0)
+        return ORC_BAD_ARG;
+    const int group = H_q / H_kv;
+    int status = ORC_OK;
+
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H_q; ++h) {
+            double *o = out + ((size_t)b * H_q + h) * d;
+            for (int k = 0; k < d; ++k) o[k] = 0.0;
+            if (probs)
+                for (int j = 0; j < max_T; ++j)
+                    probs[((size_t)b * H_q + h) * max_T + j] = 0.0;
+            const int T = seq_lens[b];
+            if (T <= 0) continue;
+            const int kvh = h / group;
+            /* the visible keys, in increasing order */
+            int *keys = (int *)malloc(sizeof(int) * (size_t)T);
+            double *s = (double *)malloc(sizeof(double) * (size_t)T);
+            if (!keys || !s) {
+                free(keys); free(s);
+#pragma omp atomic write
+                status = ORC_NO_MEM;
+                continue;
+            }
+            int n = 0;
+            for (int j = 0; j < T; ++j)
+                if (window <= 0 || j >= T - window || j < sink) keys[n++] = j;
+            const size_t q_off = ((size_t)b * H_q + h) * d;
+            for (int t = 0; t < n; ++t) {
+                const int j = keys[t];
+                const int slot = orc_slot(j / block_size, sink, ring, block_size);
+                const int32_t phys = block_table[(size_t)b * max_blocks + slot];
+                const size_t r = (((size_t)phys * H_kv + kvh) * block_size + j % block_size) * d;
+                double dot = 0.0;
+                for (int k = 0; k < d; ++k)
+                    dot += orc_read(q, q_off + k, dtype) * orc_read(k_cache, r + k, dtype);
+                s[t] = scale * dot;
+            }
+            double m = s[0];
+            for (int t = 1; t < n; ++t)
+                if (s[t] > m) m = s[t];
+            double z = 0.0;
+            for (int t = 0; t < n; ++t) {
+                s[t] = exp(s[t] - m);
+                z += s[t];
+            }
+            for (int t = 0; t < n; ++t) s[t] /= z;
+            for (int t = 0; t < n; ++t) {
+                const int j = keys[t];
+                const int slot = orc_slot(j / block_size, sink, ring, block_size);
+                const int32_t phys = block_table[(size_t)b * max_blocks + slot];
+                const size_t r = (((size_t)phys * H_kv + kvh) * block_size + j % block_size) * d;
+                for (int k = 0; k < d; ++k) o[k] += s[t] * orc_read(v_cache, r + k, dtype);
+                if (probs && j < max_T) probs[((size_t)b * H_q + h) * max_T + j] = s[t];
+            }
+            free(keys);
+            free(s);
+        }
+    }
+    return status;
+}
+
 int orc_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
                    const int32_t *seq_lens, const int32_t *block_table,
                    double *out, double *probs, int max_T, int B, int H_q,

@@ -25,6 +25,8 @@ def _load():
         c_p, c_i, c_d = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         lib.orc_decode_gqa.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i, c_i]
         lib.orc_decode_gqa.restype = c_i
+        lib.orc_decode_gqa_vis.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i, c_i, c_i, c_i]
+        lib.orc_decode_gqa_vis.restype = c_i
         lib.orc_decode_mla.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i]
         lib.orc_decode_mla.restype = c_i
         lib.orc_mla_explicit.argtypes = [c_p] * 8 + [c_i] * 8 + [c_d]
@@ -111,6 +113,37 @@ def decode_gqa(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
         B, H_q, H_kv, d, bs, max_blocks, float(scale), int(window), dt)
     if rc != 0:
         raise RuntimeError(f"oracle decode_gqa failed with status {rc}")
+    return (out, probs) if return_probs else out
+
+
+def decode_gqa_vis(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
+                   sink=0, ring=0, return_probs=False):
+    """decode_gqa with global (sink) tokens and a ring-buffer table (fp64).
+
+    Key j < T is visible when window <= 0, j >= T - window or j < sink.  With
+    ring > 0, logical block i lives in table slot i for i < A = ceil(sink /
+    block_size) (the sink blocks) and in slot A + i % ring after them.  Same arrays as
+    decode_gqa.
+    """
+    B, H_q, d = q.shape
+    _, H_kv, bs, d2 = k_cache.shape
+    assert d2 == d and tuple(v_cache.shape) == tuple(k_cache.shape)
+    qa, qp, dt = _as_input(q)
+    ka, kp, dt_k = _as_input(k_cache)
+    va, vp, dt_v = _as_input(v_cache)
+    if not (dt == dt_k == dt_v):
+        raise TypeError("q, k_cache and v_cache must share one dtype")
+    sl, slp = _as_i32(seq_lens)
+    bt, btp = _as_i32(block_table)
+    out = np.zeros((B, H_q, d), dtype=np.float64)
+    max_T = int(sl.max().item()) if return_probs and B > 0 else 0
+    probs = np.zeros((B, H_q, max_T), dtype=np.float64) if return_probs else None
+    rc = _load().orc_decode_gqa_vis(
+        qp, kp, vp, slp, btp, out.ctypes.data,
+        probs.ctypes.data if probs is not None else None, max_T,
+        B, H_q, H_kv, d, bs, bt.shape[1], float(scale), int(window), int(sink), int(ring), dt)
+    if rc != 0:
+        raise RuntimeError(f"oracle decode_gqa_vis failed with status {rc}")
     return (out, probs) if return_probs else out
 
 

@@ -402,3 +402,76 @@ def test_workload_block_tables_are_permutations():
     ids = table[table >= 0].tolist()
     assert sorted(ids) == list(range(nblk))
     assert [(table[b] >= 0).sum().item() for b in range(4)] == [1, 1, 2, 16]
+
+
+# ------------------------------------------- global (sink) tokens, ring table
+def _contiguous_case(rng, H_q, H_kv, d, T):
+    """One sequence with an identity block table: the cache holds keys
+    0..T-1 in order, so rows can also be selected directly."""
+    nb = (T + 63) // 64
+    q = rng.standard_normal((1, H_q, d))
+    k = rng.standard_normal((nb, H_kv, 64, d))
+    v = rng.standard_normal((nb, H_kv, 64, d))
+    table = np.arange(nb, dtype=np.int32)[None, :]
+    return q, k, v, table
+
+
+def test_vis_without_sink_or_ring_is_decode_gqa():
+    """Sink 0 and no ring: the same keys in the same order as the plain
+    decode, so the results are bit-identical (with and without a window)."""
+    rng = np.random.default_rng(31)
+    q, k, v, table = _contiguous_case(rng, 4, 2, 16, 300)
+    for w in (0, 1, 70, 299, 5000):
+        a = orc.decode_gqa(q, k, v, np.array([300], dtype=np.int32), table, 0.2, window=w)
+        b = orc.decode_gqa_vis(q, k, v, np.array([300], dtype=np.int32), table, 0.2, window=w, sink=0, ring=0)
+        assert np.array_equal(a, b), w
+
+
+def test_vis_window_plus_sink_selects_those_keys():
+    """Window w=5 and sink g=3 at T=20: exactly keys {0,1,2} and {15..19}
+    carry weight (attention-head §3, window plus global tokens), and the
+    output is the softmax over just those rows, computed directly."""
+    rng = np.random.default_rng(32)
+    q, k, v, table = _contiguous_case(rng, 2, 1, 8, 20)
+    out, p = orc.decode_gqa_vis(q, k, v, np.array([20], dtype=np.int32), table, 0.7, window=5, sink=3,
+                                return_probs=True)
+    for h in range(2):
+        assert set(np.nonzero(p[0, h])[0].tolist()) == {0, 1, 2, 15, 16, 17, 18, 19}
+        assert abs(p[0, h].sum() - 1.0) < 1e-12
+    rows = [0, 1, 2, 15, 16, 17, 18, 19]
+    K = k[0, 0, rows]
+    V = v[0, 0, rows]
+    for h in range(2):
+        s = 0.7 * K @ q[0, h]
+        e = np.exp(s - s.max())
+        np.testing.assert_allclose(out[0, h], (e / e.sum()) @ V, rtol=0, atol=1e-12)
+
+
+def test_vis_sink_covering_all_keys_is_full_attention():
+    rng = np.random.default_rng(33)
+    q, k, v, table = _contiguous_case(rng, 4, 4, 8, 150)
+    full = orc.decode_gqa(q, k, v, np.array([150], dtype=np.int32), table, 0.3, window=0)
+    got = orc.decode_gqa_vis(q, k, v, np.array([150], dtype=np.int32), table, 0.3, window=10, sink=150)
+    np.testing.assert_allclose(got, full, rtol=0, atol=1e-12)
+
+
+def test_vis_ring_table_reads_the_same_rows():
+    """A ring table whose slots hold the blocks the window (and the sink)
+    reach gives exactly the result of the full, identity-table cache: the
+    ring only changes where the rows live.  Sink 10 keeps slot 0; the window
+    blocks 9 and 10 of T=700, w=100 live in slots 1 + i % 3."""
+    rng = np.random.default_rng(34)
+    T, w, g, R = 700, 100, 10, 3
+    q, k, v, table = _contiguous_case(rng, 4, 2, 16, T)
+    ref = orc.decode_gqa_vis(q, k, v, np.array([T], dtype=np.int32), table, 0.25, window=w, sink=g)
+    A = 1
+    slots = A + R
+    kr = rng.standard_normal((slots + 2, 2, 64, 16))     # unused blocks hold noise
+    vr = rng.standard_normal((slots + 2, 2, 64, 16))
+    ring_table = np.array([[5, 2, 0, 4]], dtype=np.int32)  # slot -> physical block
+    for logical in [0, 9, 10]:
+        slot = logical if logical < A else A + logical % R
+        kr[ring_table[0, slot]] = k[logical]
+        vr[ring_table[0, slot]] = v[logical]
+    got = orc.decode_gqa_vis(q, kr, vr, np.array([T], dtype=np.int32), ring_table, 0.25, window=w, sink=g, ring=R)
+    assert np.array_equal(got, ref)

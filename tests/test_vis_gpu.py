@@ -1,0 +1,133 @@
+"""GPU parity of decode with global (sink) tokens and a ring-buffer block
+table (attn_decode_gqa_ext, kv_append_ext) vs the oracle's decode_gqa_vis,
+through the C ABI, on every GQA kernel.  Bars: bf16 max-abs <= 1e-2,
+rel-L2 <= 2e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from tests.parity import assert_parity
+from workloads import BLOCK_SIZE
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _inputs(seed, B, H_q, H_kv, d, n_blocks, slots):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, H_q, d), generator=g).bfloat16()
+    k = torch.randn((n_blocks, H_kv, BLOCK_SIZE, d), generator=g).bfloat16()
+    v = torch.randn((n_blocks, H_kv, BLOCK_SIZE, d), generator=g).bfloat16()
+    table = torch.randperm(n_blocks, generator=g)[: B * slots].reshape(B, slots)
+    return q, k, v, table.to(torch.int32)
+
+
+def _oracle(q, k, v, lens, table, scale, window, sink, ring):
+    return orc.decode_gqa_vis(q, k, v, np.asarray(lens, dtype=np.int32), table.numpy(), scale,
+                              window=window, sink=sink, ring=ring)
+
+
+VIS_CASES = [
+    # (H_q, H_kv, d, lens, window, sink)
+    (32, 8, 128, [1000, 70, 5, 4097], 100, 4),
+    (32, 1, 128, [3000, 64, 130], 500, 64),
+    (8, 8, 64, [700, 300, 1], 33, 100),
+    (24, 4, 256, [5000, 129], 1000, 7),
+]
+
+
+@pytest.mark.parametrize("path", [0, 1, 2], ids=["cuda_core", "tcgen05", "tcgen05_m64"])
+@pytest.mark.parametrize("H_q,H_kv,d,lens,window,sink", VIS_CASES,
+                         ids=[f"q{c[0]}_kv{c[1]}_d{c[2]}_w{c[4]}_g{c[5]}" for c in VIS_CASES])
+def test_window_plus_sink_matches_oracle(lib, path, H_q, H_kv, d, lens, window, sink):
+    B = len(lens)
+    slots = max((T + 63) // 64 for T in lens)
+    q, k, v, table = _inputs(7000 + H_q + d + window, B, H_q, H_kv, d, B * slots + 3, slots)
+    scale = 1.0 / np.sqrt(d)
+    ref = _oracle(q, k, v, lens, table, scale, window, sink, 0)
+    lib.set_gqa_path(path)
+    try:
+        got = lib.decode_gqa_ext(q.to(DEV), k.to(DEV), v.to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                 table.to(DEV), scale, window=window, sink_tokens=sink)
+        assert lib.last_error() == lib.OK
+    finally:
+        lib.set_gqa_path(-1)
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, f"vis path {path}")
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["cuda_core", "tcgen05"])
+def test_ring_table_matches_oracle(lib, path):
+    """Sequences far longer than the table row: the ring of 4 blocks after
+    one sink block holds the window (w=150); the oracle reads the same cache
+    through the same slot mapping."""
+    lens, window, sink, ring = [9000, 640, 151, 20000], 150, 10, 4
+    H_q, H_kv, d = 16, 2 if path == 0 else 1, 128
+    slots = 1 + ring
+    q, k, v, table = _inputs(7100 + path, len(lens), H_q, H_kv, d, len(lens) * slots + 5,
+                             slots)
+    scale = 0.09
+    ref = _oracle(q, k, v, lens, table, scale, window, sink, ring)
+    lib.set_gqa_path(path)
+    try:
+        got = lib.decode_gqa_ext(q.to(DEV), k.to(DEV), v.to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                 table.to(DEV), scale, window=window, sink_tokens=sink,
+                                 ring_blocks=ring)
+        assert lib.last_error() == lib.OK
+    finally:
+        lib.set_gqa_path(-1)
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, f"ring path {path}")
+
+
+def test_ring_append_evicts_and_decode_matches_full_cache(lib):
+    """Append every token of two sequences one step at a time into a ring
+    table (window 100 + sink 5 in 1 + 3 slots): blocks that leave the window
+    are overwritten, the sink block is kept, and the final decode equals the
+    oracle over the full (never evicted) cache with the same visibility."""
+    T, window, sink, ring, H_kv, H_q, d = 700, 100, 5, 3, 2, 8, 64
+    B = 2
+    g = torch.Generator().manual_seed(7200)
+    k_all = torch.randn((B, T, H_kv, d), generator=g).bfloat16()
+    v_all = torch.randn((B, T, H_kv, d), generator=g).bfloat16()
+    q = torch.randn((B, H_q, d), generator=g).bfloat16()
+    slots = 1 + ring
+    table = torch.tensor([[3, 0, 6, 1], [7, 2, 4, 5]], dtype=torch.int32)
+    kc = torch.zeros((8, H_kv, BLOCK_SIZE, d), dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    td = table.to(DEV)
+    kd, vd = k_all.to(DEV), v_all.to(DEV)
+    for t in range(T):
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        lib.kv_append_ext(kd[:, t].contiguous(), vd[:, t].contiguous(), kc, vc, pos, td,
+                          window=window, sink_tokens=sink, ring_blocks=ring)
+    assert lib.last_error() == lib.OK
+    lens = torch.full((B,), T, dtype=torch.int32, device=DEV)
+    got = lib.decode_gqa_ext(q.to(DEV), kc, vc, lens, td, 0.15, window=window,
+                             sink_tokens=sink, ring_blocks=ring)
+    assert lib.last_error() == lib.OK
+    # Full, never-evicted cache with an identity table per sequence.
+    nb = (T + 63) // 64
+    full_k = torch.zeros((B * nb, H_kv, BLOCK_SIZE, d), dtype=torch.bfloat16)
+    full_v = torch.zeros_like(full_k)
+    for b in range(B):
+        for t in range(T):
+            full_k[b * nb + t // 64, :, t % 64] = k_all[b, t]
+            full_v[b * nb + t // 64, :, t % 64] = v_all[b, t]
+    full_table = torch.arange(B * nb, dtype=torch.int32).reshape(B, nb)
+    ref = _oracle(q, full_k, full_v, [T] * B, full_table, 0.15, window, sink, 0)
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, "ring append")
+
+
+def test_visibility_host_validation(lib):
+    q, k, v, table = _inputs(1, 1, 4, 2, 64, 8, 4)
+    args = (q.to(DEV), k.to(DEV), v.to(DEV), torch.tensor([100], dtype=torch.int32,
+                                                          device=DEV), table.to(DEV), 0.1)
+    for kw in (dict(ring_blocks=2),                              # ring needs a window
+               dict(window=200, ring_blocks=3),                  # ring too small for w
+               dict(window=64, sink_tokens=65, ring_blocks=3),   # 2 sink + 3 ring > 4
+               dict(window=10, sink_tokens=-1)):
+        with pytest.raises(lib.AttnError) as e:
+            lib.decode_gqa_ext(*args, **kw)
+        assert e.value.status == lib.ERR_ARG, kw

@@ -36,6 +36,8 @@ class GQAConfig:
     T: int = 0
     dtype: torch.dtype = torch.bfloat16
     window: int = 0
+    sink: int = 0                          # global tokens kept visible (with a window)
+    ring: int = 0                          # ring table of this many blocks after the sink ones
     contiguous: bool = False               # identity block table
     seed: int = SEED_BASE
     ragged: Optional[tuple] = None         # (lo, hi) inclusive range of T_b
@@ -89,10 +91,19 @@ def ragged_config(window: int) -> GQAConfig:
 
 RAGGED_FULL = ragged_config(0)
 RAGGED_WINDOW = ragged_config(4096)
+# Window plus 64 global tokens on the same shape; and the same on a ring table
+# that keeps only the 1 sink block and the 65 blocks a 4096-key window can reach.
+RAGGED_WINDOW_SINK = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_g64", B=8, H_q=24,
+                               H_kv=4, d=256, ragged=(1024, 131072), window=4096, sink=64,
+                               seed=SEED_BASE + 3)
+RAGGED_WINDOW_RING = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_g64_ring65", B=8,
+                               H_q=24, H_kv=4, d=256, ragged=(1024, 131072), window=4096,
+                               sink=64, ring=65, seed=SEED_BASE + 3)
 MLA_DSV2 = MLAConfig("mla_absorbed_bf16_B32_H128_dc512_dr64_T8192", B=32)
 
 WORKLOADS = {c.name: c for c in [TINY, LLAMA3_8B, *SWEEP, RAGGED_FULL,
-                                 RAGGED_WINDOW, MLA_DSV2]}
+                                 RAGGED_WINDOW, RAGGED_WINDOW_SINK, RAGGED_WINDOW_RING,
+                                 MLA_DSV2]}
 
 
 def _generator(seed: int, device) -> torch.Generator:
@@ -174,8 +185,14 @@ def make_gqa_inputs(cfg: GQAConfig, device="cpu", seed: Optional[int] = None,
                     window: Optional[int] = None) -> GQAInputs:
     g = _generator(cfg.seed if seed is None else seed, device)
     seq = draw_seq_lens(cfg, g)
-    table, nblk = make_block_table(seq, g, cfg.contiguous,
-                                   extra_blocks_per_seq, pool_slack)
+    if cfg.ring > 0:
+        # Every sequence owns the sink blocks and the ring slots, whatever T.
+        slots = (cfg.sink + BLOCK_SIZE - 1) // BLOCK_SIZE + cfg.ring
+        table, nblk = make_block_table([slots * BLOCK_SIZE] * cfg.B, g, cfg.contiguous,
+                                       extra_blocks_per_seq, pool_slack)
+    else:
+        table, nblk = make_block_table(seq, g, cfg.contiguous,
+                                       extra_blocks_per_seq, pool_slack)
     q = randn((cfg.B, cfg.H_q, cfg.d), g, cfg.dtype)
     k = randn((nblk, cfg.H_kv, BLOCK_SIZE, cfg.d), g, cfg.dtype)
     v = randn((nblk, cfg.H_kv, BLOCK_SIZE, cfg.d), g, cfg.dtype)
