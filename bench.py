@@ -61,6 +61,7 @@ WORKLOAD_ALIASES = {
     "ragged_window": W.RAGGED_WINDOW.name,
     "ragged_window_sink": W.RAGGED_WINDOW_SINK.name,
     "ragged_window_ring": W.RAGGED_WINDOW_RING.name,
+    "llama3_8b_fp8": W.LLAMA3_8B_FP8.name,
     "mla": W.MLA_DSV2.name,
 }
 
@@ -247,6 +248,14 @@ def visible_tiles(T, window, sink):
     return w1 if a >= w0 else a + w1 - w0
 
 
+def kv_row_bytes(cfg):
+    """Cache bytes of one (token, KV head) row, K and V together: 2 d s, or
+    2 (d + 4) for the fp8 cache (one byte per element plus a fp32 row scale)."""
+    if cfg.kv_fp8:
+        return 2 * (cfg.d + 4)
+    return 2 * cfg.d * (torch.finfo(cfg.dtype).bits // 8)
+
+
 def algorithmic_bytes_gqa(inp):
     """K+V bytes of visible keys (both caches) + q + out."""
     cfg = inp.cfg
@@ -254,7 +263,7 @@ def algorithmic_bytes_gqa(inp):
     vis = 0
     for T in inp.seq_list:
         vis += visible_keys(T, inp.window, cfg.sink)
-    kv = vis * cfg.H_kv * cfg.d * 2 * s
+    kv = vis * cfg.H_kv * kv_row_bytes(cfg)
     qo = 2 * cfg.B * cfg.H_q * cfg.d * s
     return kv, kv + qo
 
@@ -266,7 +275,7 @@ def tile_bytes_gqa(inp):
     blocks = 0
     for T in inp.seq_list:
         blocks += visible_tiles(T, inp.window, cfg.sink)
-    return blocks * 64 * cfg.H_kv * cfg.d * 2 * s
+    return blocks * 64 * cfg.H_kv * kv_row_bytes(cfg)
 
 
 def algorithmic_bytes_mla(inp):
@@ -316,9 +325,15 @@ def run_native(args, rank, world, local):  # noqa: C901
             attn.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
                             x.block_table, x.scale, out=outs[i % reps])
         else:
-            attn.decode_gqa_ext(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                                x.scale, window=x.window, sink_tokens=cfg.sink,
-                                ring_blocks=cfg.ring, out=outs[i % reps])
+            if cfg.kv_fp8:
+                attn.decode_gqa_fp8(x.q, x.k_cache, x.v_cache, x.k_scale, x.v_scale,
+                                    x.seq_lens, x.block_table, x.scale, window=x.window,
+                                    sink_tokens=cfg.sink, ring_blocks=cfg.ring,
+                                    out=outs[i % reps])
+            else:
+                attn.decode_gqa_ext(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                                    x.scale, window=x.window, sink_tokens=cfg.sink,
+                                    ring_blocks=cfg.ring, out=outs[i % reps])
 
     for i in range(max(args.warmup, 3)):
         step(i)
@@ -385,7 +400,8 @@ def run_native(args, rank, world, local):  # noqa: C901
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_max / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32",
+        "dtype": ("fp8e4m3 cache, bf16 q/out, f32 accumulate" if getattr(cfg, "kv_fp8", False)
+                  else "bf16" if cfg.dtype == torch.bfloat16 else "f32"),
         "data": "synthetic (seeded N(0,1) q/K/V, random-permutation block table)",
         "config": {"workload": wl_name, "global_batch": B * world,
                    "seq_len": getattr(cfg, "T", None) or max(base.seq_list),
@@ -476,11 +492,16 @@ def e2e_native(attn, cfg, x, is_mla, K, world, dev):
         else:
             d_k.copy_(h_k, non_blocking=True)
             d_v.copy_(h_v, non_blocking=True)
-            attn.kv_append_ext(d_k, d_v, x.k_cache, x.v_cache, pos, x.block_table,
-                               window=x.window, sink_tokens=cfg.sink, ring_blocks=cfg.ring)
-            attn.decode_gqa_ext(d_q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                                x.scale, window=x.window, sink_tokens=cfg.sink,
-                                ring_blocks=cfg.ring, out=d_out)
+            vis = dict(window=x.window, sink_tokens=cfg.sink, ring_blocks=cfg.ring)
+            if cfg.kv_fp8:
+                attn.kv_append_fp8(d_k, d_v, x.k_cache, x.v_cache, x.k_scale, x.v_scale, pos,
+                                   x.block_table, **vis)
+                attn.decode_gqa_fp8(d_q, x.k_cache, x.v_cache, x.k_scale, x.v_scale,
+                                    x.seq_lens, x.block_table, x.scale, out=d_out, **vis)
+            else:
+                attn.kv_append_ext(d_k, d_v, x.k_cache, x.v_cache, pos, x.block_table, **vis)
+                attn.decode_gqa_ext(d_q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
+                                    x.scale, out=d_out, **vis)
         h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(3):
@@ -517,7 +538,8 @@ def _oracle_problem(cfg, is_mla, seqs, seed):
         lens = W.draw_seq_lens(cfg, g)[:seqs]
     sub = W.GQAConfig(cfg.name, B=seqs, H_q=cfg.H_q, H_kv=cfg.H_kv, d=cfg.d,
                       seq_lens=lens, T=cfg.T, dtype=cfg.dtype, window=cfg.window,
-                      sink=cfg.sink, ring=cfg.ring, contiguous=cfg.contiguous, seed=seed)
+                      sink=cfg.sink, ring=cfg.ring, kv_fp8=cfg.kv_fp8,
+                      contiguous=cfg.contiguous, seed=seed)
     return W.make_gqa_inputs(sub)
 
 
@@ -525,6 +547,11 @@ def _oracle_call(orc, x, is_mla):
     if is_mla:
         return orc.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
                               x.block_table, x.scale)
+    if x.cfg.kv_fp8:
+        k = orc.dequantize_e4m3(x.k_cache.numpy(), x.k_scale.numpy())
+        v = orc.dequantize_e4m3(x.v_cache.numpy(), x.v_scale.numpy())
+        return orc.decode_gqa_vis(x.q.double().numpy(), k, v, x.seq_lens, x.block_table,
+                                  x.scale, window=x.window, sink=x.cfg.sink, ring=x.cfg.ring)
     return orc.decode_gqa_vis(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
                               x.scale, window=x.window, sink=x.cfg.sink, ring=x.cfg.ring)
 

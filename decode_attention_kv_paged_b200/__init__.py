@@ -29,6 +29,7 @@ C_SYMBOLS = (
     "attn_debug_force_timeout", "attn_decode_last_error",
     "attn_status_string", "attn_version", "attn_decode_gqa_noalloc",
     "attn_mla_absorb_q", "attn_mla_project_out", "attn_decode_gqa_ext", "kv_append_ext",
+    "attn_decode_gqa_fp8", "kv_append_fp8",
 )
 
 
@@ -65,6 +66,9 @@ def load():
     lib.attn_decode_gqa_ext.argtypes = ([p] * 6 + [i] * 4 +
                                         [f, ctypes.POINTER(Visibility), p, i, i, i])
     lib.kv_append_ext.argtypes = [p] * 6 + [i] * 6 + [ctypes.POINTER(Visibility), p]
+    lib.attn_decode_gqa_fp8.argtypes = ([p] * 8 + [i] * 4 +
+                                        [f, ctypes.POINTER(Visibility), p, i, i])
+    lib.kv_append_fp8.argtypes = [p] * 8 + [i] * 5 + [ctypes.POINTER(Visibility), p]
     lib.attn_mla_absorb_q.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.attn_mla_project_out.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.kv_append.argtypes = [p] * 6 + [i] * 6 + [p]
@@ -163,6 +167,47 @@ def decode_gqa_ext(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
         block_table.shape[1], nblk, dt)
     _check(rc, "attn_decode_gqa_ext")
     return out
+
+
+def decode_gqa_fp8(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_table, scale,
+                   window=0, sink_tokens=0, ring_blocks=0, out=None, stream=None):
+    """out [B][H_q][d] (bf16) = decode attention over an fp8 cache: k_cache /
+    v_cache uint8 E4M3 codes [num_blocks][H_kv][64][d], k_scale / v_scale
+    fp32 row scales [num_blocks][H_kv][64] (value = code * row scale)."""
+    B, H_q, d = q.shape
+    nblk, H_kv, bs, d2 = k_cache.shape
+    if bs != BLOCK_SIZE or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("cache must be [num_blocks][H_kv][64][d] for K and V")
+    if tuple(k_scale.shape) != (nblk, H_kv, bs) or tuple(v_scale.shape) != (nblk, H_kv, bs):
+        raise ValueError("scales must be [num_blocks][H_kv][64]")
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    if out is None:
+        out = torch.empty_like(q)
+    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    rc = load().attn_decode_gqa_fp8(
+        _dev(q, "q", bf), _dev(k_cache, "k_cache", u8), _dev(v_cache, "v_cache", u8),
+        _dev(k_scale, "k_scale", f32), _dev(v_scale, "v_scale", f32),
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(block_table, "block_table", torch.int32),
+        _dev(out, "out", bf), B, H_q, H_kv, d, float(scale), ctypes.byref(vis),
+        _stream_ptr(stream), block_table.shape[1], nblk)
+    _check(rc, "attn_decode_gqa_fp8")
+    return out
+
+
+def kv_append_fp8(k_new, v_new, k_cache, v_cache, k_scale, v_scale, positions, block_table,
+                  window=0, sink_tokens=0, ring_blocks=0, stream=None):
+    """Quantise the current token's K/V rows (bf16 [B][H_kv][d]) to E4M3 with
+    one scale per row (amax / 448) and write them at positions[b]."""
+    B, H_kv, d = k_new.shape
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    rc = load().kv_append_fp8(
+        _dev(k_new, "k_new", bf), _dev(v_new, "v_new", bf), _dev(k_cache, "k_cache", u8),
+        _dev(v_cache, "v_cache", u8), _dev(k_scale, "k_scale", f32),
+        _dev(v_scale, "v_scale", f32), _dev(positions, "positions", torch.int32),
+        _dev(block_table, "block_table", torch.int32), B, H_kv, d, block_table.shape[1],
+        k_cache.shape[0], ctypes.byref(vis), _stream_ptr(stream))
+    _check(rc, "kv_append_fp8")
 
 
 def decode_gqa_noalloc(q, k_cache, v_cache, seq_lens, block_table, scale,

@@ -248,14 +248,23 @@ int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype, int *num_
 }
 
 // Shared body of attn_decode_gqa and attn_decode_gqa_ext.
+// dtype: ATTN_F32 / ATTN_BF16 for q, cache and out alike, or kFp8Cache: bf16
+// q and out over an e4m3 cache with per-row scales (k_scale, v_scale).
+constexpr int kFp8Cache = 100;
+
 static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *seq_lens, const int32_t *block_table, void *out,
                            int B, int H_q, int H_kv, int d, float scale, Visibility vis,
-                           void *stream, int max_blocks_per_seq, int num_blocks, int dtype) {
+                           void *stream, int max_blocks_per_seq, int num_blocks, int dtype,
+                           const float *k_scale = nullptr, const float *v_scale = nullptr) {
     if (!q || !k_cache || !v_cache || !seq_lens || !block_table || !out) return ATTN_ERR_ARG;
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return ATTN_ERR_ARG;
     if (max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
-    if (dtype != ATTN_F32 && dtype != ATTN_BF16) return ATTN_ERR_ARG;
+    const bool fp8 = dtype == kFp8Cache;
+    if (dtype != ATTN_F32 && dtype != ATTN_BF16 && !fp8) return ATTN_ERR_ARG;
+    if (fp8 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale)))
+        return ATTN_ERR_ARG;
+    if (fp8 && d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
     if (!std::isfinite(scale)) return ATTN_ERR_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return ATTN_ERR_ARG;
@@ -269,7 +278,8 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     cudaStream_t s = (cudaStream_t)stream;
 
     const int G = H_q / H_kv;
-    const bool tc = use_tc_path(G, d, dtype);
+    // The fp8 cache is read by the CUDA-core kernel for every group size.
+    const bool tc = !fp8 && use_tc_path(G, d, dtype);
     const int HC = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
     const int n_hc = G / HC;
     const long long units_total = (long long)B * H_kv * n_hc;
@@ -299,6 +309,8 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     kp.ws_prefix = reinterpret_cast<long long *>(ws + o_bytes + lse_bytes);
     kp.err = st->err;
     kp.out = out;
+    kp.k_scale = k_scale;
+    kp.v_scale = v_scale;
     if (!tc) {
         rc = ensure_counters(st, (size_t)units_total, s);
         if (rc) return rc;
@@ -324,6 +336,14 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     cudaError_t e;
     if (tc) {
         e = tc128 ? launch_gqa_tc128(L, d, HC) : launch_gqa_tc(L, d, HC);
+        return cuda_status(e);
+    }
+    if (fp8) {
+        switch (d) {
+            case 64: e = launch_gqa_fp8_d64(HC, L); break;
+            case 128: e = launch_gqa_fp8_d128(HC, L); break;
+            default: e = launch_gqa_fp8_d256(HC, L); break;
+        }
         return cuda_status(e);
     }
     switch (d) {
@@ -372,6 +392,54 @@ int attn_decode_gqa_ext(const void *q, const void *k_cache, const void *v_cache,
     if (rc) return rc;
     return decode_gqa_impl(q, k_cache, v_cache, seq_lens, block_table, out, B, H_q, H_kv, d,
                            scale, vis, stream, max_blocks_per_seq, num_blocks, dtype);
+}
+
+int attn_decode_gqa_fp8(const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale, const int32_t *seq_lens,
+                        const int32_t *block_table, void *out, int B, int H_q, int H_kv, int d,
+                        float scale, const attn_visibility *visibility, void *stream,
+                        int max_blocks_per_seq, int num_blocks) {
+    Visibility vis{0, 0, 0};
+    if (visibility) {
+        const int rc = check_visibility(visibility, max_blocks_per_seq, &vis);
+        if (rc) return rc;
+    }
+    return decode_gqa_impl(q, k_cache, v_cache, seq_lens, block_table, out, B, H_q, H_kv, d,
+                           scale, vis, stream, max_blocks_per_seq, num_blocks, kFp8Cache,
+                           k_scale, v_scale);
+}
+
+int kv_append_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                  float *k_scale, float *v_scale, const int32_t *positions,
+                  const int32_t *block_table, int B, int H_kv, int d, int max_blocks_per_seq,
+                  int num_blocks, const attn_visibility *visibility, void *stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !k_scale || !v_scale || !positions ||
+        !block_table)
+        return ATTN_ERR_ARG;
+    if (B <= 0 || H_kv <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
+    if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+    Visibility vis{0, 0, 0};
+    if (visibility) {
+        const int rc = check_visibility(visibility, max_blocks_per_seq, &vis);
+        if (rc) return rc;
+    }
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    KvAppendFp8Params p{};
+    p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    p.k_cache = static_cast<uint8_t *>(k_cache);
+    p.v_cache = static_cast<uint8_t *>(v_cache);
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.positions = positions;
+    p.block_table = block_table;
+    p.err = st->err;
+    p.B = B; p.H_kv = H_kv; p.d = d;
+    p.max_blocks = max_blocks_per_seq; p.num_blocks = num_blocks;
+    p.vis = vis;
+    return cuda_status(launch_kv_append_fp8(p, (cudaStream_t)stream));
 }
 
 int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent_cache,

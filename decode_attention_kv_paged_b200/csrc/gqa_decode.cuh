@@ -77,6 +77,8 @@ struct GqaParams {
     float *ws_lse;        // [slots][HC]  log2-sum-exp of the scaled scores
     long long *ws_prefix; // [B + 1]
     unsigned *ws_cnt;     // [B * units] split arrival counters, zero between launches
+    const float *k_scale; // fp8 cache only: [num_blocks][H_kv][64] row scales
+    const float *v_scale;
     unsigned *err;
     unsigned long long timeout_ns;
     float scale_log2;     // scale * log2(e)
@@ -85,9 +87,12 @@ struct GqaParams {
     int force_timeout;
 };
 
-template <int D, int HC, typename T>
+// T: query / output element type; TK: cache element type (T, or uint8_t
+// for fp8 e4m3 codes with one fp32 scale per cached row).
+template <int D, int HC, typename T, typename TK = T>
 struct GqaCfg {
-    static constexpr int kS = (int)sizeof(T);
+    static constexpr int kS = (int)sizeof(TK);                   // cache bytes / element
+    static constexpr bool kFp8 = sizeof(TK) == 1;
     // Warp specialisation: warpgroup 0 is the producer (its warp 0 streams
     // the tiles; the other three exit at once), warpgroups 1 and 2 are the
     // kNW compute warps.  setmaxnreg moves the producer group's registers to
@@ -125,14 +130,15 @@ struct GqaCfg {
     static constexpr int kPasses = (HC + kHPP - 1) / kHPP;        // softmax passes
     static constexpr int kHCP = (HC == 3) ? 4 : (HC > 4 ? 8 : HC);// padded heads
     static constexpr int kTileBytes = kTileTok * D * kS;
-    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kScaleBytes = kFp8 ? kTileTok * 4 : 0;   // one fp32 per row
+    static constexpr int kStageBytes = 2 * (kTileBytes + kScaleBytes);
     // shared memory carve-up (bytes)
     static constexpr int kScoreBytes = kNW * kTPW * kHCP * 4;
     static constexpr int kMergeOBytes = kNW * HC * D * 4;
     static constexpr int kMergeMLBytes = 2 * kNW * HC * 4;
     static constexpr int kEpiBytes = (kNW + 2) * HC * 4;         // merge weights
     static constexpr int kEpiThreads = 96;                        // producer WG warps 1-3
-    static constexpr int kQBytes = HC * D * kS;                   // one unit's queries
+    static constexpr int kQBytes = HC * D * (int)sizeof(T);      // one unit's queries
     static constexpr int kQRingBytes = 2 * ((kQBytes + 127) / 128 * 128);
     static constexpr int kMiscBytes = 1024;  // barriers + plan scratch + flags
     static constexpr int kOther =
@@ -148,35 +154,50 @@ struct GqaCfg {
     static_assert(kTileBytes % 16 == 0, "bulk copy size");
 };
 
-// Load kLE consecutive elements (16 or 8 bytes) and widen to fp32.
-template <typename T, int LE>
-__device__ __forceinline__ void load_widen(const T *p, float *f) {
-    if constexpr (sizeof(T) * LE == 16) {
-        uint4 v = *reinterpret_cast<const uint4 *>(p);
-        Chunk<T>::unpack(v, f);
-    } else {
-        static_assert(sizeof(T) * LE == 8, "load width");
-        uint2 v = *reinterpret_cast<const uint2 *>(p);
-        if constexpr (sizeof(T) == 2) {
-            f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
-            f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-        } else {
-            f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
-        }
-    }
-}
-
 // Load kLE consecutive elements and widen them to fp32 pairs (element 2j in
 // .x, 2j+1 in .y), ready for packed fp32x2 arithmetic.
+// fp8 e4m3 byte I of w as an fp32 equal to its value times 2^-120, exactly
+// (subnormals included): the sign and the 7 exponent/mantissa bits placed at
+// the top of an fp32, whose exponent bias (127) exceeds e4m3's (7) by 120.
+template <int I>
+__device__ __forceinline__ float e4m3_scaled(uint32_t w) {
+    const uint32_t t = (I == 3) ? w : (w << (24 - 8 * I));
+    return __uint_as_float((uint32_t)((int32_t)t >> 4) & 0x87F00000u);
+}
+constexpr float kE4m3Half = 1.152921504606846976e18f;   // 2^60: half of 2^120
+
+// Load kLE consecutive elements and widen them to fp32 pairs (element 2j in
+// .x, 2j+1 in .y), ready for packed fp32x2 arithmetic.  fp8 (e4m3) codes are
+// widened times 2^-120 (see e4m3_scaled); the caller folds 2^120 back in.
 template <typename T, int LE>
 __device__ __forceinline__ void load_pairs(const T *p, float2 *f) {
-    if constexpr (sizeof(T) == 2) {
-        if constexpr (LE == 8) {
+    if constexpr (sizeof(T) == 1) {
+        static_assert(LE == 4 || LE == 8 || LE == 16, "load width");
+        uint32_t w[LE / 4];
+        if constexpr (LE == 16) {
             const uint4 v = *reinterpret_cast<const uint4 *>(p);
-            f[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
-            f[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
-            f[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
-            f[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+        } else if constexpr (LE == 8) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(p);
+            w[0] = v.x; w[1] = v.y;
+        } else {
+            w[0] = *reinterpret_cast<const uint32_t *>(p);
+        }
+#pragma unroll
+        for (int k = 0; k < LE / 4; ++k) {
+            f[2 * k] = make_float2(e4m3_scaled<0>(w[k]), e4m3_scaled<1>(w[k]));
+            f[2 * k + 1] = make_float2(e4m3_scaled<2>(w[k]), e4m3_scaled<3>(w[k]));
+        }
+    } else if constexpr (sizeof(T) == 2) {
+        if constexpr (LE == 8 || LE == 16) {
+#pragma unroll
+            for (int k = 0; k < LE / 8; ++k) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(p + 8 * k);
+                f[4 * k] = make_float2(bf16lo(v.x), bf16hi(v.x));
+                f[4 * k + 1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+                f[4 * k + 2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+                f[4 * k + 3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+            }
         } else {
             static_assert(LE == 4, "load width");
             const uint2 v = *reinterpret_cast<const uint2 *>(p);
@@ -315,6 +336,7 @@ __device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor 
                                           int phys, int sub, unsigned char *dst,
                                           uint64_t *full, uint64_t pol) {
     constexpr uint32_t kTileBytes = kTileTok * D * sizeof(T);
+    constexpr uint32_t kScaleBytes = sizeof(T) == 1 ? kTileTok * 4 : 0;
     const int kvh = cur.w.unit / p.n_hc;
     if (phys < 0 || phys >= p.num_blocks) {
         raise_error(p.err, kErrBadBlock);
@@ -322,10 +344,16 @@ __device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor 
         return;
     }
     const size_t off = (((size_t)phys * p.H_kv + kvh) * kBlockSize + (size_t)sub * kTileTok) * D;
-    mbar_arrive_expect_tx(full, 2 * kTileBytes);
+    mbar_arrive_expect_tx(full, 2 * (kTileBytes + kScaleBytes));
     bulk_load(dst, static_cast<const T *>(p.k_cache) + off, kTileBytes, full, pol);
     bulk_load(dst + kTileBytes, static_cast<const T *>(p.v_cache) + off, kTileBytes,
               full, pol);
+    if constexpr (kScaleBytes > 0) {
+        // The tile's row scales (fp8 cache), after the K and V codes.
+        const size_t srow = off / D;
+        bulk_load(dst + 2 * kTileBytes, p.k_scale + srow, kScaleBytes, full, pol);
+        bulk_load(dst + 2 * kTileBytes + kScaleBytes, p.v_scale + srow, kScaleBytes, full, pol);
+    }
 }
 
 // Arrival of one split of a unit: true for the last of its `ns` splits,
@@ -342,14 +370,15 @@ __device__ __forceinline__ bool unit_arrive(unsigned *cnt, int ns) {
 // released by the compute warps; then waits for the copies still in flight
 // (the last S issued) so none lands after the CTA exits.  All 32 lanes run
 // it; lane 0 issues the copies.
-template <int D, int HC, typename T, int S, int kTileTok, int kSub>
+template <int D, int HC, typename T, typename TK, int S, int kTileTok, int kSub>
 __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long lo,
                               long long hi, int seq, long long base,
                               unsigned char *stage_base, uint64_t *full_bar,
                               uint64_t *empty_bar, unsigned char *q_ring, int q_slot_bytes,
                               uint64_t *q_full, uint64_t *q_empty, int lane,
                               volatile int *abort_flag) {
-    constexpr int kStageBytes = 2 * kTileTok * D * (int)sizeof(T);
+    constexpr int kStageBytes =
+        2 * (kTileTok * D * (int)sizeof(TK) + (sizeof(TK) == 1 ? kTileTok * 4 : 0));
     constexpr uint32_t kQBytes = HC * D * sizeof(T);
     const uint64_t pol = l2_policy_evict_first();
     Producer prod;
@@ -386,7 +415,7 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
         }
         if (sub == 0) phys = prod.block_id(p, lane);
         if (lane == 0)
-            issue_tile<D, T, kTileTok>(p, prod.cur, phys, sub,
+            issue_tile<D, TK, kTileTok>(p, prod.cur, phys, sub,
                                        stage_base + (size_t)s * kStageBytes, &full_bar[s],
                                        pol);
         if (++sub == kSub) {
@@ -534,10 +563,10 @@ __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0
     }
 }
 
-template <int D, int HC, typename T>
-__global__ void __launch_bounds__(GqaCfg<D, HC, T>::kThreads, 1)
+template <int D, int HC, typename T, typename TK>
+__global__ void __launch_bounds__(GqaCfg<D, HC, T, TK>::kThreads, 1)
 gqa_split_kernel(const GqaParams p) {
-    using C = GqaCfg<D, HC, T>;
+    using C = GqaCfg<D, HC, T, TK>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *stage_base = smem;
@@ -601,7 +630,7 @@ gqa_split_kernel(const GqaParams p) {
     if (tid < 128) {
         regs_decrease<C::kProducerRegs>();
         if (tid < 32) {
-            produce_tiles<D, HC, T, S, C::kTileTok, C::kSub>(
+            produce_tiles<D, HC, T, TK, S, C::kTileTok, C::kSub>(
                 p, pa, lo, hi, plan_sh->seq, plan_sh->base, stage_base, full_bar, empty_bar,
                 q_ring, kQSlot, q_full, q_empty, lane, abort_flag);
         } else {
@@ -692,7 +721,10 @@ gqa_split_kernel(const GqaParams p) {
             break;
         const T *qs = reinterpret_cast<const T *>(q_ring + (n_seg & 1) * kQSlot);
         float2 q2[HC][EP];
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        // fp8 cache: half of the 2^120 the widened codes lack goes into q,
+        // the other half into each row's scale.
+        const float qsc = C::kFp8 ? p.scale_log2 * kE4m3Half : p.scale_log2;
+        const float2 sc2 = make_float2(qsc, qsc);
 #pragma unroll
         for (int g = 0; g < HC; ++g) {
 #pragma unroll
@@ -724,8 +756,11 @@ gqa_split_kernel(const GqaParams p) {
                 ok = false;
                 break;
             }
-            const T *Ks = reinterpret_cast<const T *>(stage_base + stage * C::kStageBytes);
-            const T *Vs = Ks + C::kTileTok * D;
+            const TK *Ks = reinterpret_cast<const TK *>(stage_base + stage * C::kStageBytes);
+            const TK *Vs = Ks + C::kTileTok * D;
+            // fp8 cache: row scales after the codes
+            const float *ksc = reinterpret_cast<const float *>(Vs + C::kTileTok * D);
+            const float *vsc = ksc + C::kTileTok;
             const int tl = (int)(n - seg_t0);
             const int tok0 = walk.logical(walk.blk_off + tl / C::kSub) * kBlockSize +
                              (tl % C::kSub) * C::kTileTok + wig * C::kTPW;
@@ -738,13 +773,13 @@ gqa_split_kernel(const GqaParams p) {
 #pragma unroll
                 for (int i = 0; i < C::kChunk; ++i) {
                     const int it = ch * C::kChunk + i;
-                    const T *krow = Ks + (row0 + it * C::kRPW + rg) * D;
+                    const TK *krow = Ks + (row0 + it * C::kRPW + rg) * D;
 #pragma unroll
                     for (int g = 0; g < HC; ++g) acc[i * HC + g] = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int c = 0; c < C::kCPL; ++c) {
                         float2 kp[LP];
-                        load_pairs<T, C::kLE>(krow + col[c], kp);
+                        load_pairs<TK, C::kLE>(krow + col[c], kp);
 #pragma unroll
                         for (int g = 0; g < HC; ++g)
 #pragma unroll
@@ -762,7 +797,9 @@ gqa_split_kernel(const GqaParams p) {
                 for (int i = 0; i < RR::final_count(); ++i) {
                     const int v = base + i;
                     const int it = ch * C::kChunk + v / HC, g = v % HC;
-                    sc[(it * C::kRPW + rg) * C::kHCP + g] = part[i];
+                    float sv = part[i];
+                    if constexpr (C::kFp8) sv *= ksc[row0 + it * C::kRPW + rg] * kE4m3Half;
+                    sc[(it * C::kRPW + rg) * C::kHCP + g] = sv;
                 }
             }
             __syncwarp();
@@ -811,16 +848,18 @@ gqa_split_kernel(const GqaParams p) {
 #pragma unroll
             for (int it = 0; it < C::kIters; ++it) {
                 const int rl = it * C::kRPW + rg;
-                const T *vrow = Vs + (row0 + rl) * D;
+                const TK *vrow = Vs + (row0 + rl) * D;
                 float pg[C::kHCP];
                 load_row<C::kHCP>(sc + rl * C::kHCP, pg);
+                float vf = 1.f;
+                if constexpr (C::kFp8) vf = vsc[row0 + rl] * kE4m3Half;
                 float2 pp[HC];
 #pragma unroll
-                for (int g = 0; g < HC; ++g) pp[g] = make_float2(pg[g], pg[g]);
+                for (int g = 0; g < HC; ++g) pp[g] = make_float2(pg[g] * vf, pg[g] * vf);
 #pragma unroll
                 for (int c = 0; c < C::kCPL; ++c) {
                     float2 vp[LP];
-                    load_pairs<T, C::kLE>(vrow + col[c], vp);
+                    load_pairs<TK, C::kLE>(vrow + col[c], vp);
 #pragma unroll
                     for (int g = 0; g < HC; ++g)
 #pragma unroll
@@ -885,7 +924,9 @@ gqa_split_kernel(const GqaParams p) {
 #pragma unroll
                     for (int j = 0; j < LP; ++j)
                         *reinterpret_cast<float2 *>(&s_mo[(warp * HC + g) * D + col[c] + 2 * j]) =
-                            o2[g][c * LP + j];
+                            C::kFp8 ? __fmul2_rn(o2[g][c * LP + j],
+                                                 make_float2(kE4m3Half, kE4m3Half))
+                                    : o2[g][c * LP + j];
         }
         if ((lane % C::kTPW) == 0) {
 #pragma unroll

@@ -17,24 +17,24 @@ struct GqaLaunch {
 };
 
 // Shared-memory bytes the split kernel of this instantiation needs.
-template <int D, int HC, typename T>
-int gqa_smem_bytes() { return GqaCfg<D, HC, T>::kSmemBytes; }
+template <int D, int HC, typename T, typename TK = T>
+int gqa_smem_bytes() { return GqaCfg<D, HC, T, TK>::kSmemBytes; }
 
-template <int D, int HC, typename T>
+template <int D, int HC, typename T, typename TK = T>
 cudaError_t launch_gqa_impl(const GqaLaunch &L) {
-    using C = GqaCfg<D, HC, T>;
+    using C = GqaCfg<D, HC, T, TK>;
     static bool configured = false;   // per-process; attribute is per function
     cudaError_t e;
     if (!configured) {
         // The warpgroups' setmaxnreg shares must fit in the registers the
         // kernel is launched with, or the increase would never be granted.
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T>);
+        e = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T, TK>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs * C::kThreads <
             4 * 32 * C::kProducerRegs + C::kNW * 32 * C::kConsumerRegs)
             return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T>,
+        e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T, TK>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes);
         if (e != cudaSuccess) return e;
@@ -53,7 +53,7 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gqa_split_kernel<D, HC, T>, L.kp);
+    e = cudaLaunchKernelEx(&cfg, gqa_split_kernel<D, HC, T, TK>, L.kp);
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
     return cudaSuccess;
@@ -84,6 +84,23 @@ cudaError_t launch_gqa_d32(int HC, int bf16, const GqaLaunch &L);
 cudaError_t launch_gqa_d64(int HC, int bf16, const GqaLaunch &L);
 cudaError_t launch_gqa_d128(int HC, int bf16, const GqaLaunch &L);
 cudaError_t launch_gqa_d256(int HC, int bf16, const GqaLaunch &L);
+
+// bf16 queries over an fp8 (e4m3 + per-row fp32 scale) cache, d in {64, 128, 256}.
+template <int D>
+cudaError_t launch_gqa_fp8_d(int HC, const GqaLaunch &L) {
+    switch (HC) {
+        case 1: return launch_gqa_impl<D, 1, __nv_bfloat16, uint8_t>(L);
+        case 2: return launch_gqa_impl<D, 2, __nv_bfloat16, uint8_t>(L);
+        case 3: return launch_gqa_impl<D, 3, __nv_bfloat16, uint8_t>(L);
+        case 4: return launch_gqa_impl<D, 4, __nv_bfloat16, uint8_t>(L);
+        case 6: return launch_gqa_impl<D, 6, __nv_bfloat16, uint8_t>(L);
+        case 8: return launch_gqa_impl<D, 8, __nv_bfloat16, uint8_t>(L);
+        default: return cudaErrorInvalidValue;
+    }
+}
+cudaError_t launch_gqa_fp8_d64(int HC, const GqaLaunch &L);
+cudaError_t launch_gqa_fp8_d128(int HC, const GqaLaunch &L);
+cudaError_t launch_gqa_fp8_d256(int HC, const GqaLaunch &L);
 
 }  // namespace attn
 

@@ -19,4 +19,20 @@ struct KvAppendParams {
 
 cudaError_t launch_kv_append(const KvAppendParams &p, cudaStream_t stream);
 
+struct KvAppendFp8Params {
+    const __nv_bfloat16 *k_new;   // [B][H_kv][d]
+    const __nv_bfloat16 *v_new;
+    uint8_t *k_cache;             // [num_blocks][H_kv][64][d] e4m3 codes
+    uint8_t *v_cache;
+    float *k_scale;               // [num_blocks][H_kv][64] row scales
+    float *v_scale;
+    const int32_t *positions;
+    const int32_t *block_table;
+    unsigned *err;
+    int B, H_kv, d, max_blocks, num_blocks;
+    Visibility vis;
+};
+
+cudaError_t launch_kv_append_fp8(const KvAppendFp8Params &p, cudaStream_t stream);
+
 }  // namespace attn

@@ -288,6 +288,37 @@ int attn_decode_gqa_noalloc(const void *q, const void *k_cache,
                             int num_blocks, int dtype);
 
 /*
+ * attn_decode_gqa_fp8 -- attn_decode_gqa over an fp8 KV cache: quantised
+ * K/V halve the bytes the bandwidth-bound decode reads.  k_cache / v_cache
+ * [num_blocks][H_kv][64][d] hold OCP FP8 E4M3 codes (1 byte); k_scale /
+ * v_scale [num_blocks][H_kv][64] fp32 hold one scale per cached row, so the
+ * key/value used is code_value * row_scale (as written by kv_append_fp8).
+ * q and out are bf16 [B][H_q][d]; d in {64, 128, 256}; every group size runs
+ * on the CUDA-core kernel.  visibility may be null (full causal, identity
+ * table) or as for attn_decode_gqa_ext.  Scale arrays 16-byte aligned; other
+ * arguments, workspace and errors as attn_decode_gqa.
+ */
+int attn_decode_gqa_fp8(const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale, const int32_t *seq_lens,
+                        const int32_t *block_table, void *out, int B, int H_q, int H_kv, int d,
+                        float scale, const attn_visibility *visibility, void *stream,
+                        int max_blocks_per_seq, int num_blocks);
+
+/*
+ * kv_append_fp8 -- quantise and append the current token's K and V rows
+ * (bf16 [B][H_kv][d]) into the fp8 cache at positions[b] (through the table
+ * mapping of `visibility`, which may be null).  Each row x of d values is
+ * stored as E4M3 codes of x * (448 / amax), rounded to nearest even and
+ * saturated to +-448, with row scale amax / 448 (amax = max |x| in fp32; a
+ * zero row gets scale 0 and zero codes); both divisions are IEEE
+ * round-to-nearest.  Errors as kv_append.
+ */
+int kv_append_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                  float *k_scale, float *v_scale, const int32_t *positions,
+                  const int32_t *block_table, int B, int H_kv, int d, int max_blocks_per_seq,
+                  int num_blocks, const attn_visibility *visibility, void *stream);
+
+/*
  * attn_mla_absorb_q -- the key up-projection folded into the query, before
  * the absorbed MLA decode (attention-head §5.2): per sequence b and head h,
  *     q_latent[b][h][:] = sum_i q_c[b][h][i] * u_k[h][:][i]

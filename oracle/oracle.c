@@ -440,3 +440,52 @@ int orc_slot_offset(const int32_t *block_table, int max_blocks, int b, int pos,
                                       block_size, n_heads, head, row_width);
     return ORC_OK;
 }
+
+/*
+ * OCP FP8 E4M3 (the fp8 KV-cache format): 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent field 0 is subnormal (m/8 * 2^-6); no
+ * infinities; S.1111.111 is NaN; the largest finite magnitude is 448.
+ */
+double orc_e4m3_value(int code) {
+    const int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = (e == 0) ? (m / 8.0) * ldexp(1.0, -6)
+                              : (1.0 + m / 8.0) * ldexp(1.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Nearest finite E4M3 code to x, ties to the even code (mantissa bit 0),
+ * magnitudes past 448 saturating to 448, the sign kept (so -0 -> 0x80). */
+int orc_e4m3_encode(float x) {
+    const double a = fabs((double)x);
+    int best = 0;
+    double best_err = a;                       /* code 0x00 has value 0 */
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double err = fabs(orc_e4m3_value(c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return signbit(x) ? (best | 0x80) : best;
+}
+
+/* Row quantisation of the fp8 cache: amax = max |x| (fp32), scale = amax / 448,
+ * codes = e4m3(x * (448 / amax)), all fp32 arithmetic rounded to nearest; a
+ * zero row gets scale 0 and zero codes.  x [rows][d] fp32. */
+void orc_quantize_rows_e4m3(const float *x, int rows, int d, uint8_t *codes, float *scales) {
+    for (int r = 0; r < rows; ++r) {
+        const float *xr = x + (size_t)r * d;
+        float amax = 0.f;
+        for (int i = 0; i < d; ++i) {
+            const float v = fabsf(xr[i]);
+            if (v > amax) amax = v;
+        }
+        const float inv = amax > 0.f ? 448.f / amax : 0.f;
+        for (int i = 0; i < d; ++i) {
+            const float y = xr[i] * inv;
+            codes[(size_t)r * d + i] = (uint8_t)orc_e4m3_encode(y);
+        }
+        scales[r] = amax / 448.f;
+    }
+}

@@ -27,6 +27,12 @@ def _load():
         lib.orc_decode_gqa.restype = c_i
         lib.orc_decode_gqa_vis.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i, c_i, c_i, c_i]
         lib.orc_decode_gqa_vis.restype = c_i
+        lib.orc_e4m3_value.argtypes = [c_i]
+        lib.orc_e4m3_value.restype = c_d
+        lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.orc_e4m3_encode.restype = c_i
+        lib.orc_quantize_rows_e4m3.argtypes = [c_p, c_i, c_i, c_p, c_p]
+        lib.orc_quantize_rows_e4m3.restype = None
         lib.orc_decode_mla.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i]
         lib.orc_decode_mla.restype = c_i
         lib.orc_mla_explicit.argtypes = [c_p] * 8 + [c_i] * 8 + [c_d]
@@ -204,6 +210,35 @@ def mla_explicit(q_c, q_rope, latent_cache, seq_lens, block_table, U_K, U_V,
     if rc != 0:
         raise RuntimeError(f"oracle mla_explicit failed with status {rc}")
     return out
+
+
+def e4m3_table():
+    """Values of the 256 OCP FP8 E4M3 codes (fp64; NaN for the two NaN codes)."""
+    lib = _load()
+    return np.array([lib.orc_e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(x):
+    """Nearest E4M3 code of fp32 x (ties to even, saturating at 448)."""
+    return _load().orc_e4m3_encode(float(np.float32(x)))
+
+
+def quantize_rows_e4m3(x):
+    """(codes uint8 [..., d], scales fp32 [...]) of the fp8 cache row
+    quantisation: scale = amax / 448, codes = E4M3(x * (448 / amax)) in fp32."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    d = x.shape[-1]
+    rows = int(np.prod(x.shape[:-1])) if x.ndim > 1 else 1
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    scales = np.zeros(x.shape[:-1], dtype=np.float32)
+    _load().orc_quantize_rows_e4m3(x.ctypes.data, rows, d, codes.ctypes.data,
+                                   scales.ctypes.data)
+    return codes, scales
+
+
+def dequantize_e4m3(codes, scales):
+    """fp64 cache rows: code value times its row scale."""
+    return e4m3_table()[np.asarray(codes)] * np.asarray(scales, dtype=np.float64)[..., None]
 
 
 def mla_absorb_q(q_c, U_K):

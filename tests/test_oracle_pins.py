@@ -475,3 +475,49 @@ def test_vis_ring_table_reads_the_same_rows():
         vr[ring_table[0, slot]] = v[logical]
     got = orc.decode_gqa_vis(q, kr, vr, np.array([T], dtype=np.int32), ring_table, 0.25, window=w, sink=g, ring=R)
     assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------- fp8 (E4M3) KV cache
+def test_e4m3_values_match_the_format():
+    """Closed forms of the OCP FP8 E4M3 format: bias 7, 3 mantissa bits,
+    subnormals m/8 * 2^-6, largest finite 448, S.1111.111 NaN."""
+    t = orc.e4m3_table()
+    assert t[0x00] == 0.0 and t[0x38] == 1.0 and t[0xB8] == -1.0
+    assert t[0x7E] == 448.0 and t[0xFE] == -448.0
+    assert t[0x08] == 2.0 ** -6 and t[0x01] == 2.0 ** -9 and t[0x07] == 7 * 2.0 ** -9
+    assert t[0x40] == 2.0 and t[0x3F] == 1.875
+    assert np.isnan(t[0x7F]) and np.isnan(t[0xFF])
+    assert np.sum(np.isnan(t)) == 2
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    t = orc.e4m3_table()
+    for c in range(256):
+        if c in (0x7F, 0xFF):
+            continue
+        assert orc.e4m3_encode(t[c]) == c, hex(c)
+    assert orc.e4m3_encode(1.0625) == 0x38      # tie 1.0 / 1.125 -> even mantissa
+    assert orc.e4m3_encode(1.1875) == 0x3A      # tie 1.125 / 1.25 -> 1.25
+    assert orc.e4m3_encode(1.9375) == 0x40      # tie across the binade -> 2.0
+    assert orc.e4m3_encode(1000.0) == 0x7E and orc.e4m3_encode(-1000.0) == 0xFE
+    assert orc.e4m3_encode(460.0) == 0x7E       # past 448 saturates
+
+
+def test_quantize_rows_error_bound():
+    """Each row's largest element maps to 448 (within rounding) and every
+    element is reproduced to e4m3's half-ulp: relative 2^-4 for normals,
+    absolute 2^-10 * scale below the normal range."""
+    rng = np.random.default_rng(40)
+    x = (rng.standard_normal((50, 128)) * rng.uniform(0.01, 30, (50, 1))).astype(np.float32)
+    x[7] = 0.0                                        # a zero row
+    codes, scales = orc.quantize_rows_e4m3(x)
+    assert scales[7] == 0.0 and not codes[7].any()
+    deq = orc.dequantize_e4m3(codes, scales)
+    amax = np.abs(x).max(axis=1)
+    for r in range(50):
+        if amax[r] == 0:
+            continue
+        assert abs(np.abs(deq[r]).max() - amax[r]) <= 1e-6 * amax[r]
+        err = np.abs(deq[r] - x[r])
+        bound = np.maximum(np.abs(x[r]) * 2.0 ** -4, scales[r] * 2.0 ** -10) * (1 + 1e-6)
+        assert np.all(err <= bound), r

@@ -38,6 +38,7 @@ class GQAConfig:
     window: int = 0
     sink: int = 0                          # global tokens kept visible (with a window)
     ring: int = 0                          # ring table of this many blocks after the sink ones
+    kv_fp8: bool = False                   # fp8 (E4M3 + per-row scale) cache, bf16 q
     contiguous: bool = False               # identity block table
     seed: int = SEED_BASE
     ragged: Optional[tuple] = None         # (lo, hi) inclusive range of T_b
@@ -91,6 +92,9 @@ def ragged_config(window: int) -> GQAConfig:
 
 RAGGED_FULL = ragged_config(0)
 RAGGED_WINDOW = ragged_config(4096)
+# The Llama-3-8B shape over an fp8 (E4M3 + per-row scale) KV cache.
+LLAMA3_8B_FP8 = GQAConfig("llama3_8b_gqa_fp8kv_B16_Hq32_Hkv8_d128_T4096", B=16, H_q=32,
+                          H_kv=8, d=128, T=4096, kv_fp8=True, seed=SEED_BASE + 1)
 # Window plus 64 global tokens on the same shape; and the same on a ring table
 # that keeps only the 1 sink block and the 65 blocks a 4096-key window can reach.
 RAGGED_WINDOW_SINK = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_g64", B=8, H_q=24,
@@ -103,7 +107,7 @@ MLA_DSV2 = MLAConfig("mla_absorbed_bf16_B32_H128_dc512_dr64_T8192", B=32)
 
 WORKLOADS = {c.name: c for c in [TINY, LLAMA3_8B, *SWEEP, RAGGED_FULL,
                                  RAGGED_WINDOW, RAGGED_WINDOW_SINK, RAGGED_WINDOW_RING,
-                                 MLA_DSV2]}
+                                 LLAMA3_8B_FP8, MLA_DSV2]}
 
 
 def _generator(seed: int, device) -> torch.Generator:
@@ -172,12 +176,16 @@ class GQAInputs:
     window: int
     scale: float
     seq_list: List[int] = field(default_factory=list)
+    k_scale: Optional[torch.Tensor] = None   # fp8 cache: [num_blocks][H_kv][64] row scales
+    v_scale: Optional[torch.Tensor] = None
 
     def to(self, device):
+        mv = (lambda t: None if t is None else t.to(device))
         return GQAInputs(self.cfg, self.q.to(device), self.k_cache.to(device),
                          self.v_cache.to(device), self.seq_lens.to(device),
                          self.block_table.to(device), self.num_blocks,
-                         self.window, self.scale, list(self.seq_list))
+                         self.window, self.scale, list(self.seq_list),
+                         mv(self.k_scale), mv(self.v_scale))
 
 
 def make_gqa_inputs(cfg: GQAConfig, device="cpu", seed: Optional[int] = None,
@@ -194,11 +202,24 @@ def make_gqa_inputs(cfg: GQAConfig, device="cpu", seed: Optional[int] = None,
         table, nblk = make_block_table(seq, g, cfg.contiguous,
                                        extra_blocks_per_seq, pool_slack)
     q = randn((cfg.B, cfg.H_q, cfg.d), g, cfg.dtype)
+    sl = torch.tensor(seq, dtype=torch.int32, device=g.device)
+    win = cfg.window if window is None else window
+    if cfg.kv_fp8:
+        # Stand-in quantised rows: uniform E4M3 codes (the two NaN codes
+        # replaced by +-448) with row scales of N(0,1)-like rows (amax ~3).
+        shape = (nblk, cfg.H_kv, BLOCK_SIZE, cfg.d)
+        codes = []
+        for _ in range(2):
+            c = torch.randint(0, 256, shape, generator=g, device=g.device, dtype=torch.int32)
+            c = torch.where((c & 0x7F) == 0x7F, c - 1, c)
+            codes.append(c.to(torch.uint8))
+        scales = [(torch.rand(shape[:3], generator=g, device=g.device) * 2 + 2) / 448
+                  for _ in range(2)]
+        return GQAInputs(cfg, q, codes[0], codes[1], sl, table, nblk, win, cfg.scale, seq,
+                         scales[0], scales[1])
     k = randn((nblk, cfg.H_kv, BLOCK_SIZE, cfg.d), g, cfg.dtype)
     v = randn((nblk, cfg.H_kv, BLOCK_SIZE, cfg.d), g, cfg.dtype)
-    sl = torch.tensor(seq, dtype=torch.int32, device=g.device)
-    return GQAInputs(cfg, q, k, v, sl, table, nblk,
-                     cfg.window if window is None else window, cfg.scale, seq)
+    return GQAInputs(cfg, q, k, v, sl, table, nblk, win, cfg.scale, seq)
 
 
 @dataclass
