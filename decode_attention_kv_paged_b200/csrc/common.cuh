@@ -78,6 +78,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+// As mbar_try_wait, with a short suspend hint (kWatchNs), for a waiter that
+// has something else to look at between polls.
+constexpr uint32_t kWatchNs = 1000;
+__device__ __forceinline__ bool mbar_try_wait_short(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kWatchNs)
+        : "memory");
+    return done != 0;
+}
+
 // Non-blocking probe of an mbarrier phase.
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t done;
@@ -116,6 +131,48 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
             }
         }
     }
+}
+
+// mbar_wait for a whole warp (all 32 lanes call it together) that runs
+// `idle()` between polls of at most kWatchNs each.  Same bounds and results
+// as mbar_wait; the lanes leave together.
+template <typename F>
+__device__ __forceinline__ bool mbar_wait_watch(uint64_t *bar, uint32_t parity,
+                                                unsigned long long timeout_ns,
+                                                unsigned *err, volatile int *abort,
+                                                F &&idle) {
+    unsigned long long t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (__any_sync(0xffffffffu, mbar_try_wait_short(bar, parity))) return true;
+        if (*abort) return false;
+        idle();
+        if ((it & 7u) == 7u) {
+            const unsigned long long now = global_timer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > timeout_ns) {
+                if ((threadIdx.x & 31) == 0) raise_error(err, kErrTimeout);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// GPU-scope relaxed load and store of a 32-bit word, and an acquire-release
+// fence: a relaxed read that observes a value written by another CTA's
+// release sequence, followed by the fence, orders this CTA's later reads
+// after that CTA's writes.
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_gpu(unsigned *p, unsigned v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // Named barrier among `count` threads (multiple of 32), id 1..15.

@@ -94,13 +94,15 @@ struct GqaCfg {
     static constexpr int kS = (int)sizeof(TK);                   // cache bytes / element
     static constexpr bool kFp8 = sizeof(TK) == 1;
     // Warp specialisation: warpgroup 0 is the producer (its warp 0 streams
-    // the tiles; the other three exit at once), warpgroups 1 and 2 are the
-    // kNW compute warps.  setmaxnreg moves the producer group's registers to
-    // the compute groups; the shares add up to the launch's 384 x 168.
+    // the tiles, warps 1-3 run the segment epilogues), warpgroups 1 and 2
+    // are the kNW compute warps.  setmaxnreg moves registers from the
+    // producer group to the compute groups; the shares add up to the
+    // launch's 384 x 168.  200 per compute thread is what their loop needs;
+    // the rest keeps the epilogue's merge and combine out of local memory.
     static constexpr int kNW = 8;                                 // compute warps
     static constexpr int kThreads = 32 * (4 + kNW);
-    static constexpr int kProducerRegs = 40;
-    static constexpr int kConsumerRegs = 232;
+    static constexpr int kProducerRegs = 104;
+    static constexpr int kConsumerRegs = 200;
     static constexpr int kLaunchRegs = 168;
     static_assert(4 * 32 * kProducerRegs + kNW * 32 * kConsumerRegs <=
                       kThreads * kLaunchRegs, "register split exceeds the launch");
@@ -136,7 +138,7 @@ struct GqaCfg {
     static constexpr int kScoreBytes = kNW * kTPW * kHCP * 4;
     static constexpr int kMergeOBytes = kNW * HC * D * 4;
     static constexpr int kMergeMLBytes = 2 * kNW * HC * 4;
-    static constexpr int kEpiBytes = (kNW + 2) * HC * 4;         // merge weights
+    static constexpr int kEpiBytes = ((kNW + 2) * HC * 4 + 15) / 16 * 16;  // merge weights
     static constexpr int kEpiThreads = 96;                        // producer WG warps 1-3
     static constexpr int kQBytes = HC * D * (int)sizeof(T);      // one unit's queries
     static constexpr int kQRingBytes = 2 * ((kQBytes + 127) / 128 * 128);
@@ -146,7 +148,12 @@ struct GqaCfg {
     static constexpr int kStagesRaw = (kSmemBudget - kOther) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static_assert(kTPW * kHPP == 32, "softmax lane map");
-    static constexpr int kSmemBytes = kStages * kStageBytes + kOther;
+    // What the ring leaves over holds up to kPreMax other splits' partials
+    // (fp32 O and lse of one unit), prefetched by the epilogue warps.
+    static constexpr int kPreUnit = HC * D * 4 + HC * 4;
+    static constexpr int kPreRaw = (kSmemBudget - kStages * kStageBytes - kOther) / kPreUnit;
+    static constexpr int kPreMax = kPreRaw > 8 ? 8 : kPreRaw;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kOther + kPreMax * kPreUnit;
     static_assert(kStages >= kNG + 2, "not enough shared memory for the ring");
     static_assert(kLPR >= 4 && kLPR <= 32 && (kLPR & (kLPR - 1)) == 0, "LPR");
     static_assert(kIters >= 1 && kIters * kRPW == kTPW, "rows per warp");
@@ -433,18 +440,61 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
     }
 }
 
+// Loads the published partials of a unit's other splits (slots slot0 ..
+// slot0 + ns - 1 except this CTA's own, `own`) into shared memory: pf_o
+// [ns - 1][HC][D] and pf_lse [ns - 1][HC], other split i at index
+// i - (i > own).  Each thread loads the elements it later combines (the same
+// thread-to-element map as the combine), so no barrier is needed between.
+template <int D, int HC, int NT>
+__device__ __forceinline__ void prefetch_splits(const GqaParams &p, int et, long long slot0,
+                                                int ns, int own, float *pf_o, float *pf_lse) {
+    for (int e = et * 4; e < HC * D; e += NT * 4) {
+        for (int i0 = 0; i0 < ns; i0 += 4) {
+            float4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (i0 + k < ns && i0 + k != own)
+                    v[k] = __ldcg(reinterpret_cast<const float4 *>(
+                        p.ws_o + (slot0 + i0 + k) * HC * D + e));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + k;
+                if (i < ns && i != own)
+                    *reinterpret_cast<float4 *>(pf_o + (size_t)(i - (i > own)) * HC * D + e) =
+                        v[k];
+            }
+        }
+    }
+    for (int k = et; k < ns * HC; k += NT) {
+        const int i = k / HC;
+        if (i != own) pf_lse[(i - (i > own)) * HC + k % HC] = __ldcg(p.ws_lse + slot0 * HC + k);
+    }
+}
+
 // Segment epilogue, run by the kEpiThreads epilogue threads (et = 0 ..) on the
 // compute warps' stashed states: s_mo [NW][HC][D] partial outputs, s_mm /
 // s_ml [NW][HC] running max / sum of each warp.  Merges them, then writes the
-// unit's output (one split) or its fp32 partial; the last split of a unit to
-// arrive combines the unit's partials in CTA order (fixed, deterministic):
-//     out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L).
-template <int D, int HC, typename T, int NW, int NT>
+// unit's output (one split) or combines the unit's splits:
+//     out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L),
+// over the splits in CTA order (fixed, deterministic).  A split that finds
+// every other split of its unit already arrived is the last one: it combines
+// at once, taking its own (O, lse) from shared memory, without publishing
+// them -- the common case for the last segment of a CTA, whose unit's other
+// split ran at the start of the next CTA's range.  `pre` says this thread
+// has already loaded the other splits' partials into pf_o / pf_lse (while
+// the segment ran).  Otherwise the split publishes its fp32 partial and
+// arrives on the unit's counter, and the last split to arrive combines.
+// Either way the same values are summed in the same order.
+template <int D, int HC, typename T, int NW, int NT, int PRE>
 __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0, int ns,
                                  long long slot, T *out_u, float *s_mo, const float *s_mm,
-                                 const float *s_ml, float *s_w, volatile int *last_flag) {
+                                 const float *s_ml, float *s_w, volatile int *last_flag,
+                                 bool pre, float *pf_o, float *pf_lse) {
     float *s_inv = s_w + NW * HC;          // [HC]
     float *s_lse = s_inv + HC;             // [HC]
+    // Other splits already arrived?  Read early; used after the merge.
+    unsigned seen = 0;
+    if (ns > 1 && et == 0) seen = pre ? (unsigned)(ns - 1) : ld_relaxed_gpu(p.ws_cnt + u);
     // Per head: the common max, each warp's weight, the normaliser.
     if (et < HC) {
         const int g = et;
@@ -462,6 +512,8 @@ __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0
         s_lse[g] = M + log2f(den);
     }
     named_barrier(1, NT);
+    // The merged output; for a split unit it replaces warp 0's stash (each
+    // element is read and rewritten by the same thread).
     for (int e = et * 4; e < HC * D; e += NT * 4) {
         const int g = e / D;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -482,28 +534,89 @@ __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0
             out_u[e + 2] = ElemTraits<T>::from_float(acc.z);
             out_u[e + 3] = ElemTraits<T>::from_float(acc.w);
         } else {
-            *reinterpret_cast<float4 *>(p.ws_o + slot * HC * D + e) = acc;
+            *reinterpret_cast<float4 *>(s_mo + e) = acc;
         }
     }
     if (ns == 1) return;
-    if (et < HC) p.ws_lse[slot * HC + et] = s_lse[et];
-    // The barrier orders every thread's partial before thread 0's fence,
-    // which publishes them, cumulatively, before the arrival (and orders the
-    // last arrival's reads after the other splits' partials).
-    named_barrier(1, NT);
+    // The other splits' (O, lse) fit in the prefetch buffer: the combine
+    // reads them from shared memory, and the last split need not publish.
+    const bool fits = ns - 1 <= PRE;
     if (et == 0) {
-        __threadfence();
-        const bool last = unit_arrive(p.ws_cnt + u, ns);
-        if (last) __threadfence();
-        *last_flag = last ? 1 : 0;
+        const bool fast = fits && seen == (unsigned)(ns - 1);
+        if (fast) {
+            fence_acq_rel_gpu();               // the other splits' partials, then
+            st_relaxed_gpu(p.ws_cnt + u, 0u);  // the counter back to zero
+        }
+        *last_flag = fast ? 2 : 0;
     }
     named_barrier(1, NT);
-    if (!*last_flag) return;
+    if (*last_flag != 2) {
+        // Publish this split's partial and arrive.  The barrier orders every
+        // thread's stores before thread 0's fence, which publishes them,
+        // cumulatively, before the arrival (and orders the last arrival's
+        // reads after the other splits' partials).
+        for (int e = et * 4; e < HC * D; e += NT * 4)
+            *reinterpret_cast<float4 *>(p.ws_o + slot * HC * D + e) =
+                *reinterpret_cast<const float4 *>(s_mo + e);
+        if (et < HC) p.ws_lse[slot * HC + et] = s_lse[et];
+        named_barrier(1, NT);
+        if (et == 0) {
+            __threadfence();
+            const bool last = unit_arrive(p.ws_cnt + u, ns);
+            if (last) __threadfence();
+            *last_flag = last ? 1 : 0;
+        }
+        named_barrier(1, NT);
+        if (!*last_flag) return;
+    }
     const long long slot0 = u + c0;
-    if (ns <= NW * D) {
-        // Split weights 2^(lse - L) in shared memory (the stash is no longer
-        // needed), then each output is one weighted sum.
-        float *wts = s_mo;                 // [ns][HC]
+    const int own = (int)(slot - slot0);
+    float *wts = s_mo + HC * D;            // [ns][HC] split weights
+    if (fits) {
+        // The other splits' (O, lse) in shared memory (loaded here, in one
+        // round trip, unless already prefetched), this split's own from the
+        // merge; then the split weights 2^(lse - L), and each output is one
+        // weighted sum.
+        if (!pre) prefetch_splits<D, HC, NT>(p, et, slot0, ns, own, pf_o, pf_lse);
+        for (int i = et; i < ns * HC; i += NT) {
+            const int si = i / HC;
+            wts[i] = si == own ? s_lse[i % HC] : pf_lse[(si - (si > own)) * HC + i % HC];
+        }
+        named_barrier(1, NT);
+        if (et < HC) {
+            const int g = et;
+            float L = kNegInf;
+            for (int i = 0; i < ns; ++i) L = fmaxf(L, wts[i * HC + g]);
+            float den = 0.f;
+            for (int i = 0; i < ns; ++i) {
+                const float w = exp2f(wts[i * HC + g] - L);
+                wts[i * HC + g] = w;
+                den += w;
+            }
+            s_inv[g] = 1.f / den;
+        }
+        named_barrier(1, NT);
+        for (int e = et * 4; e < HC * D; e += NT * 4) {
+            const int g = e / D;
+            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+            for (int i = 0; i < ns; ++i) {
+                const float w = wts[i * HC + g];
+                const float4 v = *reinterpret_cast<const float4 *>(
+                    i == own ? s_mo + e : pf_o + (size_t)(i - (i > own)) * HC * D + e);
+                r0 = fmaf(w, v.x, r0);
+                r1 = fmaf(w, v.y, r1);
+                r2 = fmaf(w, v.z, r2);
+                r3 = fmaf(w, v.w, r3);
+            }
+            const float iv = s_inv[g];
+            out_u[e] = ElemTraits<T>::from_float(r0 * iv);
+            out_u[e + 1] = ElemTraits<T>::from_float(r1 * iv);
+            out_u[e + 2] = ElemTraits<T>::from_float(r2 * iv);
+            out_u[e + 3] = ElemTraits<T>::from_float(r3 * iv);
+        }
+    } else if (ns <= (NW - 1) * D) {
+        // More splits: weights in shared memory, partials from the
+        // published copies (this split's own included), eight loads in flight.
         for (int i = et; i < ns * HC; i += NT) wts[i] = __ldcg(p.ws_lse + slot0 * HC + i);
         named_barrier(1, NT);
         if (et < HC) {
@@ -523,7 +636,7 @@ __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0
             const int g = e / D;
             const float *src = p.ws_o + slot0 * HC * D + e;
             float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
-#pragma unroll 4
+#pragma unroll 8
             for (int i = 0; i < ns; ++i) {
                 const float w = wts[i * HC + g];
                 const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)i * HC * D));
@@ -539,6 +652,7 @@ __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0
             out_u[e + 3] = ElemTraits<T>::from_float(r3 * iv);
         }
     } else {
+        // Many splits: everything from the published partials.
         for (int e = et * 4; e < HC * D; e += NT * 4) {
             const int g = e / D, k = e % D;
             float L = kNegInf;
@@ -578,6 +692,8 @@ gqa_split_kernel(const GqaParams p) {
     float *s_ml = s_mm + C::kNW * HC;
     float *s_w = s_ml + C::kNW * HC;                    // epilogue scratch
     unsigned char *misc = reinterpret_cast<unsigned char *>(s_w + C::kEpiBytes / 4);
+    float *pf_o = reinterpret_cast<float *>(misc + C::kMiscBytes);   // [kPreMax][HC][D]
+    float *pf_lse = pf_o + C::kPreMax * HC * D;                       // [kPreMax][HC]
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(misc);
     uint64_t *empty_bar = full_bar + S;
     uint64_t *q_full = empty_bar + S;                   // [2]
@@ -651,17 +767,33 @@ gqa_split_kernel(const GqaParams p) {
             SegmentWalker ew;
             ew.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
             for (int es = 0; !ew.done(); ++es) {
-                if (!mbar_wait(epi_full, (uint32_t)(es & 1), p.timeout_ns, p.err, abort_flag))
-                    break;
                 const int len = ew.seg_len();
                 const long long u = (long long)ew.b * units + ew.unit;
                 const long long s_u = ew.pos - ew.blk_off;     // the unit's first block
                 const int c0 = cta_of(s_u, W, P);
                 const int ns = cta_of(s_u + ew.nb - 1, W, P) - c0 + 1;
+                const int own = (int)blockIdx.x - c0;
+                // While the segment runs, watch the unit's counter: once the
+                // other splits have all arrived, load their partials.
+                bool pre = false;
+                const bool watch = ns > 1 && ns - 1 <= C::kPreMax;
+                const unsigned *cnt = p.ws_cnt + u;
+                auto idle = [&]() {
+                    if (watch && !pre && ld_relaxed_gpu(cnt) == (unsigned)(ns - 1)) {
+                        fence_acq_rel_gpu();
+                        prefetch_splits<D, HC, C::kEpiThreads>(p, et, u + c0, ns, own, pf_o,
+                                                                pf_lse);
+                        pre = true;
+                    }
+                };
+                if (!mbar_wait_watch(epi_full, (uint32_t)(es & 1), p.timeout_ns, p.err,
+                                     abort_flag, idle))
+                    break;
                 const int head0 = (ew.unit / p.n_hc) * p.group + (ew.unit % p.n_hc) * HC;
                 T *out_u = static_cast<T *>(p.out) + ((size_t)ew.b * p.H_q + head0) * D;
-                segment_epilogue<D, HC, T, C::kNW, C::kEpiThreads>(
-                    p, et, u, c0, ns, u + blockIdx.x, out_u, s_mo, s_mm, s_ml, s_w, last_flag);
+                segment_epilogue<D, HC, T, C::kNW, C::kEpiThreads, C::kPreMax>(
+                    p, et, u, c0, ns, u + blockIdx.x, out_u, s_mo, s_mm, s_ml, s_w, last_flag,
+                    pre, pf_o, pf_lse);
                 mbar_arrive(epi_empty);
                 ew.advance(len);
             }
