@@ -13,8 +13,8 @@
 //   * One CTA per SM over the split-KV partition (plan.cuh).  Warp 0 issues
 //     2-D TMA loads (128-byte swizzle) of each 64-token K and V tile of the
 //     paged cache into a multi-stage ring and of the unit's query rows; one
-//     thread of warp 1 issues tcgen05 MMAs as their inputs become ready;
-//     warps 4-7 run the softmax and the epilogue.
+//     thread of warp 1 issues the S MMAs and one of warp 2 the P V MMAs as
+//     their inputs become ready; warps 4-7 run the softmax and the epilogue.
 //   * S: M = 64 query rows, N = 64 tokens, K = d, both operands in shared
 //     memory, fp32 accumulator in TMEM (double-buffered).  The M = 64
 //     accumulator puts row r in TMEM lane (r % 16) + 32 (r / 16), so each
@@ -136,7 +136,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_init(&bars->pv_done[0], 1);
         mbar_init(&bars->pv_done[1], 1);
         mbar_init(&bars->o_free, 128);
-        mbar_init(&bars->mma_final, 1);
+        mbar_init(&bars->mma_final, 2);     // one commit per issuing thread
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -198,19 +198,17 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mbar_wait(&bars->q_full, (uint32_t)((seg - 1) & 1), p.timeout_ns, p.err, nullptr);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2) {
         // ============================================================ MMA
-        // One thread issues in a fixed order -- S(0), S(1), then S(i + 2) and
-        // P V(i) for each tile i -- polling each barrier it needs (a sleeping
-        // wait wakes up too late for this chain).
+        // Two issuing threads: lane 0 of warp 1 issues S(n) = Q K(n)^T for
+        // every tile in order, lane 0 of warp 2 issues O += P(i) V(i).  Each
+        // chain waits only on its own inputs (S on the staged tile and a free
+        // S buffer, P V on the softmax's P), so the two streams of MMAs
+        // overlap instead of queueing behind one thread.  A stage is released
+        // by the commit after P V(i): S(i) has completed by then, since the
+        // softmax read it before producing P(i).  Barriers are polled (a
+        // sleeping wait wakes up too late for these chains).
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16(kTcM, 64, 0, 0);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, 0, 1);
-            const uint32_t q_base = smem_u32(sQ), c_base = smem_u32(sC), p_base = smem_u32(sP);
-            TileCursor cs, cv;
-            cs.init(pa, lo, hi, first_seq, first_base);
-            cv.init(pa, lo, hi, first_seq, first_base);
-            int seg_s = 0, seg_v = 0;
             auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
                 unsigned long long t0 = 0;
                 for (uint32_t it = 0;; ++it) {
@@ -231,57 +229,70 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             };
-            // S(n) = Q K(n)^T into S buffer n % 2.
-            auto issue_s = [&](int n) -> bool {
-                const bool first = cs.t == 0, last = cs.t == cs.len - 1;
-                const int st = n % C::kStages, sb = n & 1;
-                if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) return false;
-                if (!wait(&bars->c_full[st], (uint32_t)((n / C::kStages) & 1))) return false;
-                if (n >= 2 && !wait(&bars->s_free[sb], (uint32_t)(((n - 2) >> 1) & 1)))
-                    return false;
-                tc_fence_after();
-                const uint32_t kst = c_base + st * C::kStageBytes;
-                for (int j = 0; j < C::kBoxes; ++j)
+            const uint32_t c_base = smem_u32(sC);
+            if (warp == 1) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16(kTcM, 64, 0, 0);
+                const uint32_t q_base = smem_u32(sQ);
+                TileCursor cs;
+                cs.init(pa, lo, hi, first_seq, first_base);
+                int seg_s = 0;
+                for (int n = 0; n < n_tiles; ++n) {
+                    // S(n) into S buffer n % 2, once the softmax of tile
+                    // n - 2 has read it.
+                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
+                    const int st = n % C::kStages, sb = n & 1;
+                    if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) break;
+                    if (!wait(&bars->c_full[st], (uint32_t)((n / C::kStages) & 1))) break;
+                    if (n >= 2 && !wait(&bars->s_free[sb], (uint32_t)(((n - 2) >> 1) & 1)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t kst = c_base + st * C::kStageBytes;
+                    for (int j = 0; j < C::kBoxes; ++j)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t a =
+                                umma_desc_sw128(q_base + j * kTcBox + k * 32, 16, 1024);
+                            const uint64_t b = umma_desc_sw128(kst + j * kTcBox + k * 32, 16, 1024);
+                            umma_bf16(tmem + C::kTmemS + 64 * sb, a, b, idesc_s, (j | k) != 0);
+                        }
+                    umma_commit(&bars->s_full[sb]);
+                    if (last) umma_commit(&bars->q_empty);
+                    if (first) ++seg_s;
+                    cs.next();
+                }
+            } else {
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, 0, 1);
+                const uint32_t p_base = smem_u32(sP);
+                TileCursor cv;
+                cv.init(pa, lo, hi, first_seq, first_base);
+                int seg_v = 0;
+                for (int i = 0; i < n_tiles; ++i) {
+                    // O += P(i) V(i), P from buffer i % 2 (hi and lo halves); a
+                    // segment's first P V overwrites O once the previous
+                    // segment's output has been read.
+                    const bool first = cv.t == 0;
+                    if (!wait(&bars->p_full[i & 1], (uint32_t)((i >> 1) & 1))) break;
+                    if (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))
+                        break;
+                    tc_fence_after();
+                    const int st = i % C::kStages;
+                    const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kTcBox;
+                    const uint32_t pb = p_base + (i & 1) * 2 * kTcPBytes;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t a = umma_desc_sw128(q_base + j * kTcBox + k * 32, 16, 1024);
-                        const uint64_t b = umma_desc_sw128(kst + j * kTcBox + k * 32, 16, 1024);
-                        umma_bf16(tmem + C::kTmemS + 64 * sb, a, b, idesc_s, (j | k) != 0);
+                        const uint64_t b = umma_desc_sw128(vst + k * 2048, kTcBox, 1024);
+                        const uint64_t a_hi = umma_desc_sw128(pb + k * 32, 16, 1024);
+                        const uint64_t a_lo = umma_desc_sw128(pb + kTcPBytes + k * 32, 16, 1024);
+                        umma_bf16(tmem + C::kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
+                        umma_bf16(tmem + C::kTmemO, a_lo, b, idesc_pv, 1);
                     }
-                umma_commit(&bars->s_full[sb]);
-                if (last) umma_commit(&bars->q_empty);
-                if (first) ++seg_s;
-                cs.next();
-                return true;
-            };
-            bool ok = true;
-            for (int n = 0; ok && n < 2 && n < n_tiles; ++n) ok = issue_s(n);
-            for (int i = 0; ok && i < n_tiles; ++i) {
-                if (i + 2 < n_tiles && !issue_s(i + 2)) break;
-                // O += P(i) V(i), P from buffer i % 2 (hi and lo halves).
-                const bool first = cv.t == 0;
-                if (!wait(&bars->p_full[i & 1], (uint32_t)((i >> 1) & 1)) ||
-                    (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))) {
-                    ok = false;
-                    break;
+                    umma_commit(&bars->c_empty[st]);
+                    umma_commit(&bars->pv_done[i & 1]);
+                    if (first) ++seg_v;
+                    cv.next();
                 }
-                tc_fence_after();
-                const int st = i % C::kStages;
-                const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kTcBox;
-                const uint32_t pb = p_base + (i & 1) * 2 * kTcPBytes;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t b = umma_desc_sw128(vst + k * 2048, kTcBox, 1024);
-                    const uint64_t a_hi = umma_desc_sw128(pb + k * 32, 16, 1024);
-                    const uint64_t a_lo = umma_desc_sw128(pb + kTcPBytes + k * 32, 16, 1024);
-                    umma_bf16(tmem + C::kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
-                    umma_bf16(tmem + C::kTmemO, a_lo, b, idesc_pv, 1);
-                }
-                umma_commit(&bars->c_empty[st]);
-                umma_commit(&bars->pv_done[i & 1]);
-                if (first) ++seg_v;
-                cv.next();
             }
+            // Both issuers' MMAs complete before the tensor memory is freed.
             umma_commit(&bars->mma_final);
             mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
         }

@@ -14,8 +14,12 @@ int gqa_tc_heads_per_cta(int G);
 // Copies of a group of HC heads in the 64 MMA rows (each takes a token
 // slice); the kernel writes this many partials per (unit, CTA) slot.
 int gqa_tc_copies(int HC);
-// Group size from which the tensor-core path is the default.
-constexpr int kTcMinGroup = 8;
+// Group size from which the tensor-core path is the default.  Measured on
+// B200 (T = 32768, d = 128): at G = 8 the CUDA-core kernel and the M = 64
+// tensor-core kernel tie (d = 64: CUDA cores 20% faster); from G = 16 the
+// tensor cores win by 1.8x or more (the CUDA-core kernel then splits the
+// group and reads each K/V tile once per chunk of 8 heads).
+constexpr int kTcMinGroup = 9;
 
 cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC);
 

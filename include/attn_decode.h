@@ -218,10 +218,11 @@ int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype,
 int attn_set_num_ctas(int num_ctas);
 
 /*
- * attn_set_gqa_path -- testing/tuning hook: -1 = automatic, 0 = force the
- * CUDA-core kernel, 1 = force the tensor-core path where it is supported (the
- * M = 128 kernel for d <= 128 and units of <= 32 heads, else the M = 64
- * kernel), 2 = force the M = 64 tensor-core kernel.
+ * attn_set_gqa_path -- testing/tuning hook: -1 = automatic (the CUDA-core
+ * kernel for groups of up to 8 heads, the M = 64 tensor-core kernel for
+ * larger groups), 0 = force the CUDA-core kernel, 1 = force the tensor-core
+ * path with the M = 128 kernel where it applies (d <= 128 and units of <= 32
+ * heads, else the M = 64 kernel), 2 = force the M = 64 tensor-core kernel.
  */
 int attn_set_gqa_path(int path);
 

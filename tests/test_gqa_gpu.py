@@ -332,3 +332,43 @@ def test_each_kernel_matches_oracle(lib, path, H_q, H_kv, d, lens, window):
     finally:
         lib.set_gqa_path(-1)
     assert_parity(got, ref, torch.bfloat16, f"path {path}")
+
+
+MANY_TILE_CASES = [
+    # (H_q, H_kv, d, lens, window): few CTAs, so each walks many tiles and
+    # several units -- the tensor-core kernels' rings wrap many times.
+    (32, 4, 256, [2000, 700], 0),          # G=8, d=256: two-stage ring
+    (48, 2, 256, [1500, 64], 300),         # G=24, d=256, window
+    (32, 1, 128, [3000, 129], 0),          # MQA
+    (16, 2, 64, [2500, 1], 0),             # G=8, d=64
+]
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["tcgen05", "tcgen05_m64"])
+@pytest.mark.parametrize("H_q,H_kv,d,lens,window", MANY_TILE_CASES,
+                         ids=[f"q{c[0]}_kv{c[1]}_d{c[2]}_w{c[4]}" for c in MANY_TILE_CASES])
+def test_tensor_core_kernels_many_tiles_per_cta(lib, path, H_q, H_kv, d, lens, window):
+    """Three CTAs for the whole batch: every CTA streams tens of tiles through
+    its ring and crosses unit boundaries, against the oracle."""
+    cfg = GQAConfig("many", B=len(lens), H_q=H_q, H_kv=H_kv, d=d, seq_lens=lens,
+                    window=window, seed=4500 + H_q + d)
+    inp = make_gqa_inputs(cfg)
+    ref = full_oracle(inp)
+    lib.set_gqa_path(path)
+    lib.set_num_ctas(3)
+    try:
+        got = run_gpu(lib, inp).float().cpu().numpy()
+    finally:
+        lib.set_gqa_path(-1)
+        lib.set_num_ctas(0)
+    assert_parity(got, ref, torch.bfloat16, f"path {path}, 3 CTAs")
+
+
+@pytest.mark.parametrize("H_q,H_kv,d,expect", [
+    (32, 32, 128, 0), (32, 8, 128, 0), (32, 4, 128, 0), (16, 2, 64, 0), (24, 4, 256, 0),
+    (36, 4, 128, 2), (32, 2, 128, 2), (32, 1, 128, 2), (128, 1, 64, 2), (48, 2, 256, 2)])
+def test_automatic_kernel_choice(lib, H_q, H_kv, d, expect):
+    """bf16: CUDA cores up to groups of 8 heads, the M=64 tensor-core kernel
+    above (the measured crossover)."""
+    _, _, used = lib.gqa_config(4, H_q, H_kv, d)
+    assert used == expect
