@@ -365,9 +365,9 @@ def set_num_ctas(n):
 
 
 def set_gqa_path(path):
-    """Testing/tuning hook: -1 automatic (CUDA cores for groups of up to 8
-    heads, else the M=64 tensor-core kernel), 0 CUDA cores, 1 tensor cores
-    with the M=128 kernel where it applies, 2 the M=64 tensor-core kernel."""
+    """Testing/tuning hook: -1 automatic (bf16: CUDA cores for groups of up
+    to 4 heads, else the tensor cores), 0 CUDA cores, 1 tensor cores (the
+    M=128 kernel where it applies, else M=64), 2 the M=64 tensor-core kernel."""
     _check(load().attn_set_gqa_path(int(path)), "attn_set_gqa_path")
 
 

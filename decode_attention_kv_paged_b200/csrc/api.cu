@@ -122,12 +122,14 @@ static bool use_tc_path(int G, int d, int dtype) {
     return ok && G >= kTcMinGroup;
 }
 
-// Which tensor-core kernel runs a unit of HC heads: the M = 64 one, unless
-// the testing hook (path 1) asks for the M = 128 one (Q and P in tensor
-// memory) where it applies.  Measured on B200 the M = 128 kernel is never
-// ahead (MQA T = 32768: 53.3 vs 49.2 us at B = 8; G = 16: 88.1 vs 82.0 us).
+// Which tensor-core kernel runs a unit of HC heads: the M = 128 one (Q and P
+// in tensor memory) where it applies, else the M = 64 one; the testing hook
+// path 2 forces the M = 64 kernel.  Measured on B200 (T = 32768, B = 8) the
+// M = 128 kernel is ahead or level everywhere it applies: MQA 41.0 vs
+// 49.1 us, G = 24 60.3 vs 83.9 us, G = 8 96.2 vs 98.3 us, G = 16 59.6 vs
+// 58.3 us.
 static bool use_tc128(int d, int HC) {
-    return tl_gqa_path == 1 && gqa_tc128_supported(d, HC);
+    return tl_gqa_path != 2 && gqa_tc128_supported(d, HC);
 }
 
 // Query heads per CTA for a group of G: the largest instantiated divisor.

@@ -15,11 +15,13 @@ int gqa_tc_heads_per_cta(int G);
 // slice); the kernel writes this many partials per (unit, CTA) slot.
 int gqa_tc_copies(int HC);
 // Group size from which the tensor-core path is the default.  Measured on
-// B200 (T = 32768, d = 128): at G = 8 the CUDA-core kernel and the M = 64
-// tensor-core kernel tie (d = 64: CUDA cores 20% faster); from G = 16 the
-// tensor cores win by 1.8x or more (the CUDA-core kernel then splits the
-// group and reads each K/V tile once per chunk of 8 heads).
-constexpr int kTcMinGroup = 9;
+// B200 (B = 8, T = 32768): G = 2 CUDA cores 3% faster; G = 4 (d = 128) CUDA
+// cores 3% faster at B = 8, level at B = 16 / T = 4096, 11% slower at
+// B = 1 (kept on the CUDA cores); G = 6 tensor cores
+// 1.3x (d = 128), 1.06x (d = 64), 1.13x (d = 256, ragged); G = 8 1.5x; from
+// G = 16 1.8x-3.5x (the CUDA-core kernel splits larger groups and reads each
+// K/V tile once per chunk of 8 heads).
+constexpr int kTcMinGroup = 5;
 
 cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC);
 

@@ -20,11 +20,11 @@
 //   * P = P_hi + P_lo (bf16 rounding remainder) keeps ~16 significant bits;
 //     O += P_hi V + P_lo V with V read MN-major from its swizzled tile.
 //     S and P are double-buffered, each buffer with its own barriers.
-//   * One thread issues the MMAs in order: P V(i), then S up to tile i + 2.
-//     The softmax threads write a segment's queries into TMEM when they reach
-//     it, after reading the previous segment's O (which waits for that
-//     segment's last P V), so S of a segment's first tile n is issued only
-//     once P V(n - 1) has been: no wait can depend on itself.
+//   * Two threads issue the MMAs: one the S products in tile order, the
+//     other the P V products.  The softmax threads write a segment's queries
+//     into TMEM when they reach it, after reading the previous segment's O
+//     (which waits for that segment's last P V), so the S issuer's wait for
+//     new queries depends only on the other issuer: no wait depends on itself.
 //   * Lazy rescale: the running max is raised only when it grows by more
 //     than 2^8 (exact either way).  Every wait is bounded; TMEM is freed.
 #include "attn_decode.h"
@@ -110,7 +110,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_init(&bars->pv_done[s], 1);
         }
         mbar_init(&bars->o_free, 128);
-        mbar_init(&bars->mma_final, 1);
+        mbar_init(&bars->mma_final, 2);     // one commit per issuing thread
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -159,16 +159,16 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                           p.timeout_ns, p.err, nullptr);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2) {
         // ============================================================ MMA
+        // Lane 0 of warp 1 issues S(n) = Q K(n)^T for every tile in order,
+        // lane 0 of warp 2 issues O += P(i) V(i); each waits only on its own
+        // inputs, so the two streams overlap.  A segment's first S waits for
+        // its queries, which the softmax threads write only after reading the
+        // previous segment's O (after its last P V): that chain runs through
+        // the other issuer, never back to this one.  Barriers are polled.
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
             const uint32_t c_base = smem_u32(sC);
-            TileCursor cs, cv;
-            cs.init(pa, lo, hi, first_seq, first_base);
-            cv.init(pa, lo, hi, first_seq, first_base);
-            int seg_s = 0, seg_v = 0;
             auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
                 unsigned long long t0 = 0;
                 for (uint32_t it = 0;; ++it) {
@@ -189,63 +189,62 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                 }
             };
-            // S(n) = Q K(n)^T into S buffer n % 2; A = Q from TMEM.
-            auto issue_s = [&](int n) -> bool {
-                const bool first = cs.t == 0, last = cs.t == cs.len - 1;
-                const int st = n % C::kStages, sb = n & 1;
-                if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) return false;
-                if (!wait(&bars->c_full[st], (uint32_t)((n / C::kStages) & 1))) return false;
-                if (n >= 2 && !wait(&bars->s_free[sb], (uint32_t)(((n - 2) >> 1) & 1)))
-                    return false;
-                tc_fence_after();
-                const uint32_t kst = c_base + st * C::kStageBytes;
+            if (warp == 1) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
+                TileCursor cs;
+                cs.init(pa, lo, hi, first_seq, first_base);
+                int seg_s = 0;
+                for (int n = 0; n < n_tiles; ++n) {
+                    // S(n) into S buffer n % 2; A = Q from TMEM.
+                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
+                    const int st = n % C::kStages, sb = n & 1;
+                    if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) break;
+                    if (!wait(&bars->c_full[st], (uint32_t)((n / C::kStages) & 1))) break;
+                    if (n >= 2 && !wait(&bars->s_free[sb], (uint32_t)(((n - 2) >> 1) & 1)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t kst = c_base + st * C::kStageBytes;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t b =
-                        umma_desc_sw128(kst + (ks >> 2) * kT2Box + (ks & 3) * 32, 16, 1024);
-                    umma_bf16_ts(tmem + C::kTmemS + 64 * sb, tmem + C::kTmemQ + 8 * ks, b,
-                                 idesc_s, ks != 0);
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t b =
+                            umma_desc_sw128(kst + (ks >> 2) * kT2Box + (ks & 3) * 32, 16, 1024);
+                        umma_bf16_ts(tmem + C::kTmemS + 64 * sb, tmem + C::kTmemQ + 8 * ks, b,
+                                     idesc_s, ks != 0);
+                    }
+                    umma_commit(&bars->s_full[sb]);
+                    if (last) umma_commit(&bars->q_empty);
+                    if (first) ++seg_s;
+                    cs.next();
                 }
-                umma_commit(&bars->s_full[sb]);
-                if (last) umma_commit(&bars->q_empty);
-                if (first) ++seg_s;
-                cs.next();
-                return true;
-            };
-            // Issue S in order up to tile `upto`; a segment's first tile waits
-            // until P V of the tile before it has been issued.
-            int next_s = 0;
-            auto issue_s_upto = [&](int upto, int pv_issued) -> bool {
-                while (next_s < n_tiles && next_s <= upto) {
-                    if (cs.t == 0 && next_s > 0 && pv_issued < next_s - 1) break;
-                    if (!issue_s(next_s)) return false;
-                    ++next_s;
-                }
-                return true;
-            };
-            bool ok = issue_s_upto(1, -1);
-            for (int i = 0; ok && i < n_tiles; ++i) {
-                // O += P(i) V(i); A = P from TMEM buffer i % 2 (hi, then lo).
-                const bool first = cv.t == 0;
-                if (!wait(&bars->p_full[i & 1], (uint32_t)((i >> 1) & 1)) ||
-                    (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1))))
-                    break;
-                tc_fence_after();
-                const int st = i % C::kStages;
-                const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kT2Box;
-                const uint32_t pb = tmem + C::kTmemP + 64 * (i & 1);
+            } else {
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
+                TileCursor cv;
+                cv.init(pa, lo, hi, first_seq, first_base);
+                int seg_v = 0;
+                for (int i = 0; i < n_tiles; ++i) {
+                    // O += P(i) V(i); A = P from TMEM buffer i % 2 (hi, then lo).
+                    const bool first = cv.t == 0;
+                    if (!wait(&bars->p_full[i & 1], (uint32_t)((i >> 1) & 1))) break;
+                    if (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))
+                        break;
+                    tc_fence_after();
+                    const int st = i % C::kStages;
+                    const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kT2Box;
+                    const uint32_t pb = tmem + C::kTmemP + 64 * (i & 1);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t b = umma_desc_sw128(vst + ks * 2048, kT2Box, 1024);
-                    umma_bf16_ts(tmem + C::kTmemO, pb + 8 * ks, b, idesc_pv, !(first && ks == 0));
-                    umma_bf16_ts(tmem + C::kTmemO, pb + 32 + 8 * ks, b, idesc_pv, 1);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t b = umma_desc_sw128(vst + ks * 2048, kT2Box, 1024);
+                        umma_bf16_ts(tmem + C::kTmemO, pb + 8 * ks, b, idesc_pv,
+                                     !(first && ks == 0));
+                        umma_bf16_ts(tmem + C::kTmemO, pb + 32 + 8 * ks, b, idesc_pv, 1);
+                    }
+                    umma_commit(&bars->c_empty[st]);
+                    umma_commit(&bars->pv_done[i & 1]);
+                    if (first) ++seg_v;
+                    cv.next();
                 }
-                umma_commit(&bars->c_empty[st]);
-                umma_commit(&bars->pv_done[i & 1]);
-                if (first) ++seg_v;
-                cv.next();
-                ok = issue_s_upto(i + 2, i);
             }
+            // Both issuers' MMAs complete before the tensor memory is freed.
             umma_commit(&bars->mma_final);
             mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
         }

@@ -218,10 +218,10 @@ int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype,
 int attn_set_num_ctas(int num_ctas);
 
 /*
- * attn_set_gqa_path -- testing/tuning hook: -1 = automatic (the CUDA-core
- * kernel for groups of up to 8 heads, the M = 64 tensor-core kernel for
+ * attn_set_gqa_path -- testing/tuning hook: -1 = automatic (bf16: the
+ * CUDA-core kernel for groups of up to 4 heads, the tensor-core path for
  * larger groups), 0 = force the CUDA-core kernel, 1 = force the tensor-core
- * path with the M = 128 kernel where it applies (d <= 128 and units of <= 32
+ * path (the M = 128 kernel where it applies, d <= 128 and units of <= 32
  * heads, else the M = 64 kernel), 2 = force the M = 64 tensor-core kernel.
  */
 int attn_set_gqa_path(int path);

@@ -365,10 +365,12 @@ def test_tensor_core_kernels_many_tiles_per_cta(lib, path, H_q, H_kv, d, lens, w
 
 
 @pytest.mark.parametrize("H_q,H_kv,d,expect", [
-    (32, 32, 128, 0), (32, 8, 128, 0), (32, 4, 128, 0), (16, 2, 64, 0), (24, 4, 256, 0),
-    (36, 4, 128, 2), (32, 2, 128, 2), (32, 1, 128, 2), (128, 1, 64, 2), (48, 2, 256, 2)])
+    (32, 32, 128, 0), (32, 16, 128, 0), (32, 8, 128, 0), (24, 4, 128, 1), (32, 4, 128, 1),
+    (16, 2, 64, 1), (24, 4, 256, 2), (36, 4, 128, 1), (32, 1, 128, 1), (48, 1, 64, 2),
+    (128, 1, 64, 2), (48, 2, 256, 2)])
 def test_automatic_kernel_choice(lib, H_q, H_kv, d, expect):
-    """bf16: CUDA cores up to groups of 8 heads, the M=64 tensor-core kernel
-    above (the measured crossover)."""
+    """bf16: CUDA cores up to groups of 4 heads; above, the M=128 tensor-core
+    kernel where it applies (d <= 128, units of <= 32 heads), else the M=64
+    one (the measured crossovers)."""
     _, _, used = lib.gqa_config(4, H_q, H_kv, d)
     assert used == expect
