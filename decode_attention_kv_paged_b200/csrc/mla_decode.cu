@@ -33,9 +33,9 @@
 //     8; both halves (128 x 64, swizzled like a TMA tile) are A operands of
 //     O += P_hi C + P_lo C, 128 x 256 MMAs whose B operand is the same C tile
 //     read MN-major.  Each CTA keeps its 256 output columns in TMEM.
-//   * Warp 0 issues TMA; one thread of warp 1 issues MMAs, polling the S and
-//     P V dependencies and issuing whichever is ready (no head-of-line
-//     blocking); warps 4-7 load Q, run the softmax and the epilogue.  Every
+//   * Warp 0 issues TMA; one thread of warp 1 issues the S MMAs and one of
+//     warp 2 the P V MMAs, each as its inputs become ready; warps 4-11 load
+//     Q, run the softmax and the epilogue.  Every
 //     wait is bounded; TMEM is always freed; the final cluster handshake is a
 //     bounded mbarrier exchange.
 // Each (sequence, cluster) segment writes an fp32 partial (O/l and log2-sum-
@@ -154,7 +154,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         mbar_init(&bars->red_bar, kSoftThreads);
         mbar_init(&bars->sum_bar, kSoftThreads);
         mbar_init(&bars->end_bar, 1);
-        mbar_init(&bars->mma_final, 1);
+        mbar_init(&bars->mma_final, 2);            // one commit per issuing thread
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -214,89 +214,93 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                           p.timeout_ns, p.err, nullptr);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2) {
         // ============================================================ MMA
+        // Lane 0 of warp 1 issues S(n) = Q C(n)^T for every tile in order,
+        // lane 0 of warp 2 issues O += P(i) C(i); each waits only on its own
+        // inputs, so the two streams of MMAs overlap.  The stage is released
+        // by the commit after P V(i): S(i) has completed by then (the softmax
+        // read it before producing P(i)).  Barriers are polled.
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 256, 0, 1);
-            const uint32_t c_base = smem_u32(sC), p_base = smem_u32(sP);
-            TileCursor cs, cv;           // next tile to issue S for / P V for
-            cs.init(pa, lo, hi, first_seq, first_base);
-            cv.init(pa, lo, hi, first_seq, first_base);
-            int next_s = 0, next_pv = 0, seg_s = 0, seg_v = 0;
-            unsigned long long idle_since = 0;
-            uint32_t idle_polls = 0;
-            while (next_pv < n_tiles) {
-                bool did = false;
-                if (next_s < n_tiles) {
-                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
-                    const int st = next_s % kMlaStages;
-                    const bool ready =
-                        (!first || mbar_test(&bars->q_full, (uint32_t)(seg_s & 1))) &&
-                        mbar_test(&bars->c_full[st], (uint32_t)((next_s / kMlaStages) & 1)) &&
-                        (next_s == 0 || mbar_test(&bars->s_free, (uint32_t)((next_s - 1) & 1)));
-                    if (ready) {
-                        tc_fence_after();
-                        const uint32_t cst = c_base + st * kMlaStageBytes;
-                        for (int bx = 0; bx < nbox; ++bx)
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const uint64_t b =
-                                    umma_desc_sw128(cst + bx * kMlaCBox + k * 32, 16, 1024);
-                                umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 32 * bx + 8 * k, b,
-                                             idesc_s, (bx | k) != 0);
-                            }
-                        umma_commit(&bars->s_full);
-                        if (last) umma_commit(&bars->q_empty);
-                        if (first) ++seg_s;
-                        cs.next();
-                        ++next_s;
-                        did = true;
+            const uint32_t c_base = smem_u32(sC);
+            auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+                unsigned long long t0 = 0;
+                for (uint32_t it = 0;; ++it) {
+                    if (mbar_test(bar, parity)) return true;
+                    if ((it & 15u) == 15u) {
+                        if (*abort_flag) return false;
+                        __nanosleep(20);
+                    }
+                    if ((it & 1023u) == 1023u) {
+                        const unsigned long long now = global_timer_ns();
+                        if (t0 == 0) {
+                            t0 = now;
+                        } else if (now - t0 > p.timeout_ns) {
+                            raise_error(p.err, kErrTimeout);
+                            *abort_flag = 1;
+                            return false;
+                        }
                     }
                 }
-                if (next_pv < next_s) {
-                    const bool first = cv.t == 0;
-                    const bool ready =
-                        mbar_test(&bars->p_full, (uint32_t)(next_pv & 1)) &&
-                        (!first || seg_v == 0 ||
-                         mbar_test(&bars->o_free, (uint32_t)((seg_v - 1) & 1)));
-                    if (ready) {
-                        tc_fence_after();
-                        const int st = next_pv % kMlaStages;
-                        const uint32_t cst = c_base + st * kMlaStageBytes;
+            };
+            if (warp == 1) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
+                TileCursor cs;
+                cs.init(pa, lo, hi, first_seq, first_base);
+                int seg_s = 0;
+                for (int n = 0; n < n_tiles; ++n) {
+                    // S(n) into the S buffer once the softmax has read S(n - 1).
+                    const bool first = cs.t == 0, last = cs.t == cs.len - 1;
+                    const int st = n % kMlaStages;
+                    if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) break;
+                    if (!wait(&bars->c_full[st], (uint32_t)((n / kMlaStages) & 1))) break;
+                    if (n > 0 && !wait(&bars->s_free, (uint32_t)((n - 1) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t cst = c_base + st * kMlaStageBytes;
+                    for (int bx = 0; bx < nbox; ++bx)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const uint64_t b = umma_desc_sw128(cst + k * 2048, kMlaCBox, 1024);
-                            const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
-                            const uint64_t a_lo =
-                                umma_desc_sw128(p_base + kPBytes + k * 32, 16, 1024);
-                            umma_bf16(tmem + kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
-                            umma_bf16(tmem + kTmemO, a_lo, b, idesc_pv, 1);
+                            const uint64_t b =
+                                umma_desc_sw128(cst + bx * kMlaCBox + k * 32, 16, 1024);
+                            umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 32 * bx + 8 * k, b,
+                                         idesc_s, (bx | k) != 0);
                         }
-                        umma_commit(&bars->c_empty[st]);
-                        umma_commit(&bars->pv_done);
-                        if (first) ++seg_v;
-                        cv.next();
-                        ++next_pv;
-                        did = true;
-                    }
+                    umma_commit(&bars->s_full);
+                    if (last) umma_commit(&bars->q_empty);
+                    if (first) ++seg_s;
+                    cs.next();
                 }
-                if (did) {
-                    idle_since = 0;
-                    idle_polls = 0;
-                } else if ((++idle_polls & 7u) == 0 && (__nanosleep(32), (idle_polls & 63u) == 0)) {
-                    // the clock is read only every 64 idle polls
-                    const unsigned long long now = global_timer_ns();
-                    if (idle_since == 0) idle_since = now;
-                    if (*abort_flag) break;
-                    if (now - idle_since > p.timeout_ns) {
-                        raise_error(p.err, kErrTimeout);
-                        *abort_flag = 1;
+            } else {
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 256, 0, 1);
+                const uint32_t p_base = smem_u32(sP);
+                TileCursor cv;
+                cv.init(pa, lo, hi, first_seq, first_base);
+                int seg_v = 0;
+                for (int i = 0; i < n_tiles; ++i) {
+                    // O += P_hi C + P_lo C; a segment's first P V overwrites O
+                    // once the previous segment's output has been read.
+                    const bool first = cv.t == 0;
+                    if (!wait(&bars->p_full, (uint32_t)(i & 1))) break;
+                    if (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))
                         break;
+                    tc_fence_after();
+                    const int st = i % kMlaStages;
+                    const uint32_t cst = c_base + st * kMlaStageBytes;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t b = umma_desc_sw128(cst + k * 2048, kMlaCBox, 1024);
+                        const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
+                        const uint64_t a_lo = umma_desc_sw128(p_base + kPBytes + k * 32, 16, 1024);
+                        umma_bf16(tmem + kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
+                        umma_bf16(tmem + kTmemO, a_lo, b, idesc_pv, 1);
                     }
+                    umma_commit(&bars->c_empty[st]);
+                    umma_commit(&bars->pv_done);
+                    if (first) ++seg_v;
+                    cv.next();
                 }
             }
-            // All MMAs issued so far complete before TMEM is released.
+            // Both issuers' MMAs complete before TMEM is released.
             umma_commit(&bars->mma_final);
             mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
         }

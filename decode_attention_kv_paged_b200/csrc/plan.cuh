@@ -115,7 +115,7 @@ struct PlanScratch {          // shared memory used by plan_locate
 
 // Block-wide: total work W, and the sequence holding flattened block
 // `target(W)` together with the work (blocks x units) before that sequence.
-// Every thread of the block must call it.  When prefix_out is non-null the
+// Every thread of the block must call it (blockDim.x >= 32).  When prefix_out is non-null the
 // exclusive prefix sums of work per sequence (B + 1 values) are written.
 // `target_cta` selects target = cta_bound(target_cta, W, P') (none if the
 // CTA has no work).
@@ -124,6 +124,49 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
                             unsigned *err) {
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = (nt + 31) >> 5;
+    if (a.B <= 32) {
+        // One warp: lane b holds sequence b; a warp scan gives the prefix
+        // sums and W, a ballot the sequence holding the target (one round
+        // trip to seq_lens and one block-wide barrier).
+        if (warp == 0) {
+            long long w = 0;
+            bool bad = false;
+            if (lane < a.B) {
+                int fb, sb;
+                w = (long long)visible_blocks(a.seq_lens[lane], a.vis, a.max_blocks, &fb, &sb,
+                                              &bad) *
+                    a.units_per_seq;
+            }
+            long long x = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            const long long W = __shfl_sync(0xffffffffu, x, 31);
+            const int P = working_ctas(W, a.num_ctas);
+            const long long target =
+                (W > 0 && target_cta < P) ? cta_bound(target_cta, W, P) : W;
+            const long long excl = x - w;
+            const unsigned hit =
+                __ballot_sync(0xffffffffu, lane < a.B && w > 0 && excl <= target &&
+                                               target < excl + w);
+            const bool any_bad = __any_sync(0xffffffffu, bad);
+            const int src = hit ? __ffs(hit) - 1 : 0;
+            const long long base = __shfl_sync(0xffffffffu, excl, src);
+            if (prefix_out && lane < a.B) prefix_out[lane] = excl;
+            if (lane == 0) {
+                sh->total = W;
+                sh->seq = hit ? src : -1;
+                sh->base = hit ? base : 0;
+                sh->bad = any_bad ? 1 : 0;
+                if (prefix_out) prefix_out[a.B] = W;
+                if (any_bad && err) raise_error(err, kErrBadSeqLen);
+            }
+        }
+        __syncthreads();
+        return;
+    }
     bool any_bad = false;
 
     // Pass 1: W.

@@ -151,6 +151,8 @@ def test_window_at_least_T_equals_full(lib):
     ([131072, 1024, 5000, 77777], 4, 4096, 148),
     ([5] * 300, 2, 0, 64),
     ([100, 0, 0], 1, 0, 1000),
+    ([64 * (i % 5) + i for i in range(32)], 3, 0, 148),     # B = 32: one-warp planner
+    ([64 * (i % 5) + i for i in range(33)], 3, 100, 148),   # B = 33: block-wide planner
 ])
 def test_device_planner_matches_host_model(lib, lens, units, window, P):
     from decode_attention_kv_paged_b200 import planner
