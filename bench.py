@@ -571,13 +571,18 @@ def cpu_baseline(cfg, is_mla, target_s):
     orc.set_threads(cores)
     n, _ = _pick_sample(cfg, is_mla, orc, target_s)
     x = _oracle_problem(cfg, is_mla, n, cfg.seed)
-    t0 = time.perf_counter()
-    _oracle_call(orc, x, is_mla)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": orc.get_threads(),
+    # Repeat the pass until about target_s seconds of CPU work have run.
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_call(orc, x, is_mla)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s or passes >= 100000:
+            break
+    return {"value": n * passes / dt, "unit": "tokens/s", "cores": orc.get_threads(),
             "kind": "oracle",
             "sample": f"{n} of the workload's {cfg.B} sequences (fp64 C oracle, "
-                      f"OpenMP), one pass, {dt:.1f} s"}
+                      f"OpenMP), {passes} pass(es), {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
