@@ -34,9 +34,20 @@ C_SYMBOLS = (
 
 
 class Visibility(ctypes.Structure):
-    """attn_visibility: window, global (sink) tokens, ring table (blocks)."""
+    """attn_visibility: window, global (sink) tokens, ring table (blocks),
+    explicit global positions (device int32 [B][n_global])."""
     _fields_ = [("window", ctypes.c_int), ("sink_tokens", ctypes.c_int),
-                ("ring_blocks", ctypes.c_int)]
+                ("ring_blocks", ctypes.c_int), ("global_pos", ctypes.c_void_p),
+                ("n_global", ctypes.c_int)]
+
+
+def _visibility(window, sink_tokens, ring_blocks, global_pos=None, B=None):
+    if global_pos is None:
+        return Visibility(int(window), int(sink_tokens), int(ring_blocks), None, 0)
+    if global_pos.dim() != 2 or (B is not None and global_pos.shape[0] != B):
+        raise ValueError("global_pos must be [B][n_global]")
+    return Visibility(int(window), int(sink_tokens), int(ring_blocks),
+                      _dev(global_pos, "global_pos", torch.int32).value, int(global_pos.shape[1]))
 
 _lib = None
 
@@ -146,10 +157,12 @@ def decode_gqa(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
 
 
 def decode_gqa_ext(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
-                   sink_tokens=0, ring_blocks=0, out=None, stream=None):
-    """decode_gqa with global (sink) tokens and a ring-buffer block table:
-    key j < T is visible when window <= 0, j >= T - window or j < sink_tokens;
-    with ring_blocks > 0 logical block i lives in table slot i for the sink
+                   sink_tokens=0, ring_blocks=0, out=None, stream=None, global_pos=None):
+    """decode_gqa with global tokens and a ring-buffer block table: key
+    j < T is visible when window <= 0, j >= T - window, j < sink_tokens, j is
+    in the sequence's row of global_pos (int32 [B][n_global], ascending, -1
+    padded), or T - 1 is in it (a global query sees everything); with
+    ring_blocks > 0 logical block i lives in table slot i for the sink
     blocks and in slot A + i % ring_blocks after them (A = ceil(sink / 64))."""
     B, H_q, d = q.shape
     nblk, H_kv, bs, d2 = k_cache.shape
@@ -158,7 +171,7 @@ def decode_gqa_ext(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
     dt = _dtype_code(q.dtype)
     if out is None:
         out = torch.empty_like(q)
-    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    vis = _visibility(window, sink_tokens, ring_blocks, global_pos, B)
     rc = load().attn_decode_gqa_ext(
         _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
         _dev(v_cache, "v_cache", q.dtype), _dev(seq_lens, "seq_lens", torch.int32),
@@ -170,7 +183,8 @@ def decode_gqa_ext(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
 
 
 def decode_gqa_fp8(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_table, scale,
-                   window=0, sink_tokens=0, ring_blocks=0, out=None, stream=None):
+                   window=0, sink_tokens=0, ring_blocks=0, out=None, stream=None,
+                   global_pos=None):
     """out [B][H_q][d] (bf16) = decode attention over an fp8 cache: k_cache /
     v_cache uint8 E4M3 codes [num_blocks][H_kv][64][d], k_scale / v_scale
     fp32 row scales [num_blocks][H_kv][64] (value = code * row scale)."""
@@ -183,7 +197,7 @@ def decode_gqa_fp8(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_table,
     bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
     if out is None:
         out = torch.empty_like(q)
-    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    vis = _visibility(window, sink_tokens, ring_blocks, global_pos, B)
     rc = load().attn_decode_gqa_fp8(
         _dev(q, "q", bf), _dev(k_cache, "k_cache", u8), _dev(v_cache, "v_cache", u8),
         _dev(k_scale, "k_scale", f32), _dev(v_scale, "v_scale", f32),
@@ -200,7 +214,7 @@ def kv_append_fp8(k_new, v_new, k_cache, v_cache, k_scale, v_scale, positions, b
     one scale per row (amax / 448) and write them at positions[b]."""
     B, H_kv, d = k_new.shape
     bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
-    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    vis = _visibility(window, sink_tokens, ring_blocks)
     rc = load().kv_append_fp8(
         _dev(k_new, "k_new", bf), _dev(v_new, "v_new", bf), _dev(k_cache, "k_cache", u8),
         _dev(v_cache, "v_cache", u8), _dev(k_scale, "k_scale", f32),
@@ -297,7 +311,7 @@ def kv_append_ext(k_new, v_new, k_cache, v_cache, positions, block_table,
     then the ring): with a ring, writing past the window overwrites the block
     that left it."""
     B, H_kv, d = k_new.shape
-    vis = Visibility(int(window), int(sink_tokens), int(ring_blocks))
+    vis = _visibility(window, sink_tokens, ring_blocks)
     rc = load().kv_append_ext(
         _dev(k_new, "k_new"), _dev(v_new, "v_new", k_new.dtype),
         _dev(k_cache, "k_cache", k_new.dtype), _dev(v_cache, "v_cache", k_new.dtype),

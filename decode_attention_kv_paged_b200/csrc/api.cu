@@ -371,8 +371,17 @@ int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
 // Validates a visibility record against the table width; fills `out`.
 static int check_visibility(const attn_visibility *v, int max_blocks_per_seq, Visibility *out) {
     if (!v) return ATTN_ERR_ARG;
-    if (v->sink_tokens < 0 || v->ring_blocks < 0) return ATTN_ERR_ARG;
+    if (v->sink_tokens < 0 || v->ring_blocks < 0 || v->n_global < 0) return ATTN_ERR_ARG;
     Visibility vis{v->window > 0 ? v->window : 0, v->sink_tokens, v->ring_blocks};
+    if (v->n_global > 0) {
+        // An explicit global set replaces the sink prefix and has no ring.
+        if (!v->global_pos || (reinterpret_cast<uintptr_t>(v->global_pos) & 3u) ||
+            v->sink_tokens > 0 || v->ring_blocks > 0)
+            return ATTN_ERR_ARG;
+        if (v->n_global > 64) return ATTN_ERR_UNSUPPORTED;
+        vis.gpos = v->global_pos;
+        vis.n_g = v->n_global;
+    }
     if (vis.ring > 0) {
         // The ring must hold every block a window can reach, after the sink
         // blocks, inside the table row.

@@ -377,13 +377,13 @@ __device__ __forceinline__ bool unit_arrive(unsigned *cnt, int ns) {
 // released by the compute warps; then waits for the copies still in flight
 // (the last S issued) so none lands after the CTA exits.  All 32 lanes run
 // it; lane 0 issues the copies.
-template <int D, int HC, typename T, typename TK, int S, int kTileTok, int kSub>
+template <int D, int HC, typename T, typename TK, int S, int kTileTok, int kSub, bool G>
 __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long lo,
                               long long hi, int seq, long long base,
                               unsigned char *stage_base, uint64_t *full_bar,
                               uint64_t *empty_bar, unsigned char *q_ring, int q_slot_bytes,
                               uint64_t *q_full, uint64_t *q_empty, int lane,
-                              volatile int *abort_flag) {
+                              volatile int *abort_flag, unsigned long long *s_gmask) {
     constexpr int kStageBytes =
         2 * (kTileTok * D * (int)sizeof(TK) + (sizeof(TK) == 1 ? kTileTok * 4 : 0));
     constexpr uint32_t kQBytes = HC * D * sizeof(T);
@@ -421,6 +421,15 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
             if (!__all_sync(0xffffffffu, fr)) break;
         }
         if (sub == 0) phys = prod.block_id(p, lane);
+        if constexpr (G) {
+            // The block's global positions, for the masking of keys below
+            // the window (ordered before the stage's arrival below).
+            const int blk = prod.cur.logical_block();
+            const unsigned long long gm = blk * kBlockSize < prod.cur.w.lo
+                                              ? global_mask(p.vis, prod.cur.w.b, blk, lane)
+                                              : 0ull;
+            if (lane == 0) s_gmask[s] = gm;
+        }
         if (lane == 0)
             issue_tile<D, TK, kTileTok>(p, prod.cur, phys, sub,
                                        stage_base + (size_t)s * kStageBytes, &full_bar[s],
@@ -677,7 +686,10 @@ __device__ void segment_epilogue(const GqaParams &p, int et, long long u, int c0
     }
 }
 
-template <int D, int HC, typename T, typename TK>
+// G: the call has an explicit global set (p.vis.n_g > 0).  It is a template
+// flag so that calls without one run a loop free of its masking code, which
+// measurably slowed the common case when present but not taken.
+template <int D, int HC, typename T, typename TK, bool G>
 __global__ void __launch_bounds__(GqaCfg<D, HC, T, TK>::kThreads, 1)
 gqa_split_kernel(const GqaParams p) {
     using C = GqaCfg<D, HC, T, TK>;
@@ -704,6 +716,12 @@ gqa_split_kernel(const GqaParams p) {
     PlanScratch *plan_sh = reinterpret_cast<PlanScratch *>(never_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(plan_sh + 1);
     volatile int *last_flag = abort_flag + 1;
+    // Per stage: global positions among the staged block's keys below the
+    // window (bit t: key 64 * block + t), written by the producer before it
+    // arms the stage, read by the compute warps after they wait on it.
+    unsigned long long *s_gmask = reinterpret_cast<unsigned long long *>(misc + 768);
+    static_assert((2 * S + 7) * 8 + sizeof(PlanScratch) + 8 <= 768 && 768 + 8 * S <= C::kMiscBytes,
+                  "misc shared-memory layout");
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -746,9 +764,9 @@ gqa_split_kernel(const GqaParams p) {
     if (tid < 128) {
         regs_decrease<C::kProducerRegs>();
         if (tid < 32) {
-            produce_tiles<D, HC, T, TK, S, C::kTileTok, C::kSub>(
+            produce_tiles<D, HC, T, TK, S, C::kTileTok, C::kSub, G>(
                 p, pa, lo, hi, plan_sh->seq, plan_sh->base, stage_base, full_bar, empty_bar,
-                q_ring, kQSlot, q_full, q_empty, lane, abort_flag);
+                q_ring, kQSlot, q_full, q_empty, lane, abort_flag, s_gmask);
         } else {
             const int et = tid - 32;
             // A sequence without a visible block (empty) has a zero output
@@ -756,7 +774,7 @@ gqa_split_kernel(const GqaParams p) {
             for (int b = blockIdx.x; b < p.B; b += P) {
                 int fb, sb;
                 bool bad;
-                if (visible_blocks(p.seq_lens[b], p.vis, p.max_blocks, &fb, &sb, &bad) == 0) {
+                if (visible_blocks(p.seq_lens[b], p.vis, p.max_blocks, &fb, &sb, &bad, b) == 0) {
                     T *o = static_cast<T *>(p.out) + (size_t)b * p.H_q * D;
                     for (int i = et; i < p.H_q * D; i += C::kEpiThreads)
                         o[i] = ElemTraits<T>::from_float(0.f);
@@ -844,7 +862,7 @@ gqa_split_kernel(const GqaParams p) {
         const int len = walk.seg_len();
         const long long seg_t1 = seg_t0 + (long long)len * C::kSub;
         const int Tb = walk.T;
-        const int lo_tok = window_lo(p.vis, Tb);
+        const int lo_tok = walk.lo;
         const int sink = p.vis.sink;
 
         // The unit's queries, staged in shared memory by the producer.
@@ -894,9 +912,14 @@ gqa_split_kernel(const GqaParams p) {
             const float *ksc = reinterpret_cast<const float *>(Vs + C::kTileTok * D);
             const float *vsc = ksc + C::kTileTok;
             const int tl = (int)(n - seg_t0);
-            const int tok0 = walk.logical(walk.blk_off + tl / C::kSub) * kBlockSize +
-                             (tl % C::kSub) * C::kTileTok + wig * C::kTPW;
+            const int blk = walk.logical(walk.blk_off + tl / C::kSub);
+            const int tok0 = blk * kBlockSize + (tl % C::kSub) * C::kTileTok + wig * C::kTPW;
             const int row0 = wig * C::kTPW;
+            // Global positions among this block's keys below the window
+            // (bit t: key blk * 64 + t), staged by the producer.
+            unsigned long long gmask = 0ull;
+            if constexpr (G)
+                if (blk * kBlockSize < lo_tok) gmask = s_gmask[stage];
 
             // ---- scores: partial dot products, reduced over the row group
 #pragma unroll
@@ -948,7 +971,9 @@ gqa_split_kernel(const GqaParams p) {
                 const int tt = lane % C::kTPW;
                 const bool active = gs < HC;
                 const int pos = tok0 + tt;
-                const bool valid = active && pos < Tb && (pos >= lo_tok || pos < sink);
+                const bool valid = active && pos < Tb &&
+                                   (pos >= lo_tok || pos < sink ||
+                                    ((gmask >> (pos - blk * kBlockSize)) & 1ull));
                 const float s = valid ? sc[tt * C::kHCP + gs] : kNegInf;
                 if (__any_sync(0xffffffffu, s > m_run[ps] + kRescaleLog2)) {
                     float mx = s;
@@ -1128,7 +1153,7 @@ combine_kernel(const CombineParams p) {
     if (tid == 0) {
         int fb, sb;
         bool bad;
-        const int nb = visible_blocks(p.seq_lens[b], p.vis, p.max_blocks, &fb, &sb, &bad);
+        const int nb = visible_blocks(p.seq_lens[b], p.vis, p.max_blocks, &fb, &sb, &bad, b);
         s_nb = nb;
         s_n = 0;
         s_first = 0;

@@ -20,7 +20,7 @@ struct GqaLaunch {
 template <int D, int HC, typename T, typename TK = T>
 int gqa_smem_bytes() { return GqaCfg<D, HC, T, TK>::kSmemBytes; }
 
-template <int D, int HC, typename T, typename TK = T>
+template <int D, int HC, typename T, typename TK = T, bool G = false>
 cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     using C = GqaCfg<D, HC, T, TK>;
     static bool configured = false;   // per-process; attribute is per function
@@ -29,12 +29,12 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
         // The warpgroups' setmaxnreg shares must fit in the registers the
         // kernel is launched with, or the increase would never be granted.
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T, TK>);
+        e = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T, TK, G>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs * C::kThreads <
             4 * 32 * C::kProducerRegs + C::kNW * 32 * C::kConsumerRegs)
             return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T, TK>,
+        e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T, TK, G>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes);
         if (e != cudaSuccess) return e;
@@ -53,7 +53,7 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gqa_split_kernel<D, HC, T, TK>, L.kp);
+    e = cudaLaunchKernelEx(&cfg, gqa_split_kernel<D, HC, T, TK, G>, L.kp);
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
     return cudaSuccess;
@@ -62,10 +62,15 @@ cudaError_t launch_gqa_impl(const GqaLaunch &L) {
 // Dispatch over heads-per-CTA and dtype for one head dimension D.
 template <int D>
 cudaError_t launch_gqa_d(int HC, int dtype_bf16, const GqaLaunch &L) {
-#define ATTN_CASE(hc)                                                        \
-    case hc:                                                                 \
-        if (dtype_bf16) return launch_gqa_impl<D, hc, __nv_bfloat16>(L);     \
-        if constexpr (D <= 128) return launch_gqa_impl<D, hc, float>(L);     \
+    const bool g = L.kp.vis.n_g > 0;
+#define ATTN_CASE(hc)                                                                  \
+    case hc:                                                                           \
+        if (dtype_bf16)                                                                \
+            return g ? launch_gqa_impl<D, hc, __nv_bfloat16, __nv_bfloat16, true>(L)   \
+                     : launch_gqa_impl<D, hc, __nv_bfloat16>(L);                       \
+        if constexpr (D <= 128)                                                        \
+            return g ? launch_gqa_impl<D, hc, float, float, true>(L)                   \
+                     : launch_gqa_impl<D, hc, float>(L);                               \
         return cudaErrorNotSupported;
     switch (HC) {
         ATTN_CASE(1)
@@ -88,15 +93,21 @@ cudaError_t launch_gqa_d256(int HC, int bf16, const GqaLaunch &L);
 // bf16 queries over an fp8 (e4m3 + per-row fp32 scale) cache, d in {64, 128, 256}.
 template <int D>
 cudaError_t launch_gqa_fp8_d(int HC, const GqaLaunch &L) {
+    const bool g = L.kp.vis.n_g > 0;
+#define ATTN_FP8(hc)                                                                   \
+    case hc:                                                                           \
+        return g ? launch_gqa_impl<D, hc, __nv_bfloat16, uint8_t, true>(L)             \
+                 : launch_gqa_impl<D, hc, __nv_bfloat16, uint8_t>(L);
     switch (HC) {
-        case 1: return launch_gqa_impl<D, 1, __nv_bfloat16, uint8_t>(L);
-        case 2: return launch_gqa_impl<D, 2, __nv_bfloat16, uint8_t>(L);
-        case 3: return launch_gqa_impl<D, 3, __nv_bfloat16, uint8_t>(L);
-        case 4: return launch_gqa_impl<D, 4, __nv_bfloat16, uint8_t>(L);
-        case 6: return launch_gqa_impl<D, 6, __nv_bfloat16, uint8_t>(L);
-        case 8: return launch_gqa_impl<D, 8, __nv_bfloat16, uint8_t>(L);
+        ATTN_FP8(1)
+        ATTN_FP8(2)
+        ATTN_FP8(3)
+        ATTN_FP8(4)
+        ATTN_FP8(6)
+        ATTN_FP8(8)
         default: return cudaErrorInvalidValue;
     }
+#undef ATTN_FP8
 }
 cudaError_t launch_gqa_fp8_d64(int HC, const GqaLaunch &L);
 cudaError_t launch_gqa_fp8_d128(int HC, const GqaLaunch &L);

@@ -76,13 +76,18 @@ struct TcBars {
     // finish two tiles before the MMA thread tests the first, which a single
     // barrier could not tell apart.
     uint64_t p_full[2], pv_done[2], o_free, mma_final;
+    // Per stage: global positions among the staged block's keys below the
+    // window (bit t: key 64 * block + t), written before the stage is armed.
+    unsigned long long gmask[6];
     uint32_t tmem_base;
     int abort;
     PlanScratch plan;
 };
 static_assert(sizeof(TcBars) <= 1024, "barrier block");
 
-template <int D, int TPC>
+// G: the call has an explicit global set (its masking code is compiled only
+// into that instantiation, keeping the common loop as tight as before).
+template <int D, int TPC, bool G>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const GqaParams p, int HC) {
@@ -182,6 +187,11 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 const int row = (phys * p.H_kv + kvh) * 64;
                 unsigned char *dst = sC + st * C::kStageBytes;
+                if constexpr (G) {
+                    const int blk = cur.logical_block();
+                    bars->gmask[st] = blk * 64 < cur.w.lo
+                                          ? global_mask_thread(p.vis, cur.w.b, blk) : 0ull;
+                }
                 mbar_arrive_expect_tx(&bars->c_full[st], C::kStageBytes);
                 for (int j = 0; j < C::kBoxes; ++j) {
                     tma_load_2d(dst + j * kTcBox, &tm_k, 64 * j, row, &bars->c_full[st], pol);
@@ -316,8 +326,21 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int i = 0; i < n_tiles; ++i) {
             const bool first = cur.t == 0, last = cur.t == cur.len - 1;
             const int b = cur.w.b, T = cur.w.T;
-            const int lo_tok = window_lo(p.vis, T), sink = p.vis.sink;
-            const int tok0 = cur.logical_block() * 64 + copy * TPC;
+            const int lo_tok = cur.w.lo, sink = p.vis.sink;
+            const int blk = cur.logical_block();
+            const int tok0 = blk * 64 + copy * TPC;
+            // Global positions among this block's keys below the window.
+            unsigned long long gmask = 0ull;
+            if (G && blk * 64 < lo_tok) {
+                // The stage of tile i is still armed for it (it is refilled only
+                // after this tile's P V), so this wait returns at once and orders
+                // the producer's mask before the read.
+                const int st = i % C::kStages;
+                if (!all(mbar_wait(&bars->c_full[st], (uint32_t)((i / C::kStages) & 1),
+                                   p.timeout_ns, p.err, abort_flag)))
+                    break;
+                gmask = bars->gmask[st];
+            }
             const int sb = i & 1;
             if (!all(mbar_wait(&bars->s_full[sb], (uint32_t)((i >> 1) & 1), p.timeout_ns, p.err,
                                abort_flag)))
@@ -339,11 +362,13 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 s[j] = v.x;
                 s[j + 1] = v.y;
             }
-            if (tok0 + TPC > T || (tok0 < lo_tok && tok0 + TPC > sink)) {
+            if (tok0 + TPC > T || (tok0 < lo_tok && (tok0 + TPC > sink || gmask))) {
 #pragma unroll
                 for (int j = 0; j < TPC; ++j) {
                     const int pos = tok0 + j;
-                    if (pos >= T || (pos < lo_tok && pos >= sink)) s[j] = kNegInf;
+                    if (pos >= T || (pos < lo_tok && pos >= sink &&
+                                     !((gmask >> (pos - blk * 64)) & 1ull)))
+                        s[j] = kNegInf;
                 }
             }
             float mx;
@@ -513,12 +538,12 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
 
 namespace {
 
-template <int D, int TPC>
-cudaError_t launch_tc(const GqaLaunch &L, int HC) {
+template <int D, int TPC, bool G>
+cudaError_t launch_tc_g(const GqaLaunch &L, int HC) {
     using C = TcCfg<D>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_tc_kernel<D, TPC>,
+        cudaError_t e = cudaFuncSetAttribute(gqa_tc_kernel<D, TPC, G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -530,7 +555,7 @@ cudaError_t launch_tc(const GqaLaunch &L, int HC) {
         !tc_make_map(&tv, kp.v_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64))
         return cudaErrorInvalidValue;
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
-    gqa_tc_kernel<D, TPC><<<kp.num_ctas, kTcThreads, C::kSmem, L.stream>>>(tq, tk, tv, kp, HC);
+    gqa_tc_kernel<D, TPC, G><<<kp.num_ctas, kTcThreads, C::kSmem, L.stream>>>(tq, tk, tv, kp, HC);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
@@ -553,6 +578,12 @@ cudaError_t launch_tc(const GqaLaunch &L, int HC) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, combine_kernel<__nv_bfloat16>, cp);
+}
+
+template <int D, int TPC>
+cudaError_t launch_tc(const GqaLaunch &L, int HC) {
+    return L.kp.vis.n_g > 0 ? launch_tc_g<D, TPC, true>(L, HC)
+                            : launch_tc_g<D, TPC, false>(L, HC);
 }
 
 }  // namespace

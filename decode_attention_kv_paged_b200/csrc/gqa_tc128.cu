@@ -63,13 +63,18 @@ struct T2Bars {
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], pv_done[2];
     uint64_t o_free, mma_final;
+    // Per stage: global positions among the staged block's keys below the
+    // window (bit t: key 64 * block + t), written before the stage is armed.
+    unsigned long long gmask[6];
     uint32_t tmem_base;
     int abort;
     PlanScratch plan;
 };
 static_assert(sizeof(T2Bars) <= 1024, "barrier block");
 
-template <int D, int HCP>
+// G: the call has an explicit global set (its masking code is compiled only
+// into that instantiation, keeping the common loop as tight as before).
+template <int D, int HCP, bool G>
 __global__ void __launch_bounds__(kT2Threads, 1)
 gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const GqaParams p, int HC) {
@@ -144,6 +149,11 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
                 const int row = (phys * p.H_kv + kvh) * 64;
                 unsigned char *dst = sC + st * C::kStageBytes;
+                if constexpr (G) {
+                    const int blk = cur.logical_block();
+                    bars->gmask[st] = blk * 64 < cur.w.lo
+                                          ? global_mask_thread(p.vis, cur.w.b, blk) : 0ull;
+                }
                 mbar_arrive_expect_tx(&bars->c_full[st], C::kStageBytes);
                 for (int j = 0; j < C::kBoxes; ++j) {
                     tma_load_2d(dst + j * kT2Box, &tm_k, 64 * j, row, &bars->c_full[st], pol);
@@ -280,7 +290,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         for (int i = 0; i < n_tiles; ++i) {
             const bool first = cur.t == 0, last = cur.t == cur.len - 1;
             const int b = cur.w.b, T = cur.w.T;
-            const int lo_tok = window_lo(p.vis, T), sink = p.vis.sink;
+            const int lo_tok = cur.w.lo, sink = p.vis.sink;
             if (first) {
                 // This segment's queries into TMEM (rows beyond the group: 0),
                 // once the previous segment's last S has read the old ones.
@@ -317,7 +327,20 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_arrive(&bars->s_free[sb]);
 
             // This lane's kTPC tokens: window positions [half kTPC, + kTPC).
-            const int tok0 = cur.logical_block() * 64 + 16 * q4 + half * kTPC;
+            const int blk = cur.logical_block();
+            const int tok0 = blk * 64 + 16 * q4 + half * kTPC;
+            // Global positions among this block's keys below the window.
+            unsigned long long gmask = 0ull;
+            if (G && blk * 64 < lo_tok) {
+                // The stage of tile i is still armed for it (it is refilled only
+                // after this tile's P V), so this wait returns at once and orders
+                // the producer's mask before the read.
+                const int st = i % C::kStages;
+                if (!all(mbar_wait(&bars->c_full[st], (uint32_t)((i / C::kStages) & 1),
+                                   p.timeout_ns, p.err, abort_flag)))
+                    break;
+                gmask = bars->gmask[st];
+            }
             float s[kTPC];
 #pragma unroll
             for (int j = 0; j < kTPC; ++j) {
@@ -325,11 +348,13 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if constexpr (kTPC == 8) v = half ? w16[8 + j] : w16[j];
                 s[j] = v * p.scale_log2;
             }
-            if (tok0 + kTPC > T || (tok0 < lo_tok && tok0 + kTPC > sink)) {
+            if (tok0 + kTPC > T || (tok0 < lo_tok && (tok0 + kTPC > sink || gmask))) {
 #pragma unroll
                 for (int j = 0; j < kTPC; ++j) {
                     const int pos = tok0 + j;
-                    if (pos >= T || (pos < lo_tok && pos >= sink)) s[j] = kNegInf;
+                    if (pos >= T || (pos < lo_tok && pos >= sink &&
+                                     !((gmask >> (pos - blk * 64)) & 1ull)))
+                        s[j] = kNegInf;
                 }
             }
             float mx = s[0];
@@ -448,12 +473,12 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 // -------------------------------------------------------------- host side
 namespace {
 
-template <int D, int HCP>
-cudaError_t launch_tc128(const GqaLaunch &L, int HC) {
+template <int D, int HCP, bool G>
+cudaError_t launch_tc128_g(const GqaLaunch &L, int HC) {
     using C = T2Cfg<D>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_tc128_kernel<D, HCP>,
+        cudaError_t e = cudaFuncSetAttribute(gqa_tc128_kernel<D, HCP, G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -464,7 +489,7 @@ cudaError_t launch_tc128(const GqaLaunch &L, int HC) {
         !tc_make_map(&tv, kp.v_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64))
         return cudaErrorInvalidValue;
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
-    gqa_tc128_kernel<D, HCP><<<kp.num_ctas, kT2Threads, C::kSmem, L.stream>>>(tk, tv, kp, HC);
+    gqa_tc128_kernel<D, HCP, G><<<kp.num_ctas, kT2Threads, C::kSmem, L.stream>>>(tk, tv, kp, HC);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
@@ -486,6 +511,12 @@ cudaError_t launch_tc128(const GqaLaunch &L, int HC) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, combine_kernel<__nv_bfloat16>, cp);
+}
+
+template <int D, int HCP>
+cudaError_t launch_tc128(const GqaLaunch &L, int HC) {
+    return L.kp.vis.n_g > 0 ? launch_tc128_g<D, HCP, true>(L, HC)
+                            : launch_tc128_g<D, HCP, false>(L, HC);
 }
 
 }  // namespace

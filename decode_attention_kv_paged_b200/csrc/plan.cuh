@@ -19,16 +19,41 @@ namespace attn {
 
 // Which cached keys a query sees, and where the block table keeps them
 // (attention-head article, §3: sliding window, and window plus global
-// tokens).  Key j of a sequence with T cached tokens is visible when j < T
-// and (no window, or j >= T - window, or j < sink).  With ring > 0 the table
-// row is a ring: the blocks holding the sink keys keep slots [0, A)
-// (A = ceil(sink / 64)); logical block i >= A lives in slot A + i % ring, so
-// a window layer stores only the blocks its window can reach.
+// tokens G).  Key j of a sequence with T cached tokens is visible to the
+// decode query (position T - 1) when j < T and (no window, or j >= T -
+// window, or j < sink, or j is in the sequence's global set G_b, or T - 1 is
+// itself in G_b: a global query sees the whole history).  G_b is row b of
+// gpos ([B][n_g], positions in ascending order; an entry below the previous
+// one, e.g. a -1 pad, ends the row).  With ring > 0 the table row is a ring:
+// the blocks holding the sink keys keep slots [0, A) (A = ceil(sink / 64));
+// logical block i >= A lives in slot A + i % ring, so a window layer stores
+// only the blocks its window can reach.
 struct Visibility {
     int window;   // > 0: sliding window of the last `window` keys
     int sink;     // > 0: the first `sink` keys stay visible (global tokens)
     int ring;     // > 0: ring of this many table slots after the sink blocks
+    const int32_t *gpos = nullptr;   // n_g > 0: global positions per sequence
+    int n_g = 0;
 };
+
+// Global set of sequence b: walks G_b's positions below T in ascending order.
+__host__ __device__ __forceinline__ const int32_t *global_row(const Visibility &v, int b) {
+    return v.gpos + (size_t)b * v.n_g;
+}
+
+// Whether the decode query of a sequence with T keys is a global position.
+__device__ __forceinline__ bool global_query(const Visibility &v, int b, int T) {
+    if (v.n_g <= 0 || T <= 0) return false;
+    const int32_t *g = global_row(v, b);
+    int prev = -1;
+    for (int i = 0; i < v.n_g; ++i) {
+        const int p = g[i];
+        if (p <= prev || p >= T) break;
+        if (p == T - 1) return true;
+        prev = p;
+    }
+    return false;
+}
 
 __host__ __device__ __forceinline__ int sink_blocks(const Visibility &v) {
     return v.sink > 0 ? (v.sink + kBlockSize - 1) / kBlockSize : 0;
@@ -46,17 +71,101 @@ __host__ __device__ __forceinline__ int window_lo(const Visibility &v, int T) {
     return (v.window > 0 && T > v.window) ? T - v.window : 0;
 }
 
-__host__ __device__ __forceinline__ bool key_visible(const Visibility &v, int j, int T) {
-    return j < T && (j >= window_lo(v, T) || j < v.sink);
+// First key of the contiguous visible run of sequence b: the window's start,
+// or 0 when the query itself is global.
+__device__ __forceinline__ int seq_window_lo(const Visibility &v, int b, int T) {
+    return global_query(v, b, T) ? 0 : window_lo(v, T);
 }
 
-// Visible blocks of a sequence with T cached tokens (current one included):
-// blocks holding at least one visible key, in order.  They are the first
-// *sink_blks logical blocks (the sink part) followed by a run starting at
-// logical block *first_block; visible block v is logical block
-// v < sink_blks ? v : first_block + v - sink_blks.
+// Logical block of the i-th distinct block (ascending) holding a global
+// position of sequence b below block w0 (i < the count visible_blocks gave).
+__device__ __forceinline__ int global_block(const Visibility &v, int b, int i) {
+    const int32_t *g = global_row(v, b);
+    int prev = -1, last = -1, n = 0;
+    for (int k = 0; k < v.n_g; ++k) {
+        const int p = g[k];
+        if (p <= prev) break;
+        prev = p;
+        const int blk = p / kBlockSize;
+        if (blk != last) {
+            if (n == i) return blk;
+            ++n;
+            last = blk;
+        }
+    }
+    return last;   // not reached for i < count
+}
+
+// Bit t set when token blk * 64 + t of sequence b is a global position.
+// One warp, all 32 lanes; rows of up to 64 entries.
+__device__ __forceinline__ unsigned long long global_mask(const Visibility &v, int b, int blk,
+                                                       int lane) {
+    const int32_t *g = global_row(v, b);
+    const int k0 = lane, k1 = lane + 32;
+    const int p0 = k0 < v.n_g ? g[k0] : 0, p1 = k1 < v.n_g ? g[k1] : 0;
+    const int q0 = k0 == 0 ? -1 : (k0 < v.n_g ? g[k0 - 1] : 0);
+    const int q1 = k1 < v.n_g ? g[k1 - 1] : 0;
+    // The row ends at its first entry that does not exceed the one before.
+    const unsigned e0 = __ballot_sync(0xffffffffu, k0 >= v.n_g || p0 <= q0);
+    const unsigned e1 = __ballot_sync(0xffffffffu, k1 >= v.n_g || p1 <= q1);
+    const int end = e0 ? __ffs(e0) - 1 : (e1 ? 32 + __ffs(e1) - 1 : 64);
+    unsigned lo = 0u, hi = 0u;
+    const int t0 = p0 - blk * kBlockSize, t1 = p1 - blk * kBlockSize;
+    if (k0 < end && t0 >= 0 && t0 < kBlockSize) (t0 < 32 ? lo : hi) |= 1u << (t0 & 31);
+    if (k1 < end && t1 >= 0 && t1 < kBlockSize) (t1 < 32 ? lo : hi) |= 1u << (t1 & 31);
+    lo = __reduce_or_sync(0xffffffffu, lo);
+    hi = __reduce_or_sync(0xffffffffu, hi);
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+// visible_blocks with a global set: the distinct blocks of global
+// positions before the window, then the window run.
+__device__ __forceinline__ int visible_blocks_global(int T, const Visibility &v, int b, int w1,
+                                                   int *first_block, int *sink_blks) {
+    const int w0 = seq_window_lo(v, b, T) / kBlockSize;
+    if (w0 == 0) return w1;                               // one run [0, w1)
+    const int32_t *g = global_row(v, b);
+    int prev = -1, last = -1, n = 0;
+    for (int k = 0; k < v.n_g; ++k) {
+        const int p = g[k];
+        if (p <= prev || p / kBlockSize >= w0) break;
+        prev = p;
+        if (p / kBlockSize != last) {
+            ++n;
+            last = p / kBlockSize;
+        }
+    }
+    *sink_blks = n;
+    *first_block = w0;
+    return n + (w1 - w0);
+}
+
+// global_mask computed by one thread.
+__device__ __forceinline__ unsigned long long global_mask_thread(const Visibility &v, int b,
+                                                                 int blk) {
+    const int32_t *g = global_row(v, b);
+    unsigned long long m = 0ull;
+    int prev = -1;
+    for (int k = 0; k < v.n_g; ++k) {
+        const int p = g[k];
+        if (p <= prev) break;
+        prev = p;
+        const int t = p - blk * kBlockSize;
+        if (t >= kBlockSize) break;
+        if (t >= 0) m |= 1ull << t;
+    }
+    return m;
+}
+
+// Visible blocks of sequence b with T cached tokens (current one included):
+// blocks holding at least one visible key, in order.  They are *sink_blks
+// blocks before the window (the sink blocks [0, A), or the distinct blocks
+// of global positions) followed by a run starting at logical block
+// *first_block; visible block v is logical block first_block + v -
+// sink_blks for v >= sink_blks, else v (sink) or global_block(v) (set G).
 __device__ __forceinline__ int visible_blocks(int T, const Visibility &v, int max_blocks,
-                                              int *first_block, int *sink_blks, bool *bad) {
+                                              int *first_block, int *sink_blks, bool *bad,
+                                              int b = 0) {
     *first_block = 0;
     *sink_blks = 0;
     if (T <= 0) {
@@ -68,8 +177,9 @@ __device__ __forceinline__ int visible_blocks(int T, const Visibility &v, int ma
         return 0;
     }
     *bad = false;
-    const int w0 = window_lo(v, T) / kBlockSize;        // first window block
     const int w1 = (T - 1) / kBlockSize + 1;             // one past the last block
+    if (v.n_g > 0) return visible_blocks_global(T, v, b, w1, first_block, sink_blks);
+    const int w0 = window_lo(v, T) / kBlockSize;        // first window block
     const int a = sink_blocks(v) < w1 ? sink_blocks(v) : w1;
     if (a >= w0) return w1;                               // one run [0, w1)
     *sink_blks = a;
@@ -134,7 +244,7 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
             if (lane < a.B) {
                 int fb, sb;
                 w = (long long)visible_blocks(a.seq_lens[lane], a.vis, a.max_blocks, &fb, &sb,
-                                              &bad) *
+                                              &bad, lane) *
                     a.units_per_seq;
             }
             long long x = w;
@@ -174,7 +284,7 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
     for (int b = tid; b < a.B; b += nt) {
         int fb, sb;
         bool bad;
-        mine += (long long)visible_blocks(a.seq_lens[b], a.vis, a.max_blocks, &fb, &sb, &bad) *
+        mine += (long long)visible_blocks(a.seq_lens[b], a.vis, a.max_blocks, &fb, &sb, &bad, b) *
                 a.units_per_seq;
         any_bad |= bad;
     }
@@ -202,7 +312,7 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
         if (b < a.B) {
             int fb, sb;
             bool bad;
-            w = (long long)visible_blocks(a.seq_lens[b], a.vis, a.max_blocks, &fb, &sb, &bad) *
+            w = (long long)visible_blocks(a.seq_lens[b], a.vis, a.max_blocks, &fb, &sb, &bad, b) *
                 a.units_per_seq;
         }
         long long x = w;
@@ -250,16 +360,19 @@ struct SegmentWalker {
     // state
     long long pos, end;
     int b, unit, blk_off, nb, first_blk, sink_blks, T;
+    int lo;   // first key of the contiguous visible run (window start, or 0)
 
     __device__ void load_seq() {
         bool bad;
         T = seq_lens[b];
-        nb = visible_blocks(T, vis, max_blocks, &first_blk, &sink_blks, &bad);
+        nb = visible_blocks(T, vis, max_blocks, &first_blk, &sink_blks, &bad, b);
+        lo = vis.n_g > 0 ? seq_window_lo(vis, b, T) : window_lo(vis, T);
     }
 
     // Logical block of visible block v of the current sequence.
     __device__ int logical(int v) const {
-        return v < sink_blks ? v : first_blk + (v - sink_blks);
+        if (v >= sink_blks) return first_blk + (v - sink_blks);
+        return vis.n_g > 0 ? global_block(vis, b, v) : v;
     }
 
     __device__ void init(const PlanArgs &a, long long lo, long long hi,

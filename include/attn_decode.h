@@ -140,8 +140,18 @@ int kv_append_mla(const void *latent_new, void *latent_cache,
 /*
  * attn_visibility -- which cached keys each query sees, and how the block
  * table row maps them (attention-head article, §3 sliding window; window plus
- * global tokens).  Key j of a sequence with T = seq_lens[b] cached tokens is
- * visible when j < T and (window <= 0, or j >= T - window, or j < sink_tokens).
+ * global tokens G).  Key j of a sequence with T = seq_lens[b] cached tokens is
+ * visible to the decode query (position T - 1) when j < T and (window <= 0,
+ * or j >= T - window, or j < sink_tokens, or j is a global position of the
+ * sequence, or T - 1 is itself a global position: a global query sees the
+ * whole history).  Global positions: global_pos is a device int32 array
+ * [B][n_global], row b holding sequence b's positions in ascending order;
+ * the row ends at its first entry that does not exceed the previous one (pad
+ * with -1).  0 < n_global <= 64; global_pos needs sink_tokens = 0 and
+ * ring_blocks = 0 (ATTN_ERR_ARG otherwise; n_global > 64:
+ * ATTN_ERR_UNSUPPORTED); n_global = 0 ignores global_pos.  Blocks before the
+ * window hold visible keys only where a global position lies, and only those
+ * blocks are read.
  * ring_blocks > 0 makes the table row a ring for window layers: the blocks
  * holding the sink keys keep slots [0, A) with A = ceil(sink_tokens / 64),
  * and logical block i >= A lives in slot A + (i mod ring_blocks), so a
@@ -156,6 +166,8 @@ typedef struct attn_visibility {
     int window;
     int sink_tokens;
     int ring_blocks;
+    const int32_t *global_pos;   /* device, [B][n_global]; may be NULL if n_global == 0 */
+    int n_global;
 } attn_visibility;
 
 /*

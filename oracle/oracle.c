@@ -105,15 +105,29 @@ static size_t orc_row_offset(const int32_t *block_table, int max_blocks, int b,
  * a zero output row.
  */
 /*
- * Decode attention with global (sink) tokens and a ring-buffer table
- * (attention-head article, §3: sliding window; window plus global tokens).
- * Key j of sequence b (T = seq_lens[b]) is visible when j < T and
- * (window <= 0 or j >= T - window or j < sink).  The row of key j sits in
+ * Decode attention with global tokens and a ring-buffer table
+ * (attention-head article, §3: sliding window; window plus global tokens G,
+ * whose figure has G = {0, 5}: row 8 sees {0, 5, 6, 7, 8} with w = 3, and
+ * the global query of row 5 sees all of 0..5).  Key j of sequence b
+ * (T = seq_lens[b]; the query is position T - 1) is visible when j < T and
+ * (window <= 0 or j >= T - window or j < sink or j in G_b or T - 1 in G_b).
+ * G_b is row b of gpos [B][n_g] (n_g = 0: empty), read in order up to its
+ * first entry that does not exceed the one before.  The row of key j sits in
  * the block of table slot slot(j / block_size): with ring > 0, logical block
  * i < A = ceil(sink / block_size) keeps slot i and i >= A goes to slot
  * A + i % ring; without ring, slot i = i.  Softmax over the visible keys only.
  * Same arrays and dtypes as orc_decode_gqa; probs (optional) [B][H_q][max_T].
  */
+static int orc_in_set(const int32_t *row, int n, int x) {
+    int prev = -1;
+    for (int k = 0; k < n; ++k) {
+        if (row[k] <= prev) break;
+        if (row[k] == x) return 1;
+        prev = row[k];
+    }
+    return 0;
+}
+
 static int orc_slot(int i, int sink, int ring, int block_size) {
     if (ring <= 0) return i;
     const int a = sink > 0 ? (sink + block_size - 1) / block_size : 0;
@@ -124,9 +138,10 @@ int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *seq_lens, const int32_t *block_table,
                        double *out, double *probs, int max_T, int B, int H_q,
                        int H_kv, int d, int block_size, int max_blocks,
-                       double scale, int window, int sink, int ring, int dtype) {
+                       double scale, int window, int sink, int ring, int dtype,
+                       const int32_t *gpos, int n_g) {
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || d <= 0 || block_size <= 0 ||
-        H_q % H_kv != 0 || sink < 0 || ring < 0)
+        H_q % H_kv != 0 || sink < 0 || ring < 0 || n_g < 0 || (n_g > 0 && !gpos))
         return ORC_BAD_ARG;
     const int group = H_q / H_kv;
     int status = ORC_OK;
@@ -151,9 +166,13 @@ int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
                 status = ORC_NO_MEM;
                 continue;
             }
+            const int32_t *grow = n_g > 0 ? gpos + (size_t)b * n_g : NULL;
+            const int q_global = grow && orc_in_set(grow, n_g, T - 1);
             int n = 0;
             for (int j = 0; j < T; ++j)
-                if (window <= 0 || j >= T - window || j < sink) keys[n++] = j;
+                if (window <= 0 || j >= T - window || j < sink || q_global ||
+                    (grow && orc_in_set(grow, n_g, j)))
+                    keys[n++] = j;
             const size_t q_off = ((size_t)b * H_q + h) * d;
             for (int t = 0; t < n; ++t) {
                 const int j = keys[t];

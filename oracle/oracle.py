@@ -25,7 +25,8 @@ def _load():
         c_p, c_i, c_d = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         lib.orc_decode_gqa.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i, c_i]
         lib.orc_decode_gqa.restype = c_i
-        lib.orc_decode_gqa_vis.argtypes = [c_p] * 7 + [c_i] * 7 + [c_d, c_i, c_i, c_i, c_i]
+        lib.orc_decode_gqa_vis.argtypes = ([c_p] * 7 + [c_i] * 7 + [c_d, c_i, c_i, c_i, c_i] +
+                                           [c_p, c_i])
         lib.orc_decode_gqa_vis.restype = c_i
         lib.orc_e4m3_value.argtypes = [c_i]
         lib.orc_e4m3_value.restype = c_d
@@ -123,13 +124,16 @@ def decode_gqa(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
 
 
 def decode_gqa_vis(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
-                   sink=0, ring=0, return_probs=False):
-    """decode_gqa with global (sink) tokens and a ring-buffer table (fp64).
+                   sink=0, ring=0, return_probs=False, global_pos=None):
+    """decode_gqa with global tokens and a ring-buffer table (fp64).
 
-    Key j < T is visible when window <= 0, j >= T - window or j < sink.  With
-    ring > 0, logical block i lives in table slot i for i < A = ceil(sink /
-    block_size) (the sink blocks) and in slot A + i % ring after them.  Same arrays as
-    decode_gqa.
+    Key j < T is visible when window <= 0, j >= T - window, j < sink, j is in
+    the sequence's global set, or T - 1 is in it (attention-head article, §3:
+    a global query sees the whole history).  global_pos: int [B][n_g], each
+    row ascending and read up to its first entry that does not exceed the one
+    before (pad with -1).  With ring > 0, logical block i lives in table slot
+    i for i < A = ceil(sink / block_size) (the sink blocks) and in slot
+    A + i % ring after them.  Same arrays as decode_gqa.
     """
     B, H_q, d = q.shape
     _, H_kv, bs, d2 = k_cache.shape
@@ -144,10 +148,18 @@ def decode_gqa_vis(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
     out = np.zeros((B, H_q, d), dtype=np.float64)
     max_T = int(sl.max().item()) if return_probs and B > 0 else 0
     probs = np.zeros((B, H_q, max_T), dtype=np.float64) if return_probs else None
+    if global_pos is None:
+        gp, gpp, n_g = None, None, 0
+    else:
+        gp, gpp = _as_i32(global_pos)
+        if gp.ndim != 2 or gp.shape[0] != B:
+            raise ValueError("global_pos must be [B][n_g]")
+        n_g = gp.shape[1]
     rc = _load().orc_decode_gqa_vis(
         qp, kp, vp, slp, btp, out.ctypes.data,
         probs.ctypes.data if probs is not None else None, max_T,
-        B, H_q, H_kv, d, bs, bt.shape[1], float(scale), int(window), int(sink), int(ring), dt)
+        B, H_q, H_kv, d, bs, bt.shape[1], float(scale), int(window), int(sink), int(ring), dt,
+        gpp, n_g)
     if rc != 0:
         raise RuntimeError(f"oracle decode_gqa_vis failed with status {rc}")
     return (out, probs) if return_probs else out

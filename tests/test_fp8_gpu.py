@@ -117,3 +117,27 @@ def test_fp8_append_then_decode(lib):
                          orc.dequantize_e4m3(vc, vs), np.full(B, T, dtype=np.int32),
                          table.numpy(), 0.1)
     assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, "fp8 append+decode")
+
+
+def test_fp8_decode_with_global_positions(lib):
+    """The fp8 cache under a window plus an explicit global set."""
+    lens, window = [2000, 700], 300
+    rows = [[0, 5, 640, 1650], [699, -1, -1, -1]]
+    H_q, H_kv, d = 32, 8, 128
+    B = len(lens)
+    slots = max((T + 63) // 64 for T in lens)
+    n_blocks = B * slots + 2
+    kc, ks, vc, vs = _fp8_cache(8400, n_blocks, H_kv, d)
+    g = torch.Generator().manual_seed(8401)
+    q = torch.randn((B, H_q, d), generator=g).bfloat16()
+    table = torch.randperm(n_blocks, generator=g)[: B * slots].reshape(B, slots).to(torch.int32)
+    gp = torch.tensor(rows, dtype=torch.int32)
+    got = lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV), torch.from_numpy(vc).to(DEV),
+                             torch.from_numpy(ks).to(DEV), torch.from_numpy(vs).to(DEV),
+                             torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV),
+                             0.09, window=window, global_pos=gp.to(DEV))
+    assert lib.last_error() == lib.OK
+    ref = orc.decode_gqa_vis(q.double().numpy(), orc.dequantize_e4m3(kc, ks),
+                             orc.dequantize_e4m3(vc, vs), np.asarray(lens, dtype=np.int32),
+                             table.numpy(), 0.09, window=window, global_pos=gp.numpy())
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, "fp8 global set")

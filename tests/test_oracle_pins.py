@@ -477,6 +477,64 @@ def test_vis_ring_table_reads_the_same_rows():
     assert np.array_equal(got, ref)
 
 
+def _visible_keys(p):
+    return [set(np.nonzero(p[b, h])[0].tolist()) for b in range(p.shape[0])
+            for h in range(p.shape[1])]
+
+
+def test_vis_global_set_matches_page_figure():
+    """The attention-head §3 figure (right panel): w=3, G={0,5}.  The decode
+    query of a sequence with T keys is row T-1: row 8 sees {0,5,6,7,8}, the
+    global row 5 sees all of 0..5 (fixture tests/golden/global_tokens.json)."""
+    fx = json.load(open(os.path.join(GOLDEN, "global_tokens.json")))
+    rng = np.random.default_rng(35)
+    for case in fx["cases"]:
+        T = case["T"]
+        q, k, v, table = _contiguous_case(rng, 2, 1, 8, T)
+        gp = np.array([fx["global"]], dtype=np.int32)
+        _, p = orc.decode_gqa_vis(q, k, v, np.array([T], dtype=np.int32), table, 0.5,
+                                  window=fx["window"], global_pos=gp, return_probs=True)
+        assert all(ks == set(case["visible"]) for ks in _visible_keys(p)), T
+
+
+def test_vis_global_set_brute_force_membership():
+    """Every (T, G) over small cases: exactly the keys the definition lists
+    carry weight -- window, global keys, and everything for a global query;
+    a -1 pad or an entry that does not ascend ends the row."""
+    rng = np.random.default_rng(36)
+    for T in range(1, 20):
+        for row in ([0, 5], [3], [T - 1], [2, 9, 11, -1, -1], [4, 7, 6, 12], [-1, 3]):
+            w = 3
+            q, k, v, table = _contiguous_case(rng, 1, 1, 4, T)
+            gp = np.array([row], dtype=np.int32)
+            _, p = orc.decode_gqa_vis(q, k, v, np.array([T], dtype=np.int32), table, 0.5,
+                                      window=w, global_pos=gp, return_probs=True)
+            G, prev = set(), -1
+            for x in row:
+                if x <= prev:
+                    break
+                G.add(x)
+                prev = x
+            if (T - 1) in G:
+                want = set(range(T))
+            else:
+                want = {j for j in range(T) if j >= T - w or j in G}
+            assert _visible_keys(p)[0] == want, (T, row)
+
+
+def test_vis_global_prefix_equals_sink_tokens():
+    """G = {0..g-1} is the sink prefix: same keys, same order, bit-identical
+    (attention-head §3, window plus global tokens)."""
+    rng = np.random.default_rng(37)
+    q, k, v, table = _contiguous_case(rng, 4, 2, 16, 500)
+    lens = np.array([500], dtype=np.int32)
+    for g in (1, 7, 64, 70):
+        a = orc.decode_gqa_vis(q, k, v, lens, table, 0.2, window=100, sink=g)
+        gp = np.arange(g, dtype=np.int32)[None, :]
+        b = orc.decode_gqa_vis(q, k, v, lens, table, 0.2, window=100, global_pos=gp)
+        assert np.array_equal(a, b), g
+
+
 # ------------------------------------------------------- fp8 (E4M3) KV cache
 def test_e4m3_values_match_the_format():
     """Closed forms of the OCP FP8 E4M3 format: bias 7, 3 mantissa bits,

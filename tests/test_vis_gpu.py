@@ -131,3 +131,81 @@ def test_visibility_host_validation(lib):
         with pytest.raises(lib.AttnError) as e:
             lib.decode_gqa_ext(*args, **kw)
         assert e.value.status == lib.ERR_ARG, kw
+
+
+GLOBAL_CASES = [
+    # (H_q, H_kv, d, lens, window, global rows (-1 padded))
+    (32, 8, 128, [1000, 300, 4097, 65],
+     [[0, 5, 130, 700], [299, -1, -1, -1], [1, 2, 64, 3000], [-1, -1, -1, -1]], 200),
+    (32, 1, 128, [3000, 640, 1],
+     [[0, 70, 71, 200, 1500, 2990], [0, 639, -1, -1, -1, -1], [0, -1, -1, -1, -1, -1]], 100),
+    (24, 4, 256, [5000, 129],
+     [[10, 64 * 20 + 3, 64 * 40, 4000], [5, 6, 7, -1]], 700),
+    (8, 8, 64, [700, 300], [[4, 7, 6, 600], [3] + [-1] * 3], 33),
+]
+
+
+@pytest.mark.parametrize("path", [0, 1, 2], ids=["cuda_core", "tcgen05", "tcgen05_m64"])
+@pytest.mark.parametrize("H_q,H_kv,d,lens,rows,window", GLOBAL_CASES,
+                         ids=[f"q{c[0]}_kv{c[1]}_d{c[2]}_w{c[5]}" for c in GLOBAL_CASES])
+def test_global_positions_match_oracle(lib, path, H_q, H_kv, d, lens, rows, window):
+    """Window plus an explicit global set per sequence (attention-head §3,
+    G = {0, 5} in its figure): blocks before the window are read only where
+    a global position lies, keys in them are masked to the set, and a query
+    that is itself global sees everything; every kernel vs the oracle."""
+    B = len(lens)
+    slots = max((T + 63) // 64 for T in lens)
+    q, k, v, table = _inputs(7300 + H_q + d, B, H_q, H_kv, d, B * slots + 3, slots)
+    gp = torch.tensor(rows, dtype=torch.int32)
+    scale = 1.0 / np.sqrt(d)
+    ref = orc.decode_gqa_vis(q, k, v, np.asarray(lens, dtype=np.int32), table.numpy(), scale,
+                             window=window, global_pos=gp.numpy())
+    lib.set_gqa_path(path)
+    try:
+        got = lib.decode_gqa_ext(q.to(DEV), k.to(DEV), v.to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                 table.to(DEV), scale, window=window, global_pos=gp.to(DEV))
+        assert lib.last_error() == lib.OK
+    finally:
+        lib.set_gqa_path(-1)
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, f"global set, path {path}")
+
+
+def test_global_positions_many_tiles_per_cta(lib):
+    """Three CTAs over the batch: global blocks and window runs of several
+    sequences in one CTA's range, on both tensor-core kernels and CUDA cores."""
+    lens = [2000, 1500, 700]
+    rows = [[0, 1, 500, 1000], [64, 900, -1, -1], [699, -1, -1, -1]]
+    for path, (H_q, H_kv, d) in ((0, (32, 8, 128)), (1, (32, 2, 128)), (2, (48, 2, 256))):
+        B = len(lens)
+        slots = max((T + 63) // 64 for T in lens)
+        q, k, v, table = _inputs(7400 + path, B, H_q, H_kv, d, B * slots + 2, slots)
+        gp = torch.tensor(rows, dtype=torch.int32)
+        ref = orc.decode_gqa_vis(q, k, v, np.asarray(lens, dtype=np.int32), table.numpy(), 0.1,
+                                 window=250, global_pos=gp.numpy())
+        lib.set_gqa_path(path)
+        lib.set_num_ctas(3)
+        try:
+            got = lib.decode_gqa_ext(q.to(DEV), k.to(DEV), v.to(DEV),
+                                     torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                     table.to(DEV), 0.1, window=250, global_pos=gp.to(DEV))
+            assert lib.last_error() == lib.OK
+        finally:
+            lib.set_gqa_path(-1)
+            lib.set_num_ctas(0)
+        assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, f"path {path}")
+
+
+def test_global_positions_host_validation(lib):
+    q, k, v, table = _inputs(2, 1, 4, 2, 64, 8, 4)
+    args = (q.to(DEV), k.to(DEV), v.to(DEV), torch.tensor([100], dtype=torch.int32,
+                                                          device=DEV), table.to(DEV), 0.1)
+    gp = torch.tensor([[0, 5]], dtype=torch.int32, device=DEV)
+    for kw, status in ((dict(window=10, sink_tokens=4, global_pos=gp), lib.ERR_ARG),
+                       (dict(window=64, ring_blocks=3, global_pos=gp), lib.ERR_ARG),
+                       (dict(window=10, global_pos=torch.zeros((1, 65), dtype=torch.int32,
+                                                               device=DEV)),
+                        lib.ERR_UNSUPPORTED)):
+        with pytest.raises(lib.AttnError) as e:
+            lib.decode_gqa_ext(*args, **kw)
+        assert e.value.status == status, kw
