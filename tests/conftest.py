@@ -29,7 +29,7 @@ def oracle():
 
 @pytest.fixture(scope="session")
 def lib():
-    """The CUDA library (C-ABI) -- loading it must succeed on a GPU machine."""
+    """The CUDA library (C-ABI) -- loading it must succeed wherever a GPU is present."""
     import decode_attention_kv_paged_b200 as attn
     attn.load()
     return attn
