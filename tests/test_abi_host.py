@@ -93,3 +93,43 @@ def test_host_planner_partition_properties(lens, units, window, P):
                 s = b * units + u + c
                 assert s not in slots and s < U + P
                 slots.add(s)
+
+
+def test_visibility_struct_layout_matches_header(tmp_path):
+    """The Python binding's attn_visibility has the header's layout (field
+    offsets and size, as a C compiler lays it out)."""
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "attn_decode.h"\n'
+                   'int main(void) { printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(attn_visibility),'
+                   ' offsetof(attn_visibility, window), offsetof(attn_visibility, sink_tokens),'
+                   ' offsetof(attn_visibility, ring_blocks), offsetof(attn_visibility, global_pos),'
+                   ' offsetof(attn_visibility, n_global)); return 0; }\n')
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    V = attn.Visibility
+    want = [ctypes.sizeof(V), V.window.offset, V.sink_tokens.offset, V.ring_blocks.offset,
+            V.global_pos.offset, V.n_global.offset]
+    assert got == want
+
+
+def test_global_set_validated_on_the_host():
+    """An explicit global set with sink tokens or a ring, a null set, or more
+    than 64 positions is refused before any launch."""
+    lib = attn.load()
+    p = ctypes.c_void_p(16)      # never dereferenced: validation fails first
+    g = ctypes.c_void_p(64)
+
+    def call(vis):
+        return lib.attn_decode_gqa_ext(p, p, p, p, p, p, 1, 8, 2, 64, ctypes.c_float(0.1),
+                                       ctypes.byref(vis), None, 4, 8, attn.BF16)
+    V = attn.Visibility
+    assert call(V(10, 4, 0, g.value, 2)) == attn.ERR_ARG        # with sink tokens
+    assert call(V(64, 0, 3, g.value, 2)) == attn.ERR_ARG        # with a ring
+    assert call(V(10, 0, 0, None, 2)) == attn.ERR_ARG           # no positions
+    assert call(V(10, 0, 0, g.value, -1)) == attn.ERR_ARG       # negative count
+    assert call(V(10, 0, 0, ctypes.c_void_p(66).value, 2)) == attn.ERR_ARG   # misaligned
+    assert call(V(10, 0, 0, g.value, 65)) == attn.ERR_UNSUPPORTED
