@@ -109,15 +109,25 @@ def traffic_for(kernel, wl_name):
     """dram bytes per launch of `kernel` on `wl_name` from the committed ncu
     summary, if the kernel's sources are unchanged since it was taken; else
     None."""
+    return traffic_entry(kernel, wl_name)[0]
+
+
+def traffic_entry(kernel, wl_name):
+    """(dram bytes per launch or None, note): the note says why the figure is
+    missing (no capture of this kernel on this workload, or a capture of
+    different kernel sources)."""
     if not os.path.exists(TRAFFIC_FILE):
-        return None
+        return None, "no ncu capture committed"
     with open(TRAFFIC_FILE) as f:
         j = json.load(f)
     e = j.get(wl_name)
-    if (not e or e.get("kernel") != kernel
-            or e.get("kernel_hash") != kernel_hash(kernel)):
-        return None
-    return e.get("dram_bytes_per_launch")
+    if not e or e.get("kernel") != kernel:
+        return None, "no ncu capture of this kernel on this workload"
+    if e.get("kernel_hash") != kernel_hash(kernel):
+        return None, ("the committed capture (%s, %.1f MB per launch) was taken on other "
+                      "sources of this kernel" % (e.get("summary"),
+                                                  e.get("dram_bytes_per_launch", 0) / 1e6))
+    return e.get("dram_bytes_per_launch"), None
 
 
 # ------------------------------------------------------------------ clocks
@@ -393,7 +403,9 @@ def run_native(args, rank, world, local):  # noqa: C901
     roof["kernel"] = kernel
     roof["kernel_ms_avg"] = kern_avg
     roof["algorithmic_bytes_per_launch"] = alg_bytes
-    roof["traffic"] = traffic_for(kernel, wl_name)
+    roof["traffic"], note = traffic_entry(kernel, wl_name)
+    if note:
+        roof["traffic_note"] = note
 
     line = {
         "metric": "decode tokens/s and KV-cache read GB/s (% of B200 HBM peak), 1 GPU",
