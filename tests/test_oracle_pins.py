@@ -535,6 +535,36 @@ def test_vis_global_prefix_equals_sink_tokens():
         assert np.array_equal(a, b), g
 
 
+@pytest.mark.parametrize("T,w,g,R", [(700, 100, 10, 3), (65, 64, 0, 2), (1000, 200, 70, 5),
+                                     (129, 1, 0, 1), (5000, 640, 64, 11), (300, 63, 130, 2)])
+def test_vis_ring_table_any_geometry_reads_the_same_rows(T, w, g, R):
+    """For any ring large enough for the window (R * 64 >= w + 63), a table
+    row of A sink slots + R ring slots holding the sink blocks and the blocks
+    the window reaches gives the full table's result bit for bit; every other
+    block of the ring-side pool holds noise that must never be read."""
+    if R * 64 < w + 63:
+        pytest.skip("ring smaller than the window")
+    rng = np.random.default_rng(T + w + g + R)
+    q, k, v, table = _contiguous_case(rng, 2, 1, 8, T)
+    lens = np.array([T], dtype=np.int32)
+    ref = orc.decode_gqa_vis(q, k, v, lens, table, 0.3, window=w, sink=g)
+    A = (g + 63) // 64
+    nb = (T + 63) // 64
+    lo_blk = max(0, T - w) // 64
+    slots = A + R
+    perm = rng.permutation(slots + 3).astype(np.int32)
+    ring_table = perm[:slots][None, :]
+    kr = rng.standard_normal((slots + 3, 1, 64, 8))
+    vr = rng.standard_normal((slots + 3, 1, 64, 8))
+    needed = set(range(min(A, nb))) | set(range(lo_blk, nb))
+    for logical in needed:
+        slot = logical if logical < A else A + logical % R
+        kr[ring_table[0, slot]] = k[logical]
+        vr[ring_table[0, slot]] = v[logical]
+    got = orc.decode_gqa_vis(q, kr, vr, lens, ring_table, 0.3, window=w, sink=g, ring=R)
+    assert np.array_equal(got, ref)
+
+
 # ------------------------------------------------------- fp8 (E4M3) KV cache
 def test_e4m3_values_match_the_format():
     """Closed forms of the OCP FP8 E4M3 format: bias 7, 3 mantissa bits,
