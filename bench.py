@@ -61,6 +61,7 @@ WORKLOAD_ALIASES = {
     "ragged_window": W.RAGGED_WINDOW.name,
     "ragged_window_sink": W.RAGGED_WINDOW_SINK.name,
     "ragged_window_ring": W.RAGGED_WINDOW_RING.name,
+    "ragged_window_global": W.RAGGED_WINDOW_GLOBAL.name,
     "llama3_8b_fp8": W.LLAMA3_8B_FP8.name,
     "mla": W.MLA_DSV2.name,
 }
@@ -74,7 +75,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="llama3_8b",
                     help="llama3_8b | tiny | ragged_full | ragged_window | "
-                         "ragged_window_sink | ragged_window_ring | mla "
+                         "ragged_window_sink | ragged_window_ring | ragged_window_global | mla "
                          "| a sweep name such as sweep_bf16_B8_Hq32_Hkv8_d128_T32768")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true",
@@ -258,6 +259,40 @@ def visible_tiles(T, window, sink):
     return w1 if a >= w0 else a + w1 - w0
 
 
+def _global_set(row):
+    """The positions a global-position row holds (ascending run, -1 pads)."""
+    out, prev = [], -1
+    for p in row:
+        if p <= prev:
+            break
+        out.append(p)
+        prev = p
+    return out
+
+
+def visible_keys_global(T, window, row):
+    """visible_keys with an explicit global set: the window, the global
+    positions before it, or every key when the query (T - 1) is global."""
+    G = [p for p in _global_set(row) if p < T]
+    if T <= 0:
+        return 0
+    if window <= 0 or T - 1 in G:
+        return T
+    lo = max(0, T - window)
+    return T - lo + sum(1 for p in G if p < lo)
+
+
+def visible_tiles_global(T, window, row):
+    if T <= 0:
+        return 0
+    G = [p for p in _global_set(row) if p < T]
+    w1 = (T - 1) // 64 + 1
+    if window <= 0 or T - 1 in G:
+        return w1
+    w0 = max(0, T - window) // 64
+    return len({p // 64 for p in G if p // 64 < w0}) + w1 - w0
+
+
 def kv_row_bytes(cfg):
     """Cache bytes of one (token, KV head) row, K and V together: 2 d s, or
     2 (d + 4) for the fp8 cache (one byte per element plus a fp32 row scale)."""
@@ -271,8 +306,10 @@ def algorithmic_bytes_gqa(inp):
     cfg = inp.cfg
     s = torch.finfo(cfg.dtype).bits // 8
     vis = 0
-    for T in inp.seq_list:
-        vis += visible_keys(T, inp.window, cfg.sink)
+    rows = inp.global_pos.tolist() if inp.global_pos is not None else None
+    for b, T in enumerate(inp.seq_list):
+        vis += (visible_keys_global(T, inp.window, rows[b]) if rows
+                else visible_keys(T, inp.window, cfg.sink))
     kv = vis * cfg.H_kv * kv_row_bytes(cfg)
     qo = 2 * cfg.B * cfg.H_q * cfg.d * s
     return kv, kv + qo
@@ -283,8 +320,10 @@ def tile_bytes_gqa(inp):
     cfg = inp.cfg
     s = torch.finfo(cfg.dtype).bits // 8
     blocks = 0
-    for T in inp.seq_list:
-        blocks += visible_tiles(T, inp.window, cfg.sink)
+    rows = inp.global_pos.tolist() if inp.global_pos is not None else None
+    for b, T in enumerate(inp.seq_list):
+        blocks += (visible_tiles_global(T, inp.window, rows[b]) if rows
+                   else visible_tiles(T, inp.window, cfg.sink))
     return blocks * 64 * cfg.H_kv * kv_row_bytes(cfg)
 
 
@@ -343,7 +382,8 @@ def run_native(args, rank, world, local):  # noqa: C901
             else:
                 attn.decode_gqa_ext(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
                                     x.scale, window=x.window, sink_tokens=cfg.sink,
-                                    ring_blocks=cfg.ring, out=outs[i % reps])
+                                    ring_blocks=cfg.ring, out=outs[i % reps],
+                                    global_pos=x.global_pos)
 
     for i in range(max(args.warmup, 3)):
         step(i)
@@ -513,7 +553,7 @@ def e2e_native(attn, cfg, x, is_mla, K, world, dev):
             else:
                 attn.kv_append_ext(d_k, d_v, x.k_cache, x.v_cache, pos, x.block_table, **vis)
                 attn.decode_gqa_ext(d_q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                                    x.scale, out=d_out, **vis)
+                                    x.scale, out=d_out, global_pos=x.global_pos, **vis)
         h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(3):
@@ -551,7 +591,7 @@ def _oracle_problem(cfg, is_mla, seqs, seed):
     sub = W.GQAConfig(cfg.name, B=seqs, H_q=cfg.H_q, H_kv=cfg.H_kv, d=cfg.d,
                       seq_lens=lens, T=cfg.T, dtype=cfg.dtype, window=cfg.window,
                       sink=cfg.sink, ring=cfg.ring, kv_fp8=cfg.kv_fp8,
-                      contiguous=cfg.contiguous, seed=seed)
+                      contiguous=cfg.contiguous, seed=seed, n_global=cfg.n_global)
     return W.make_gqa_inputs(sub)
 
 
@@ -565,7 +605,8 @@ def _oracle_call(orc, x, is_mla):
         return orc.decode_gqa_vis(x.q.double().numpy(), k, v, x.seq_lens, x.block_table,
                                   x.scale, window=x.window, sink=x.cfg.sink, ring=x.cfg.ring)
     return orc.decode_gqa_vis(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                              x.scale, window=x.window, sink=x.cfg.sink, ring=x.cfg.ring)
+                              x.scale, window=x.window, sink=x.cfg.sink, ring=x.cfg.ring,
+                              global_pos=x.global_pos)
 
 
 def _pick_sample(cfg, is_mla, orc, target_s):

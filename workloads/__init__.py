@@ -42,6 +42,7 @@ class GQAConfig:
     contiguous: bool = False               # identity block table
     seed: int = SEED_BASE
     ragged: Optional[tuple] = None         # (lo, hi) inclusive range of T_b
+    n_global: int = 0                      # explicit global positions per sequence (global_rows)
 
     @property
     def scale(self) -> float:
@@ -103,11 +104,26 @@ RAGGED_WINDOW_SINK = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_g64", B=
 RAGGED_WINDOW_RING = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_g64_ring65", B=8,
                                H_q=24, H_kv=4, d=256, ragged=(1024, 131072), window=4096,
                                sink=64, ring=65, seed=SEED_BASE + 3)
+RAGGED_WINDOW_GLOBAL = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_G16", B=8, H_q=24,
+                                 H_kv=4, d=256, ragged=(1024, 131072), window=4096,
+                                 n_global=16, seed=SEED_BASE + 3)
 MLA_DSV2 = MLAConfig("mla_absorbed_bf16_B32_H128_dc512_dr64_T8192", B=32)
 
 WORKLOADS = {c.name: c for c in [TINY, LLAMA3_8B, *SWEEP, RAGGED_FULL,
                                  RAGGED_WINDOW, RAGGED_WINDOW_SINK, RAGGED_WINDOW_RING,
-                                 LLAMA3_8B_FP8, MLA_DSV2]}
+                                 RAGGED_WINDOW_GLOBAL, LLAMA3_8B_FP8, MLA_DSV2]}
+
+
+def global_rows(seq_lens, n: int) -> torch.Tensor:
+    """[B][n] int32 global positions: per sequence of T tokens the first 4
+    positions and n - 4 positions spread evenly over [0, T) (a prompt's
+    leading tokens and periodic summary tokens), ascending, -1 padded."""
+    rows = []
+    for T in seq_lens:
+        pos = set(range(min(4, T))) | {T * k // (n - 3) for k in range(1, n - 3)}
+        pos = sorted(p for p in pos if 0 <= p < T)[:n]
+        rows.append(pos + [-1] * (n - len(pos)))
+    return torch.tensor(rows, dtype=torch.int32)
 
 
 def _generator(seed: int, device) -> torch.Generator:
@@ -178,6 +194,7 @@ class GQAInputs:
     seq_list: List[int] = field(default_factory=list)
     k_scale: Optional[torch.Tensor] = None   # fp8 cache: [num_blocks][H_kv][64] row scales
     v_scale: Optional[torch.Tensor] = None
+    global_pos: Optional[torch.Tensor] = None   # [B][n_global] int32 (cfg.n_global > 0)
 
     def to(self, device):
         mv = (lambda t: None if t is None else t.to(device))
@@ -185,7 +202,7 @@ class GQAInputs:
                          self.v_cache.to(device), self.seq_lens.to(device),
                          self.block_table.to(device), self.num_blocks,
                          self.window, self.scale, list(self.seq_list),
-                         mv(self.k_scale), mv(self.v_scale))
+                         mv(self.k_scale), mv(self.v_scale), mv(self.global_pos))
 
 
 def make_gqa_inputs(cfg: GQAConfig, device="cpu", seed: Optional[int] = None,
@@ -219,7 +236,8 @@ def make_gqa_inputs(cfg: GQAConfig, device="cpu", seed: Optional[int] = None,
                          scales[0], scales[1])
     k = randn((nblk, cfg.H_kv, BLOCK_SIZE, cfg.d), g, cfg.dtype)
     v = randn((nblk, cfg.H_kv, BLOCK_SIZE, cfg.d), g, cfg.dtype)
-    return GQAInputs(cfg, q, k, v, sl, table, nblk, win, cfg.scale, seq)
+    gp = global_rows(seq, cfg.n_global).to(g.device) if cfg.n_global > 0 else None
+    return GQAInputs(cfg, q, k, v, sl, table, nblk, win, cfg.scale, seq, global_pos=gp)
 
 
 @dataclass
