@@ -3,11 +3,20 @@
 One step = one decode-attention call of the whole hot path (split planning,
 paged block gather, K/V tile streaming, scores, online softmax, P V, split
 partials, log-sum-exp combine) over one batch of synthetic inputs resident in
-HBM.  Default workload: Llama-3-8B-shaped GQA (B=16, H_q=32, H_kv=8, d=128,
-T=4096, bf16, 64-token blocks, random-permutation block table).
+HBM.  Default (headline) workload: the largest single-GPU shape of the
+head-sharing sweep, MHA with B=32, H_q=H_kv=32, d=128, T=32768, bf16, 64-token
+blocks, random-permutation block table (a 16 GiB cache, far larger than L2).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--impl native|reference]
+                  [--impl native|reference] [--no-per-config]
+
+Timing: W warm-up steps, then blocks of exactly K steps, each bracketed by a
+barrier and a device synchronisation and timed with CUDA events on the
+launching stream; blocks repeat until about --min-seconds of timed work has
+run (so the clock sampler sees the region) and the median block is reported.
+The line also carries `per_config`: every other workload of the benchmark
+plan timed the same way (kernel and step time, algorithmic bytes, fraction of
+the measured HBM peak).
 
 N > 1 runs under torch.distributed.run, one rank per GPU, each rank with its
 own batch (weak scaling; ranks share nothing on the data path -- the only
@@ -67,16 +76,24 @@ WORKLOAD_ALIASES = {
 }
 
 
+HEADLINE = W.sweep_config(32, 32).name
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="llama3_8b",
-                    help="llama3_8b | tiny | ragged_full | ragged_window | "
-                         "ragged_window_sink | ragged_window_ring | ragged_window_global | mla "
-                         "| a sweep name such as sweep_bf16_B8_Hq32_Hkv8_d128_T32768")
+    ap.add_argument("--workload", default=HEADLINE,
+                    help="headline (default: the largest sweep shape) | llama3_8b | tiny | "
+                         "ragged_full | ragged_window | ragged_window_sink | ragged_window_ring "
+                         "| ragged_window_global | llama3_8b_fp8 | mla | a sweep name such as "
+                         "sweep_bf16_B8_Hq32_Hkv8_d128_T32768")
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="repeat K-step blocks until this much timed work has run")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true",
                     help="skip the oracle CPU baseline (profiling runs)")
@@ -86,6 +103,8 @@ def parse():
 
 
 def workload(name):
+    if name == "headline":
+        name = HEADLINE
     return W.WORKLOADS[WORKLOAD_ALIASES.get(name, name)]
 
 
@@ -108,32 +127,36 @@ def kernel_hash(kind):
 
 def traffic_for(kernel, wl_name):
     """dram bytes per launch of `kernel` on `wl_name` from the committed ncu
-    summary, if the kernel's sources are unchanged since it was taken; else
+    capture, if the kernel's sources are unchanged since it was taken; else
     None."""
     return traffic_entry(kernel, wl_name)[0]
 
 
 def traffic_entry(kernel, wl_name):
-    """(dram bytes per launch or None, note): the note says why the figure is
-    missing (no capture of this kernel on this workload, or a capture of
-    different kernel sources)."""
+    """(dram bytes per launch or None, note).  A capture taken on a smaller
+    case of the same shape is scaled to a full launch by the units processed
+    (its entry records the factor).  The note says why the figure is missing:
+    no capture of this kernel on this workload, or a capture of other
+    sources of the kernel."""
     if not os.path.exists(TRAFFIC_FILE):
-        return None, "no ncu capture committed"
+        return None, f"no ncu capture of {kernel}"
     with open(TRAFFIC_FILE) as f:
         j = json.load(f)
     e = j.get(wl_name)
     if not e or e.get("kernel") != kernel:
-        return None, "no ncu capture of this kernel on this workload"
+        return None, f"no ncu capture of {kernel} on this workload"
     if e.get("kernel_hash") != kernel_hash(kernel):
-        return None, ("the committed capture (%s, %.1f MB per launch) was taken on other "
-                      "sources of this kernel" % (e.get("summary"),
-                                                  e.get("dram_bytes_per_launch", 0) / 1e6))
+        return None, (f"the ncu capture of {kernel} on this workload "
+                      f"({e.get('dram_bytes_per_launch', 0) / 1e6:.1f} MB per launch) was "
+                      "taken on other sources of the kernel")
     return e.get("dram_bytes_per_launch"), None
 
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock and throttle-reason samples every 50 ms; the summary
+    keeps the samples taken inside the marked timed windows."""
+    QUERY = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -141,6 +164,7 @@ class ClockSampler:
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.windows = []
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -149,15 +173,20 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         time.sleep(0.3)
         return self
 
+    def mark(self, t0, t1):
+        """Record a timed window (host wall-clock seconds)."""
+        self.windows.append((t0, t1))
+
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -167,6 +196,7 @@ class ClockSampler:
         return False
 
     def summary(self):
+        import datetime
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         rows = []
@@ -176,22 +206,28 @@ class ClockSampler:
                 if len(parts) < 9:
                     continue
                 try:
-                    rows.append((float(parts[1]), float(parts[2]), parts))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts))
                 except ValueError:
                     continue
         os.unlink(self.path)
-        if not rows:
+        inside = [r for r in rows if any(t0 <= r[0] <= t1 for t0, t1 in self.windows)]
+        use = inside or rows
+        if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
         reasons = set()
-        for _, _, parts in rows:
+        for *_, parts in use:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(r[0] for r in rows),
-                "sm_max_mhz": max(r[1] for r in rows),
-                "samples": len(rows), "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in use),
+                "power_w_max": max((float(r[3][3]) for r in use
+                                    if r[3][3].replace(".", "", 1).isdigit()), default=None),
+                "samples": len(use), "samples_in_timed_region": len(inside),
+                "reasons": sorted(reasons)}
 
 
 # ------------------------------------------------------------ distributed
@@ -340,143 +376,244 @@ def mla_flops(inp):
 
 
 # ------------------------------------------------------------ native arm
-def run_native(args, rank, world, local):  # noqa: C901
-    import decode_attention_kv_paged_b200 as attn
-    attn.load()
-    cfg = workload(args.workload)
-    is_mla = isinstance(cfg, W.MLAConfig)
-    dev = torch.device("cuda", local)
-    seed = rank_seed(cfg.seed, rank)
-    if is_mla:
-        base = W.make_mla_inputs(cfg, device=dev, seed=seed)
-        kv_bytes, alg_bytes = algorithmic_bytes_mla(base)
-        cache_bytes = base.latent_cache.numel() * 2
-    else:
-        base = W.make_gqa_inputs(cfg, device=dev, seed=seed)
-        kv_bytes, alg_bytes = algorithmic_bytes_gqa(base)
-        cache_bytes = (base.k_cache.numel() + base.v_cache.numel()) * \
-            base.k_cache.element_size()
-    # Rotate among enough cache replicas that consecutive steps never find
-    # the previous step's cache in the 126 MB L2.
-    reps = max(2, math.ceil(3 * L2_BYTES / max(cache_bytes, 1)))
-    reps = min(reps, 64)
-    inputs = [base]
-    for r in range(1, reps):
-        if is_mla:
-            inputs.append(W.make_mla_inputs(cfg, device=dev, seed=seed + r))
-        else:
-            inputs.append(W.make_gqa_inputs(cfg, device=dev, seed=seed + r))
-    outs = [torch.empty_like(i.q_lat if is_mla else i.q) for i in inputs]
+def kernel_name(attn, cfg):
+    """The main kernel a decode call of this workload launches."""
+    if isinstance(cfg, W.MLAConfig):
+        return "mla_decode_kernel"
+    if cfg.kv_fp8:
+        return "gqa_split_kernel"
+    _, _, path = attn.gqa_config(cfg.B, cfg.H_q, cfg.H_kv, cfg.d, cfg.dtype)
+    return {0: "gqa_split_kernel", 1: "gqa_tc128_kernel", 2: "gqa_tc_kernel"}[path]
 
-    def step(i):
-        x = inputs[i % reps]
-        if is_mla:
-            attn.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
-                            x.block_table, x.scale, out=outs[i % reps])
-        else:
-            if cfg.kv_fp8:
-                attn.decode_gqa_fp8(x.q, x.k_cache, x.v_cache, x.k_scale, x.v_scale,
-                                    x.seq_lens, x.block_table, x.scale, window=x.window,
-                                    sink_tokens=cfg.sink, ring_blocks=cfg.ring,
-                                    out=outs[i % reps])
-            else:
-                attn.decode_gqa_ext(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table,
-                                    x.scale, window=x.window, sink_tokens=cfg.sink,
-                                    ring_blocks=cfg.ring, out=outs[i % reps],
-                                    global_pos=x.global_pos)
 
-    for i in range(max(args.warmup, 3)):
+def launches_per_step(kernel):
+    """Library kernels one decode call launches: the CUDA-core split kernel
+    combines its own splits; the tensor-core and MLA paths add a combine."""
+    return 1 if kernel == "gqa_split_kernel" else 2
+
+
+class Problem:
+    """Device-resident inputs of one workload and the decode call over them.
+    Caches smaller than 8x the L2 are replicated and rotated so consecutive
+    steps never find the previous step's cache in L2."""
+
+    def __init__(self, attn, cfg, dev, seed):
+        self.attn, self.cfg = attn, cfg
+        self.is_mla = isinstance(cfg, W.MLAConfig)
+        make = W.make_mla_inputs if self.is_mla else W.make_gqa_inputs
+        base = make(cfg, device=dev, seed=seed)
+        if self.is_mla:
+            self.kv_bytes, self.alg_bytes = algorithmic_bytes_mla(base)
+            cache = base.latent_cache.numel() * 2
+        else:
+            self.kv_bytes, self.alg_bytes = algorithmic_bytes_gqa(base)
+            cache = 2 * base.k_cache.numel() * base.k_cache.element_size()
+            if base.k_scale is not None:
+                cache += 2 * base.k_scale.numel() * 4
+        self.reps = 1 if cache >= 8 * L2_BYTES else min(64, max(2, math.ceil(3 * L2_BYTES / cache)))
+        self.cache_bytes = cache
+        self.inputs = [base] + [make(cfg, device=dev, seed=seed + r) for r in range(1, self.reps)]
+        self.outs = [torch.empty_like(i.q_lat if self.is_mla else i.q) for i in self.inputs]
+        self.base = base
+        if self.reps * cache > 2 * L2_BYTES:
+            self.l2 = (f"inputs larger than L2: {self.reps} cache replica(s) of "
+                       f"{cache / 2**20:.0f} MiB, rotated")
+        else:
+            self.l2 = (f"L2-resident: {self.reps} replicas of {cache / 2**10:.0f} KiB "
+                       "(launch-bound case)")
+
+    def step(self, i):
+        attn, cfg = self.attn, self.cfg
+        x, out = self.inputs[i % self.reps], self.outs[i % self.reps]
+        if self.is_mla:
+            attn.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens, x.block_table,
+                            x.scale, out=out)
+        elif cfg.kv_fp8:
+            attn.decode_gqa_fp8(x.q, x.k_cache, x.v_cache, x.k_scale, x.v_scale, x.seq_lens,
+                                x.block_table, x.scale, window=x.window, sink_tokens=cfg.sink,
+                                ring_blocks=cfg.ring, out=out)
+        else:
+            attn.decode_gqa_ext(x.q, x.k_cache, x.v_cache, x.seq_lens, x.block_table, x.scale,
+                                window=x.window, sink_tokens=cfg.sink, ring_blocks=cfg.ring,
+                                out=out, global_pos=x.global_pos)
+
+
+def time_blocks(attn, step, K, warmup, min_s, world, clk=None, max_blocks=200):
+    """W warm-up steps, then blocks of exactly K steps, each between a barrier
+    and a device synchronisation, timed with CUDA events on the launching
+    stream; the library records events around its main kernel.  Blocks repeat
+    until min_s seconds of (slowest-rank) timed work.  Every rank takes the
+    same number of blocks (the stop test uses the max over ranks)."""
+    for i in range(max(warmup, 3)):
         step(i)
     torch.cuda.synchronize()
     if attn.last_error() != attn.OK:
         raise SystemExit("device error during warm-up")
-
-    K = args.steps
-    prof = attn.ProfileEvents(K)
+    n = max(warmup, 3)
+    block_ms, kern_ms = [], []
+    total = 0.0
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    while True:
+        prof = attn.ProfileEvents(K)
         barrier(world)
         torch.cuda.synchronize()
+        t0 = time.time()
         with prof:
             ev0.record()
             for i in range(K):
-                step(i)
+                step(n + i)
             ev1.record()
         torch.cuda.synchronize()
         barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    kern_ms = prof.times_ms(K)
+        t1 = time.time()
+        if clk is not None:
+            clk.mark(t0, t1)
+        ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+        block_ms.append(ms)
+        kern_ms.extend(prof.times_ms(K))
+        n += K
+        total += ms / 1e3
+        if total >= min_s or len(block_ms) >= max_blocks:
+            break
     if attn.last_error() != attn.OK:
         raise SystemExit("device error during the timed region")
-    ms_max = max_over_ranks(ms, world)
-    kern_avg = max_over_ranks(sum(kern_ms) / K, world)
+    return {"block_ms": block_ms,
+            "ms_per_step": statistics.median(block_ms) / K,
+            "kernel_ms_avg": max_over_ranks(sum(kern_ms) / len(kern_ms), world),
+            "kernel_ms_median": max_over_ranks(statistics.median(kern_ms), world)}
 
-    B = cfg.B
-    value = whole_job_tokens_per_s(world, B, K, ms_max)
-    kv_gbs = world * kv_bytes * K / (ms_max / 1e3) / 1e9
-    pk, pk_kind = peaks()
-    wl_name = cfg.name
-    if is_mla:
-        kernel = "mla_decode_kernel"
-    else:
-        _, _, path = attn.gqa_config(cfg.B, cfg.H_q, cfg.H_kv, cfg.d, cfg.dtype)
-        kernel = {0: "gqa_split_kernel", 1: "gqa_tc128_kernel", 2: "gqa_tc_kernel"}[path]
-    if is_mla:
-        flops = mla_flops(base)
-        t_hbm = alg_bytes / (pk["hbm_gbs"] * 1e9)
+
+def roofline_entry(prob, kernel, kern_ms, pk):
+    """Fraction of the binding roofline of the dominant kernel: HBM bytes for
+    the GQA family; for MLA the tighter of HBM bytes and tensor-core FLOPs."""
+    cfg = prob.cfg
+    t = kern_ms / 1e3
+    roof = None
+    if prob.is_mla:
+        flops = mla_flops(prob.base)
+        t_hbm = prob.alg_bytes / (pk["hbm_gbs"] * 1e9)
         t_tc = flops / (pk.get("bf16_tflops", 1590.0) * 1e12)
         if t_tc > t_hbm:
-            achieved = flops / (kern_avg / 1e3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved,
+            roof = {"bound": "tensor", "achieved": flops / t / 1e12,
                     "peak": pk.get("bf16_tflops"), "unit": "TFLOP/s"}
-        else:
-            achieved = alg_bytes / (kern_avg / 1e3) / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                    "unit": "GB/s"}
-    else:
-        achieved = alg_bytes / (kern_avg / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+    if roof is None:
+        roof = {"bound": "hbm", "achieved": prob.alg_bytes / t / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["peak_source"] = pk_kind
     roof["kernel"] = kernel
-    roof["kernel_ms_avg"] = kern_avg
-    roof["algorithmic_bytes_per_launch"] = alg_bytes
-    roof["traffic"], note = traffic_entry(kernel, wl_name)
+    roof["kernel_ms_avg"] = kern_ms
+    roof["algorithmic_bytes_per_launch"] = prob.alg_bytes
+    roof["traffic"], note = traffic_entry(kernel, cfg.name)
     if note:
         roof["traffic_note"] = note
+    if prob.is_mla:
+        roof["flops_per_launch"] = mla_flops(prob.base)
+        roof["tensor_frac"] = (mla_flops(prob.base) / t / 1e12) / pk.get("bf16_tflops", 1590.0)
+        roof["hbm_frac"] = (prob.alg_bytes / t / 1e9) / pk["hbm_gbs"]
+    return roof
 
+
+def config_entry(attn, cfg, dev, seed, K, warmup, min_s, pk, clk=None):
+    """Time one workload (one rank) and describe it for `per_config`."""
+    prob = Problem(attn, cfg, dev, seed)
+    r = time_blocks(attn, prob.step, K, warmup, min_s, 1, clk=clk, max_blocks=50)
+    kernel = kernel_name(attn, cfg)
+    roof = roofline_entry(prob, kernel, r["kernel_ms_avg"], pk)
+    e = {"workload": cfg.name, "kernel": kernel,
+         "kernel_us": r["kernel_ms_avg"] * 1e3, "step_us": r["ms_per_step"] * 1e3,
+         "algorithmic_bytes": prob.alg_bytes, "kv_bytes": prob.kv_bytes,
+         "tokens_per_s": cfg.B / (r["ms_per_step"] / 1e3),
+         "kernel_gbs": prob.alg_bytes / (r["kernel_ms_avg"] / 1e3) / 1e9,
+         "frac_of_measured_hbm": prob.alg_bytes / (r["kernel_ms_avg"] / 1e3) / 1e9
+         / pk["hbm_gbs"],
+         "frac_of_8tbs_spec": prob.alg_bytes / (r["kernel_ms_avg"] / 1e3) / 1e9 / 8000.0,
+         "bound": roof["bound"], "frac": roof["frac"], "traffic": roof["traffic"],
+         "steps_timed": K * len(r["block_ms"]), "l2": prob.l2}
+    if "traffic_note" in roof:
+        e["traffic_note"] = roof["traffic_note"]
+    if prob.is_mla:
+        e["tensor_frac"] = roof["tensor_frac"]
+        e["flops"] = roof["flops_per_launch"]
+        e["mla_absorb"] = mla_absorb_timing(attn, cfg, dev, seed)
+    else:
+        e["tile_overread_bytes"] = tile_bytes_gqa(prob.base) - prob.kv_bytes
+    del prob
+    torch.cuda.empty_cache()
+    return e
+
+
+# Every workload of the benchmark plan, by what it is (the headline excluded
+# at run time): the tiny fp32 case, the Llama-3-8B shape, the nine points of
+# the head-sharing sweep, the ragged 24/4/256 shape full and with w=4096, the
+# DeepSeek-V2 MLA shape; then the window/global/ring and fp8-cache variants.
+PER_CONFIG = [W.TINY, W.LLAMA3_8B, *W.SWEEP, W.RAGGED_FULL, W.RAGGED_WINDOW, W.MLA_DSV2,
+              W.LLAMA3_8B_FP8, W.RAGGED_WINDOW_SINK, W.RAGGED_WINDOW_RING,
+              W.RAGGED_WINDOW_GLOBAL]
+
+
+def run_native(args, rank, world, local):
+    import decode_attention_kv_paged_b200 as attn
+    attn.load()
+    cfg = workload(args.workload)
+    dev = torch.device("cuda", local)
+    pk, pk_kind = peaks()
+    K = args.steps
+    prob = Problem(attn, cfg, dev, rank_seed(cfg.seed, rank))
+    with ClockSampler(local) as clk:
+        r = time_blocks(attn, prob.step, K, args.warmup, args.min_seconds, world, clk=clk)
+    kernel = kernel_name(attn, cfg)
+    roof = roofline_entry(prob, kernel, r["kernel_ms_avg"], pk)
+    roof["peak_source"] = pk_kind
+    ms = r["ms_per_step"]
+    B = cfg.B
+    kv_gbs = world * prob.kv_bytes / (ms / 1e3) / 1e9
     line = {
         "metric": "decode tokens/s and KV-cache read GB/s (% of B200 HBM peak), 1 GPU",
-        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": max(args.warmup, 3), "ms_per_step": ms_max / K,
+        "value": whole_job_tokens_per_s(world, B, 1, ms), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": ("fp8e4m3 cache, bf16 q/out, f32 accumulate" if getattr(cfg, "kv_fp8", False)
                   else "bf16" if cfg.dtype == torch.bfloat16 else "f32"),
         "data": "synthetic (seeded N(0,1) q/K/V, random-permutation block table)",
-        "config": {"workload": wl_name, "global_batch": B * world,
-                   "seq_len": getattr(cfg, "T", None) or max(base.seq_list),
+        "config": {"workload": cfg.name, "global_batch": B * world,
+                   "seq_len": getattr(cfg, "T", None) or max(prob.base.seq_list),
                    "parallelism": f"dp{world} (independent batches, no collective)",
-                   "l2": f"inputs larger than L2, rotated among {reps} cache "
-                         f"replicas ({cache_bytes / 2**20:.0f} MiB each)"},
+                   "l2": prob.l2},
+        "timing": {"blocks": len(r["block_ms"]), "steps_per_block": K,
+                   "ms_per_step_median_block": ms,
+                   "ms_per_step_min_block": min(r["block_ms"]) / K,
+                   "ms_per_step_max_block": max(r["block_ms"]) / K,
+                   "kernel_ms_median": r["kernel_ms_median"]},
         "kv_gbs": kv_gbs,
         "kv_frac_of_peak": kv_gbs / world / pk["hbm_gbs"],
         "kv_frac_of_8tbs_spec": kv_gbs / world / 8000.0,
         "roofline": roof,
-        # main kernel per step, plus the combine kernel on the tensor-core
-        # paths (the CUDA-core GQA kernel combines its splits itself)
-        "gpu_launches": (1 if kernel == "gqa_split_kernel" else 2) * K,
+        "gpu_launches": launches_per_step(kernel) * K * len(r["block_ms"]),
+        "gpu_launches_per_step": launches_per_step(kernel),
         "clocks": clk.summary(),
     }
-    if not is_mla:
-        line["tile_overread_bytes_per_step"] = tile_bytes_gqa(base) - kv_bytes
-    if is_mla:
-        line["mla_absorb"] = mla_absorb_timing(attn, cfg, dev, rank_seed(cfg.seed, rank))
+    if not prob.is_mla:
+        line["tile_overread_bytes_per_step"] = tile_bytes_gqa(prob.base) - prob.kv_bytes
+    e2e_input = prob.inputs[0]
+    del prob
     if not args.no_e2e:
-        line["e2e"] = e2e_native(attn, cfg, inputs[0], is_mla, K, world, dev)
+        line["e2e"] = e2e_native(attn, cfg, e2e_input, isinstance(cfg, W.MLAConfig), K, world,
+                                 dev)
+    del e2e_input
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_per_config:
+        entries = []
+        with ClockSampler(local) as pclk:
+            for c in PER_CONFIG:
+                if c.name == cfg.name:
+                    continue
+                entries.append(config_entry(attn, c, dev, c.seed, K, args.warmup, 0.05, pk,
+                                            clk=pclk))
+        line["per_config"] = {"peak_gbs": pk["hbm_gbs"], "peak_source": pk_kind,
+                              "clocks": pclk.summary(), "entries": entries}
     if rank == 0 and world == 1 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline(cfg, is_mla, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(cfg, isinstance(cfg, W.MLAConfig), args.cpu_seconds)
     return line
 
 
@@ -559,6 +696,19 @@ def e2e_native(attn, cfg, x, is_mla, K, world, dev):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    # Host round trip per step: the host has each step's output in hand
+    # before it issues the next step's copies (a decode loop's latency).
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        step()
+        stream.synchronize()
+    t1 = time.perf_counter()
+    barrier(world)
+    ms = max_over_ranks((t1 - t0) * 1e3, world)
+    # The same steps issued back to back without a host wait in between.
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -569,12 +719,16 @@ def e2e_native(attn, cfg, x, is_mla, K, world, dev):
     e1.record()
     torch.cuda.synchronize()
     barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_pipe = max_over_ranks(e0.elapsed_time(e1), world)
     return {"value": world * B * K / (ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms / K,
-            "note": "cache stays resident (L2 not rotated); step = H2D of the new "
-                    "token's inputs + kv_append + decode + D2H of the output"}
+            "pipelined_tokens_per_s": world * B * K / (ms_pipe / 1e3),
+            "pipelined_ms_per_step": ms_pipe / K,
+            "note": "step = H2D of the new token's q/K/V from pinned host memory + kv_append "
+                    "+ decode + D2H of the output, and the host waits for the output before "
+                    "the next step (wall clock, max over ranks); pipelined_* issue the same "
+                    "steps without the host wait (CUDA events)"}
 
 
 # ------------------------------------------------------------- oracle arm

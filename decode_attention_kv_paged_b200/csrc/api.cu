@@ -5,11 +5,11 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
-#include <vector>
 
 #include "attn_decode.h"
 #include "gqa_launch.cuh"
 #include "gqa_tc.cuh"
+#include "host_state.cuh"
 #include "kv_append.cuh"
 #include "mla_launch.cuh"
 
@@ -27,8 +27,10 @@ struct DeviceState {
     size_t cnt_elems = 0;
 };
 
+// One record per device ordinal; a pointer to a record stays valid for the
+// life of the process.
 static std::mutex g_mu;
-static std::vector<DeviceState> g_dev;
+static DeviceState g_dev[kMaxDevices];
 static thread_local int tl_num_ctas = 0;
 static thread_local int tl_gqa_path = -1;
 static std::atomic<int> g_force_timeout{0};
@@ -41,10 +43,9 @@ static int cuda_status(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN
 
 // Per-device state of the current device (created on first use).
 static int device_state(DeviceState **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int dev = current_device();
+    if (dev < 0) return ATTN_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
     DeviceState &st = g_dev[dev];
     if (!st.ready) {
         if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) !=

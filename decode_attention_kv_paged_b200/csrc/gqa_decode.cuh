@@ -716,12 +716,15 @@ gqa_split_kernel(const GqaParams p) {
     PlanScratch *plan_sh = reinterpret_cast<PlanScratch *>(never_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(plan_sh + 1);
     volatile int *last_flag = abort_flag + 1;
+    volatile int *epi_vote = last_flag + 1;             // [2][4]: epilogue warps' wait outcomes
     // Per stage: global positions among the staged block's keys below the
     // window (bit t: key 64 * block + t), written by the producer before it
     // arms the stage, read by the compute warps after they wait on it.
     unsigned long long *s_gmask = reinterpret_cast<unsigned long long *>(misc + 768);
-    static_assert((2 * S + 7) * 8 + sizeof(PlanScratch) + 8 <= 768 && 768 + 8 * S <= C::kMiscBytes,
+    static_assert((2 * S + 7) * 8 + sizeof(PlanScratch) + 8 + 32 <= 768 &&
+                      768 + 8 * S <= C::kMiscBytes,
                   "misc shared-memory layout");
+    static_assert(C::kEpiThreads % 32 == 0 && C::kEpiThreads / 32 <= 4, "epilogue vote slots");
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -804,9 +807,21 @@ gqa_split_kernel(const GqaParams p) {
                         pre = true;
                     }
                 };
-                if (!mbar_wait_watch(epi_full, (uint32_t)(es & 1), p.timeout_ns, p.err,
-                                     abort_flag, idle))
-                    break;
+                const bool got = mbar_wait_watch(epi_full, (uint32_t)(es & 1), p.timeout_ns,
+                                                 p.err, abort_flag, idle);
+                // The epilogue warps leave that wait separately: a stash that
+                // completes just as an abort is raised can end one warp's
+                // wait with the phase and another's with the abort.  Every
+                // warp reaches this barrier either way (each wait is bounded)
+                // and all go on only if all saw the stash, so no warp is ever
+                // left waiting at a barrier of the epilogue below.
+                volatile int *vote = epi_vote + 4 * (es & 1);
+                if (lane == 0) vote[et >> 5] = got ? 1 : 0;
+                named_barrier(1, C::kEpiThreads);
+                bool all_got = true;
+#pragma unroll
+                for (int w = 0; w < C::kEpiThreads / 32; ++w) all_got = all_got && vote[w];
+                if (!all_got) break;
                 const int head0 = (ew.unit / p.n_hc) * p.group + (ew.unit % p.n_hc) * HC;
                 T *out_u = static_cast<T *>(p.out) + ((size_t)ew.b * p.H_q + head0) * D;
                 segment_epilogue<D, HC, T, C::kNW, C::kEpiThreads, C::kPreMax>(

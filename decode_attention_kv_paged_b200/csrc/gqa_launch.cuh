@@ -4,6 +4,7 @@
 #pragma once
 
 #include "gqa_decode.cuh"
+#include "host_state.cuh"
 
 namespace attn {
 
@@ -23,23 +24,22 @@ int gqa_smem_bytes() { return GqaCfg<D, HC, T, TK>::kSmemBytes; }
 template <int D, int HC, typename T, typename TK = T, bool G = false>
 cudaError_t launch_gqa_impl(const GqaLaunch &L) {
     using C = GqaCfg<D, HC, T, TK>;
-    static bool configured = false;   // per-process; attribute is per function
-    cudaError_t e;
-    if (!configured) {
+    // The attribute is set on the function for the current device only.
+    static PerDeviceFlag configured;
+    cudaError_t e = configure_once_per_device(configured, [] {
         // The warpgroups' setmaxnreg shares must fit in the registers the
         // kernel is launched with, or the increase would never be granted.
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T, TK, G>);
-        if (e != cudaSuccess) return e;
+        cudaError_t r = cudaFuncGetAttributes(&fa, gqa_split_kernel<D, HC, T, TK, G>);
+        if (r != cudaSuccess) return r;
         if (fa.numRegs * C::kThreads <
             4 * 32 * C::kProducerRegs + C::kNW * 32 * C::kConsumerRegs)
             return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(gqa_split_kernel<D, HC, T, TK, G>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+        return cudaFuncSetAttribute(gqa_split_kernel<D, HC, T, TK, G>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
     // The split partials are combined inside the kernel (by the last split
     // of each unit), so this is the call's only launch.

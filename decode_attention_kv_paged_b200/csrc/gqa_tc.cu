@@ -37,6 +37,7 @@
 #include "gqa_decode.cuh"
 #include "gqa_tc.cuh"
 #include "tc_common.cuh"
+#include "host_state.cuh"
 
 namespace attn {
 
@@ -541,12 +542,13 @@ namespace {
 template <int D, int TPC, bool G>
 cudaError_t launch_tc_g(const GqaLaunch &L, int HC) {
     using C = TcCfg<D>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_tc_kernel<D, TPC, G>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    static PerDeviceFlag configured;   // the attribute is per function and device
+    {
+        const cudaError_t e = configure_once_per_device(configured, [] {
+            return cudaFuncSetAttribute(gqa_tc_kernel<D, TPC, G>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        });
         if (e != cudaSuccess) return e;
-        configured = true;
     }
     const GqaParams &kp = L.kp;
     CUtensorMap tq, tk, tv;

@@ -31,6 +31,7 @@
 #include "gqa_decode.cuh"
 #include "gqa_tc.cuh"
 #include "tc_common.cuh"
+#include "host_state.cuh"
 
 namespace attn {
 
@@ -476,12 +477,13 @@ namespace {
 template <int D, int HCP, bool G>
 cudaError_t launch_tc128_g(const GqaLaunch &L, int HC) {
     using C = T2Cfg<D>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_tc128_kernel<D, HCP, G>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    static PerDeviceFlag configured;   // the attribute is per function and device
+    {
+        const cudaError_t e = configure_once_per_device(configured, [] {
+            return cudaFuncSetAttribute(gqa_tc128_kernel<D, HCP, G>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        });
         if (e != cudaSuccess) return e;
-        configured = true;
     }
     const GqaParams &kp = L.kp;
     CUtensorMap tk, tv;

@@ -47,6 +47,7 @@
 #include "gqa_decode.cuh"
 #include "mla_launch.cuh"
 #include "tc_common.cuh"
+#include "host_state.cuh"
 
 namespace attn {
 
@@ -631,13 +632,12 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     if (H != kMlaH) return ATTN_ERR_UNSUPPORTED;
     if ((long long)num_blocks * 64 > (1ll << 31) - 64 || (long long)B * kMlaH > (1ll << 31))
         return ATTN_ERR_ARG;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kMlaSmem) != cudaSuccess)
-            return ATTN_ERR_CUDA;
-        configured = true;
-    }
+    static PerDeviceFlag configured;   // the attribute is per function and device
+    if (configure_once_per_device(configured, [] {
+            return cudaFuncSetAttribute(mla_decode_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
+        }) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     int clusters = forced_ctas > 0 ? forced_ctas : max_resident_clusters(num_sms);
     if (clusters <= 0) return ATTN_ERR_CUDA;
     const long long slots = (long long)B + clusters;

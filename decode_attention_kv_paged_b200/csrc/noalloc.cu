@@ -14,10 +14,10 @@
 // address is looked up once per device (cudaGetSymbolAddress, with that
 // device current) by the first call made on the device.
 #include <mutex>
-#include <vector>
 
 #include "attn_decode.h"
 #include "gqa_launch.cuh"
+#include "host_state.cuh"
 
 namespace attn {
 
@@ -36,16 +36,17 @@ struct NoAllocDevice {
     int num_sms = 0;
 };
 
+// One record per device ordinal (fixed array: a pointer to a record stays
+// valid while other threads set up other devices).
 std::mutex g_noalloc_mu;
-std::vector<NoAllocDevice> g_noalloc_dev;
+NoAllocDevice g_noalloc_dev[kMaxDevices];
 
 // First call on a device: resolve the scratch array's device address (the
 // name is only a host-side stand-in) and the SM count.  No allocation.
 int noalloc_setup(NoAllocDevice **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int dev = current_device();
+    if (dev < 0) return ATTN_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if ((int)g_noalloc_dev.size() <= dev) g_noalloc_dev.resize(dev + 1);
     NoAllocDevice &d = g_noalloc_dev[dev];
     if (!d.ready) {
         void *ptr = nullptr, *cptr = nullptr;
