@@ -60,7 +60,7 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
     if (force or not os.path.exists(LIB) or
             os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs)):
         tmp = LIB + ".tmp%d" % os.getpid()
-        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lcublas"]
+        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

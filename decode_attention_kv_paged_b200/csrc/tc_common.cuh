@@ -27,6 +27,12 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
                  : "memory");
 }
 
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+    uint64_t policy;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
+    return policy;
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t policy;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
@@ -268,6 +274,9 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *local, uint32_t rank
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)),
                  "r"(rank));
     return r;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c,
                                               float d) {

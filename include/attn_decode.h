@@ -338,9 +338,10 @@ int kv_append_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_c
  * i.e. q_c (U^K_h)^T with k^C_j = c_j U^K_h.  q_c [B][H][d_h], u_k
  * [H][d_c][d_h], q_latent [B][H][d_c] (the q_latent input of
  * attn_decode_mla); all bf16, device, 16-byte aligned, row-major; fp32
- * accumulation, result rounded to bf16.  d_c and d_h multiples of 8
- * (ATTN_ERR_UNSUPPORTED otherwise).  Stream-ordered; a plain batched GEMM
- * over the heads (cuBLAS).
+ * accumulation, result rounded to bf16 (nearest even).  d_c a multiple of
+ * 128 and d_h a multiple of 64, H <= 65535 (ATTN_ERR_UNSUPPORTED otherwise).
+ * Stream-ordered; a tcgen05 tensor-core kernel that reads each head's weight
+ * once per call and reuses it for all B sequences.  Allocates nothing.
  */
 int attn_mla_absorb_q(const void *q_c, const void *u_k, void *q_latent, int B, int H,
                       int d_c, int d_h, void *stream);
@@ -351,8 +352,10 @@ int attn_mla_absorb_q(const void *q_c, const void *u_k, void *q_latent, int B, i
  *     o[b][h][:] = sum_c z[b][h][c] * u_v[h][c][:]
  * i.e. z U^V_h with v_j = c_j U^V_h.  z [B][H][d_c] (the output of
  * attn_decode_mla), u_v [H][d_c][d_v], o [B][H][d_v]; bf16, device, 16-byte
- * aligned, row-major; fp32 accumulation, result rounded to bf16.  d_c and
- * d_v multiples of 8.  Stream-ordered; a plain batched GEMM (cuBLAS).
+ * aligned, row-major; fp32 accumulation, result rounded to bf16 (nearest
+ * even).  d_v a multiple of 128 and d_c a multiple of 64, H <= 65535
+ * (ATTN_ERR_UNSUPPORTED otherwise).  Stream-ordered; the same tensor-core
+ * kernel as attn_mla_absorb_q, U^V_h read once per call.  Allocates nothing.
  */
 int attn_mla_project_out(const void *z, const void *u_v, void *o, int B, int H, int d_c,
                          int d_v, void *stream);
