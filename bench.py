@@ -73,6 +73,7 @@ WORKLOAD_ALIASES = {
     "ragged_window_global": W.RAGGED_WINDOW_GLOBAL.name,
     "llama3_8b_fp8": W.LLAMA3_8B_FP8.name,
     "mla": W.MLA_DSV2.name,
+    "mla_fp8": W.MLA_DSV2_FP8.name,
 }
 
 
@@ -364,8 +365,11 @@ def tile_bytes_gqa(inp):
 
 
 def algorithmic_bytes_mla(inp):
+    """Latent rows of the visible keys (bf16, or fp8 codes plus a fp32 row
+    scale) + q + out."""
     cfg = inp.cfg
-    lat = sum(inp.seq_list) * (cfg.d_c + cfg.d_r) * 2
+    row = (cfg.d_c + cfg.d_r + 4) if cfg.kv_fp8 else (cfg.d_c + cfg.d_r) * 2
+    lat = sum(inp.seq_list) * row
     qo = cfg.B * cfg.H * (2 * cfg.d_c + cfg.d_r) * 2
     return lat, lat + qo
 
@@ -404,7 +408,9 @@ class Problem:
         base = make(cfg, device=dev, seed=seed)
         if self.is_mla:
             self.kv_bytes, self.alg_bytes = algorithmic_bytes_mla(base)
-            cache = base.latent_cache.numel() * 2
+            cache = base.latent_cache.numel() * base.latent_cache.element_size()
+            if base.latent_scale is not None:
+                cache += base.latent_scale.numel() * 4
         else:
             self.kv_bytes, self.alg_bytes = algorithmic_bytes_gqa(base)
             cache = 2 * base.k_cache.numel() * base.k_cache.element_size()
@@ -425,7 +431,10 @@ class Problem:
     def step(self, i):
         attn, cfg = self.attn, self.cfg
         x, out = self.inputs[i % self.reps], self.outs[i % self.reps]
-        if self.is_mla:
+        if self.is_mla and cfg.kv_fp8:
+            attn.decode_mla_fp8(x.q_lat, x.q_rope, x.latent_cache, x.latent_scale, x.seq_lens,
+                                x.block_table, x.scale, out=out)
+        elif self.is_mla:
             attn.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens, x.block_table,
                             x.scale, out=out)
         elif cfg.kv_fp8:
@@ -535,7 +544,8 @@ def config_entry(attn, cfg, dev, seed, K, warmup, min_s, pk, clk=None):
     if prob.is_mla:
         e["tensor_frac"] = roof["tensor_frac"]
         e["flops"] = roof["flops_per_launch"]
-        e["mla_absorb"] = mla_absorb_timing(attn, cfg, dev, seed)
+        if not cfg.kv_fp8:
+            e["mla_absorb"] = mla_absorb_timing(attn, cfg, dev, seed)
     else:
         e["tile_overread_bytes"] = tile_bytes_gqa(prob.base) - prob.kv_bytes
     del prob
@@ -548,7 +558,7 @@ def config_entry(attn, cfg, dev, seed, K, warmup, min_s, pk, clk=None):
 # the head-sharing sweep, the ragged 24/4/256 shape full and with w=4096, the
 # DeepSeek-V2 MLA shape; then the window/global/ring and fp8-cache variants.
 PER_CONFIG = [W.TINY, W.LLAMA3_8B, *W.SWEEP, W.RAGGED_FULL, W.RAGGED_WINDOW, W.MLA_DSV2,
-              W.LLAMA3_8B_FP8, W.RAGGED_WINDOW_SINK, W.RAGGED_WINDOW_RING,
+              W.LLAMA3_8B_FP8, W.MLA_DSV2_FP8, W.RAGGED_WINDOW_SINK, W.RAGGED_WINDOW_RING,
               W.RAGGED_WINDOW_GLOBAL]
 
 
@@ -706,9 +716,15 @@ def e2e_native(attn, cfg, x, is_mla, K, world, dev):
         if is_mla:
             d_r.copy_(h_r, non_blocking=True)
             d_lat.copy_(h_lat, non_blocking=True)
-            attn.kv_append_mla(d_lat, x.latent_cache, pos, x.block_table)
-            attn.decode_mla(d_q, d_r, x.latent_cache, x.seq_lens, x.block_table,
-                            x.scale, out=d_out)
+            if cfg.kv_fp8:
+                attn.kv_append_mla_fp8(d_lat, x.latent_cache, x.latent_scale, pos,
+                                       x.block_table)
+                attn.decode_mla_fp8(d_q, d_r, x.latent_cache, x.latent_scale, x.seq_lens,
+                                    x.block_table, x.scale, out=d_out)
+            else:
+                attn.kv_append_mla(d_lat, x.latent_cache, pos, x.block_table)
+                attn.decode_mla(d_q, d_r, x.latent_cache, x.seq_lens, x.block_table,
+                                x.scale, out=d_out)
         else:
             d_k.copy_(h_k, non_blocking=True)
             d_v.copy_(h_v, non_blocking=True)
@@ -767,7 +783,7 @@ def _oracle_problem(cfg, is_mla, seqs, seed):
     """Host-resident inputs of the first `seqs` sequences of the workload."""
     if is_mla:
         sub = W.MLAConfig(cfg.name, B=seqs, H=cfg.H, d_c=cfg.d_c, d_r=cfg.d_r,
-                          T=cfg.T, seed=seed)
+                          T=cfg.T, seed=seed, kv_fp8=cfg.kv_fp8)
         return W.make_mla_inputs(sub)
     lens = None
     if cfg.ragged:
@@ -781,6 +797,10 @@ def _oracle_problem(cfg, is_mla, seqs, seed):
 
 
 def _oracle_call(orc, x, is_mla):
+    if is_mla and x.cfg.kv_fp8:
+        lat = orc.dequantize_e4m3(x.latent_cache.numpy(), x.latent_scale.numpy())
+        return orc.decode_mla(x.q_lat.double().numpy(), x.q_rope.double().numpy(), lat,
+                              x.seq_lens, x.block_table, x.scale)
     if is_mla:
         return orc.decode_mla(x.q_lat, x.q_rope, x.latent_cache, x.seq_lens,
                               x.block_table, x.scale)

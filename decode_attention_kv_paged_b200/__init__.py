@@ -29,7 +29,7 @@ C_SYMBOLS = (
     "attn_debug_force_timeout", "attn_decode_last_error",
     "attn_status_string", "attn_version", "attn_decode_gqa_noalloc",
     "attn_mla_absorb_q", "attn_mla_project_out", "attn_decode_gqa_ext", "kv_append_ext",
-    "attn_decode_gqa_fp8", "kv_append_fp8",
+    "attn_decode_gqa_fp8", "kv_append_fp8", "attn_decode_mla_fp8", "kv_append_mla_fp8",
 )
 
 
@@ -80,6 +80,8 @@ def load():
     lib.attn_decode_gqa_fp8.argtypes = ([p] * 8 + [i] * 4 +
                                         [f, ctypes.POINTER(Visibility), p, i, i])
     lib.kv_append_fp8.argtypes = [p] * 8 + [i] * 5 + [ctypes.POINTER(Visibility), p]
+    lib.attn_decode_mla_fp8.argtypes = [p] * 7 + [i] * 4 + [f, p, i, i]
+    lib.kv_append_mla_fp8.argtypes = [p] * 5 + [i] * 5 + [p]
     lib.attn_mla_absorb_q.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.attn_mla_project_out.argtypes = [p] * 3 + [i] * 4 + [p]
     lib.kv_append.argtypes = [p] * 6 + [i] * 6 + [p]
@@ -271,6 +273,47 @@ def decode_mla(q_latent, q_rope, latent_cache, seq_lens, block_table, scale,
         nblk)
     _check(rc, "attn_decode_mla")
     return out
+
+
+def decode_mla_fp8(q_latent, q_rope, latent_codes, latent_scale, seq_lens, block_table,
+                   scale, out=None, stream=None):
+    """z [B][H][d_c] (bf16) = absorbed MLA decode over an fp8 latent cache:
+    latent_codes uint8 E4M3 [num_blocks][64][d_c + d_r], latent_scale fp32
+    [num_blocks][64] (value = code value * row scale)."""
+    B, H, d_c = q_latent.shape
+    d_r = q_rope.shape[2]
+    nblk, bs, width = latent_codes.shape
+    if bs != BLOCK_SIZE or width != d_c + d_r:
+        raise ValueError("latent_codes must be [num_blocks][64][d_c + d_r]")
+    if tuple(latent_scale.shape) != (nblk, bs):
+        raise ValueError("latent_scale must be [num_blocks][64]")
+    if out is None:
+        out = torch.empty_like(q_latent)
+    bf = torch.bfloat16
+    rc = load().attn_decode_mla_fp8(
+        _dev(q_latent, "q_latent", bf), _dev(q_rope, "q_rope", bf),
+        _dev(latent_codes, "latent_codes", torch.uint8),
+        _dev(latent_scale, "latent_scale", torch.float32),
+        _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(block_table, "block_table", torch.int32), _dev(out, "out", bf),
+        B, H, d_c, d_r, float(scale), _stream_ptr(stream), block_table.shape[1], nblk)
+    _check(rc, "attn_decode_mla_fp8")
+    return out
+
+
+def kv_append_mla_fp8(latent_new, latent_codes, latent_scale, positions, block_table,
+                      d_c=512, stream=None):
+    """Quantise latent_new [B][d_c + d_r] (bf16) to E4M3 with one scale per row
+    and write it into the fp8 latent cache at positions[b]."""
+    B, width = latent_new.shape
+    rc = load().kv_append_mla_fp8(
+        _dev(latent_new, "latent_new", torch.bfloat16),
+        _dev(latent_codes, "latent_codes", torch.uint8),
+        _dev(latent_scale, "latent_scale", torch.float32),
+        _dev(positions, "positions", torch.int32),
+        _dev(block_table, "block_table", torch.int32), B, d_c, width - d_c,
+        block_table.shape[1], latent_codes.shape[0], _stream_ptr(stream))
+    _check(rc, "kv_append_mla_fp8")
 
 
 def mla_absorb_q(q_c, u_k, out=None, stream=None):

@@ -4,7 +4,9 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <thread>
 
 #include "attn_decode.h"
 #include "gqa_launch.cuh"
@@ -17,14 +19,30 @@ namespace attn {
 
 __device__ unsigned g_err_word;   // per-device error word (bits kErr*)
 
-struct DeviceState {
-    bool ready = false;
-    int num_sms = 0;
-    unsigned *err = nullptr;      // device address of g_err_word
+// Split workspace of one stream: calls on different streams may run at the
+// same time, so each stream keeps its own partials and arrival counters.
+struct StreamWork {
+    cudaStream_t stream = nullptr;
+    unsigned long long key2 = 0;  // per-thread default stream: the calling thread
+    bool used = false;
+    unsigned long long last_use = 0;
     void *ws = nullptr;
     size_t ws_bytes = 0;
     unsigned *cnt = nullptr;      // split arrival counters (zero between launches)
     size_t cnt_elems = 0;
+};
+
+// Streams per device with a workspace of their own; the least recently used
+// one gives up its workspace to a new stream (freed with cudaFree, which
+// waits for the work still using it).
+constexpr int kMaxStreams = 16;
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned *err = nullptr;      // device address of g_err_word
+    unsigned long long tick = 0;
+    StreamWork work[kMaxStreams];
 };
 
 // One record per device ordinal; a pointer to a record stays valid for the
@@ -60,46 +78,83 @@ static int device_state(DeviceState **out) {
     return ATTN_OK;
 }
 
-// Grow the device's split workspace to at least `bytes`.  Never during
-// stream capture (a graph must not depend on an allocation made inside it).
-static int ensure_workspace(DeviceState *st, size_t bytes, cudaStream_t stream) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (st->ws_bytes >= bytes) return ATTN_OK;
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (cs != cudaStreamCaptureStatusNone) return ATTN_ERR_UNSUPPORTED;
-    size_t want = bytes < 2 * st->ws_bytes ? 2 * st->ws_bytes : bytes;
-    want = (want + (1u << 20) - 1) & ~(size_t)((1u << 20) - 1);
-    if (st->ws) {
-        cudaFree(st->ws);   // implicitly waits for work that may still use it
-        st->ws = nullptr;
-        st->ws_bytes = 0;
+// The workspace record of `stream` on this device (taken over from the least
+// recently used stream when all records are in use).  The per-thread default
+// stream is one handle for many streams, so it is keyed by the calling thread
+// as well.  Caller holds g_mu.
+static StreamWork *stream_work_locked(DeviceState *st, cudaStream_t stream) {
+    const unsigned long long key2 =
+        stream == cudaStreamPerThread
+            ? (unsigned long long)std::hash<std::thread::id>()(std::this_thread::get_id())
+            : 0ull;
+    StreamWork *victim = nullptr;
+    for (StreamWork &w : st->work) {
+        if (w.used && w.stream == stream && w.key2 == key2) {
+            w.last_use = ++st->tick;
+            return &w;
+        }
+        if (!victim || (!w.used && victim->used) ||
+            (w.used == victim->used && w.last_use < victim->last_use))
+            victim = &w;
     }
-    if (cudaMalloc(&st->ws, want) != cudaSuccess) return ATTN_ERR_CUDA;
-    st->ws_bytes = want;
+    if (victim->used) {
+        // cudaFree waits for all work on the device, the old stream's included.
+        if (victim->ws) cudaFree(victim->ws);
+        if (victim->cnt) cudaFree(victim->cnt);
+        *victim = StreamWork{};
+    }
+    victim->used = true;
+    victim->stream = stream;
+    victim->key2 = key2;
+    victim->last_use = ++st->tick;
+    return victim;
+}
+
+// Grow `stream`'s split workspace to at least `bytes`; returns it in *ws.
+// Never during stream capture (a graph must not depend on an allocation made
+// inside it).
+static int ensure_workspace(DeviceState *st, size_t bytes, cudaStream_t stream, void **ws) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    StreamWork *w = stream_work_locked(st, stream);
+    if (w->ws_bytes < bytes) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return ATTN_ERR_UNSUPPORTED;
+        size_t want = bytes < 2 * w->ws_bytes ? 2 * w->ws_bytes : bytes;
+        want = (want + (1u << 20) - 1) & ~(size_t)((1u << 20) - 1);
+        if (w->ws) {
+            cudaFree(w->ws);   // implicitly waits for work that may still use it
+            w->ws = nullptr;
+            w->ws_bytes = 0;
+        }
+        if (cudaMalloc(&w->ws, want) != cudaSuccess) return ATTN_ERR_CUDA;
+        w->ws_bytes = want;
+    }
+    *ws = w->ws;
     return ATTN_OK;
 }
 
-// Grow the device's split arrival counters to at least `n` (zeroed when
+// Grow `stream`'s split arrival counters to at least `n` (zeroed when
 // allocated; every launch leaves them at zero).  Never during capture.
-static int ensure_counters(DeviceState *st, size_t n, cudaStream_t stream) {
+static int ensure_counters(DeviceState *st, size_t n, cudaStream_t stream, unsigned **cnt) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (st->cnt_elems >= n) return ATTN_OK;
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (cs != cudaStreamCaptureStatusNone) return ATTN_ERR_UNSUPPORTED;
-    size_t want = n < 2 * st->cnt_elems ? 2 * st->cnt_elems : n;
-    want = (want + 4095) & ~(size_t)4095;
-    if (st->cnt) {
-        cudaFree(st->cnt);
-        st->cnt = nullptr;
-        st->cnt_elems = 0;
+    StreamWork *w = stream_work_locked(st, stream);
+    if (w->cnt_elems < n) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return ATTN_ERR_UNSUPPORTED;
+        size_t want = n < 2 * w->cnt_elems ? 2 * w->cnt_elems : n;
+        want = (want + 4095) & ~(size_t)4095;
+        if (w->cnt) {
+            cudaFree(w->cnt);
+            w->cnt = nullptr;
+            w->cnt_elems = 0;
+        }
+        if (cudaMalloc(&w->cnt, want * sizeof(unsigned)) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaMemset(w->cnt, 0, want * sizeof(unsigned)) != cudaSuccess) return ATTN_ERR_CUDA;
+        w->cnt_elems = want;
     }
-    if (cudaMalloc(&st->cnt, want * sizeof(unsigned)) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    if (cudaMemset(st->cnt, 0, want * sizeof(unsigned)) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    st->cnt_elems = want;
+    *cnt = w->cnt;
     return ATTN_OK;
 }
 
@@ -300,9 +355,10 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     const size_t o_bytes = align256((size_t)slots * copies * HC * d * sizeof(float));
     const size_t lse_bytes = align256((size_t)slots * copies * HC * sizeof(float));
     const size_t pre_bytes = align256((size_t)(B + 1) * sizeof(long long));
-    rc = ensure_workspace(st, o_bytes + lse_bytes + pre_bytes, s);
+    void *ws_raw = nullptr;
+    rc = ensure_workspace(st, o_bytes + lse_bytes + pre_bytes, s, &ws_raw);
     if (rc) return rc;
-    unsigned char *ws = static_cast<unsigned char *>(st->ws);
+    unsigned char *ws = static_cast<unsigned char *>(ws_raw);
 
     GqaLaunch L{};
     GqaParams &kp = L.kp;
@@ -316,9 +372,8 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     kp.k_scale = k_scale;
     kp.v_scale = v_scale;
     if (!tc) {
-        rc = ensure_counters(st, (size_t)units_total, s);
+        rc = ensure_counters(st, (size_t)units_total, s, &kp.ws_cnt);
         if (rc) return rc;
-        kp.ws_cnt = st->cnt;
     }
     take_force_timeout(&kp.force_timeout, &kp.timeout_ns);
     kp.scale_log2 = scale * 1.4426950408889634f;
@@ -455,10 +510,12 @@ int kv_append_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_c
     return cuda_status(launch_kv_append_fp8(p, (cudaStream_t)stream));
 }
 
-int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent_cache,
-                    const int32_t *seq_lens, const int32_t *block_table, void *out, int B,
-                    int H, int d_c, int d_r, float scale, void *stream,
-                    int max_blocks_per_seq, int num_blocks) {
+// Shared body of attn_decode_mla (latent_scale null: bf16 cache) and
+// attn_decode_mla_fp8 (E4M3 codes with per-row scales).
+static int decode_mla_impl(const void *q_latent, const void *q_rope, const void *latent_cache,
+                           const float *latent_scale, const int32_t *seq_lens,
+                           const int32_t *block_table, void *out, int B, int H, int d_c, int d_r,
+                           float scale, void *stream, int max_blocks_per_seq, int num_blocks) {
     if (!q_latent || !q_rope || !latent_cache || !seq_lens || !block_table || !out)
         return ATTN_ERR_ARG;
     if (B <= 0 || H <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
@@ -473,15 +530,58 @@ int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent
     if (rc) return rc;
     cudaEvent_t ev_start, ev_stop;
     take_profile_events(&ev_start, &ev_stop);
-    return mla_decode_entry(q_latent, q_rope, latent_cache, seq_lens, block_table, out, B,
-                            H, scale, (cudaStream_t)stream, max_blocks_per_seq, num_blocks,
-                            st->num_sms, tl_num_ctas, st->err,
+    return mla_decode_entry(q_latent, q_rope, latent_cache, latent_scale, seq_lens, block_table,
+                            out, B, H, scale, (cudaStream_t)stream, max_blocks_per_seq,
+                            num_blocks, st->num_sms, tl_num_ctas, st->err,
                             [&](size_t bytes, void **ws) {
-                                int r = ensure_workspace(st, bytes, (cudaStream_t)stream);
-                                *ws = st->ws;
-                                return r;
+                                return ensure_workspace(st, bytes, (cudaStream_t)stream, ws);
                             },
                             ev_start, ev_stop);
+}
+
+int attn_decode_mla(const void *q_latent, const void *q_rope, const void *latent_cache,
+                    const int32_t *seq_lens, const int32_t *block_table, void *out, int B,
+                    int H, int d_c, int d_r, float scale, void *stream,
+                    int max_blocks_per_seq, int num_blocks) {
+    return decode_mla_impl(q_latent, q_rope, latent_cache, nullptr, seq_lens, block_table, out,
+                           B, H, d_c, d_r, scale, stream, max_blocks_per_seq, num_blocks);
+}
+
+int attn_decode_mla_fp8(const void *q_latent, const void *q_rope, const void *latent_codes,
+                        const float *latent_scale, const int32_t *seq_lens,
+                        const int32_t *block_table, void *out, int B, int H, int d_c, int d_r,
+                        float scale, void *stream, int max_blocks_per_seq, int num_blocks) {
+    if (!latent_scale || !aligned16(latent_scale)) return ATTN_ERR_ARG;
+    return decode_mla_impl(q_latent, q_rope, latent_codes, latent_scale, seq_lens, block_table,
+                           out, B, H, d_c, d_r, scale, stream, max_blocks_per_seq, num_blocks);
+}
+
+int kv_append_mla_fp8(const void *latent_new, void *latent_codes, float *latent_scale,
+                      const int32_t *positions, const int32_t *block_table, int B, int d_c,
+                      int d_r, int max_blocks_per_seq, int num_blocks, void *stream) {
+    if (!latent_new || !latent_codes || !latent_scale || !positions || !block_table)
+        return ATTN_ERR_ARG;
+    if (B <= 0 || d_c <= 0 || d_r < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return ATTN_ERR_ARG;
+    if ((d_c + d_r) % 2 || !aligned16(latent_new) || !aligned16(latent_codes))
+        return ATTN_ERR_ARG;
+    DeviceState *st;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    KvAppendFp8Params p{};
+    p.k_new = static_cast<const __nv_bfloat16 *>(latent_new);
+    p.v_new = nullptr;                 // one latent row per token, no separate V
+    p.k_cache = static_cast<uint8_t *>(latent_codes);
+    p.v_cache = nullptr;
+    p.k_scale = latent_scale;
+    p.v_scale = nullptr;
+    p.positions = positions;
+    p.block_table = block_table;
+    p.err = st->err;
+    p.B = B; p.H_kv = 1; p.d = d_c + d_r;
+    p.max_blocks = max_blocks_per_seq; p.num_blocks = num_blocks;
+    p.vis = Visibility{0, 0, 0};
+    return cuda_status(launch_kv_append_fp8(p, (cudaStream_t)stream));
 }
 
 static int kv_append_impl(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -53,13 +53,14 @@ cudaError_t launch_kv_append(const KvAppendParams &p, cudaStream_t stream) {
 
 namespace attn {
 
-// fp8 append: one warp per (sequence, KV head) row of K and one of V.  Each
+// fp8 append: one warp per (sequence, KV head) row of K and one of V (K only
+// for the MLA latent cache, whose row is c_j followed by kR_j).  Each
 // row of d bf16 values x is stored as e4m3 codes of x * (448 / amax) (round to
 // nearest even, saturating) with the fp32 row scale amax / 448, amax =
 // max |x| (a zero row: scale 0, codes 0).  Divisions are IEEE round-to-nearest.
 __global__ void kv_append_fp8_kernel(const KvAppendFp8Params p) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    const int rows = p.B * p.H_kv * 2;               // K rows, then V rows
+    const int rows = p.B * p.H_kv * (p.v_new ? 2 : 1);   // K rows, then V rows (if any)
     if (warp >= rows) return;
     const bool is_v = warp >= p.B * p.H_kv;
     const int bh = is_v ? warp - p.B * p.H_kv : warp;
@@ -93,7 +94,7 @@ __global__ void kv_append_fp8_kernel(const KvAppendFp8Params p) {
 }
 
 cudaError_t launch_kv_append_fp8(const KvAppendFp8Params &p, cudaStream_t stream) {
-    const int rows = p.B * p.H_kv * 2;
+    const int rows = p.B * p.H_kv * (p.v_new ? 2 : 1);
     const int threads = 256;
     const int blocks = (rows * 32 + threads - 1) / threads;
     kv_append_fp8_kernel<<<blocks, threads, 0, stream>>>(p);

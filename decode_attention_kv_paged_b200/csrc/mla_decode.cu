@@ -40,8 +40,16 @@
 //     bounded mbarrier exchange.
 // Each (sequence, cluster) segment writes an fp32 partial (O/l and log2-sum-
 // exp) that the combine kernel reduces in cluster order.
+//
+// FP8 latent cache (template flag F8): rows stored as OCP E4M3 codes with one
+// fp32 scale per row (value = code value x scale).  The TMA loads each tile's
+// code boxes and 64 row scales into a raw stage; warp 3 widens the codes to
+// bf16 exactly (every E4M3 value is a bf16 value) into the same swizzled
+// stage layout the MMAs read, so the tensor-core path is unchanged.  The row
+// scale multiplies the token's score column (scores) and its probability
+// before the hi/lo split (values); the softmax sums use the unscaled
+// probabilities.
 #include <mutex>
-#include <vector>
 
 #include "attn_decode.h"
 #include "gqa_decode.cuh"
@@ -55,28 +63,40 @@ constexpr int kMlaH = 128;                 // heads = MMA M
 constexpr int kMlaDc = 512, kMlaDr = 64, kMlaWidth = 576;
 constexpr int kMlaCBox = 64 * 128;         // [64 tokens][64 cols] bf16
 constexpr int kMlaMaxBoxes = 5;
-constexpr int kMlaStages = 3;
 constexpr int kMlaPrefetch = 4;            // blocks pulled into L2 ahead of the ring
 constexpr int kMlaStageBytes = kMlaMaxBoxes * kMlaCBox;
-constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA, 4-11 softmax
+constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA/widening, 4-11 softmax
 constexpr int kSoftThreads = 256;
 constexpr int kPBytes = kMlaH * 128;       // one P half: [128 heads][64 tokens] bf16
 constexpr int kXBytes = kMlaH * 64 * 4;    // exchange buffer: 16 chunks x [128 rows] x 16 B
-constexpr int kOffC = 0;
-constexpr int kOffP = kOffC + kMlaStages * kMlaStageBytes;
-constexpr int kOffX = kOffP + 2 * kPBytes;   // receives the peer's partial S
-constexpr int kOffStg = kOffX + kXBytes;     // stages this CTA's partial S
-constexpr int kOffBar = kOffStg + kXBytes;
-constexpr int kOffRed = kOffBar + 512;     // [2][2][128] row-max halves + [2][2][128] sums
-constexpr int kMlaSmemUsed = kOffRed + 2 * 2 * 2 * 128 * 4;
-constexpr int kMlaSmem = kMlaSmemUsed + 1024;       // + alignment slack
+constexpr int kRawBox = 64 * 64;           // fp8: one box of codes, [64 tokens][64 columns]
+
+// Shared-memory layout of one variant (bf16 cache, or fp8 codes + row scales).
+template <bool F8> struct MlaCfg {
+    static constexpr int kStages = F8 ? 2 : 3;      // bf16 stages the MMAs read
+    static constexpr int kOffC = 0;
+    static constexpr int kOffP = kOffC + kStages * kMlaStageBytes;
+    static constexpr int kOffX = kOffP + 2 * kPBytes;   // receives the peer's partial S
+    static constexpr int kOffStg = kOffX + kXBytes;     // stages this CTA's partial S
+    static constexpr int kOffBar = kOffStg + kXBytes;
+    static constexpr int kOffRed = kOffBar + 512;       // [2][2][128] row maxima + sums
+    static constexpr int kOffRaw = kOffRed + 4096;      // fp8: raw code stages
+    static constexpr int kRawStages = 2;
+    static constexpr int kRawStageBytes = kMlaMaxBoxes * kRawBox + 1024;   // + 64 row scales
+    static constexpr int kOffScale = kOffRaw + (F8 ? kRawStages * kRawStageBytes : 0);
+    static constexpr int kSmemUsed = kOffScale + (F8 ? kStages * 64 * 4 : 0);
+    static constexpr int kSmem = kSmemUsed + 1024;     // + alignment slack
+    static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+};
+constexpr int kMlaMaxStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320;   // Q: 32 columns per box
 constexpr float kRescaleThreshold = 8.0f;           // log2 units
 
 struct MlaBars {
     uint64_t q_full, q_empty;
-    uint64_t c_full[kMlaStages], c_empty[kMlaStages];
+    uint64_t c_full[kMlaMaxStages], c_empty[kMlaMaxStages];
+    uint64_t raw_full[2], raw_empty[2];   // fp8: code stages landed / widened
     uint64_t s_full, s_free;
     uint64_t p_full, pv_done, o_free;
     uint64_t x_full, x_free, stg_full;
@@ -87,13 +107,13 @@ struct MlaBars {
     PlanScratch plan;
 };
 static_assert(sizeof(MlaBars) <= 512, "barrier block");
-static_assert(kMlaSmem <= 227 * 1024, "shared memory per CTA");
 static_assert(kTmemQ + 32 * kMlaMaxBoxes <= kTmemCols, "TMEM columns");
 
 struct MlaParams {
     const __nv_bfloat16 *q_lat;    // [B][128][512]
     const __nv_bfloat16 *q_rope;   // [B][128][64]
-    const __nv_bfloat16 *latent;   // [num_blocks][64][576]
+    const void *latent;            // [num_blocks][64][576] bf16, or E4M3 codes (fp8)
+    const float *lscale;           // fp8: [num_blocks][64] row scales
     const int32_t *seq_lens;
     const int32_t *block_table;
     float *ws_o;          // [slots][128][512]
@@ -105,8 +125,13 @@ struct MlaParams {
     int B, max_blocks, num_blocks, num_clusters;
 };
 
+template <bool F8>
 __global__ void __launch_bounds__(kMlaThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
+    using C = MlaCfg<F8>;
+    constexpr int kMlaStages = C::kStages;
+    constexpr int kOffC = C::kOffC, kOffP = C::kOffP, kOffX = C::kOffX, kOffStg = C::kOffStg,
+                  kOffBar = C::kOffBar, kOffRed = C::kOffRed;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -141,8 +166,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         mbar_init(&bars->q_full, kSoftThreads);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMlaStages; ++s) {
-            mbar_init(&bars->c_full[s], 1);
+            mbar_init(&bars->c_full[s], F8 ? 32 : 1);   // widening warp, or the TMA
             mbar_init(&bars->c_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->raw_full[s], 1);
+            mbar_init(&bars->raw_empty[s], 32);
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->s_free, kSoftThreads);
@@ -170,6 +199,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         // ============================================================ TMA
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
+            constexpr uint32_t kElem = F8 ? 1 : 2;     // bytes per cached value
             tma_prefetch_map(&tm_c);
             TileCursor cur;
             cur.init(pa, lo, hi, first_seq, first_base);
@@ -182,37 +212,55 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 if (rank != 0 || pf.done()) return;
                 const int pb = p.block_table[(size_t)pf.w.b * p.max_blocks + pf.logical_block()];
                 if (pb >= 0 && pb < p.num_blocks)
-                    bulk_prefetch_l2(p.latent + (size_t)pb * 64 * kMlaWidth,
-                                     64 * kMlaWidth * (uint32_t)sizeof(__nv_bfloat16));
+                    bulk_prefetch_l2(static_cast<const unsigned char *>(p.latent) +
+                                         (size_t)pb * 64 * kMlaWidth * kElem,
+                                     64 * kMlaWidth * kElem);
                 pf.next();
             };
             for (int k = 0; k < kMlaPrefetch; ++k) prefetch_next();
+            // bf16: straight into the stages the MMAs read; fp8: codes and
+            // row scales into a raw stage that warp 3 widens.
+            constexpr int kRing = F8 ? C::kRawStages : kMlaStages;
+            uint64_t *ring_full = F8 ? bars->raw_full : bars->c_full;
+            uint64_t *ring_empty = F8 ? bars->raw_empty : bars->c_empty;
             int tile = 0;
             while (!cur.done()) {
                 prefetch_next();
-                const int st = tile % kMlaStages;
-                if (tile >= kMlaStages &&
-                    !mbar_wait(&bars->c_empty[st],
-                               (uint32_t)(((tile - kMlaStages) / kMlaStages) & 1),
+                const int st = tile % kRing;
+                if (tile >= kRing &&
+                    !mbar_wait(&ring_empty[st], (uint32_t)(((tile - kRing) / kRing) & 1),
                                p.timeout_ns, p.err, abort_flag))
                     break;
                 int phys = p.block_table[(size_t)cur.w.b * p.max_blocks + cur.logical_block()];
-                if (phys < 0 || phys >= p.num_blocks) {
+                const bool bad = phys < 0 || phys >= p.num_blocks;
+                if (bad) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;            // wholly out of bounds: zero fill
                 }
-                unsigned char *dst = sC + st * kMlaStageBytes;
-                mbar_arrive_expect_tx(&bars->c_full[st], nbox * kMlaCBox);
-                for (int i = 0; i < nbox; ++i)
-                    tma_load_2d(dst + i * kMlaCBox, &tm_c, col0 + i * 64, phys * 64,
-                                &bars->c_full[st], pol);
+                if constexpr (F8) {
+                    unsigned char *dst = smem + C::kOffRaw + st * C::kRawStageBytes;
+                    float *dsc = reinterpret_cast<float *>(dst + kMlaMaxBoxes * kRawBox);
+                    if (bad)   // no scale row to copy: zeros (the codes are zero-filled too)
+                        for (int t = 0; t < 64; ++t) dsc[t] = 0.f;
+                    mbar_arrive_expect_tx(&ring_full[st], nbox * kRawBox + (bad ? 0 : 256));
+                    for (int i = 0; i < nbox; ++i)
+                        tma_load_2d(dst + i * kRawBox, &tm_c, col0 + i * 64, phys * 64,
+                                    &ring_full[st], pol);
+                    if (!bad) bulk_load(dsc, p.lscale + (size_t)phys * 64, 256, &ring_full[st]);
+                } else {
+                    unsigned char *dst = sC + st * kMlaStageBytes;
+                    mbar_arrive_expect_tx(&ring_full[st], nbox * kMlaCBox);
+                    for (int i = 0; i < nbox; ++i)
+                        tma_load_2d(dst + i * kMlaCBox, &tm_c, col0 + i * 64, phys * 64,
+                                    &ring_full[st], pol);
+                }
                 cur.next();
                 ++tile;
             }
             // Every issued load must have landed before the CTA exits.
-            for (int t = tile - kMlaStages < 0 ? 0 : tile - kMlaStages; t < tile; ++t)
-                mbar_wait(&bars->c_full[t % kMlaStages], (uint32_t)((t / kMlaStages) & 1),
-                          p.timeout_ns, p.err, nullptr);
+            for (int t = tile - kRing < 0 ? 0 : tile - kRing; t < tile; ++t)
+                mbar_wait(&ring_full[t % kRing], (uint32_t)((t / kRing) & 1), p.timeout_ns,
+                          p.err, nullptr);
         }
         __syncwarp();
     } else if (warp == 1 || warp == 2) {
@@ -306,6 +354,60 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
         }
         __syncwarp();
+    } else if (warp == 3) {
+        // ================================================ fp8 -> bf16 widening
+        // An E4M3 code's 7 magnitude bits, shifted so the 4-bit exponent and
+        // 3-bit mantissa sit at the top of an fp32's exponent and mantissa
+        // fields, are the fp32 pattern of value x 2^-120 (subnormal codes
+        // included: they become fp32 subnormals); one exact multiply by 2^120
+        // gives the value, whose top 16 bits are its bf16 pattern (at most 4
+        // significant bits, so nothing is rounded).
+        if constexpr (F8) {
+            TileCursor cur;
+            cur.init(pa, lo, hi, first_seq, first_base);
+            for (int tile = 0; tile < n_tiles; ++tile) {
+                const int rs = tile % C::kRawStages, st = tile % kMlaStages;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&bars->raw_full[rs], (uint32_t)((tile / C::kRawStages) & 1),
+                                          p.timeout_ns, p.err, abort_flag)))
+                    break;
+                if (tile >= kMlaStages &&
+                    !__all_sync(0xffffffffu,
+                                mbar_wait(&bars->c_empty[st],
+                                          (uint32_t)(((tile - kMlaStages) / kMlaStages) & 1),
+                                          p.timeout_ns, p.err, abort_flag)))
+                    break;
+                const unsigned char *raw = smem + C::kOffRaw + rs * C::kRawStageBytes;
+                unsigned char *dst = sC + st * kMlaStageBytes;
+                for (int idx = lane; idx < nbox * 512; idx += 32) {
+                    const int bx = idx >> 9, t = (idx >> 3) & 63, c = idx & 7;
+                    const uint2 codes =
+                        *reinterpret_cast<const uint2 *>(raw + bx * kRawBox + t * 64 + c * 8);
+                    uint32_t w[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t src = k < 2 ? codes.x : codes.y;
+                        const uint32_t u0 = (src >> (16 * (k & 1))) & 0xFFu;
+                        const uint32_t u1 = (src >> (16 * (k & 1) + 8)) & 0xFFu;
+                        const float f0 = __uint_as_float(((u0 & 0x7Fu) << 20) | ((u0 & 0x80u) << 24)) *
+                                         0x1p120f;
+                        const float f1 = __uint_as_float(((u1 & 0x7Fu) << 20) | ((u1 & 0x80u) << 24)) *
+                                         0x1p120f;
+                        w[k] = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
+                    }
+                    *reinterpret_cast<uint4 *>(dst + bx * kMlaCBox + t * 128 + ((c ^ (t & 7)) * 16)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                const float *rsc = reinterpret_cast<const float *>(raw + kMlaMaxBoxes * kRawBox);
+                float *ssc = reinterpret_cast<float *>(smem + C::kOffScale) + st * 64;
+                ssc[lane] = rsc[lane];
+                ssc[lane + 32] = rsc[lane + 32];
+                fence_proxy_async_smem();      // the MMAs read the widened stage
+                mbar_arrive(&bars->raw_empty[rs]);
+                mbar_arrive(&bars->c_full[st]);
+                cur.next();
+            }
+        }
     } else if (warp >= 4) {
         // ============================================ Q load, softmax, epilogue
         // Two threads per head row: warps w and w + 4 share TMEM lanes
@@ -405,6 +507,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 break;
             const unsigned char *xrow = sX + row * 16;
             const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+            // fp8: this half's 32 row scales of tile i (kept with its stage)
+            const float *tsc = reinterpret_cast<const float *>(smem + C::kOffScale) +
+                               (i % kMlaStages) * 64 + 32 * h;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const float4 v =
@@ -413,6 +518,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 float2 bb = __fadd2_rn(make_float2(s[4 * c + 2], s[4 * c + 3]), make_float2(v.z, v.w));
                 a = __fmul2_rn(a, sl2);
                 bb = __fmul2_rn(bb, sl2);
+                if constexpr (F8) {
+                    const float4 r = *reinterpret_cast<const float4 *>(tsc + 4 * c);
+                    a = __fmul2_rn(a, make_float2(r.x, r.y));
+                    bb = __fmul2_rn(bb, make_float2(r.z, r.w));
+                }
                 s[4 * c] = a.x; s[4 * c + 1] = a.y; s[4 * c + 2] = bb.x; s[4 * c + 3] = bb.y;
             }
             mbar_arrive_remote(x_free_peer);
@@ -464,6 +574,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 sum2 = __fadd2_rn(sum2, make_float2(s[j], s[j + 1]));
             }
             l_run += sum2.x + sum2.y;
+            if constexpr (F8) {
+                // the values are code values x row scale: scale each token's weight
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 r = *reinterpret_cast<const float4 *>(tsc + j);
+                    s[j] *= r.x; s[j + 1] *= r.y; s[j + 2] *= r.z; s[j + 3] *= r.w;
+                }
+            }
 
             // P and O may be touched once the previous P V has completed
             if (i >= 1 && !all(mbar_wait(&bars->pv_done, (uint32_t)((i - 1) & 1),
@@ -573,18 +691,20 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Row-major bf16 matrix [rows][cols] with row stride `stride` bytes, boxes of
-// [box_rows][64] with 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
-              uint64_t stride, uint32_t box_rows) {
+// The latent cache as a row-major matrix [num_blocks * 64][576] with boxes of
+// [64 rows][64 values]: bf16 with 128-byte swizzle (the MMAs read the boxes
+// directly), or fp8 codes unswizzled (widened into the swizzled layout).
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, bool fp8) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {stride};
-    cuuint32_t box[2] = {64, box_rows};
+    const uint64_t elem = fp8 ? 1 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)kMlaWidth, rows};
+    cuuint64_t strides[1] = {kMlaWidth * elem};
+    cuuint32_t box[2] = {64, 64};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -592,19 +712,19 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Clusters of two that can be resident at once (one CTA per SM), so that the
-// persistent ranges all run in a single wave.  Cached per device.
+// persistent ranges all run in a single wave.  Cached per device and variant.
+template <bool F8>
 int max_resident_clusters(int num_sms) {
     static std::mutex mu;
-    static std::vector<int> cache;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    static int cache[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0) return -1;
     std::lock_guard<std::mutex> lk(mu);
-    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
     if (cache[dev] == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(num_sms);
         cfg.blockDim = dim3(kMlaThreads);
-        cfg.dynamicSmemBytes = kMlaSmem;
+        cfg.dynamicSmemBytes = MlaCfg<F8>::kSmem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -613,7 +733,8 @@ int max_resident_clusters(int num_sms) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, mla_decode_kernel, &cfg) != cudaSuccess || n <= 0)
+        if (cudaOccupancyMaxActiveClusters(&n, mla_decode_kernel<F8>, &cfg) != cudaSuccess ||
+            n <= 0)
             n = num_sms / 2;
         cache[dev] = n < num_sms / 2 ? n : num_sms / 2;
         if (cache[dev] <= 0) cache[dev] = 1;
@@ -621,24 +742,50 @@ int max_resident_clusters(int num_sms) {
     return cache[dev];
 }
 
+template <bool F8>
+int mla_launch(const MlaParams &mp, const CUtensorMap &tc, int clusters, cudaStream_t stream,
+               cudaEvent_t ev_start, cudaEvent_t ev_stop) {
+    static PerDeviceFlag configured;   // the attribute is per function and device
+    if (configure_once_per_device(configured, [] {
+            return cudaFuncSetAttribute(mla_decode_kernel<F8>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        MlaCfg<F8>::kSmem);
+        }) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(kMlaThreads);
+    cfg.dynamicSmemBytes = MlaCfg<F8>::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (ev_start) cudaEventRecord(ev_start, stream);
+    if (cudaLaunchKernelEx(&cfg, mla_decode_kernel<F8>, tc, mp) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (ev_stop) cudaEventRecord(ev_stop, stream);
+    return ATTN_OK;
+}
+
 }  // namespace
 
 int mla_decode_entry(const void *q_latent, const void *q_rope, const void *latent_cache,
-                     const int32_t *seq_lens, const int32_t *block_table, void *out, int B,
-                     int H, float scale, cudaStream_t stream, int max_blocks, int num_blocks,
-                     int num_sms, int forced_ctas, unsigned *err,
-                     const WorkspaceFn &workspace, cudaEvent_t ev_start,
-                     cudaEvent_t ev_stop) {
+                     const float *latent_scale, const int32_t *seq_lens,
+                     const int32_t *block_table, void *out, int B, int H, float scale,
+                     cudaStream_t stream, int max_blocks, int num_blocks, int num_sms,
+                     int forced_ctas, unsigned *err, const WorkspaceFn &workspace,
+                     cudaEvent_t ev_start, cudaEvent_t ev_stop) {
     if (H != kMlaH) return ATTN_ERR_UNSUPPORTED;
     if ((long long)num_blocks * 64 > (1ll << 31) - 64 || (long long)B * kMlaH > (1ll << 31))
         return ATTN_ERR_ARG;
-    static PerDeviceFlag configured;   // the attribute is per function and device
-    if (configure_once_per_device(configured, [] {
-            return cudaFuncSetAttribute(mla_decode_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
-        }) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    int clusters = forced_ctas > 0 ? forced_ctas : max_resident_clusters(num_sms);
+    const bool fp8 = latent_scale != nullptr;
+    int clusters = forced_ctas > 0 ? forced_ctas
+                                   : (fp8 ? max_resident_clusters<true>(num_sms)
+                                          : max_resident_clusters<false>(num_sms));
     if (clusters <= 0) return ATTN_ERR_CUDA;
     const long long slots = (long long)B + clusters;
     const size_t o_bytes = round256((size_t)slots * kMlaH * kMlaDc * sizeof(float));
@@ -650,13 +797,13 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     unsigned char *w = static_cast<unsigned char *>(ws);
 
     CUtensorMap tc;
-    if (!make_map(&tc, latent_cache, kMlaWidth, (uint64_t)num_blocks * 64, kMlaWidth * 2, 64))
-        return ATTN_ERR_CUDA;
+    if (!make_map(&tc, latent_cache, (uint64_t)num_blocks * 64, fp8)) return ATTN_ERR_CUDA;
 
     MlaParams mp{};
     mp.q_lat = static_cast<const __nv_bfloat16 *>(q_latent);
     mp.q_rope = static_cast<const __nv_bfloat16 *>(q_rope);
-    mp.latent = static_cast<const __nv_bfloat16 *>(latent_cache);
+    mp.latent = latent_cache;
+    mp.lscale = latent_scale;
     mp.seq_lens = seq_lens;
     mp.block_table = block_table;
     mp.ws_o = reinterpret_cast<float *>(w);
@@ -669,23 +816,9 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     mp.max_blocks = max_blocks;
     mp.num_blocks = num_blocks;
     mp.num_clusters = clusters;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * clusters);
-    cfg.blockDim = dim3(kMlaThreads);
-    cfg.dynamicSmemBytes = kMlaSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (ev_start) cudaEventRecord(ev_start, stream);
-    if (cudaLaunchKernelEx(&cfg, mla_decode_kernel, tc, mp) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    if (ev_stop) cudaEventRecord(ev_stop, stream);
+    rc = fp8 ? mla_launch<true>(mp, tc, clusters, stream, ev_start, ev_stop)
+             : mla_launch<false>(mp, tc, clusters, stream, ev_start, ev_stop);
+    if (rc) return rc;
 
     CombineParams cp{};
     cp.seq_lens = seq_lens;

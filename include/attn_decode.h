@@ -81,9 +81,15 @@ typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
  *          is always fp32.
  * Requirements: H_q % H_kv == 0; d in {16, 32, 64, 128, 256}; pointers
  * 16-byte aligned; B >= 1; max_blocks_per_seq >= 1; num_blocks >= 1.
- * Uses a library-owned per-device workspace for the split partials; it is
- * grown (cudaMalloc) on first use outside stream capture.  Growing it while
- * the stream is being captured returns ATTN_ERR_UNSUPPORTED.
+ * Uses a library-owned split workspace (partials and arrival counters) per
+ * device and stream, so calls on different streams may run at the same time.
+ * A stream's workspace is grown (cudaMalloc) on first use outside stream
+ * capture; growing it while the stream is being captured returns
+ * ATTN_ERR_UNSUPPORTED.  Up to 16 streams per device keep their own; another
+ * stream takes over the least recently used one's (after a cudaFree, which
+ * waits for the device).  The per-thread default stream is keyed by the
+ * calling thread.  The device error word read by attn_decode_last_error is
+ * shared by all streams of the device.
  */
 int attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
                     const int32_t *seq_lens, const int32_t *block_table,
@@ -271,8 +277,11 @@ int attn_decode_last_error(void *stream);
  * Some callers cannot call cudaMalloc/cudaFree after start-up: a serving
  * process that gives all device memory to its own pool, or a latency-critical
  * thread that cannot take the device-wide synchronisation cudaFree implies.
- * This entry point computes exactly what attn_decode_gqa computes, with the
- * same arguments and layouts, but keeps its split scratch in a fixed array
+ * This entry point computes the same operation as attn_decode_gqa, with the
+ * same arguments and layouts, always on the CUDA-core split kernel (so it
+ * agrees with attn_decode_gqa within the parity tolerance, not bit for bit
+ * where that call picks a tensor-core kernel), but keeps its split scratch
+ * in a fixed array
  * of ATTN_NOALLOC_SCRATCH_BYTES compiled into the library (every GPU that
  * loads the library holds that array until the process exits).  It never
  * allocates.  The caller still passes all inputs and the output.
@@ -330,6 +339,39 @@ int kv_append_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_c
                   float *k_scale, float *v_scale, const int32_t *positions,
                   const int32_t *block_table, int B, int H_kv, int d, int max_blocks_per_seq,
                   int num_blocks, const attn_visibility *visibility, void *stream);
+
+/*
+ * attn_decode_mla_fp8 -- attn_decode_mla over an fp8 latent cache: the
+ * shared latent rows (the cache MLA keeps, attention-head §5.4) stored as
+ * OCP FP8 E4M3 codes, halving the bytes a decode streams ([BAIDU] §4.3: the
+ * cache-quantisation schemes a serving stack carries).
+ * latent_codes [num_blocks][64][d_c + d_r] uint8 E4M3 codes; latent_scale
+ * [num_blocks][64] fp32, one scale per cached row, so c_j / kR_j are the code
+ * values times the row scale (as written by kv_append_mla_fp8).  q_latent,
+ * q_rope and out are bf16 as for attn_decode_mla; d_c = 512, d_r = 64,
+ * H = 128.  The codes are widened to bf16 exactly on the chip; NaN codes
+ * (S.1111.111, never written by kv_append_mla_fp8) read as +-480.
+ * latent_scale 16-byte aligned; other arguments, workspace and errors as
+ * attn_decode_mla.
+ */
+int attn_decode_mla_fp8(const void *q_latent, const void *q_rope, const void *latent_codes,
+                        const float *latent_scale, const int32_t *seq_lens,
+                        const int32_t *block_table, void *out, int B, int H, int d_c, int d_r,
+                        float scale, void *stream, int max_blocks_per_seq, int num_blocks);
+
+/*
+ * kv_append_mla_fp8 -- quantise and append each sequence's new latent row
+ * (latent_new [B][d_c + d_r] bf16, c followed by kR) into the fp8 latent cache
+ * at positions[b]: codes of x * (448 / amax), rounded to nearest even and
+ * saturated to +-448, with row scale amax / 448 (amax = max |x| over the whole
+ * row, fp32; a zero row gets scale 0 and zero codes; both divisions IEEE
+ * round-to-nearest), exactly as kv_append_fp8 quantises a K/V row.
+ * latent_codes / latent_scale as for attn_decode_mla_fp8.  d_c + d_r even;
+ * latent_new and latent_codes 16-byte aligned.  Errors as kv_append.
+ */
+int kv_append_mla_fp8(const void *latent_new, void *latent_codes, float *latent_scale,
+                      const int32_t *positions, const int32_t *block_table, int B, int d_c,
+                      int d_r, int max_blocks_per_seq, int num_blocks, void *stream);
 
 /*
  * attn_mla_absorb_q -- the key up-projection folded into the query, before

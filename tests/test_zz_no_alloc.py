@@ -1,16 +1,17 @@
 """attn_decode_gqa_noalloc: the decode entry point for callers that must not
 allocate device memory while running (e.g. a server that gives all device
 memory to its own pool at start-up).  Its scratch is a fixed array inside the
-library; these tests call it through the C ABI and check it against the
-regular attn_decode_gqa on two consecutive calls.  This file is collected
-last so that a stop-at-first-failure run has already run everything else;
-it also passes on its own in a fresh process."""
+library; these tests call it through the C ABI and check it, on two
+consecutive calls, against the regular attn_decode_gqa and against the fp64
+oracle (both within the bf16 parity bars).  This file is collected last so
+that a stop-at-first-failure run has already run everything else; it also
+passes on its own in a fresh process."""
 import ctypes
 
 import pytest
 import torch
 
-from tests.parity import assert_parity
+from tests.parity import assert_parity, oracle_gqa_sequences
 from workloads import GQAConfig, make_gqa_inputs
 
 pytestmark = pytest.mark.gpu
@@ -42,8 +43,11 @@ def test_noalloc_matches_regular_entry_point_on_two_calls(lib):
         out = torch.full_like(x.q, float("nan"))
         assert _call_noalloc(lib, x, out) == lib.OK
         assert lib.last_error() == lib.OK
-        assert_parity(out.float().cpu().numpy(), ref.float().cpu().numpy(),
-                      torch.bfloat16, "noalloc vs attn_decode_gqa")
+        got = out.float().cpu().numpy()
+        assert_parity(got, ref.float().cpu().numpy(), torch.bfloat16,
+                      "noalloc vs attn_decode_gqa")
+        for b, r in oracle_gqa_sequences(x, range(x.cfg.B)).items():
+            assert_parity(got[b], r, torch.bfloat16, f"noalloc vs oracle b={b}")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):

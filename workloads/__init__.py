@@ -61,6 +61,7 @@ class MLAConfig:
     value_scale: float = 1.0 / math.sqrt(576.0)
     seed: int = SEED_BASE + 4
     dtype: torch.dtype = torch.bfloat16
+    kv_fp8: bool = False                   # fp8 latent cache (E4M3 codes + row scales)
 
     @property
     def scale(self) -> float:
@@ -108,10 +109,12 @@ RAGGED_WINDOW_GLOBAL = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_G16", 
                                  H_kv=4, d=256, ragged=(1024, 131072), window=4096,
                                  n_global=16, seed=SEED_BASE + 3)
 MLA_DSV2 = MLAConfig("mla_absorbed_bf16_B32_H128_dc512_dr64_T8192", B=32)
+# The DeepSeek-V2 shape over an fp8 latent cache.
+MLA_DSV2_FP8 = MLAConfig("mla_absorbed_fp8latent_B32_H128_dc512_dr64_T8192", B=32, kv_fp8=True)
 
 WORKLOADS = {c.name: c for c in [TINY, LLAMA3_8B, *SWEEP, RAGGED_FULL,
                                  RAGGED_WINDOW, RAGGED_WINDOW_SINK, RAGGED_WINDOW_RING,
-                                 RAGGED_WINDOW_GLOBAL, LLAMA3_8B_FP8, MLA_DSV2]}
+                                 RAGGED_WINDOW_GLOBAL, LLAMA3_8B_FP8, MLA_DSV2, MLA_DSV2_FP8]}
 
 
 def global_rows(seq_lens, n: int) -> torch.Tensor:
@@ -251,12 +254,14 @@ class MLAInputs:
     num_blocks: int
     scale: float
     seq_list: List[int] = field(default_factory=list)
+    latent_scale: Optional[torch.Tensor] = None   # fp8 cache: [num_blocks][64] row scales
 
     def to(self, device):
         return MLAInputs(self.cfg, self.q_lat.to(device),
                          self.q_rope.to(device), self.latent_cache.to(device),
                          self.seq_lens.to(device), self.block_table.to(device),
-                         self.num_blocks, self.scale, list(self.seq_list))
+                         self.num_blocks, self.scale, list(self.seq_list),
+                         None if self.latent_scale is None else self.latent_scale.to(device))
 
 
 def make_mla_inputs(cfg: MLAConfig, device="cpu", seed: Optional[int] = None,
@@ -267,8 +272,17 @@ def make_mla_inputs(cfg: MLAConfig, device="cpu", seed: Optional[int] = None,
     vs = cfg.value_scale
     q_lat = randn((cfg.B, cfg.H, cfg.d_c), g, cfg.dtype, vs)
     q_rope = randn((cfg.B, cfg.H, cfg.d_r), g, cfg.dtype, vs)
-    cache = randn((nblk, BLOCK_SIZE, cfg.d_c + cfg.d_r), g, cfg.dtype, vs)
     sl = torch.tensor(seq, dtype=torch.int32, device=g.device)
+    if cfg.kv_fp8:
+        # Stand-in quantised rows: uniform E4M3 codes (the two NaN codes
+        # replaced by +-448) with row scales of rows like N(0,1)*value_scale
+        # (amax ~3.2 value_scale).
+        shape = (nblk, BLOCK_SIZE, cfg.d_c + cfg.d_r)
+        c = torch.randint(0, 256, shape, generator=g, device=g.device, dtype=torch.int32)
+        c = torch.where((c & 0x7F) == 0x7F, c - 1, c).to(torch.uint8)
+        sc = (torch.rand(shape[:2], generator=g, device=g.device) * 0.8 + 2.8) * vs / 448
+        return MLAInputs(cfg, q_lat, q_rope, c, sl, table, nblk, cfg.scale, seq, sc)
+    cache = randn((nblk, BLOCK_SIZE, cfg.d_c + cfg.d_r), g, cfg.dtype, vs)
     return MLAInputs(cfg, q_lat, q_rope, cache, sl, table, nblk, cfg.scale,
                      seq)
 
