@@ -113,19 +113,34 @@ static size_t orc_row_offset(const int32_t *block_table, int max_blocks, int b,
  * (window <= 0 or j >= T - window or j < sink or j in G_b or T - 1 in G_b).
  * G_b is row b of gpos [B][n_g] (n_g = 0: empty), read in order up to its
  * first entry that does not exceed the one before.  The row of key j sits in
- * the block of table slot slot(j / block_size): with ring > 0, logical block
- * i < A = ceil(sink / block_size) keeps slot i and i >= A goes to slot
- * A + i % ring; without ring, slot i = i.  Softmax over the visible keys only.
- * Same arrays and dtypes as orc_decode_gqa; probs (optional) [B][H_q][max_T].
+ * the block of the table slot that holds logical block i = j / block_size:
+ *   - no ring: slot i;
+ *   - ring, no global set: block i < A = ceil(sink / block_size) keeps slot
+ *     i, block i >= A goes to slot A + i % ring;
+ *   - ring with a global set (a window layer that also keeps the positions
+ *     of G, §3): slots [0, n_g) are the global slots, slot k holding the
+ *     block of position G_b[k]; a key in a block before the window's first
+ *     block (there only keys of G are visible) is read through the global
+ *     slot of its own position, and block i from the window's first block
+ *     (max(0, T - window) / block_size) on through ring slot n_g + i % ring.
+ *     The ring no longer holds the history a global query (T - 1 in G_b)
+ *     would need, so such a query with T > window is refused (ORC_BAD_ARG).
+ * Softmax over the visible keys only.  Same arrays and dtypes as
+ * orc_decode_gqa; probs (optional) [B][H_q][max_T].
  */
-static int orc_in_set(const int32_t *row, int n, int x) {
+/* index k with row[k] == x in the (ascending, possibly padded) set, or -1 */
+static int orc_set_index(const int32_t *row, int n, int x) {
     int prev = -1;
     for (int k = 0; k < n; ++k) {
         if (row[k] <= prev) break;
-        if (row[k] == x) return 1;
+        if (row[k] == x) return k;
         prev = row[k];
     }
-    return 0;
+    return -1;
+}
+
+static int orc_in_set(const int32_t *row, int n, int x) {
+    return orc_set_index(row, n, x) >= 0;
 }
 
 static int orc_slot(int i, int sink, int ring, int block_size) {
@@ -141,7 +156,8 @@ int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
                        double scale, int window, int sink, int ring, int dtype,
                        const int32_t *gpos, int n_g) {
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || d <= 0 || block_size <= 0 ||
-        H_q % H_kv != 0 || sink < 0 || ring < 0 || n_g < 0 || (n_g > 0 && !gpos))
+        H_q % H_kv != 0 || sink < 0 || ring < 0 || n_g < 0 || (n_g > 0 && !gpos) ||
+        (n_g > 0 && ring > 0 && sink > 0))
         return ORC_BAD_ARG;
     const int group = H_q / H_kv;
     int status = ORC_OK;
@@ -168,6 +184,14 @@ int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
             }
             const int32_t *grow = n_g > 0 ? gpos + (size_t)b * n_g : NULL;
             const int q_global = grow && orc_in_set(grow, n_g, T - 1);
+            if (q_global && ring > 0 && window > 0 && T > window) {
+                free(keys); free(s);
+#pragma omp atomic write
+                status = ORC_BAD_ARG;
+                continue;
+            }
+            /* first block of the window (global-set ring layout) */
+            const int w0 = (window > 0 && T > window ? T - window : 0) / block_size;
             int n = 0;
             for (int j = 0; j < T; ++j)
                 if (window <= 0 || j >= T - window || j < sink || q_global ||
@@ -176,7 +200,10 @@ int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
             const size_t q_off = ((size_t)b * H_q + h) * d;
             for (int t = 0; t < n; ++t) {
                 const int j = keys[t];
-                const int slot = orc_slot(j / block_size, sink, ring, block_size);
+                const int slot = (grow && ring > 0)
+                                     ? (j / block_size < w0 ? orc_set_index(grow, n_g, j)
+                                                            : n_g + (j / block_size) % ring)
+                                     : orc_slot(j / block_size, sink, ring, block_size);
                 const int32_t phys = block_table[(size_t)b * max_blocks + slot];
                 const size_t r = (((size_t)phys * H_kv + kvh) * block_size + j % block_size) * d;
                 double dot = 0.0;
@@ -195,7 +222,10 @@ int orc_decode_gqa_vis(const void *q, const void *k_cache, const void *v_cache,
             for (int t = 0; t < n; ++t) s[t] /= z;
             for (int t = 0; t < n; ++t) {
                 const int j = keys[t];
-                const int slot = orc_slot(j / block_size, sink, ring, block_size);
+                const int slot = (grow && ring > 0)
+                                     ? (j / block_size < w0 ? orc_set_index(grow, n_g, j)
+                                                            : n_g + (j / block_size) % ring)
+                                     : orc_slot(j / block_size, sink, ring, block_size);
                 const int32_t phys = block_table[(size_t)b * max_blocks + slot];
                 const size_t r = (((size_t)phys * H_kv + kvh) * block_size + j % block_size) * d;
                 for (int k = 0; k < d; ++k) o[k] += s[t] * orc_read(v_cache, r + k, dtype);

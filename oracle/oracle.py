@@ -131,9 +131,15 @@ def decode_gqa_vis(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
     the sequence's global set, or T - 1 is in it (attention-head article, §3:
     a global query sees the whole history).  global_pos: int [B][n_g], each
     row ascending and read up to its first entry that does not exceed the one
-    before (pad with -1).  With ring > 0, logical block i lives in table slot
-    i for i < A = ceil(sink / block_size) (the sink blocks) and in slot
-    A + i % ring after them.  Same arrays as decode_gqa.
+    before (pad with -1).  With ring > 0 and no global set, logical block i
+    lives in table slot i for i < A = ceil(sink / block_size) (the sink
+    blocks) and in slot A + i % ring after them.  With ring > 0 and a global
+    set (sink must be 0), slots [0, n_g) are global slots -- slot k holds the
+    block of position global_pos[b][k] -- a visible key in a block before the
+    window's first block is read through its own position's global slot, and
+    block i from the window's first block on sits in slot n_g + i % ring; a
+    global query with T > window is refused (the ring no longer holds the
+    history it would see).  Same arrays as decode_gqa.
     """
     B, H_q, d = q.shape
     _, H_kv, bs, d2 = k_cache.shape

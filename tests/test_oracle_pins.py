@@ -565,6 +565,101 @@ def test_vis_ring_table_any_geometry_reads_the_same_rows(T, w, g, R):
     assert np.array_equal(got, ref)
 
 
+def _global_ring_table(rng, k, v, T, w, R, gp_row, spare=3):
+    """Table row of n_g global slots + R ring slots for one sequence whose
+    full-table cache is (k, v): global slot k names the block of position
+    gp_row[k] (positions sharing a block share its physical block), ring
+    slot n_g + i % R names logical block i for the blocks the window
+    reaches.  Every physical block nothing names holds noise."""
+    n_g = len(gp_row)
+    nb = (T + 63) // 64
+    w0 = max(0, T - w) // 64
+    gblocks = sorted({p // 64 for p in gp_row if p >= 0})
+    n_phys = len(gblocks) + R + spare
+    perm = rng.permutation(n_phys).astype(np.int32)
+    table = np.full((1, n_g + R), -1, dtype=np.int32)
+    kr = rng.standard_normal((n_phys,) + k.shape[1:])
+    vr = rng.standard_normal((n_phys,) + v.shape[1:])
+    phys_of = {}
+    for j, blk in enumerate(gblocks):
+        phys_of[blk] = perm[j]
+        kr[perm[j]] = k[blk]
+        vr[perm[j]] = v[blk]
+    for kk, pos in enumerate(gp_row):
+        if pos >= 0:
+            table[0, kk] = phys_of[pos // 64]
+    for i in range(w0, nb):
+        ph = perm[len(gblocks) + i % R]
+        table[0, n_g + i % R] = ph
+        kr[ph] = k[i]
+        vr[ph] = v[i]
+    return kr, vr, table
+
+
+@pytest.mark.parametrize("T,w,R,gp", [
+    (9, 3, 2, [0, 5]),                      # the §3 figure's G = {0, 5}, w = 3
+    (700, 100, 3, [0, 5, 130, 131, 640]),   # two positions share a block; one in the window
+    (1000, 200, 5, [63, 64, 799, 801]),     # 799 straddles the window's first block
+    (5000, 640, 11, [1, 2, 3, 4000, 4500, -1, -1]),
+    (129, 1, 1, [0, 127]),
+    (300, 63, 2, [10, 250, 298]),
+])
+def test_vis_global_set_ring_reads_the_same_rows(T, w, R, gp):
+    """A window layer that keeps the positions of an explicit global set G
+    (attention-head article, §3): a table row of n_g global slots + a ring
+    holding the window's blocks gives the full table's result bit for bit,
+    wherever G's positions lie (before the window, in its first block, in
+    it), and no other physical block is read."""
+    if R * 64 < w + 63:
+        pytest.skip("ring smaller than the window")
+    gp_row = list(gp)
+    if (T - 1) in gp_row and T > w:
+        pytest.skip("a global query needs the whole history")
+    rng = np.random.default_rng(T + 7 * w + R)
+    q, k, v, table = _contiguous_case(rng, 2, 1, 8, T)
+    lens = np.array([T], dtype=np.int32)
+    gpos = np.array([gp_row], dtype=np.int32)
+    ref = orc.decode_gqa_vis(q, k, v, lens, table, 0.3, window=w, global_pos=gpos)
+    kr, vr, ring_table = _global_ring_table(rng, k, v, T, w, R, gp_row)
+    got = orc.decode_gqa_vis(q, kr, vr, lens, ring_table, 0.3, window=w, ring=R,
+                             global_pos=gpos)
+    assert np.array_equal(got, ref)
+
+
+def test_vis_global_set_ring_noise_changes_result_when_a_global_block_is_lost():
+    """Negative control of the ring pin: if a global slot names a noise block
+    instead of its position's block, the result changes -- the ring layout
+    really reads the global slots."""
+    T, w, R, gp_row = 700, 100, 3, [0, 5, 130]
+    rng = np.random.default_rng(3)
+    q, k, v, table = _contiguous_case(rng, 2, 1, 8, T)
+    lens = np.array([T], dtype=np.int32)
+    gpos = np.array([gp_row], dtype=np.int32)
+    ref = orc.decode_gqa_vis(q, k, v, lens, table, 0.3, window=w, global_pos=gpos)
+    kr, vr, ring_table = _global_ring_table(rng, k, v, T, w, R, gp_row, spare=3)
+    ring_table[0, 2] = kr.shape[0] - 1          # block of position 130 -> a noise block
+    got = orc.decode_gqa_vis(q, kr, vr, lens, ring_table, 0.3, window=w, ring=R,
+                             global_pos=gpos)
+    assert not np.allclose(got, ref)
+
+
+def test_vis_global_query_with_ring_is_refused():
+    """A global query sees the whole history (§3), which a ring no longer
+    holds once T > window: the oracle refuses it; with T <= window the
+    window covers everything and the call is served."""
+    rng = np.random.default_rng(5)
+    q, k, v, table = _contiguous_case(rng, 2, 1, 8, 200)
+    gpos = np.array([[3, 199]], dtype=np.int32)          # T - 1 = 199 is global
+    with pytest.raises(RuntimeError):
+        orc.decode_gqa_vis(q, k, v, np.array([200], dtype=np.int32), table, 0.3, window=100,
+                           ring=4, global_pos=gpos)
+    kr, vr, ring_table = _global_ring_table(rng, k, v, 200, 300, 6, [3, 199])
+    ok = orc.decode_gqa_vis(q, kr, vr, np.array([200], dtype=np.int32), ring_table, 0.3,
+                            window=300, ring=6, global_pos=gpos)
+    full = orc.decode_gqa(q, k, v, np.array([200], dtype=np.int32), table, 0.3, window=0)
+    assert np.array_equal(ok, full)
+
+
 # ------------------------------------------------------- fp8 (E4M3) KV cache
 def test_e4m3_values_match_the_format():
     """Closed forms of the OCP FP8 E4M3 format: bias 7, 3 mantissa bits,
