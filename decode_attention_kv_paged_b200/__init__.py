@@ -165,7 +165,10 @@ def decode_gqa_ext(q, k_cache, v_cache, seq_lens, block_table, scale, window=0,
     in the sequence's row of global_pos (int32 [B][n_global], ascending, -1
     padded), or T - 1 is in it (a global query sees everything); with
     ring_blocks > 0 logical block i lives in table slot i for the sink
-    blocks and in slot A + i % ring_blocks after them (A = ceil(sink / 64))."""
+    blocks and in slot A + i % ring_blocks after them (A = ceil(sink / 64));
+    with ring_blocks > 0 and global_pos, slots [0, n_global) hold the blocks
+    of the global positions (read for blocks before the window) and A =
+    n_global."""
     B, H_q, d = q.shape
     nblk, H_kv, bs, d2 = k_cache.shape
     if bs != BLOCK_SIZE or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape):
@@ -349,12 +352,12 @@ def mla_project_out(z, u_v, out=None, stream=None):
 
 
 def kv_append_ext(k_new, v_new, k_cache, v_cache, positions, block_table,
-                  window=0, sink_tokens=0, ring_blocks=0, stream=None):
-    """kv_append through the table mapping of a visibility record (sink slots,
-    then the ring): with a ring, writing past the window overwrites the block
-    that left it."""
+                  window=0, sink_tokens=0, ring_blocks=0, stream=None, global_pos=None):
+    """kv_append through the table mapping of a visibility record (sink or
+    global slots, then the ring): with a ring, writing past the window
+    overwrites the block that left it."""
     B, H_kv, d = k_new.shape
-    vis = _visibility(window, sink_tokens, ring_blocks)
+    vis = _visibility(window, sink_tokens, ring_blocks, global_pos, B)
     rc = load().kv_append_ext(
         _dev(k_new, "k_new"), _dev(v_new, "v_new", k_new.dtype),
         _dev(k_cache, "k_cache", k_new.dtype), _dev(v_cache, "v_cache", k_new.dtype),

@@ -430,9 +430,10 @@ static int check_visibility(const attn_visibility *v, int max_blocks_per_seq, Vi
     if (v->sink_tokens < 0 || v->ring_blocks < 0 || v->n_global < 0) return ATTN_ERR_ARG;
     Visibility vis{v->window > 0 ? v->window : 0, v->sink_tokens, v->ring_blocks};
     if (v->n_global > 0) {
-        // An explicit global set replaces the sink prefix and has no ring.
+        // An explicit global set replaces the sink prefix; with a ring its
+        // positions' blocks keep the n_global slots ahead of the ring.
         if (!v->global_pos || (reinterpret_cast<uintptr_t>(v->global_pos) & 3u) ||
-            v->sink_tokens > 0 || v->ring_blocks > 0)
+            v->sink_tokens > 0)
             return ATTN_ERR_ARG;
         if (v->n_global > 64) return ATTN_ERR_UNSUPPORTED;
         vis.gpos = v->global_pos;
@@ -440,11 +441,11 @@ static int check_visibility(const attn_visibility *v, int max_blocks_per_seq, Vi
     }
     if (vis.ring > 0) {
         // The ring must hold every block a window can reach, after the sink
-        // blocks, inside the table row.
+        // blocks (or the global slots), inside the table row.
         if (vis.window <= 0) return ATTN_ERR_ARG;
         if ((long long)vis.ring * kBlockSize < (long long)vis.window + kBlockSize - 1)
             return ATTN_ERR_ARG;
-        if ((long long)sink_blocks(vis) + vis.ring > max_blocks_per_seq) return ATTN_ERR_ARG;
+        if ((long long)ring_base(vis) + vis.ring > max_blocks_per_seq) return ATTN_ERR_ARG;
     }
     *out = vis;
     return ATTN_OK;

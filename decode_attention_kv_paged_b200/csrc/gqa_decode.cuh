@@ -289,6 +289,7 @@ struct TileCursor {
     }
     __device__ bool done() const { return w.done(); }
     __device__ int logical_block() const { return w.logical(w.blk_off + t); }
+    __device__ int table_slot_of_tile() const { return w.slot(w.blk_off + t); }
     __device__ void next() {
         if (++t == len) {
             w.advance(len);
@@ -312,7 +313,7 @@ struct Producer {
         const int j = i + lane;
         if (j >= cur.len) return -1;
         return __ldg(p.block_table + (size_t)cur.w.b * p.max_blocks +
-                     table_slot(p.vis, cur.w.logical(cur.w.blk_off + j)));
+                     cur.w.slot(cur.w.blk_off + j));
     }
 
     // Physical block id of the current tile (warp-uniform call).
@@ -1135,9 +1136,14 @@ constexpr int kCombineThreads = 256;
 constexpr int kCombineMaxW = 4096;       // (head, partial) weights held in shared memory
 
 // Threads that share one float4 of output in the combine: more when a unit
-// has many partials (each takes every lanes-th partial), one when it has few.
+// has many partials (each takes every lanes-th partial, so the chain of
+// dependent loads per thread stays short and few-unit shapes still spread
+// over many CTAs), one when it has few.
 __host__ __device__ constexpr int combine_lanes(int expected_partials) {
-    return expected_partials >= 32 ? 8 : (expected_partials >= 8 ? 4 : 1);
+    return expected_partials >= 256 ? 32
+           : expected_partials >= 96 ? 16
+           : expected_partials >= 32 ? 8
+           : expected_partials >= 8 ? 4 : 1;
 }
 // CTAs of the combine kernel per unit.
 __host__ __device__ constexpr int combine_blocks_per_unit(int HC, int D, int lanes) {

@@ -181,7 +181,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                p.timeout_ns, p.err, abort_flag))
                     break;
                 int phys = p.block_table[(size_t)cur.w.b * p.max_blocks +
-                                         table_slot(p.vis, cur.logical_block())];
+                                         cur.table_slot_of_tile()];
                 if (phys < 0 || phys >= p.num_blocks) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;                 // wholly out of bounds: zero fill

@@ -143,7 +143,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                                p.timeout_ns, p.err, abort_flag))
                     break;
                 int phys = p.block_table[(size_t)cur.w.b * p.max_blocks +
-                                         table_slot(p.vis, cur.logical_block())];
+                                         cur.table_slot_of_tile()];
                 if (phys < 0 || phys >= p.num_blocks) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;                 // wholly out of bounds: zero fill

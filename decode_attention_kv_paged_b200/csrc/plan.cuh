@@ -27,7 +27,12 @@ namespace attn {
 // one, e.g. a -1 pad, ends the row).  With ring > 0 the table row is a ring:
 // the blocks holding the sink keys keep slots [0, A) (A = ceil(sink / 64));
 // logical block i >= A lives in slot A + i % ring, so a window layer stores
-// only the blocks its window can reach.
+// only the blocks its window can reach.  With ring > 0 and a global set
+// (sink 0) the row starts with n_g global slots instead, slot k holding the
+// block of G_b[k]: blocks before the window's first block are read through
+// the global slot of their first global position, and block i from the
+// window's first block on lives in slot n_g + i % ring.  A global query with
+// T > window would need history the ring no longer holds and is refused.
 struct Visibility {
     int window;   // > 0: sliding window of the last `window` keys
     int sink;     // > 0: the first `sink` keys stay visible (global tokens)
@@ -59,11 +64,17 @@ __host__ __device__ __forceinline__ int sink_blocks(const Visibility &v) {
     return v.sink > 0 ? (v.sink + kBlockSize - 1) / kBlockSize : 0;
 }
 
-// Table slot of logical block i.
+// Slots ahead of the ring: the sink blocks, or one per global position.
+__host__ __device__ __forceinline__ int ring_base(const Visibility &v) {
+    return v.n_g > 0 ? v.n_g : sink_blocks(v);
+}
+
+// Table slot of logical block i (for a global-set ring: of a block from the
+// window's first block on; earlier blocks use global_slot).
 __host__ __device__ __forceinline__ int table_slot(const Visibility &v, int i) {
     if (v.ring <= 0) return i;
-    const int a = sink_blocks(v);
-    return i < a ? i : a + i % v.ring;
+    const int a = ring_base(v);
+    return (v.n_g <= 0 && i < a) ? i : a + i % v.ring;
 }
 
 // First visible key of the window part (0 without a window).
@@ -94,6 +105,26 @@ __device__ __forceinline__ int global_block(const Visibility &v, int b, int i) {
         }
     }
     return last;   // not reached for i < count
+}
+
+// Global-set ring layout: table slot of the i-th distinct block (ascending)
+// holding a global position of sequence b, i.e. the index of the first
+// position of G_b in it (0 if there is none, which callers never ask for).
+__device__ __forceinline__ int global_slot(const Visibility &v, int b, int i) {
+    const int32_t *g = global_row(v, b);
+    int prev = -1, last = -1, n = 0;
+    for (int k = 0; k < v.n_g; ++k) {
+        const int p = g[k];
+        if (p <= prev) break;
+        prev = p;
+        const int blk = p / kBlockSize;
+        if (blk != last) {
+            if (n == i) return k;
+            ++n;
+            last = blk;
+        }
+    }
+    return 0;
 }
 
 // Bit t set when token blk * 64 + t of sequence b is a global position.
@@ -178,7 +209,13 @@ __device__ __forceinline__ int visible_blocks(int T, const Visibility &v, int ma
     }
     *bad = false;
     const int w1 = (T - 1) / kBlockSize + 1;             // one past the last block
-    if (v.n_g > 0) return visible_blocks_global(T, v, b, w1, first_block, sink_blks);
+    if (v.n_g > 0) {
+        if (v.ring > 0 && window_lo(v, T) > 0 && global_query(v, b, T)) {
+            *bad = true;                                  // history left the ring
+            return 0;
+        }
+        return visible_blocks_global(T, v, b, w1, first_block, sink_blks);
+    }
     const int w0 = window_lo(v, T) / kBlockSize;        // first window block
     const int a = sink_blocks(v) < w1 ? sink_blocks(v) : w1;
     if (a >= w0) return w1;                               // one run [0, w1)
@@ -373,6 +410,12 @@ struct SegmentWalker {
     __device__ int logical(int v) const {
         if (v >= sink_blks) return first_blk + (v - sink_blks);
         return vis.n_g > 0 ? global_block(vis, b, v) : v;
+    }
+
+    // Table slot of visible block v of the current sequence.
+    __device__ int slot(int v) const {
+        if (v < sink_blks && vis.n_g > 0 && vis.ring > 0) return global_slot(vis, b, v);
+        return table_slot(vis, logical(v));
     }
 
     __device__ void init(const PlanArgs &a, long long lo, long long hi,

@@ -56,7 +56,7 @@ typedef enum {
     ATTN_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
     ATTN_ERR_TIMEOUT = -4,      /* device: a bounded wait ran out */
     ATTN_ERR_BAD_BLOCK = -5,    /* device: block id outside [0, num_blocks) */
-    ATTN_ERR_BAD_SEQLEN = -6    /* device: T_b < 0 or > 64 * max_blocks */
+    ATTN_ERR_BAD_SEQLEN = -6    /* device: T_b < 0, > 64 * max_blocks, or not servable by the ring */
 } attn_status;
 
 typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
@@ -153,17 +153,28 @@ int kv_append_mla(const void *latent_new, void *latent_cache,
  * whole history).  Global positions: global_pos is a device int32 array
  * [B][n_global], row b holding sequence b's positions in ascending order;
  * the row ends at its first entry that does not exceed the previous one (pad
- * with -1).  0 < n_global <= 64; global_pos needs sink_tokens = 0 and
- * ring_blocks = 0 (ATTN_ERR_ARG otherwise; n_global > 64:
- * ATTN_ERR_UNSUPPORTED); n_global = 0 ignores global_pos.  Blocks before the
- * window hold visible keys only where a global position lies, and only those
- * blocks are read.
+ * with -1).  0 < n_global <= 64; global_pos needs sink_tokens = 0
+ * (ATTN_ERR_ARG otherwise; n_global > 64: ATTN_ERR_UNSUPPORTED);
+ * n_global = 0 ignores global_pos.  Blocks before the window hold visible
+ * keys only where a global position lies, and only those blocks are read.
  * ring_blocks > 0 makes the table row a ring for window layers: the blocks
  * holding the sink keys keep slots [0, A) with A = ceil(sink_tokens / 64),
  * and logical block i >= A lives in slot A + (i mod ring_blocks), so a
  * sequence stores only the blocks its window can reach; kv_append_ext
  * writing token T-1 then overwrites (evicts) the block that left the
- * window.  ring_blocks > 0 requires window > 0, ring_blocks * 64 >=
+ * window.  With a global set, the row instead starts with A = n_global
+ * global slots: slot k names the block holding position global_pos[b][k]
+ * (slots of positions that share a block name the same block; slots after
+ * the row's end are not read), a block before the window's first block
+ * (logical block max(0, T - window) / 64) is read through the global slot
+ * of its first global position, and logical block i from the window's first
+ * block on lives in slot A + (i mod ring_blocks).  The caller keeps a global
+ * position's block alive in its global slot when the ring moves past it
+ * (gives the ring slot a new block); kv_append_ext with the same record
+ * writes through the ring slots.  A global query (T - 1 a global position)
+ * with T > window would need keys the ring no longer holds: that sequence
+ * is refused on the device (ATTN_ERR_BAD_SEQLEN from attn_decode_last_error,
+ * zero output row).  ring_blocks > 0 requires window > 0, ring_blocks * 64 >=
  * window + 63 (the ring holds every block a window can touch) and
  * A + ring_blocks <= max_blocks_per_seq; T is then not limited by the table
  * width.  All zero: full causal attention, identity table (attn_decode_gqa).

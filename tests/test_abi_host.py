@@ -117,8 +117,9 @@ def test_visibility_struct_layout_matches_header(tmp_path):
 
 
 def test_global_set_validated_on_the_host():
-    """An explicit global set with sink tokens or a ring, a null set, or more
-    than 64 positions is refused before any launch."""
+    """An explicit global set with sink tokens, with a ring that does not fit
+    the table row after its global slots, a null set, or more than 64
+    positions is refused before any launch."""
     lib = attn.load()
     p = ctypes.c_void_p(16)      # never dereferenced: validation fails first
     g = ctypes.c_void_p(64)
@@ -128,7 +129,9 @@ def test_global_set_validated_on_the_host():
                                        ctypes.byref(vis), None, 4, 8, attn.BF16)
     V = attn.Visibility
     assert call(V(10, 4, 0, g.value, 2)) == attn.ERR_ARG        # with sink tokens
-    assert call(V(64, 0, 3, g.value, 2)) == attn.ERR_ARG        # with a ring
+    assert call(V(64, 0, 3, g.value, 2)) == attn.ERR_ARG        # 2 global + 3 ring slots > 4
+    assert call(V(64, 4, 2, g.value, 2)) == attn.ERR_ARG        # sink tokens and a ring
+    assert call(V(200, 0, 2, g.value, 2)) == attn.ERR_ARG       # ring shorter than the window
     assert call(V(10, 0, 0, None, 2)) == attn.ERR_ARG           # no positions
     assert call(V(10, 0, 0, g.value, -1)) == attn.ERR_ARG       # negative count
     assert call(V(10, 0, 0, ctypes.c_void_p(66).value, 2)) == attn.ERR_ARG   # misaligned

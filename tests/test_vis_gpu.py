@@ -209,3 +209,152 @@ def test_global_positions_host_validation(lib):
         with pytest.raises(lib.AttnError) as e:
             lib.decode_gqa_ext(*args, **kw)
         assert e.value.status == status, kw
+
+
+def _global_ring_table(rng, B, lens, window, ring, rows, n_phys):
+    """Per sequence: n_g global slots + `ring` ring slots.  Global slot k
+    names one physical block per distinct block of the positions (slots of
+    positions sharing a block share it; pads stay -1), ring slot n_g + i %
+    ring names the block of logical block i for the blocks the window
+    reaches.  All blocks are distinct; the pool holds spares nothing names."""
+    n_g = len(rows[0])
+    table = np.full((B, n_g + ring), -1, dtype=np.int32)
+    perm = iter(rng.permutation(n_phys).tolist())
+    for b in range(B):
+        by_block = {}
+        for k, pos in enumerate(rows[b]):
+            if pos < 0:
+                continue
+            if pos // 64 not in by_block:
+                by_block[pos // 64] = next(perm)
+            table[b, k] = by_block[pos // 64]
+        for r in range(ring):
+            table[b, n_g + r] = next(perm)
+    return torch.from_numpy(table)
+
+
+GLOBAL_RING_CASES = [
+    # (H_q, H_kv, d, lens, rows, window, ring)
+    (16, 2, 128, [9000, 640, 151, 20000],
+     [[0, 5, 70, 3000, 8990], [3, 600, -1, -1, -1], [0, 149, -1, -1, -1],
+      [64, 65, 19000, 19950, -1]], 150, 4),
+    (32, 1, 128, [5000, 130], [[1, 2, 4700, 4900], [129, -1, -1, -1]], 400, 8),
+    (24, 4, 256, [3000, 2999], [[10, 1300, 2900, -1], [0, 2000, 2950, -1]], 100, 3),
+]
+
+
+@pytest.mark.parametrize("path", [0, 1, 2], ids=["cuda_core", "tcgen05", "tcgen05_m64"])
+@pytest.mark.parametrize("H_q,H_kv,d,lens,rows,window,ring", GLOBAL_RING_CASES,
+                         ids=[f"q{c[0]}_kv{c[1]}_d{c[2]}_w{c[5]}_r{c[6]}"
+                              for c in GLOBAL_RING_CASES])
+def test_global_set_with_ring_matches_oracle(lib, path, H_q, H_kv, d, lens, rows, window,
+                                             ring):
+    """A window layer that also keeps an explicit global set in a ring table
+    (attention-head §3): global slots ahead of the ring, sequences far longer
+    than the row; every kernel vs the oracle through the same table."""
+    B = len(lens)
+    n_phys = B * (len(rows[0]) + ring) + 4
+    q, k, v, _ = _inputs(7500 + H_q + d, B, H_q, H_kv, d, n_phys, 1)
+    table = _global_ring_table(np.random.default_rng(7500 + d), B, lens, window, ring, rows,
+                               n_phys)
+    gp = torch.tensor(rows, dtype=torch.int32)
+    scale = 1.0 / np.sqrt(d)
+    ref = orc.decode_gqa_vis(q, k, v, np.asarray(lens, dtype=np.int32), table.numpy(), scale,
+                             window=window, ring=ring, global_pos=gp.numpy())
+    lib.set_gqa_path(path)
+    try:
+        got = lib.decode_gqa_ext(q.to(DEV), k.to(DEV), v.to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                 table.to(DEV), scale, window=window, ring_blocks=ring,
+                                 global_pos=gp.to(DEV))
+        assert lib.last_error() == lib.OK
+    finally:
+        lib.set_gqa_path(-1)
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16,
+                  f"global set + ring, path {path}")
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["cuda_core", "tcgen05"])
+def test_global_query_with_ring_is_flagged(lib, path):
+    """A global query (T - 1 in G) with T > window needs history the ring no
+    longer holds: that sequence is refused on the device (bad sequence
+    length, zero output row) and the others are served."""
+    lens, rows, window, ring = [3000, 1000], [[5, 2999], [7, -1]], 200, 5
+    H_q, H_kv, d = 16, 2, 128
+    B = len(lens)
+    n_phys = B * (2 + ring) + 2
+    q, k, v, _ = _inputs(7600 + path, B, H_q, H_kv, d, n_phys, 1)
+    table = _global_ring_table(np.random.default_rng(7600), B, lens, window, ring, rows, n_phys)
+    gp = torch.tensor(rows, dtype=torch.int32)
+    ref1 = orc.decode_gqa_vis(q[1:], k, v, np.asarray(lens[1:], dtype=np.int32),
+                              table[1:].numpy(), 0.1, window=window, ring=ring,
+                              global_pos=gp[1:].numpy())
+    lib.set_gqa_path(path)
+    try:
+        got = lib.decode_gqa_ext(q.to(DEV), k.to(DEV), v.to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                 table.to(DEV), 0.1, window=window, ring_blocks=ring,
+                                 global_pos=gp.to(DEV))
+        assert lib.last_error() == lib.ERR_BAD_SEQLEN
+        assert lib.last_error() == lib.OK            # reading clears it
+    finally:
+        lib.set_gqa_path(-1)
+    got = got.float().cpu()
+    assert torch.count_nonzero(got[0]) == 0
+    assert_parity(got[1:].numpy(), ref1, torch.bfloat16, f"served rows, path {path}")
+
+
+def test_global_set_ring_append_then_decode_matches_full_cache(lib):
+    """Append every token of two sequences one step at a time into a ring
+    table with global slots, the caller keeping a global position's block
+    alive (the ring slot gets a fresh block when it comes round): the final
+    decode equals the oracle over the full, never-evicted cache with the
+    same window and global set."""
+    T, window, ring, H_kv, H_q, d = 900, 100, 3, 2, 8, 64
+    rows = [[0, 5, 300, 301, 700], [64, 890, -1, -1, -1]]
+    B, n_g = 2, len(rows[0])
+    g = torch.Generator().manual_seed(7700)
+    k_all = torch.randn((B, T, H_kv, d), generator=g).bfloat16()
+    v_all = torch.randn((B, T, H_kv, d), generator=g).bfloat16()
+    q = torch.randn((B, H_q, d), generator=g).bfloat16()
+    n_phys = 32
+    free = list(range(n_phys))[::-1]
+    table = np.full((B, n_g + ring), -1, dtype=np.int32)
+    pinned = [set() for _ in range(B)]
+    kc = torch.zeros((n_phys, H_kv, BLOCK_SIZE, d), dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    td = torch.from_numpy(table).to(DEV)
+    gp = torch.tensor(rows, dtype=torch.int32, device=DEV)
+    kd, vd = k_all.to(DEV), v_all.to(DEV)
+    for t in range(T):
+        if t % 64 == 0:                       # a new block: the cache manager's step
+            i = t // 64
+            for b in range(B):
+                r = n_g + i % ring
+                old = table[b, r]
+                if old < 0 or old in pinned[b]:
+                    table[b, r] = free.pop()  # fresh block; a pinned one stays alive
+                for kk, pos in enumerate(rows[b]):
+                    if pos >= 0 and pos // 64 == i:
+                        table[b, kk] = table[b, r]
+                        pinned[b].add(int(table[b, r]))
+            td.copy_(torch.from_numpy(table))
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        lib.kv_append_ext(kd[:, t].contiguous(), vd[:, t].contiguous(), kc, vc, pos, td,
+                          window=window, ring_blocks=ring, global_pos=gp)
+    assert lib.last_error() == lib.OK
+    lens = torch.full((B,), T, dtype=torch.int32, device=DEV)
+    got = lib.decode_gqa_ext(q.to(DEV), kc, vc, lens, td, 0.15, window=window,
+                             ring_blocks=ring, global_pos=gp)
+    assert lib.last_error() == lib.OK
+    nb = (T + 63) // 64
+    full_k = torch.zeros((B * nb, H_kv, BLOCK_SIZE, d), dtype=torch.bfloat16)
+    full_v = torch.zeros_like(full_k)
+    for b in range(B):
+        for t in range(T):
+            full_k[b * nb + t // 64, :, t % 64] = k_all[b, t]
+            full_v[b * nb + t // 64, :, t % 64] = v_all[b, t]
+    full_table = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
+    ref = orc.decode_gqa_vis(q, full_k, full_v, np.array([T] * B, dtype=np.int32), full_table,
+                             0.15, window=window, global_pos=np.asarray(rows, dtype=np.int32))
+    assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, "global set ring append")
