@@ -43,12 +43,14 @@
 //
 // FP8 latent cache (template flag F8): rows stored as OCP E4M3 codes with one
 // fp32 scale per row (value = code value x scale).  The TMA loads each tile's
-// code boxes and 64 row scales into a raw stage; warp 3 widens the codes to
-// bf16 exactly (every E4M3 value is a bf16 value) into the same swizzled
-// stage layout the MMAs read, so the tensor-core path is unchanged.  The row
-// scale multiplies the token's score column (scores) and its probability
-// before the hi/lo split (values); the softmax sums use the unscaled
-// probabilities.
+// code boxes and 64 row scales into a raw stage; a widening warpgroup (warps
+// 12-15) converts the codes to f16 exactly (every E4M3 value is an f16
+// value) into the same swizzled stage layout the MMAs read, and this variant
+// runs its MMAs on f16 operands: the query is converted to f16 once per
+// sequence (exact within f16's range) and P is one f16 operand (11
+// significant bits, so no P_lo product).  The row scale multiplies the
+// token's score column (scores) and its probability before the P V product
+// (values); the softmax sums use the unscaled probabilities.
 #include <mutex>
 
 #include "attn_decode.h"
@@ -65,7 +67,8 @@ constexpr int kMlaCBox = 64 * 128;         // [64 tokens][64 cols] bf16
 constexpr int kMlaMaxBoxes = 5;
 constexpr int kMlaPrefetch = 4;            // blocks pulled into L2 ahead of the ring
 constexpr int kMlaStageBytes = kMlaMaxBoxes * kMlaCBox;
-constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA/widening, 4-11 softmax
+constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA, 4-11 softmax
+constexpr int kMlaThreadsF8 = 512;         // fp8: + warps 12-15 widening the codes
 constexpr int kSoftThreads = 256;
 constexpr int kPBytes = kMlaH * 128;       // one P half: [128 heads][64 tokens] bf16
 constexpr int kXBytes = kMlaH * 64 * 4;    // exchange buffer: 16 chunks x [128 rows] x 16 B
@@ -126,7 +129,7 @@ struct MlaParams {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(kMlaThreads, 1)
+__global__ void __launch_bounds__(F8 ? kMlaThreadsF8 : kMlaThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
     using C = MlaCfg<F8>;
     constexpr int kMlaStages = C::kStages;
@@ -166,12 +169,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         mbar_init(&bars->q_full, kSoftThreads);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMlaStages; ++s) {
-            mbar_init(&bars->c_full[s], F8 ? 32 : 1);   // widening warp, or the TMA
+            mbar_init(&bars->c_full[s], F8 ? 128 : 1);  // widening warps, or the TMA
             mbar_init(&bars->c_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->raw_full[s], 1);
-            mbar_init(&bars->raw_empty[s], 32);
+            mbar_init(&bars->raw_empty[s], 128);
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->s_free, kSoftThreads);
@@ -195,7 +198,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
     cluster_sync_all();   // the peer's barriers exist before any remote arrive
     const uint32_t tmem = bars->tmem_base;
 
+    // fp8: 16 warps; the launch's 512 x 128 registers are re-split so the
+    // softmax warpgroups keep 176 (TMA/MMA warpgroup 80, widening 80:
+    // 128 x 80 + 256 x 176 + 128 x 80 = 65536), each at the top of its role.
     if (warp == 0) {
+        if constexpr (F8) regs_decrease<80>();
         // ============================================================ TMA
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
@@ -264,6 +271,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         }
         __syncwarp();
     } else if (warp == 1 || warp == 2) {
+        if constexpr (F8) regs_decrease<80>();
         // ============================================================ MMA
         // Lane 0 of warp 1 issues S(n) = Q C(n)^T for every tile in order,
         // lane 0 of warp 2 issues O += P(i) C(i); each waits only on its own
@@ -293,7 +301,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 }
             };
             if (warp == 1) {
-                constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
+                constexpr uint32_t idesc_s =
+                    F8 ? umma_idesc_f16(128, 64, 0, 0) : umma_idesc_bf16(128, 64, 0, 0);
                 TileCursor cs;
                 cs.init(pa, lo, hi, first_seq, first_base);
                 int seg_s = 0;
@@ -320,14 +329,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                     cs.next();
                 }
             } else {
-                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 256, 0, 1);
+                constexpr uint32_t idesc_pv =
+                    F8 ? umma_idesc_f16(128, 256, 0, 1) : umma_idesc_bf16(128, 256, 0, 1);
                 const uint32_t p_base = smem_u32(sP);
                 TileCursor cv;
                 cv.init(pa, lo, hi, first_seq, first_base);
                 int seg_v = 0;
                 for (int i = 0; i < n_tiles; ++i) {
-                    // O += P_hi C + P_lo C; a segment's first P V overwrites O
-                    // once the previous segment's output has been read.
+                    // O += P_hi C + P_lo C (fp8: O += P C, P in f16); a
+                    // segment's first P V overwrites O once the previous
+                    // segment's output has been read.
                     const bool first = cv.t == 0;
                     if (!wait(&bars->p_full, (uint32_t)(i & 1))) break;
                     if (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))
@@ -341,7 +352,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                         const uint64_t a_hi = umma_desc_sw128(p_base + k * 32, 16, 1024);
                         const uint64_t a_lo = umma_desc_sw128(p_base + kPBytes + k * 32, 16, 1024);
                         umma_bf16(tmem + kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
-                        umma_bf16(tmem + kTmemO, a_lo, b, idesc_pv, 1);
+                        if constexpr (!F8) umma_bf16(tmem + kTmemO, a_lo, b, idesc_pv, 1);
                     }
                     umma_commit(&bars->c_empty[st]);
                     umma_commit(&bars->pv_done);
@@ -355,16 +366,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         }
         __syncwarp();
     } else if (warp == 3) {
+        if constexpr (F8) regs_decrease<80>();
+    } else if (F8 && warp >= 12) {
         // ================================================ fp8 -> bf16 widening
-        // An E4M3 code's 7 magnitude bits, shifted so the 4-bit exponent and
-        // 3-bit mantissa sit at the top of an fp32's exponent and mantissa
-        // fields, are the fp32 pattern of value x 2^-120 (subnormal codes
-        // included: they become fp32 subnormals); one exact multiply by 2^120
-        // gives the value, whose top 16 bits are its bf16 pattern (at most 4
-        // significant bits, so nothing is rounded).
+        regs_decrease<80>();
+        // The codes are widened to f16 with the hardware conversion (exact:
+        // every E4M3 value is an f16 value); the fp8 variant runs its MMAs on
+        // f16 operands.
         if constexpr (F8) {
-            TileCursor cur;
-            cur.init(pa, lo, hi, first_seq, first_base);
+            const int wt = tid - 384;            // widening thread 0..127
             for (int tile = 0; tile < n_tiles; ++tile) {
                 const int rs = tile % C::kRawStages, st = tile % kMlaStages;
                 if (!__all_sync(0xffffffffu,
@@ -379,37 +389,32 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                     break;
                 const unsigned char *raw = smem + C::kOffRaw + rs * C::kRawStageBytes;
                 unsigned char *dst = sC + st * kMlaStageBytes;
-                for (int idx = lane; idx < nbox * 512; idx += 32) {
-                    const int bx = idx >> 9, t = (idx >> 3) & 63, c = idx & 7;
-                    const uint2 codes =
-                        *reinterpret_cast<const uint2 *>(raw + bx * kRawBox + t * 64 + c * 8);
-                    uint32_t w[4];
+                // item: 16 codes (group g of row t of box bx) -> 2 swizzled chunks
+                for (int idx = wt; idx < nbox * 256; idx += 128) {
+                    const int bx = idx >> 8, t = (idx >> 2) & 63, g = idx & 3;
+                    const uint4 codes =
+                        *reinterpret_cast<const uint4 *>(raw + bx * kRawBox + t * 64 + g * 16);
+                    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+                    uint32_t w[8];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t src = k < 2 ? codes.x : codes.y;
-                        const uint32_t u0 = (src >> (16 * (k & 1))) & 0xFFu;
-                        const uint32_t u1 = (src >> (16 * (k & 1) + 8)) & 0xFFu;
-                        const float f0 = __uint_as_float(((u0 & 0x7Fu) << 20) | ((u0 & 0x80u) << 24)) *
-                                         0x1p120f;
-                        const float f1 = __uint_as_float(((u1 & 0x7Fu) << 20) | ((u1 & 0x80u) << 24)) *
-                                         0x1p120f;
-                        w[k] = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
-                    }
-                    *reinterpret_cast<uint4 *>(dst + bx * kMlaCBox + t * 128 + ((c ^ (t & 7)) * 16)) =
+                    for (int k = 0; k < 4; ++k) e4m3x4_to_f16x4(cw[k], w[2 * k], w[2 * k + 1]);
+                    unsigned char *drow = dst + bx * kMlaCBox + t * 128;
+                    *reinterpret_cast<uint4 *>(drow + (((2 * g) ^ (t & 7)) * 16)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(drow + (((2 * g + 1) ^ (t & 7)) * 16)) =
+                        make_uint4(w[4], w[5], w[6], w[7]);
                 }
                 const float *rsc = reinterpret_cast<const float *>(raw + kMlaMaxBoxes * kRawBox);
                 float *ssc = reinterpret_cast<float *>(smem + C::kOffScale) + st * 64;
-                ssc[lane] = rsc[lane];
-                ssc[lane + 32] = rsc[lane + 32];
+                if (wt < 64) ssc[wt] = rsc[wt];
                 fence_proxy_async_smem();      // the MMAs read the widened stage
                 mbar_arrive(&bars->raw_empty[rs]);
                 mbar_arrive(&bars->c_full[st]);
-                cur.next();
             }
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 12) {
         // ============================================ Q load, softmax, epilogue
+        if constexpr (F8) regs_increase<176>();
         // Two threads per head row: warps w and w + 4 share TMEM lanes
         // 32*(w%4) .. +31; half h takes tokens [32h, 32h+32) of each tile and
         // output columns [128h, 128h+128) of this CTA's 256.
@@ -445,6 +450,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 for (int j = 0; j < 8; ++j) {
                     const uint4 v = __ldg(src + j);
                     r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+                }
+                if constexpr (F8) {
+                    // f16 operands: the query pairs converted (exact within f16's range)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = bf16x2_to_f16x2(r[j]);
                 }
                 tmem_st32(trow + kTmemQ + 32 * bx, r);
             }
@@ -587,24 +597,37 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             if (i >= 1 && !all(mbar_wait(&bars->pv_done, (uint32_t)((i - 1) & 1),
                                          p.timeout_ns, p.err, abort_flag)))
                 break;
+            if constexpr (F8) {
+                // one f16 P (11 significant bits): no P_lo product needed
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {          // 8 tokens per 16-byte chunk
-                uint32_t hi_w[4], lo_w[4];
+                for (int c = 0; c < 4; ++c) {      // 8 tokens per 16-byte chunk
+                    uint32_t w[4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float a = s[8 * c + 2 * k], bb = s[8 * c + 2 * k + 1];
-                    hi_w[k] = pack_bf16x2(a, bb);
-                    const float2 r = __fadd2_rn(
-                        make_float2(a, bb),
-                        make_float2(-__uint_as_float(hi_w[k] << 16),
-                                    -__uint_as_float(hi_w[k] & 0xFFFF0000u)));
-                    lo_w[k] = pack_bf16x2(r.x, r.y);
+                    for (int k = 0; k < 4; ++k)
+                        w[k] = pack_f16x2(s[8 * c + 2 * k], s[8 * c + 2 * k + 1]);
+                    const int off = ((4 * h + c) ^ (row & 7)) * 16;
+                    *reinterpret_cast<uint4 *>(prow + off) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                const int off = ((4 * h + c) ^ (row & 7)) * 16;
-                *reinterpret_cast<uint4 *>(prow + off) =
-                    make_uint4(hi_w[0], hi_w[1], hi_w[2], hi_w[3]);
-                *reinterpret_cast<uint4 *>(prow + kPBytes + off) =
-                    make_uint4(lo_w[0], lo_w[1], lo_w[2], lo_w[3]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {          // 8 tokens per 16-byte chunk
+                    uint32_t hi_w[4], lo_w[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float a = s[8 * c + 2 * k], bb = s[8 * c + 2 * k + 1];
+                        hi_w[k] = pack_bf16x2(a, bb);
+                        const float2 r = __fadd2_rn(
+                            make_float2(a, bb),
+                            make_float2(-__uint_as_float(hi_w[k] << 16),
+                                        -__uint_as_float(hi_w[k] & 0xFFFF0000u)));
+                        lo_w[k] = pack_bf16x2(r.x, r.y);
+                    }
+                    const int off = ((4 * h + c) ^ (row & 7)) * 16;
+                    *reinterpret_cast<uint4 *>(prow + off) =
+                        make_uint4(hi_w[0], hi_w[1], hi_w[2], hi_w[3]);
+                    *reinterpret_cast<uint4 *>(prow + kPBytes + off) =
+                        make_uint4(lo_w[0], lo_w[1], lo_w[2], lo_w[3]);
+                }
             }
             tc_fence_after();
             if (__any_sync(0xffffffffu, rescale)) {   // rows without a new max use alpha = 1
@@ -723,7 +746,7 @@ int max_resident_clusters(int num_sms) {
     if (cache[dev] == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(num_sms);
-        cfg.blockDim = dim3(kMlaThreads);
+        cfg.blockDim = dim3(F8 ? kMlaThreadsF8 : kMlaThreads);
         cfg.dynamicSmemBytes = MlaCfg<F8>::kSmem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -754,7 +777,7 @@ int mla_launch(const MlaParams &mp, const CUtensorMap &tc, int clusters, cudaStr
         return ATTN_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters);
-    cfg.blockDim = dim3(kMlaThreads);
+    cfg.blockDim = dim3(F8 ? kMlaThreadsF8 : kMlaThreads);
     cfg.dynamicSmemBytes = MlaCfg<F8>::kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

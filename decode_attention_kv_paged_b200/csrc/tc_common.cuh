@@ -184,6 +184,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// Two fp32 -> packed f16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// A bf16x2 pair to f16x2 (exact for values inside f16's normal range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+    return pack_f16x2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+}
+
 // Round an fp32 (finite) to the nearest bf16, ties to even, with integer
 // operations only; returns the 16-bit pattern.
 __device__ __forceinline__ uint32_t bf16_rne_bits(float x) {
@@ -220,6 +232,24 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, i
            | (1u << 10)                  // B format: bf16
            | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f16 with f16 A/B and fp32 accumulator.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4)                     // D format: f32 (A, B format 0: f16)
+           | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Four OCP E4M3 codes (bytes of w, lowest first) to two f16x2 words with the
+// hardware conversion (exact: every E4M3 value is an f16 value).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
