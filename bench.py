@@ -384,9 +384,8 @@ def kernel_name(attn, cfg):
     """The main kernel a decode call of this workload launches."""
     if isinstance(cfg, W.MLAConfig):
         return "mla_decode_kernel"
-    if cfg.kv_fp8:
-        return "gqa_split_kernel"
-    _, _, path = attn.gqa_config(cfg.B, cfg.H_q, cfg.H_kv, cfg.d, cfg.dtype)
+    _, _, path = attn.gqa_config(cfg.B, cfg.H_q, cfg.H_kv, cfg.d,
+                                 "fp8" if cfg.kv_fp8 else cfg.dtype)
     return {0: "gqa_split_kernel", 1: "gqa_tc128_kernel", 2: "gqa_tc_kernel"}[path]
 
 
@@ -574,7 +573,8 @@ def config_entry(attn, cfg, dev, seed, K, warmup, min_s, pk, clk=None):
 # the head-sharing sweep, the ragged 24/4/256 shape full and with w=4096, the
 # DeepSeek-V2 MLA shape; then the window/global/ring and fp8-cache variants.
 PER_CONFIG = [W.TINY, W.LLAMA3_8B, *W.SWEEP, W.RAGGED_FULL, W.RAGGED_WINDOW, W.MLA_DSV2,
-              W.LLAMA3_8B_FP8, W.MLA_DSV2_FP8, W.RAGGED_WINDOW_SINK, W.RAGGED_WINDOW_RING,
+              W.LLAMA3_8B_FP8, W.MQA_B8_FP8, W.MLA_DSV2_FP8, W.RAGGED_WINDOW_SINK,
+              W.RAGGED_WINDOW_RING,
               W.RAGGED_WINDOW_GLOBAL]
 
 

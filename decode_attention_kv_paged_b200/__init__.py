@@ -19,7 +19,7 @@ BLOCK_SIZE = 64
 
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BAD_BLOCK, \
     ERR_BAD_SEQLEN = 0, -1, -2, -3, -4, -5, -6
-F32, BF16 = 0, 1
+F32, BF16, FP8_E4M3 = 0, 1, 2
 
 # Every entry point include/attn_decode.h declares.
 C_SYMBOLS = (
@@ -411,9 +411,10 @@ def plan(seq_lens, units_per_seq, window, max_blocks, num_ctas, stream=None):
 def gqa_config(B, H_q, H_kv, d, dtype=torch.bfloat16):
     """(num_ctas, heads_per_cta, path) the GQA call uses for this problem;
     path 0 = CUDA-core kernel, 1 = M=128 tensor-core kernel, 2 = M=64
-    tensor-core kernel."""
+    tensor-core kernel.  dtype "fp8" asks about decode_gqa_fp8."""
     n, h, pth = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    rc = load().attn_decode_gqa_config(B, H_q, H_kv, d, _dtype_code(dtype),
+    code = FP8_E4M3 if dtype == "fp8" else _dtype_code(dtype)
+    rc = load().attn_decode_gqa_config(B, H_q, H_kv, d, code,
                                        ctypes.byref(n), ctypes.byref(h),
                                        ctypes.byref(pth))
     _check(rc, "attn_decode_gqa_config")

@@ -188,6 +188,21 @@ static bool use_tc128(int d, int HC) {
     return tl_gqa_path != 2 && gqa_tc128_supported(d, HC);
 }
 
+// Whether an fp8 call runs the M = 128 tensor-core kernel (codes widened to
+// f16 on the chip) rather than the CUDA-core kernel: by default for groups of
+// kTcFp8MinGroup heads or more, where the CUDA-core kernel splits the group
+// into 8-head chunks and reads every tile once per chunk (measured on B200,
+// T = 32768: MQA at B = 8 168 us on CUDA cores vs 68 us on tensor cores, at
+// B = 1 41 vs 29 us; G = 4 at B = 8 207 vs 318 us, MHA 633 vs 1223 us);
+// path 1 forces it wherever it applies, path 0 forces the CUDA cores (and
+// path 2, the M = 64 kernel, has no fp8 form).
+constexpr int kTcFp8MinGroup = 16;
+static bool use_tc_fp8(int G, int d) {
+    if (tl_gqa_path == 0 || tl_gqa_path == 2) return false;
+    if (!gqa_tc128_fp8_supported(d, G)) return false;
+    return tl_gqa_path == 1 || G >= kTcFp8MinGroup;
+}
+
 // Query heads per CTA for a group of G: the largest instantiated divisor.
 static int heads_per_cta(int G) {
     static const int options[] = {8, 6, 4, 3, 2, 1};
@@ -292,14 +307,20 @@ int attn_decode_last_error(void *stream) {
 int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype, int *num_ctas,
                            int *heads, int *path) {
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv || !valid_head_dim(d) ||
-        (dtype != ATTN_F32 && dtype != ATTN_BF16))
+        (dtype != ATTN_F32 && dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3))
         return ATTN_ERR_ARG;
     DeviceState *st;
     int rc = device_state(&st);
     if (rc) return rc;
     const int G = H_q / H_kv;
-    const bool tc = use_tc_path(G, d, dtype);
     if (num_ctas) *num_ctas = tl_num_ctas > 0 ? tl_num_ctas : st->num_sms;
+    if (dtype == ATTN_FP8_E4M3) {
+        const bool tc8 = use_tc_fp8(G, d);
+        if (heads) *heads = tc8 ? gqa_tc128_fp8_heads_per_cta(G) : heads_per_cta(G);
+        if (path) *path = tc8 ? 1 : 0;
+        return ATTN_OK;
+    }
+    const bool tc = use_tc_path(G, d, dtype);
     const int hc = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
     if (heads) *heads = hc;
     if (path) *path = tc ? (use_tc128(d, hc) ? 1 : 2) : 0;
@@ -337,9 +358,10 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     cudaStream_t s = (cudaStream_t)stream;
 
     const int G = H_q / H_kv;
-    // The fp8 cache is read by the CUDA-core kernel for every group size.
-    const bool tc = !fp8 && use_tc_path(G, d, dtype);
-    const int HC = tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G);
+    const bool tc8 = fp8 && use_tc_fp8(G, d);
+    const bool tc = tc8 || (!fp8 && use_tc_path(G, d, dtype));
+    const int HC = tc8 ? gqa_tc128_fp8_heads_per_cta(G)
+                       : (tc ? gqa_tc_heads_per_cta(G) : heads_per_cta(G));
     const int n_hc = G / HC;
     const long long units_total = (long long)B * H_kv * n_hc;
     // No more CTAs than the work could possibly fill (units x table width).
@@ -350,7 +372,7 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     const long long slots = units_total + P;
 
     // The tensor-core kernels write one partial per head-group copy per slot.
-    const bool tc128 = tc && use_tc128(d, HC);
+    const bool tc128 = tc8 || (tc && use_tc128(d, HC));
     const int copies = tc ? (tc128 ? gqa_tc128_copies(HC) : gqa_tc_copies(HC)) : 1;
     const size_t o_bytes = align256((size_t)slots * copies * HC * d * sizeof(float));
     const size_t lse_bytes = align256((size_t)slots * copies * HC * sizeof(float));
@@ -394,7 +416,8 @@ static int decode_gqa_impl(const void *q, const void *k_cache, const void *v_cac
     const int bf16 = dtype == ATTN_BF16;
     cudaError_t e;
     if (tc) {
-        e = tc128 ? launch_gqa_tc128(L, d, HC) : launch_gqa_tc(L, d, HC);
+        e = tc8 ? launch_gqa_tc128_fp8(L, d, HC)
+                : (tc128 ? launch_gqa_tc128(L, d, HC) : launch_gqa_tc(L, d, HC));
         return cuda_status(e);
     }
     if (fp8) {

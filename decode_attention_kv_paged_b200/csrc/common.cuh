@@ -53,6 +53,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     (void)state;
 }
 
+// One arrival per warp (the barrier counts warps): the lanes' prior memory
+// operations are ordered before lane 0's arrival by the warp barrier, so one
+// release stands for the whole warp and the barrier word takes 1/32 of the
+// atomic traffic.  All 32 lanes must call it.
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar,
                                                       uint32_t bytes) {
     uint64_t state;

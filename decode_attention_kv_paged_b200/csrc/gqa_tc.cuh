@@ -31,6 +31,11 @@ cudaError_t launch_gqa_tc(const GqaLaunch &L, int d, int HC);
 bool gqa_tc128_supported(int d, int HC);
 int gqa_tc128_copies(int HC);
 cudaError_t launch_gqa_tc128(const GqaLaunch &L, int d, int HC);
+// Its fp8 variant (E4M3 K/V codes with per-row scales, widened to f16 on the
+// chip): the same shapes; HC = G, or 32 for groups that are multiples of 32.
+bool gqa_tc128_fp8_supported(int d, int G);
+int gqa_tc128_fp8_heads_per_cta(int G);
+cudaError_t launch_gqa_tc128_fp8(const GqaLaunch &L, int d, int HC);
 
 // 2-D tensor map over a row-major bf16 matrix [rows][cols] with 64-column,
 // box_rows-row boxes and 128-byte swizzle.

@@ -36,16 +36,28 @@
 namespace attn {
 
 constexpr int kT2Threads = 256;
+constexpr int kT2ThreadsF8 = 384;          // fp8: + warps 8-11 widening the codes
 constexpr int kT2Box = 64 * 128;           // [64 rows][64 cols] bf16, swizzled
 constexpr float kT2Rescale = 8.0f;         // lazy-rescale headroom, log2 units
 
-template <int D>
+template <int D, bool F8 = false>
 struct T2Cfg {
     static constexpr int kBoxes = D / 64;
-    static constexpr int kStageBytes = 2 * kBoxes * kT2Box;       // K then V
-    static constexpr int kStagesRaw = (227 * 1024 - 2048) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
-    static constexpr int kOffBar = kStages * kStageBytes;
+    static constexpr int kStageBytes = 2 * kBoxes * kT2Box;       // K then V (bf16 / f16)
+    // fp8: each stage also has a raw stage (K codes, V codes, K and V row
+    // scales) that the widening warps convert into it.
+    // The raw ring is the deeper one: the codes in flight from HBM are what
+    // keeps the memory system busy, the widened stages only feed the MMAs.
+    static constexpr int kRawBytes = F8 ? 2 * 64 * D + 512 : 0;
+    static constexpr int kScaleBytes = F8 ? 512 : 0;              // widened stage's scales
+    static constexpr int kStagesFit = (227 * 1024 - 4096) / kStageBytes;
+    static constexpr int kStages = F8 ? (D == 128 ? 3 : 4) : (kStagesFit > 6 ? 6 : kStagesFit);
+    static constexpr int kRawFit =
+        F8 ? (227 * 1024 - 4096 - kStages * (kStageBytes + kScaleBytes)) / kRawBytes : 0;
+    static constexpr int kRaw = kRawFit > 8 ? 8 : kRawFit;         // fp8 raw stages
+    static constexpr int kOffRaw = kStages * kStageBytes;
+    static constexpr int kOffScale = kOffRaw + kRaw * kRawBytes;
+    static constexpr int kOffBar = kOffScale + kStages * kScaleBytes;
     static constexpr int kSmem = kOffBar + 1024 + 1024;           // + alignment slack
     // TMEM columns: O [0, D), S 2 x 64, Q D/2 (bf16 pairs), P 2 x (hi 32, lo 32).
     static constexpr uint32_t kTmemO = 0;
@@ -55,11 +67,14 @@ struct T2Cfg {
     static constexpr uint32_t kTmemCols = 512;
     static_assert(kTmemP + 128 <= kTmemCols, "TMEM columns");
     static_assert(kStages >= 3, "stages");
+    static_assert(!F8 || kRaw >= 4, "raw stages");
     static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 struct T2Bars {
     uint64_t c_full[6], c_empty[6];
+    uint64_t raw_full[8], raw_empty[8];   // fp8: codes landed / widened
+    int raw_bad[8];                       // fp8: the stage's block id was invalid
     uint64_t q_full, q_empty;
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], pv_done[2];
@@ -75,11 +90,17 @@ static_assert(sizeof(T2Bars) <= 1024, "barrier block");
 
 // G: the call has an explicit global set (its masking code is compiled only
 // into that instantiation, keeping the common loop as tight as before).
-template <int D, int HCP, bool G>
-__global__ void __launch_bounds__(kT2Threads, 1)
+// F8: the cache holds OCP E4M3 codes with one fp32 scale per row (value =
+// code x scale); the codes are widened to f16 on the chip (exact) and the
+// MMAs run on f16 operands (query converted once per segment, exact within
+// f16's range; P one f16 operand of 11 significant bits, so no P_lo
+// product); the K row scale multiplies the token's score, the V row scale
+// its probability before the P V product (the softmax sums stay unscaled).
+template <int D, int HCP, bool G, bool F8>
+__global__ void __launch_bounds__(F8 ? kT2ThreadsF8 : kT2Threads, 1)
 gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const GqaParams p, int HC) {
-    using C = T2Cfg<D>;
+    using C = T2Cfg<D, F8>;
     constexpr int kCopies = 128 / HCP;      // copies of the head group in the rows
     constexpr int kTPC = 64 / kCopies;      // tokens per copy per tile (16 or 8)
     extern __shared__ unsigned char smem_raw[];
@@ -104,18 +125,22 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     if (tid == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&bars->c_full[s], 1);
+            mbar_init(&bars->c_full[s], F8 ? 4 : 1);     // widening warps, or the TMA
             mbar_init(&bars->c_empty[s], 1);
         }
-        mbar_init(&bars->q_full, 128);
+        for (int s = 0; s < C::kRaw; ++s) {
+            mbar_init(&bars->raw_full[s], 1);
+            mbar_init(&bars->raw_empty[s], 4);
+        }
+        mbar_init(&bars->q_full, 4);        // barriers count warps (one arrival each)
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
-            mbar_init(&bars->s_free[s], 128);
-            mbar_init(&bars->p_full[s], 128);
+            mbar_init(&bars->s_free[s], 4);
+            mbar_init(&bars->p_full[s], 4);
             mbar_init(&bars->pv_done[s], 1);
         }
-        mbar_init(&bars->o_free, 128);
+        mbar_init(&bars->o_free, 4);
         mbar_init(&bars->mma_final, 2);     // one commit per issuing thread
         bars->abort = 0;
         fence_barrier_init();
@@ -135,39 +160,63 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             TileCursor cur;
             cur.init(pa, lo, hi, first_seq, first_base);
             int tile = 0;
+            constexpr int kRing = F8 ? C::kRaw : C::kStages;   // the ring this thread fills
+            uint64_t *freed = F8 ? bars->raw_empty : bars->c_empty;
             while (!cur.done()) {
                 const int kvh = cur.w.unit / p.n_hc;
-                const int st = tile % C::kStages;
-                if (tile >= C::kStages &&
-                    !mbar_wait(&bars->c_empty[st], (uint32_t)(((tile - C::kStages) / C::kStages) & 1),
+                const int st = tile % kRing;
+                if (tile >= kRing &&
+                    !mbar_wait(&freed[st], (uint32_t)(((tile - kRing) / kRing) & 1),
                                p.timeout_ns, p.err, abort_flag))
                     break;
                 int phys = p.block_table[(size_t)cur.w.b * p.max_blocks +
                                          cur.table_slot_of_tile()];
-                if (phys < 0 || phys >= p.num_blocks) {
+                const bool bad = phys < 0 || phys >= p.num_blocks;
+                if (bad) {
                     raise_error(p.err, kErrBadBlock);
                     phys = p.num_blocks;                 // wholly out of bounds: zero fill
                 }
                 const int row = (phys * p.H_kv + kvh) * 64;
-                unsigned char *dst = sC + st * C::kStageBytes;
                 if constexpr (G) {
                     const int blk = cur.logical_block();
                     bars->gmask[st] = blk * 64 < cur.w.lo
                                           ? global_mask_thread(p.vis, cur.w.b, blk) : 0ull;
                 }
-                mbar_arrive_expect_tx(&bars->c_full[st], C::kStageBytes);
-                for (int j = 0; j < C::kBoxes; ++j) {
-                    tma_load_2d(dst + j * kT2Box, &tm_k, 64 * j, row, &bars->c_full[st], pol);
-                    tma_load_2d(dst + (C::kBoxes + j) * kT2Box, &tm_v, 64 * j, row,
-                                &bars->c_full[st], pol);
+                if constexpr (F8) {
+                    // codes and row scales into the raw stage (the widening
+                    // warps release it); a bad block is zeros, never read
+                    unsigned char *raw = smem + C::kOffRaw + st * C::kRawBytes;
+                    bars->raw_bad[st] = bad ? 1 : 0;
+                    if (bad) {
+                        mbar_arrive(&bars->raw_full[st]);
+                    } else {
+                        const size_t off = (size_t)row * D;
+                        mbar_arrive_expect_tx(&bars->raw_full[st], C::kRawBytes);
+                        bulk_load(raw, static_cast<const uint8_t *>(p.k_cache) + off, 64 * D,
+                                  &bars->raw_full[st], pol);
+                        bulk_load(raw + 64 * D, static_cast<const uint8_t *>(p.v_cache) + off,
+                                  64 * D, &bars->raw_full[st], pol);
+                        bulk_load(raw + 128 * D, p.k_scale + row, 256, &bars->raw_full[st], pol);
+                        bulk_load(raw + 128 * D + 256, p.v_scale + row, 256, &bars->raw_full[st],
+                                  pol);
+                    }
+                } else {
+                    unsigned char *dst = sC + st * C::kStageBytes;
+                    mbar_arrive_expect_tx(&bars->c_full[st], C::kStageBytes);
+                    for (int j = 0; j < C::kBoxes; ++j) {
+                        tma_load_2d(dst + j * kT2Box, &tm_k, 64 * j, row, &bars->c_full[st], pol);
+                        tma_load_2d(dst + (C::kBoxes + j) * kT2Box, &tm_v, 64 * j, row,
+                                    &bars->c_full[st], pol);
+                    }
                 }
                 cur.next();
                 ++tile;
             }
             // Every issued load must have landed before the CTA exits.
-            for (int t = tile - C::kStages < 0 ? 0 : tile - C::kStages; t < tile; ++t)
-                mbar_wait(&bars->c_full[t % C::kStages], (uint32_t)((t / C::kStages) & 1),
-                          p.timeout_ns, p.err, nullptr);
+            uint64_t *landed = F8 ? bars->raw_full : bars->c_full;
+            for (int t = tile - kRing < 0 ? 0 : tile - kRing; t < tile; ++t)
+                mbar_wait(&landed[t % kRing], (uint32_t)((t / kRing) & 1), p.timeout_ns, p.err,
+                          nullptr);
         }
         __syncwarp();
     } else if (warp == 1 || warp == 2) {
@@ -201,7 +250,8 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
             };
             if (warp == 1) {
-                constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
+                constexpr uint32_t idesc_s =
+                    F8 ? umma_idesc_f16(128, 64, 0, 0) : umma_idesc_bf16(128, 64, 0, 0);
                 TileCursor cs;
                 cs.init(pa, lo, hi, first_seq, first_base);
                 int seg_s = 0;
@@ -228,7 +278,8 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     cs.next();
                 }
             } else {
-                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
+                constexpr uint32_t idesc_pv =
+                    F8 ? umma_idesc_f16(128, D, 0, 1) : umma_idesc_bf16(128, D, 0, 1);
                 TileCursor cv;
                 cv.init(pa, lo, hi, first_seq, first_base);
                 int seg_v = 0;
@@ -247,7 +298,8 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         const uint64_t b = umma_desc_sw128(vst + ks * 2048, kT2Box, 1024);
                         umma_bf16_ts(tmem + C::kTmemO, pb + 8 * ks, b, idesc_pv,
                                      !(first && ks == 0));
-                        umma_bf16_ts(tmem + C::kTmemO, pb + 32 + 8 * ks, b, idesc_pv, 1);
+                        if constexpr (!F8)
+                            umma_bf16_ts(tmem + C::kTmemO, pb + 32 + 8 * ks, b, idesc_pv, 1);
                     }
                     umma_commit(&bars->c_empty[st]);
                     umma_commit(&bars->pv_done[i & 1]);
@@ -260,7 +312,66 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_wait(&bars->mma_final, 0, p.timeout_ns, p.err, nullptr);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (F8 && warp >= 8) {
+        // ============================================= fp8 -> f16 widening
+        // Each item: 16 codes of one row of K or V -> two 16-byte chunks of
+        // the row's swizzled f16 box (the layout the TMA gives bf16 tiles);
+        // the hardware conversion is exact (every E4M3 value is an f16).
+        if constexpr (F8) {
+            const int wt = tid - 256;                 // widening thread 0..127
+            constexpr int kGroups = D / 16;           // 16-code groups per row
+            for (int tile = 0; tile < n_tiles; ++tile) {
+                const int rs = tile % C::kRaw, st = tile % C::kStages;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&bars->raw_full[rs], (uint32_t)((tile / C::kRaw) & 1),
+                                          p.timeout_ns, p.err, abort_flag)))
+                    break;
+                if (tile >= C::kStages &&
+                    !__all_sync(0xffffffffu,
+                                mbar_wait(&bars->c_empty[st],
+                                          (uint32_t)(((tile - C::kStages) / C::kStages) & 1),
+                                          p.timeout_ns, p.err, abort_flag)))
+                    break;
+                const unsigned char *raw = smem + C::kOffRaw + rs * C::kRawBytes;
+                unsigned char *dst = sC + st * C::kStageBytes;
+                const bool bad = bars->raw_bad[rs] != 0;
+                // kGroups items per thread: all loads first, then convert and store
+                uint4 codes[kGroups];
+#pragma unroll
+                for (int k = 0; k < kGroups; ++k) {
+                    const int idx = wt + 128 * k;
+                    const int m = idx / (64 * kGroups), r = idx % (64 * kGroups);
+                    const int t = r / kGroups, g = r % kGroups;
+                    codes[k] = bad ? make_uint4(0u, 0u, 0u, 0u)
+                                   : *reinterpret_cast<const uint4 *>(raw + m * 64 * D + t * D +
+                                                                      16 * g);
+                }
+#pragma unroll
+                for (int k = 0; k < kGroups; ++k) {
+                    const int idx = wt + 128 * k;
+                    const int m = idx / (64 * kGroups), r = idx % (64 * kGroups);
+                    const int t = r / kGroups, g = r % kGroups;
+                    uint32_t w[8];
+                    e4m3x4_to_f16x4(codes[k].x, w[0], w[1]);
+                    e4m3x4_to_f16x4(codes[k].y, w[2], w[3]);
+                    e4m3x4_to_f16x4(codes[k].z, w[4], w[5]);
+                    e4m3x4_to_f16x4(codes[k].w, w[6], w[7]);
+                    unsigned char *drow = dst + (m * C::kBoxes + g / 4) * kT2Box + t * 128;
+                    const int c0 = 2 * (g % 4);
+                    *reinterpret_cast<uint4 *>(drow + ((c0 ^ (t & 7)) * 16)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(drow + (((c0 + 1) ^ (t & 7)) * 16)) =
+                        make_uint4(w[4], w[5], w[6], w[7]);
+                }
+                // row scales of the stage: K [0, 64), V [64, 128)
+                float *sc = reinterpret_cast<float *>(smem + C::kOffScale) + st * 128;
+                sc[wt] = bad ? 0.f : reinterpret_cast<const float *>(raw + 128 * D)[wt];
+                fence_proxy_async_smem();             // the MMAs read the widened stage
+                mbar_arrive_warp(&bars->raw_empty[rs]);
+                mbar_arrive_warp(&bars->c_full[st]);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
         // ================================================ softmax, epilogue
         // Row r = 32 q + lane lives in TMEM lane r: head r % HCP of copy
         // r / HCP.  Warp q reads the 16-token window [16 q, 16 q + 16) of S
@@ -311,10 +422,15 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         const uint4 v = active ? __ldg(src + 8 * bx + j) : make_uint4(0, 0, 0, 0);
                         r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
                     }
+                    if constexpr (F8) {
+                        // f16 operands: exact within f16's range
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) r[j] = bf16x2_to_f16x2(r[j]);
+                    }
                     tmem_st32(trow + C::kTmemQ + 32 * bx, r);
                 }
                 tc_fence_before();
-                mbar_arrive(&bars->q_full);
+                mbar_arrive_warp(&bars->q_full);
                 ++q_seg;
             }
             const int sb = i & 1;
@@ -325,7 +441,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             float w16[16];
             tmem_ld16(trow + C::kTmemS + 64 * sb + 16 * q4, w16);
             tc_fence_before();
-            mbar_arrive(&bars->s_free[sb]);
+            mbar_arrive_warp(&bars->s_free[sb]);
 
             // This lane's kTPC tokens: window positions [half kTPC, + kTPC).
             const int blk = cur.logical_block();
@@ -348,6 +464,20 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 float v = w16[j];
                 if constexpr (kTPC == 8) v = half ? w16[8 + j] : w16[j];
                 s[j] = v * p.scale_log2;
+            }
+            // fp8: this lane's tokens' K and V row scales, kept with the
+            // stage (armed for tile i until its P V: the wait returns at once
+            // and orders the widening warps' writes before the reads)
+            const float *tsc = nullptr;
+            if constexpr (F8) {
+                const int st = i % C::kStages;
+                if (!all(mbar_wait(&bars->c_full[st], (uint32_t)((i / C::kStages) & 1),
+                                   p.timeout_ns, p.err, abort_flag)))
+                    break;
+                tsc = reinterpret_cast<const float *>(smem + C::kOffScale) + st * 128 +
+                      (tok0 - blk * 64);
+#pragma unroll
+                for (int j = 0; j < kTPC; ++j) s[j] *= tsc[j];
             }
             if (tok0 + kTPC > T || (tok0 < lo_tok && (tok0 + kTPC > sink || gmask))) {
 #pragma unroll
@@ -380,12 +510,33 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 sum += s[j];
             }
             l_run += sum;
+            if constexpr (F8) {
+#pragma unroll
+                for (int j = 0; j < kTPC; ++j) s[j] *= tsc[64 + j];   // V row scales
+            }
 
             // P buffer i % 2 was last read by P V(i - 2).
             if (i >= 2 && !all(mbar_wait(&bars->pv_done[i & 1], (uint32_t)(((i >> 1) - 1) & 1),
                                          p.timeout_ns, p.err, abort_flag)))
                 break;
-            {
+            if constexpr (F8) {
+                // f16 pairs of this lane's window: own slice, zeros elsewhere.
+                uint32_t w[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) w[k] = 0u;
+#pragma unroll
+                for (int k = 0; k < kTPC / 2; ++k) {
+                    const uint32_t h = pack_f16x2(active ? s[2 * k] : 0.f,
+                                                  active ? s[2 * k + 1] : 0.f);
+                    if constexpr (kTPC == 16) {
+                        w[k] = h;
+                    } else {
+                        w[k] = half ? 0u : h;
+                        w[4 + k] = half ? h : 0u;
+                    }
+                }
+                tmem_st8(trow + C::kTmemP + 64 * (i & 1) + 8 * q4, w);
+            } else {
                 // bf16 pairs of this lane's window: own slice, zeros elsewhere.
                 uint32_t hi_w[8], lo_w[8];
 #pragma unroll
@@ -431,7 +582,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->p_full[i & 1]);
+            mbar_arrive_warp(&bars->p_full[i & 1]);
 
             if (last) {
                 if (!all(mbar_wait(&bars->pv_done[i & 1], (uint32_t)((i >> 1) & 1), p.timeout_ns,
@@ -459,7 +610,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
                 if (active) p.ws_lse[part] = empty ? kNegInf : m_run + log2f(l_run);
                 tc_fence_before();
-                mbar_arrive(&bars->o_free);
+                mbar_arrive_warp(&bars->o_free);
             }
             cur.next();
         }
@@ -474,24 +625,25 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 // -------------------------------------------------------------- host side
 namespace {
 
-template <int D, int HCP, bool G>
+template <int D, int HCP, bool G, bool F8>
 cudaError_t launch_tc128_g(const GqaLaunch &L, int HC) {
-    using C = T2Cfg<D>;
+    using C = T2Cfg<D, F8>;
     static PerDeviceFlag configured;   // the attribute is per function and device
     {
         const cudaError_t e = configure_once_per_device(configured, [] {
-            return cudaFuncSetAttribute(gqa_tc128_kernel<D, HCP, G>,
+            return cudaFuncSetAttribute(gqa_tc128_kernel<D, HCP, G, F8>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         });
         if (e != cudaSuccess) return e;
     }
     const GqaParams &kp = L.kp;
-    CUtensorMap tk, tv;
-    if (!tc_make_map(&tk, kp.k_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64) ||
-        !tc_make_map(&tv, kp.v_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64))
+    CUtensorMap tk{}, tv{};            // fp8: the codes come by bulk copies, no maps
+    if (!F8 && (!tc_make_map(&tk, kp.k_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64) ||
+                !tc_make_map(&tv, kp.v_cache, D, (uint64_t)kp.num_blocks * kp.H_kv * 64, 64)))
         return cudaErrorInvalidValue;
     if (L.ev_start) cudaEventRecord(L.ev_start, L.stream);
-    gqa_tc128_kernel<D, HCP, G><<<kp.num_ctas, kT2Threads, C::kSmem, L.stream>>>(tk, tv, kp, HC);
+    gqa_tc128_kernel<D, HCP, G, F8><<<kp.num_ctas, F8 ? kT2ThreadsF8 : kT2Threads, C::kSmem,
+                                      L.stream>>>(tk, tv, kp, HC);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.ev_stop) cudaEventRecord(L.ev_stop, L.stream);
@@ -515,10 +667,10 @@ cudaError_t launch_tc128_g(const GqaLaunch &L, int HC) {
     return cudaLaunchKernelEx(&cfg, combine_kernel<__nv_bfloat16>, cp);
 }
 
-template <int D, int HCP>
+template <int D, int HCP, bool F8>
 cudaError_t launch_tc128(const GqaLaunch &L, int HC) {
-    return L.kp.vis.n_g > 0 ? launch_tc128_g<D, HCP, true>(L, HC)
-                            : launch_tc128_g<D, HCP, false>(L, HC);
+    return L.kp.vis.n_g > 0 ? launch_tc128_g<D, HCP, true, F8>(L, HC)
+                            : launch_tc128_g<D, HCP, false, F8>(L, HC);
 }
 
 }  // namespace
@@ -527,11 +679,30 @@ bool gqa_tc128_supported(int d, int HC) { return (d == 64 || d == 128) && HC <= 
 
 int gqa_tc128_copies(int HC) { return HC <= 16 ? 8 : 4; }
 
+bool gqa_tc128_fp8_supported(int d, int G) {
+    return (d == 64 || d == 128) && (G <= 32 || G % 32 == 0);
+}
+
+int gqa_tc128_fp8_heads_per_cta(int G) { return G <= 32 ? G : 32; }
+
 cudaError_t launch_gqa_tc128(const GqaLaunch &L, int d, int HC) {
     const bool wide = HC > 16;
     switch (d) {
-        case 64: return wide ? launch_tc128<64, 32>(L, HC) : launch_tc128<64, 16>(L, HC);
-        case 128: return wide ? launch_tc128<128, 32>(L, HC) : launch_tc128<128, 16>(L, HC);
+        case 64: return wide ? launch_tc128<64, 32, false>(L, HC)
+                             : launch_tc128<64, 16, false>(L, HC);
+        case 128: return wide ? launch_tc128<128, 32, false>(L, HC)
+                              : launch_tc128<128, 16, false>(L, HC);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t launch_gqa_tc128_fp8(const GqaLaunch &L, int d, int HC) {
+    const bool wide = HC > 16;
+    switch (d) {
+        case 64: return wide ? launch_tc128<64, 32, true>(L, HC)
+                             : launch_tc128<64, 16, true>(L, HC);
+        case 128: return wide ? launch_tc128<128, 32, true>(L, HC)
+                              : launch_tc128<128, 16, true>(L, HC);
         default: return cudaErrorNotSupported;
     }
 }

@@ -59,7 +59,9 @@ typedef enum {
     ATTN_ERR_BAD_SEQLEN = -6    /* device: T_b < 0, > 64 * max_blocks, or not servable by the ring */
 } attn_status;
 
-typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
+typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1, ATTN_FP8_E4M3 = 2 } attn_dtype;
+/* ATTN_FP8_E4M3 names the cache of attn_decode_gqa_fp8 in
+ * attn_decode_gqa_config only; the decode entry points take F32 or BF16. */
 
 /* Tokens per cache block (fixed by the storage format). */
 #define ATTN_BLOCK_SIZE 64
@@ -235,7 +237,8 @@ int attn_decode_plan(const int32_t *seq_lens, int B, int units_per_seq,
  * heads a CTA processes per KV head (the group is split into
  * H_q / H_kv / heads_per_cta chunks when it does not fit), *path = 0 for the
  * CUDA-core kernel, 1 for the M = 128 tensor-core (tcgen05) kernel, 2 for
- * the M = 64 tensor-core kernel.
+ * the M = 64 tensor-core kernel.  dtype ATTN_FP8_E4M3 answers for
+ * attn_decode_gqa_fp8.
  */
 int attn_decode_gqa_config(int B, int H_q, int H_kv, int d, int dtype,
                            int *num_ctas, int *heads_per_cta, int *path);
@@ -249,9 +252,12 @@ int attn_set_num_ctas(int num_ctas);
 /*
  * attn_set_gqa_path -- testing/tuning hook: -1 = automatic (bf16: the
  * CUDA-core kernel for groups of up to 4 heads, the tensor-core path for
- * larger groups), 0 = force the CUDA-core kernel, 1 = force the tensor-core
- * path (the M = 128 kernel where it applies, d <= 128 and units of <= 32
- * heads, else the M = 64 kernel), 2 = force the M = 64 tensor-core kernel.
+ * larger groups; fp8 cache: the M = 128 tensor-core kernel for d <= 128 and
+ * groups of 16 to 32 heads or multiples of 32, else the CUDA-core kernel),
+ * 0 = force the CUDA-core kernel, 1 = force the tensor-core path (the M = 128
+ * kernel where it applies, d <= 128 and units of <= 32 heads, else the M = 64
+ * kernel, which has no fp8 form), 2 = force the M = 64 tensor-core kernel
+ * (fp8 calls then run on the CUDA cores).
  */
 int attn_set_gqa_path(int path);
 

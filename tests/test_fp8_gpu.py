@@ -2,7 +2,9 @@
 the C ABI, vs the oracle: the append's quantisation is bit-exact (codes and
 scales are integer/byte results of fp32 arithmetic both sides do alike), and
 the decode matches the oracle's decode over the dequantised cache within the
-bf16 bars (max-abs <= 1e-2, rel-L2 <= 2e-3)."""
+bf16 bars (max-abs <= 1e-2, rel-L2 <= 2e-3), on both kernels that read an
+fp8 cache: the CUDA-core split kernel (path 0) and the M = 128 tensor-core
+kernel that widens the codes to f16 on the chip (path 1, d <= 128)."""
 import numpy as np
 import pytest
 import torch
@@ -67,9 +69,28 @@ FP8_CASES = [
 ]
 
 
+class _path:
+    """Force a GQA kernel for the calls inside the block."""
+
+    def __init__(self, lib, path):
+        self.lib, self.path = lib, path
+
+    def __enter__(self):
+        self.lib.set_gqa_path(self.path)
+
+    def __exit__(self, *exc):
+        self.lib.set_gqa_path(-1)
+
+
+PATHS = pytest.mark.parametrize("path", [0, 1], ids=["cuda_core", "tcgen05"])
+
+
+@PATHS
 @pytest.mark.parametrize("H_q,H_kv,d,lens,window,sink", FP8_CASES,
                          ids=[f"q{c[0]}_kv{c[1]}_d{c[2]}_w{c[4]}_g{c[5]}" for c in FP8_CASES])
-def test_fp8_decode_matches_oracle(lib, H_q, H_kv, d, lens, window, sink):
+def test_fp8_decode_matches_oracle(lib, path, H_q, H_kv, d, lens, window, sink):
+    if path == 1 and d > 128:
+        pytest.skip("the tensor-core fp8 kernel takes d <= 128")
     B = len(lens)
     slots = max((T + 63) // 64 for T in lens)
     n_blocks = B * slots + 2
@@ -78,11 +99,13 @@ def test_fp8_decode_matches_oracle(lib, H_q, H_kv, d, lens, window, sink):
     q = torch.randn((B, H_q, d), generator=g).bfloat16()
     table = torch.randperm(n_blocks, generator=g)[: B * slots].reshape(B, slots).to(torch.int32)
     scale = 1.0 / np.sqrt(d)
-    got = lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV), torch.from_numpy(vc).to(DEV),
-                             torch.from_numpy(ks).to(DEV), torch.from_numpy(vs).to(DEV),
-                             torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV),
-                             scale, window=window, sink_tokens=sink)
-    assert lib.last_error() == lib.OK
+    with _path(lib, path):
+        got = lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV),
+                                 torch.from_numpy(vc).to(DEV), torch.from_numpy(ks).to(DEV),
+                                 torch.from_numpy(vs).to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV),
+                                 scale, window=window, sink_tokens=sink)
+        assert lib.last_error() == lib.OK
     ref = orc.decode_gqa_vis(q.double().numpy(), orc.dequantize_e4m3(kc, ks),
                              orc.dequantize_e4m3(vc, vs), np.asarray(lens, dtype=np.int32),
                              table.numpy(), scale, window=window, sink=sink)
@@ -119,7 +142,8 @@ def test_fp8_append_then_decode(lib):
     assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, "fp8 append+decode")
 
 
-def test_fp8_decode_with_global_positions(lib):
+@PATHS
+def test_fp8_decode_with_global_positions(lib, path):
     """The fp8 cache under a window plus an explicit global set."""
     lens, window = [2000, 700], 300
     rows = [[0, 5, 640, 1650], [699, -1, -1, -1]]
@@ -132,12 +156,115 @@ def test_fp8_decode_with_global_positions(lib):
     q = torch.randn((B, H_q, d), generator=g).bfloat16()
     table = torch.randperm(n_blocks, generator=g)[: B * slots].reshape(B, slots).to(torch.int32)
     gp = torch.tensor(rows, dtype=torch.int32)
-    got = lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV), torch.from_numpy(vc).to(DEV),
-                             torch.from_numpy(ks).to(DEV), torch.from_numpy(vs).to(DEV),
-                             torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV),
-                             0.09, window=window, global_pos=gp.to(DEV))
-    assert lib.last_error() == lib.OK
+    with _path(lib, path):
+        got = lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV),
+                                 torch.from_numpy(vc).to(DEV), torch.from_numpy(ks).to(DEV),
+                                 torch.from_numpy(vs).to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV),
+                                 0.09, window=window, global_pos=gp.to(DEV))
+        assert lib.last_error() == lib.OK
     ref = orc.decode_gqa_vis(q.double().numpy(), orc.dequantize_e4m3(kc, ks),
                              orc.dequantize_e4m3(vc, vs), np.asarray(lens, dtype=np.int32),
                              table.numpy(), 0.09, window=window, global_pos=gp.numpy())
     assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, "fp8 global set")
+
+
+def _fp8_unit_cache(seed, n_blocks, H_kv, d):
+    """Unit-variance bf16 K/V rows (no magnitude narrowing), quantised by the
+    oracle."""
+    g = torch.Generator().manual_seed(seed)
+    shape = (n_blocks, H_kv, BLOCK_SIZE, d)
+    k = torch.randn(shape, generator=g).bfloat16()
+    v = torch.randn(shape, generator=g).bfloat16()
+    kc, ks = orc.quantize_rows_e4m3(k.float().numpy())
+    vc, vs = orc.quantize_rows_e4m3(v.float().numpy())
+    return kc, ks, vc, vs
+
+
+def _within_one_bf16_ulp(got, ref, slack):
+    """|got - ref| within one bf16 ulp of ref (the output's own rounding)
+    plus an absolute slack for the fp32 arithmetic before it."""
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    return np.abs(np.asarray(got, dtype=np.float64) - ref) <= ulp + slack
+
+
+@PATHS
+@pytest.mark.parametrize("H_q,H_kv,d,lens", [(32, 8, 128, [1, 2, 700, 4097]),
+                                             (32, 1, 128, [3000, 64]),
+                                             (16, 16, 64, [1500, 3])],
+                         ids=["gqa8_d128", "mqa_d128", "mha_d64"])
+def test_fp8_unit_variance_rows(lib, path, H_q, H_kv, d, lens):
+    """Unit-variance K/V rows and queries, no narrowing of the input ranges
+    (one-token outputs reach |o| of 3-4, where a bf16 ulp is 2^-6): judged by
+    rel-L2 and by agreement with the exact result to one bf16 ulp plus 2e-3."""
+    B = len(lens)
+    slots = max((T + 63) // 64 for T in lens)
+    n_blocks = B * slots + 2
+    kc, ks, vc, vs = _fp8_unit_cache(8500 + H_q + d, n_blocks, H_kv, d)
+    g = torch.Generator().manual_seed(8501 + d)
+    q = torch.randn((B, H_q, d), generator=g).bfloat16()
+    table = torch.randperm(n_blocks, generator=g)[: B * slots].reshape(B, slots).to(torch.int32)
+    scale = 1.0 / np.sqrt(d)
+    with _path(lib, path):
+        got = lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV),
+                                 torch.from_numpy(vc).to(DEV), torch.from_numpy(ks).to(DEV),
+                                 torch.from_numpy(vs).to(DEV),
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV),
+                                 scale)
+        assert lib.last_error() == lib.OK
+    ref = orc.decode_gqa(q.double().numpy(), orc.dequantize_e4m3(kc, ks),
+                         orc.dequantize_e4m3(vc, vs), np.asarray(lens, dtype=np.int32),
+                         table.numpy(), scale)
+    got = got.float().cpu().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel <= 2e-3, rel
+    ok = _within_one_bf16_ulp(got, ref, 2e-3)
+    assert ok.all(), f"{(~ok).sum()} outputs off by more than one bf16 ulp + 2e-3"
+
+
+@pytest.mark.parametrize("H_q,H_kv,d", [(32, 1, 128), (64, 1, 128), (8, 2, 64), (4, 4, 128),
+                                        (24, 4, 64)],
+                         ids=["mqa32", "mqa64", "g4_d64", "mha", "g6_d64"])
+def test_fp8_tensor_core_many_tiles_and_splits(lib, H_q, H_kv, d):
+    """The tensor-core fp8 kernel over long, ragged sequences whose tiles wrap
+    the stage ring many times, with 3 and 148 CTAs (segments crossing units
+    and sequences), groups from 1 to 64 heads (64: two 32-head units)."""
+    lens = [5000, 777, 64, 65, 2100]
+    B = len(lens)
+    slots = max((T + 63) // 64 for T in lens)
+    n_blocks = B * slots + 2
+    kc, ks, vc, vs = _fp8_cache(8600 + H_q + d, n_blocks, H_kv, d)
+    g = torch.Generator().manual_seed(8601 + H_q)
+    q = torch.randn((B, H_q, d), generator=g).bfloat16()
+    table = torch.randperm(n_blocks, generator=g)[: B * slots].reshape(B, slots).to(torch.int32)
+    ref = orc.decode_gqa(q.double().numpy(), orc.dequantize_e4m3(kc, ks),
+                         orc.dequantize_e4m3(vc, vs), np.asarray(lens, dtype=np.int32),
+                         table.numpy(), 0.08)
+    args = (q.to(DEV), torch.from_numpy(kc).to(DEV), torch.from_numpy(vc).to(DEV),
+            torch.from_numpy(ks).to(DEV), torch.from_numpy(vs).to(DEV),
+            torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV), 0.08)
+    for ctas in (3, 0):
+        lib.set_num_ctas(ctas)
+        try:
+            with _path(lib, 1):
+                got = lib.decode_gqa_fp8(*args)
+                assert lib.last_error() == lib.OK
+        finally:
+            lib.set_num_ctas(0)
+        assert_parity(got.float().cpu().numpy(), ref, torch.bfloat16, f"fp8 tc, {ctas} CTAs")
+
+
+def test_fp8_tensor_core_bad_block_is_flagged(lib):
+    """A block id outside the pool on the tensor-core fp8 kernel sets the
+    bad-block error and is never dereferenced."""
+    H_q, H_kv, d, lens = 32, 1, 128, [300, 200]
+    n_blocks = 12
+    kc, ks, vc, vs = _fp8_cache(8700, n_blocks, H_kv, d)
+    q = torch.randn((2, H_q, d)).bfloat16()
+    table = torch.arange(10, dtype=torch.int32).reshape(2, 5)
+    table[1, 2] = 1 << 20                                 # outside the pool
+    with _path(lib, 1):
+        lib.decode_gqa_fp8(q.to(DEV), torch.from_numpy(kc).to(DEV), torch.from_numpy(vc).to(DEV),
+                           torch.from_numpy(ks).to(DEV), torch.from_numpy(vs).to(DEV),
+                           torch.tensor(lens, dtype=torch.int32, device=DEV), table.to(DEV), 0.1)
+        assert lib.last_error() == lib.ERR_BAD_BLOCK

@@ -97,6 +97,9 @@ RAGGED_WINDOW = ragged_config(4096)
 # The Llama-3-8B shape over an fp8 (E4M3 + per-row scale) KV cache.
 LLAMA3_8B_FP8 = GQAConfig("llama3_8b_gqa_fp8kv_B16_Hq32_Hkv8_d128_T4096", B=16, H_q=32,
                           H_kv=8, d=128, T=4096, kv_fp8=True, seed=SEED_BASE + 1)
+# MQA at B = 8, T = 32768 over an fp8 cache (the tensor-core fp8 kernel's shape).
+MQA_B8_FP8 = GQAConfig("sweep_fp8_B8_Hq32_Hkv1_d128_T32768", B=8, H_q=32, H_kv=1, d=128,
+                       T=32768, kv_fp8=True, seed=SEED_BASE + 2)
 # Window plus 64 global tokens on the same shape; and the same on a ring table
 # that keeps only the 1 sink block and the 65 blocks a 4096-key window can reach.
 RAGGED_WINDOW_SINK = GQAConfig("ragged_gqa_bf16_B8_Hq24_Hkv4_d256_w4096_g64", B=8, H_q=24,
@@ -114,7 +117,8 @@ MLA_DSV2_FP8 = MLAConfig("mla_absorbed_fp8latent_B32_H128_dc512_dr64_T8192", B=3
 
 WORKLOADS = {c.name: c for c in [TINY, LLAMA3_8B, *SWEEP, RAGGED_FULL,
                                  RAGGED_WINDOW, RAGGED_WINDOW_SINK, RAGGED_WINDOW_RING,
-                                 RAGGED_WINDOW_GLOBAL, LLAMA3_8B_FP8, MLA_DSV2, MLA_DSV2_FP8]}
+                                 RAGGED_WINDOW_GLOBAL, LLAMA3_8B_FP8, MQA_B8_FP8, MLA_DSV2,
+                                 MLA_DSV2_FP8]}
 
 
 def global_rows(seq_lens, n: int) -> torch.Tensor:
