@@ -70,6 +70,7 @@ constexpr int kMlaStageBytes = kMlaMaxBoxes * kMlaCBox;
 constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA, 4-11 softmax
 constexpr int kMlaThreadsF8 = 512;         // fp8: + warps 12-15 widening the codes
 constexpr int kSoftThreads = 256;
+constexpr int kSoftWarps = kSoftThreads / 32;   // barriers count warps (one arrival each)
 constexpr int kPBytes = kMlaH * 128;       // one P half: [128 heads][64 tokens] bf16
 constexpr int kXBytes = kMlaH * 64 * 4;    // exchange buffer: 16 chunks x [128 rows] x 16 B
 constexpr int kRawBox = 64 * 64;           // fp8: one box of codes, [64 tokens][64 columns]
@@ -166,26 +167,26 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
 
     // ---- set-up: barriers, TMEM, cluster handshake
     if (tid == 0) {
-        mbar_init(&bars->q_full, kSoftThreads);
+        mbar_init(&bars->q_full, kSoftWarps);
         mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMlaStages; ++s) {
-            mbar_init(&bars->c_full[s], F8 ? 128 : 1);  // widening warps, or the TMA
+            mbar_init(&bars->c_full[s], F8 ? 4 : 1);    // widening warps, or the TMA
             mbar_init(&bars->c_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->raw_full[s], 1);
-            mbar_init(&bars->raw_empty[s], 128);
+            mbar_init(&bars->raw_empty[s], 4);
         }
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, kSoftThreads);
-        mbar_init(&bars->p_full, kSoftThreads);
+        mbar_init(&bars->s_free, kSoftWarps);
+        mbar_init(&bars->p_full, kSoftWarps);
         mbar_init(&bars->pv_done, 1);
-        mbar_init(&bars->o_free, kSoftThreads);
-        mbar_init(&bars->x_full, 1);               // peer's arrive.expect_tx + bulk copy
-        mbar_init(&bars->x_free, kSoftThreads);    // peer's threads consumed my data
-        mbar_init(&bars->stg_full, kSoftThreads);  // my threads staged their halves
-        mbar_init(&bars->red_bar, kSoftThreads);
-        mbar_init(&bars->sum_bar, kSoftThreads);
+        mbar_init(&bars->o_free, kSoftWarps);
+        mbar_init(&bars->x_full, 1);               // own arrive.expect_tx + peer's bulk copy
+        mbar_init(&bars->x_free, kSoftWarps);      // peer's warps consumed my data
+        mbar_init(&bars->stg_full, kSoftWarps);    // my warps staged their halves
+        mbar_init(&bars->red_bar, kSoftWarps);
+        mbar_init(&bars->sum_bar, kSoftWarps);
         mbar_init(&bars->end_bar, 1);
         mbar_init(&bars->mma_final, 2);            // one commit per issuing thread
         bars->abort = 0;
@@ -408,8 +409,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 float *ssc = reinterpret_cast<float *>(smem + C::kOffScale) + st * 64;
                 if (wt < 64) ssc[wt] = rsc[wt];
                 fence_proxy_async_smem();      // the MMAs read the widened stage
-                mbar_arrive(&bars->raw_empty[rs]);
-                mbar_arrive(&bars->c_full[st]);
+                mbar_arrive_warp(&bars->raw_empty[rs]);
+                mbar_arrive_warp(&bars->c_full[st]);
             }
         }
     } else if (warp >= 4 && warp < 12) {
@@ -459,7 +460,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 tmem_st32(trow + kTmemQ + 32 * bx, r);
             }
             tc_fence_before();
-            mbar_arrive(&bars->q_full);
+            mbar_arrive_warp(&bars->q_full);
             return true;
         };
         // Read this half of the CTA's partial S(i) from TMEM, free it, stage it
@@ -473,9 +474,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             tc_fence_after();
             tmem_ld32(trow + kTmemS + 32 * h, dst);
             tc_fence_before();
-            mbar_arrive(&bars->s_free);
-            if (i >= 1 && !all(mbar_wait_cluster(&bars->x_free, (uint32_t)((i - 1) & 1),
-                                                 p.timeout_ns, p.err, abort_flag)))
+            mbar_arrive_warp(&bars->s_free);
+            if (i >= 1 && !all(mbar_wait(&bars->x_free, (uint32_t)((i - 1) & 1), p.timeout_ns,
+                                         p.err, abort_flag)))
                 return false;
             unsigned char *stg = sStg + row * 16;
 #pragma unroll
@@ -483,15 +484,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 *reinterpret_cast<float4 *>(stg + (8 * h + c) * (kMlaH * 16)) =
                     make_float4(dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3]);
             fence_proxy_async_smem();
-            mbar_arrive(&bars->stg_full);
+            mbar_arrive_warp(&bars->stg_full);
             bool sent = true;
             if (sender) {
                 sent = mbar_wait(&bars->stg_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
                                  abort_flag);
-                if (sent) {
-                    mbar_arrive_expect_tx_remote(x_full_peer, kXBytes);
-                    bulk_copy_to_peer(x_peer, sStg, kXBytes, x_full_peer);
-                }
+                if (sent) bulk_copy_to_peer(x_peer, sStg, kXBytes, x_full_peer);
             }
             return all(sent);
         };
@@ -502,6 +500,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         int q_seg = 0, n_seg = 0;
         float m_run = -1e30f, l_run = 0.f;                // l_run: this half's sum
         float s_nxt[32];
+        if (sender && n_tiles > 0) mbar_arrive_expect_tx(&bars->x_full, kXBytes);   // tile 0
         bool ok = load_q(nxt.w.b, q_seg++) && fetch_s(0, s_nxt);
         for (int i = 0; ok && i < n_tiles; ++i) {
             float s[32];
@@ -512,8 +511,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             const int nvalid = T - (cur.logical_block() * 64 + 32 * h);   // valid in this half
 
             // add the peer's partial scores of tile i, scale to log2 units
-            if (!all(mbar_wait_cluster(&bars->x_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
-                                       abort_flag)))
+            if (!all(mbar_wait(&bars->x_full, (uint32_t)(i & 1), p.timeout_ns, p.err, abort_flag)))
                 break;
             const unsigned char *xrow = sX + row * 16;
             const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
@@ -535,7 +533,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 }
                 s[4 * c] = a.x; s[4 * c + 1] = a.y; s[4 * c + 2] = bb.x; s[4 * c + 3] = bb.y;
             }
-            mbar_arrive_remote(x_free_peer);
+            // arm the receive barrier for tile i + 1 (the peer's copy may
+            // land first: the byte count then runs negative until this),
+            // then let the peer reuse the buffer
+            if (sender && i + 1 < n_tiles) mbar_arrive_expect_tx(&bars->x_full, kXBytes);
+            mbar_arrive_remote_relaxed_warp(x_free_peer);
 
             // prefetch: next tile's query (new sequence) and partial scores
             nxt.next();
@@ -555,7 +557,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             // row max across the two halves (double-buffered by tile parity)
             float *rb = red + (i & 1) * 256;
             rb[h * 128 + row] = mx;
-            mbar_arrive(&bars->red_bar);
+            mbar_arrive_warp(&bars->red_bar);
             if (!all(mbar_wait(&bars->red_bar, (uint32_t)(i & 1), p.timeout_ns, p.err,
                                abort_flag)))
                 break;
@@ -643,12 +645,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive_warp(&bars->p_full);
 
             if (last) {
                 float *sb = red + 512 + (n_seg & 1) * 256;
                 sb[h * 128 + row] = l_run;
-                mbar_arrive(&bars->sum_bar);
+                mbar_arrive_warp(&bars->sum_bar);
                 if (!all(mbar_wait(&bars->sum_bar, (uint32_t)(n_seg & 1), p.timeout_ns, p.err,
                                    abort_flag)))
                     break;
@@ -673,7 +675,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 }
                 if (rank == 0 && h == 0) p.ws_lse[slot * kMlaH + row] = m_run + log2f(l_tot);
                 tc_fence_before();
-                mbar_arrive(&bars->o_free);
+                mbar_arrive_warp(&bars->o_free);
             }
             cur.next();
         }

@@ -320,6 +320,26 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
                      remote_bar)
                  : "memory");
 }
+// Arrive without release semantics on another CTA's mbarrier: for a signal
+// that orders no memory the waiter reads (e.g. "my reads of your buffer have
+// completed": their values are already in registers), and avoids the
+// cluster-scope release fence on the signalling thread's path.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                     remote_bar)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote_relaxed_warp(uint32_t remote_bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive_remote_relaxed(remote_bar);
+}
+
+// mbar_arrive_remote once per warp (see mbar_arrive_warp).  All lanes call it.
+__device__ __forceinline__ void mbar_arrive_remote_warp(uint32_t remote_bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive_remote(remote_bar);
+}
+
 // try_wait with cluster-scope acquire (pairs with remote release arrivals).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
     uint32_t done;
