@@ -16,14 +16,16 @@
 //     pairs per 32-bit column), written once per sequence by the softmax
 //     threads; S = Q C^T is a 128 x 64 (heads x tokens) tcgen05 MMA with A in
 //     TMEM and B = the C tile in shared memory, accumulated in TMEM.
-//   * The two partial S are exchanged between the CTAs of the cluster: each
-//     thread stages its half-row in local shared memory and one thread moves
-//     the 32 KiB to the peer with a single bulk copy (shared::cta ->
-//     shared::cluster, completion on the peer's barrier); both CTAs sum the
-//     halves identically.  The softmax loop is software-pipelined: in
-//     iteration i a CTA first consumes the peer's S(i), then stages and sends
-//     its own S(i+1), then does the softmax of tile i, which hides the
-//     transfer.
+//   * The two partial S are exchanged between the CTAs of the cluster by
+//     four exchange warps per CTA (one thread per head row): they read S(i)
+//     from TMEM as soon as its MMA completes, stage it in shared memory,
+//     free the TMEM buffer for S(i + 1), and one thread moves the staged 32
+//     KiB to the peer with a single bulk copy (shared::cta ->
+//     shared::cluster, completion on the peer's barrier, which the peer
+//     arms itself).  The softmax warps only sum the staged and the received
+//     halves, so the exchange of tile i + 1 runs while they work on tile i;
+//     no cluster-scope fence sits on their path (the consume signal to the
+//     peer is a relaxed arrival).  Both CTAs sum the halves identically.
 //   * Softmax runs one thread per head row on the TMEM rows (no cross-thread
 //     reductions); the running max is only raised when it grows by more than
 //     2^8, so O is rescaled rarely (the result is exact either way: numerator
@@ -35,7 +37,7 @@
 //     read MN-major.  Each CTA keeps its 256 output columns in TMEM.
 //   * Warp 0 issues TMA; one thread of warp 1 issues the S MMAs and one of
 //     warp 2 the P V MMAs, each as its inputs become ready; warps 4-11 load
-//     Q, run the softmax and the epilogue.  Every
+//     Q, run the softmax and the epilogue; warps 12-15 exchange the scores.  Every
 //     wait is bounded; TMEM is always freed; the final cluster handshake is a
 //     bounded mbarrier exchange.
 // Each (sequence, cluster) segment writes an fp32 partial (O/l and log2-sum-
@@ -44,7 +46,7 @@
 // FP8 latent cache (template flag F8): rows stored as OCP E4M3 codes with one
 // fp32 scale per row (value = code value x scale).  The TMA loads each tile's
 // code boxes and 64 row scales into a raw stage; a widening warpgroup (warps
-// 12-15) converts the codes to f16 exactly (every E4M3 value is an f16
+// 16-19) converts the codes to f16 exactly (every E4M3 value is an f16
 // value) into the same swizzled stage layout the MMAs read, and this variant
 // runs its MMAs on f16 operands: the query is converted to f16 once per
 // sequence (exact within f16's range) and P is one f16 operand (11
@@ -67,8 +69,9 @@ constexpr int kMlaCBox = 64 * 128;         // [64 tokens][64 cols] bf16
 constexpr int kMlaMaxBoxes = 5;
 constexpr int kMlaPrefetch = 4;            // blocks pulled into L2 ahead of the ring
 constexpr int kMlaStageBytes = kMlaMaxBoxes * kMlaCBox;
-constexpr int kMlaThreads = 384;           // warps 0-3 TMA/MMA, 4-11 softmax
-constexpr int kMlaThreadsF8 = 512;         // fp8: + warps 12-15 widening the codes
+constexpr int kMlaThreads = 512;           // warps 0-3 TMA/MMA, 4-11 softmax, 12-15 exchange
+constexpr int kMlaThreadsF8 = 640;         // fp8: + warps 16-19 widening the codes
+constexpr int kXchgWarps = 4;              // exchange warps: one thread per head row
 constexpr int kSoftThreads = 256;
 constexpr int kSoftWarps = kSoftThreads / 32;   // barriers count warps (one arrival each)
 constexpr int kPBytes = kMlaH * 128;       // one P half: [128 heads][64 tokens] bf16
@@ -91,6 +94,16 @@ template <bool F8> struct MlaCfg {
     static constexpr int kSmemUsed = kOffScale + (F8 ? kStages * 64 * 4 : 0);
     static constexpr int kSmem = kSmemUsed + 1024;     // + alignment slack
     static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+    // Registers per thread by warpgroup (setmaxnreg), within the launch's
+    // threads x registers (bf16: 512 x 128; fp8: 640 x 96): TMA/MMA warps,
+    // softmax warps (two warpgroups), exchange warps, widening warps.
+    static constexpr int kRegCtl = F8 ? 48 : 56;
+    static constexpr int kRegSoft = F8 ? 152 : 184;
+    static constexpr int kRegX = F8 ? 64 : 80;
+    static constexpr int kRegW = 64;
+    static_assert(128 * kRegCtl + 256 * kRegSoft + 128 * kRegX + (F8 ? 128 * kRegW : 0) <=
+                      (F8 ? 640 * 96 : 512 * 128),
+                  "register split");
 };
 constexpr int kMlaMaxStages = 3;
 constexpr uint32_t kTmemCols = 512;
@@ -103,7 +116,7 @@ struct MlaBars {
     uint64_t raw_full[2], raw_empty[2];   // fp8: code stages landed / widened
     uint64_t s_full, s_free;
     uint64_t p_full, pv_done, o_free;
-    uint64_t x_full, x_free, stg_full;
+    uint64_t x_full, x_free, stg_full, stg_free;
     uint64_t red_bar, sum_bar;
     uint64_t end_bar, mma_final;
     uint32_t tmem_base;
@@ -178,13 +191,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             mbar_init(&bars->raw_empty[s], 4);
         }
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, kSoftWarps);
+        mbar_init(&bars->s_free, kXchgWarps);        // the exchange warps read S
         mbar_init(&bars->p_full, kSoftWarps);
         mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->o_free, kSoftWarps);
         mbar_init(&bars->x_full, 1);               // own arrive.expect_tx + peer's bulk copy
-        mbar_init(&bars->x_free, kSoftWarps);      // peer's warps consumed my data
-        mbar_init(&bars->stg_full, kSoftWarps);    // my warps staged their halves
+        mbar_init(&bars->x_free, kSoftWarps);      // peer's softmax warps consumed my data
+        mbar_init(&bars->stg_full, kXchgWarps);    // exchange warps staged my partial S
+        mbar_init(&bars->stg_free, kSoftWarps);    // my softmax warps consumed it
         mbar_init(&bars->red_bar, kSoftWarps);
         mbar_init(&bars->sum_bar, kSoftWarps);
         mbar_init(&bars->end_bar, 1);
@@ -199,11 +213,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
     cluster_sync_all();   // the peer's barriers exist before any remote arrive
     const uint32_t tmem = bars->tmem_base;
 
-    // fp8: 16 warps; the launch's 512 x 128 registers are re-split so the
-    // softmax warpgroups keep 176 (TMA/MMA warpgroup 80, widening 80:
-    // 128 x 80 + 256 x 176 + 128 x 80 = 65536), each at the top of its role.
+    // Registers are re-split by warpgroup at the top of each role (MlaCfg).
     if (warp == 0) {
-        if constexpr (F8) regs_decrease<80>();
+        regs_decrease<C::kRegCtl>();
         // ============================================================ TMA
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
@@ -272,7 +284,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         }
         __syncwarp();
     } else if (warp == 1 || warp == 2) {
-        if constexpr (F8) regs_decrease<80>();
+        regs_decrease<C::kRegCtl>();
         // ============================================================ MMA
         // Lane 0 of warp 1 issues S(n) = Q C(n)^T for every tile in order,
         // lane 0 of warp 2 issues O += P(i) C(i); each waits only on its own
@@ -367,15 +379,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         }
         __syncwarp();
     } else if (warp == 3) {
-        if constexpr (F8) regs_decrease<80>();
-    } else if (F8 && warp >= 12) {
-        // ================================================ fp8 -> bf16 widening
-        regs_decrease<80>();
+        regs_decrease<C::kRegCtl>();
+    } else if (F8 && warp >= 16) {
+        // ================================================ fp8 -> f16 widening
+        regs_decrease<C::kRegW>();
         // The codes are widened to f16 with the hardware conversion (exact:
         // every E4M3 value is an f16 value); the fp8 variant runs its MMAs on
         // f16 operands.
         if constexpr (F8) {
-            const int wt = tid - 384;            // widening thread 0..127
+            const int wt = tid - 512;            // widening thread 0..127
             for (int tile = 0; tile < n_tiles; ++tile) {
                 const int rs = tile % C::kRawStages, st = tile % kMlaStages;
                 if (!__all_sync(0xffffffffu,
@@ -415,18 +427,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
         }
     } else if (warp >= 4 && warp < 12) {
         // ============================================ Q load, softmax, epilogue
-        if constexpr (F8) regs_increase<176>();
+        regs_increase<C::kRegSoft>();
         // Two threads per head row: warps w and w + 4 share TMEM lanes
         // 32*(w%4) .. +31; half h takes tokens [32h, 32h+32) of each tile and
         // output columns [128h, 128h+128) of this CTA's 256.
         const int q4 = warp & 3, h = (warp - 4) >> 2;
         const int row = 32 * q4 + lane;                      // head = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
-        const uint32_t x_peer = map_to_rank(sX, peer);
-        const uint32_t x_full_peer = map_to_rank(&bars->x_full, peer);
         const uint32_t x_free_peer = map_to_rank(&bars->x_free, peer);
-        unsigned char *sStg = smem + kOffStg;
-        const bool sender = (warp == 4 && lane == 0);
+        const unsigned char *own_row = smem + kOffStg + row * 16;   // staged by the exchange warps
+        const unsigned char *peer_row = sX + row * 16;             // received from the peer
+        const bool sender = (warp == 4 && lane == 0);              // arms the receive barrier
         unsigned char *prow = sP + row * 128;
         float *red = reinterpret_cast<float *>(smem + kOffRed);   // [2][2][128] then sums
         // Wait outcomes are made warp-uniform: the TMEM loads and stores are
@@ -463,67 +474,38 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             mbar_arrive_warp(&bars->q_full);
             return true;
         };
-        // Read this half of the CTA's partial S(i) from TMEM, free it, stage it
-        // and (one thread) send the whole staged tile to the peer.  The peer
-        // must have consumed the previous tile (x_free) before the staging
-        // buffer and its receive buffer are reused.
-        auto fetch_s = [&](int i, float *dst) -> bool {
-            if (!all(mbar_wait(&bars->s_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
-                               abort_flag)))
-                return false;
-            tc_fence_after();
-            tmem_ld32(trow + kTmemS + 32 * h, dst);
-            tc_fence_before();
-            mbar_arrive_warp(&bars->s_free);
-            if (i >= 1 && !all(mbar_wait(&bars->x_free, (uint32_t)((i - 1) & 1), p.timeout_ns,
-                                         p.err, abort_flag)))
-                return false;
-            unsigned char *stg = sStg + row * 16;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<float4 *>(stg + (8 * h + c) * (kMlaH * 16)) =
-                    make_float4(dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3]);
-            fence_proxy_async_smem();
-            mbar_arrive_warp(&bars->stg_full);
-            bool sent = true;
-            if (sender) {
-                sent = mbar_wait(&bars->stg_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
-                                 abort_flag);
-                if (sent) bulk_copy_to_peer(x_peer, sStg, kXBytes, x_full_peer);
-            }
-            return all(sent);
-        };
-
         TileCursor cur, nxt;
         cur.init(pa, lo, hi, first_seq, first_base);
         nxt.init(pa, lo, hi, first_seq, first_base);
         int q_seg = 0, n_seg = 0;
         float m_run = -1e30f, l_run = 0.f;                // l_run: this half's sum
-        float s_nxt[32];
         if (sender && n_tiles > 0) mbar_arrive_expect_tx(&bars->x_full, kXBytes);   // tile 0
-        bool ok = load_q(nxt.w.b, q_seg++) && fetch_s(0, s_nxt);
+        bool ok = load_q(nxt.w.b, q_seg++);
         for (int i = 0; ok && i < n_tiles; ++i) {
             float s[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = s_nxt[j];
             const bool first = cur.t == 0, last = cur.t == cur.len - 1;
             const int b = cur.w.b, T = cur.w.T;
             const int nvalid = T - (cur.logical_block() * 64 + 32 * h);   // valid in this half
 
-            // add the peer's partial scores of tile i, scale to log2 units
+            // this CTA's and the peer's partial scores of tile i, summed and
+            // scaled to log2 units
+            if (!all(mbar_wait(&bars->stg_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                break;
             if (!all(mbar_wait(&bars->x_full, (uint32_t)(i & 1), p.timeout_ns, p.err, abort_flag)))
                 break;
-            const unsigned char *xrow = sX + row * 16;
             const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
             // fp8: this half's 32 row scales of tile i (kept with its stage)
             const float *tsc = reinterpret_cast<const float *>(smem + C::kOffScale) +
                                (i % kMlaStages) * 64 + 32 * h;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
+                const float4 u =
+                    *reinterpret_cast<const float4 *>(own_row + (8 * h + c) * (kMlaH * 16));
                 const float4 v =
-                    *reinterpret_cast<const float4 *>(xrow + (8 * h + c) * (kMlaH * 16));
-                float2 a = __fadd2_rn(make_float2(s[4 * c], s[4 * c + 1]), make_float2(v.x, v.y));
-                float2 bb = __fadd2_rn(make_float2(s[4 * c + 2], s[4 * c + 3]), make_float2(v.z, v.w));
+                    *reinterpret_cast<const float4 *>(peer_row + (8 * h + c) * (kMlaH * 16));
+                float2 a = __fadd2_rn(make_float2(u.x, u.y), make_float2(v.x, v.y));
+                float2 bb = __fadd2_rn(make_float2(u.z, u.w), make_float2(v.z, v.w));
                 a = __fmul2_rn(a, sl2);
                 bb = __fmul2_rn(bb, sl2);
                 if constexpr (F8) {
@@ -535,16 +517,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             }
             // arm the receive barrier for tile i + 1 (the peer's copy may
             // land first: the byte count then runs negative until this),
-            // then let the peer reuse the buffer
+            // then let the exchange warps restage and the peer resend
             if (sender && i + 1 < n_tiles) mbar_arrive_expect_tx(&bars->x_full, kXBytes);
+            mbar_arrive_warp(&bars->stg_free);
             mbar_arrive_remote_relaxed_warp(x_free_peer);
 
-            // prefetch: next tile's query (new sequence) and partial scores
+            // the next tile's query (a new sequence) into TMEM ahead of its S
             nxt.next();
-            if (i + 1 < n_tiles) {
-                if (nxt.t == 0 && !load_q(nxt.w.b, q_seg++)) break;
-                if (!fetch_s(i + 1, s_nxt)) break;
-            }
+            if (i + 1 < n_tiles && nxt.t == 0 && !load_q(nxt.w.b, q_seg++)) break;
 
             if (nvalid < 32) {
 #pragma unroll
@@ -678,6 +658,60 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 mbar_arrive_warp(&bars->o_free);
             }
             cur.next();
+        }
+    }
+
+    if (warp >= 12 && warp < 16) {
+        // ============================================= score exchange
+        // One thread per head row (TMEM lane) reads this CTA's partial S(i)
+        // (64 tokens) from TMEM, stages it in shared memory -- where this
+        // CTA's softmax reads it too -- and frees the TMEM buffer for S(i + 1);
+        // one thread then sends the staged tile to the peer with a bulk copy.
+        // Staging tile i waits until this CTA's softmax has consumed tile
+        // i - 1 (stg_free) and the peer has consumed its copy of it (x_free:
+        // the copy out of the staging buffer has completed and the peer's
+        // receive buffer is free), so the softmax threads never wait on the
+        // exchange themselves.
+        regs_decrease<C::kRegX>();
+        const int q4 = warp & 3;
+        const int row = 32 * q4 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
+        const uint32_t x_peer = map_to_rank(sX, peer);
+        const uint32_t x_full_peer = map_to_rank(&bars->x_full, peer);
+        unsigned char *sStg = smem + kOffStg;
+        unsigned char *stg = sStg + row * 16;
+        const bool issuer = warp == 12 && lane == 0;
+        auto all = [](bool v) { return __all_sync(0xffffffffu, v); };
+        for (int i = 0; i < n_tiles; ++i) {
+            if (i >= 1 &&
+                !all(mbar_wait(&bars->stg_free, (uint32_t)((i - 1) & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                break;
+            if (i >= 1 &&
+                !all(mbar_wait(&bars->x_free, (uint32_t)((i - 1) & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                break;
+            if (!all(mbar_wait(&bars->s_full, (uint32_t)(i & 1), p.timeout_ns, p.err,
+                               abort_flag)))
+                break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+                tmem_ld32(trow + kTmemS + 32 * hh, v);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4 *>(stg + (8 * hh + c) * (kMlaH * 16)) =
+                        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+            tc_fence_before();
+            mbar_arrive_warp(&bars->s_free);
+            fence_proxy_async_smem();          // the bulk copy reads the staging buffer
+            mbar_arrive_warp(&bars->stg_full);
+            if (issuer &&
+                mbar_wait(&bars->stg_full, (uint32_t)(i & 1), p.timeout_ns, p.err, abort_flag))
+                bulk_copy_to_peer(x_peer, sStg, kXBytes, x_full_peer);
+            __syncwarp();
         }
     }
 
