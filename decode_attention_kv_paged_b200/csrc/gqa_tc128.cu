@@ -51,7 +51,7 @@ struct T2Cfg {
     static constexpr int kRawBytes = F8 ? 2 * 64 * D + 512 : 0;
     static constexpr int kScaleBytes = F8 ? 512 : 0;              // widened stage's scales
     static constexpr int kStagesFit = (227 * 1024 - 4096) / kStageBytes;
-    static constexpr int kStages = F8 ? (D == 128 ? 3 : 4) : (kStagesFit > 6 ? 6 : kStagesFit);
+    static constexpr int kStages = F8 ? (D == 128 ? 4 : 6) : (kStagesFit > 6 ? 6 : kStagesFit);
     static constexpr int kRawFit =
         F8 ? (227 * 1024 - 4096 - kStages * (kStageBytes + kScaleBytes)) / kRawBytes : 0;
     static constexpr int kRaw = kRawFit > 8 ? 8 : kRawFit;         // fp8 raw stages

@@ -46,18 +46,33 @@ __host__ __device__ __forceinline__ const int32_t *global_row(const Visibility &
     return v.gpos + (size_t)b * v.n_g;
 }
 
+// Eight entries of G_b from k0 into c (entries past the row get -1), all
+// eight loads issued before any is used, so a scan of the row costs one
+// memory round trip per eight entries.
+__device__ __forceinline__ void global_chunk(const int32_t *g, int n_g, int k0, int32_t *c) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) c[j] = k0 + j < n_g ? g[k0 + j] : -1;
+}
+
 // Whether the decode query of a sequence with T keys is a global position.
 __device__ __forceinline__ bool global_query(const Visibility &v, int b, int T) {
     if (v.n_g <= 0 || T <= 0) return false;
     const int32_t *g = global_row(v, b);
     int prev = -1;
-    for (int i = 0; i < v.n_g; ++i) {
-        const int p = g[i];
-        if (p <= prev || p >= T) break;
-        if (p == T - 1) return true;
-        prev = p;
+    bool end = false, found = false;
+    for (int k0 = 0; k0 < v.n_g && !end; k0 += 8) {
+        int32_t c[8];
+        global_chunk(g, v.n_g, k0, c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            end = end || k0 + j >= v.n_g || c[j] <= prev || c[j] >= T;
+            if (!end) {
+                found = found || c[j] == T - 1;
+                prev = c[j];
+            }
+        }
     }
-    return false;
+    return found;
 }
 
 __host__ __device__ __forceinline__ int sink_blocks(const Visibility &v) {
@@ -92,19 +107,29 @@ __device__ __forceinline__ int seq_window_lo(const Visibility &v, int b, int T) 
 // position of sequence b below block w0 (i < the count visible_blocks gave).
 __device__ __forceinline__ int global_block(const Visibility &v, int b, int i) {
     const int32_t *g = global_row(v, b);
-    int prev = -1, last = -1, n = 0;
-    for (int k = 0; k < v.n_g; ++k) {
-        const int p = g[k];
-        if (p <= prev) break;
-        prev = p;
-        const int blk = p / kBlockSize;
-        if (blk != last) {
-            if (n == i) return blk;
-            ++n;
-            last = blk;
+    int prev = -1, last = -1, n = 0, found = -1;
+    bool end = false;
+    for (int k0 = 0; k0 < v.n_g && !end; k0 += 8) {
+        int32_t c[8];
+        global_chunk(g, v.n_g, k0, c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            end = end || k0 + j >= v.n_g || c[j] <= prev;
+            if (!end) {
+                prev = c[j];
+                const int blk = c[j] / kBlockSize;
+                if (blk != last) {
+                    if (n == i) {
+                        found = blk;
+                        end = true;
+                    }
+                    ++n;
+                    last = blk;
+                }
+            }
         }
     }
-    return last;   // not reached for i < count
+    return found >= 0 ? found : last;   // not reached for i < count
 }
 
 // Global-set ring layout: table slot of the i-th distinct block (ascending)
@@ -112,19 +137,29 @@ __device__ __forceinline__ int global_block(const Visibility &v, int b, int i) {
 // position of G_b in it (0 if there is none, which callers never ask for).
 __device__ __forceinline__ int global_slot(const Visibility &v, int b, int i) {
     const int32_t *g = global_row(v, b);
-    int prev = -1, last = -1, n = 0;
-    for (int k = 0; k < v.n_g; ++k) {
-        const int p = g[k];
-        if (p <= prev) break;
-        prev = p;
-        const int blk = p / kBlockSize;
-        if (blk != last) {
-            if (n == i) return k;
-            ++n;
-            last = blk;
+    int prev = -1, last = -1, n = 0, found = 0;
+    bool end = false;
+    for (int k0 = 0; k0 < v.n_g && !end; k0 += 8) {
+        int32_t c[8];
+        global_chunk(g, v.n_g, k0, c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            end = end || k0 + j >= v.n_g || c[j] <= prev;
+            if (!end) {
+                prev = c[j];
+                const int blk = c[j] / kBlockSize;
+                if (blk != last) {
+                    if (n == i) {
+                        found = k0 + j;
+                        end = true;
+                    }
+                    ++n;
+                    last = blk;
+                }
+            }
         }
     }
-    return 0;
+    return found;
 }
 
 // Bit t set when token blk * 64 + t of sequence b is a global position.
@@ -157,13 +192,20 @@ __device__ __forceinline__ int visible_blocks_global(int T, const Visibility &v,
     if (w0 == 0) return w1;                               // one run [0, w1)
     const int32_t *g = global_row(v, b);
     int prev = -1, last = -1, n = 0;
-    for (int k = 0; k < v.n_g; ++k) {
-        const int p = g[k];
-        if (p <= prev || p / kBlockSize >= w0) break;
-        prev = p;
-        if (p / kBlockSize != last) {
-            ++n;
-            last = p / kBlockSize;
+    bool end = false;
+    for (int k0 = 0; k0 < v.n_g && !end; k0 += 8) {
+        int32_t c[8];
+        global_chunk(g, v.n_g, k0, c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            end = end || k0 + j >= v.n_g || c[j] <= prev || c[j] / kBlockSize >= w0;
+            if (!end) {
+                prev = c[j];
+                if (c[j] / kBlockSize != last) {
+                    ++n;
+                    last = c[j] / kBlockSize;
+                }
+            }
         }
     }
     *sink_blks = n;
@@ -177,13 +219,21 @@ __device__ __forceinline__ unsigned long long global_mask_thread(const Visibilit
     const int32_t *g = global_row(v, b);
     unsigned long long m = 0ull;
     int prev = -1;
-    for (int k = 0; k < v.n_g; ++k) {
-        const int p = g[k];
-        if (p <= prev) break;
-        prev = p;
-        const int t = p - blk * kBlockSize;
-        if (t >= kBlockSize) break;
-        if (t >= 0) m |= 1ull << t;
+    for (int k0 = 0; k0 < v.n_g; k0 += 8) {
+        int32_t c[8];
+        global_chunk(g, v.n_g, k0, c);
+        bool end = false;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int p = c[j];
+            end = end || k0 + j >= v.n_g || p <= prev || p - blk * kBlockSize >= kBlockSize;
+            if (!end) {
+                prev = p;
+                const int t = p - blk * kBlockSize;
+                if (t >= 0) m |= 1ull << t;
+            }
+        }
+        if (end) break;
     }
     return m;
 }
