@@ -278,8 +278,9 @@ struct RowReduce {
 };
 
 // Steps through the tiles (blocks) of a CTA's range in order.
-struct TileCursor {
-    SegmentWalker w;
+template <bool G = true>
+struct TileCursorT {
+    SegmentWalkerT<G> w;
     int t, len;
     __device__ void init(const PlanArgs &a, long long lo, long long hi, int seq,
                          long long base) {
@@ -298,14 +299,16 @@ struct TileCursor {
         }
     }
 };
+using TileCursor = TileCursorT<true>;
 
 // Producer of warp 0: walks the CTA's tiles and keeps the physical block ids
 // of the current segment in registers, 32 at a time (lane i holds tile
 // bt0 + i), fetched with one coalesced load and the next batch prefetched
 // half a batch early, so no bulk copy waits on a dependent global load.
 // All 32 lanes call it together; lane 0 issues the copies.
+template <bool G>
 struct Producer {
-    TileCursor cur;
+    TileCursorT<G> cur;
     int id_cur, id_nxt, bt0;
     bool has_next;
 
@@ -339,8 +342,8 @@ struct Producer {
 // Issue the bulk copies of one tile -- tile `sub` (kTileTok tokens) of the
 // physical block `phys`, KV head of the cursor's unit -- into a stage.
 // Called by one lane.
-template <int D, typename T, int kTileTok>
-__device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursor &cur,
+template <int D, typename T, int kTileTok, bool G>
+__device__ __forceinline__ void issue_tile(const GqaParams &p, const TileCursorT<G> &cur,
                                           int phys, int sub, unsigned char *dst,
                                           uint64_t *full, uint64_t pol) {
     constexpr uint32_t kTileBytes = kTileTok * D * sizeof(T);
@@ -389,7 +392,7 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
         2 * (kTileTok * D * (int)sizeof(TK) + (sizeof(TK) == 1 ? kTileTok * 4 : 0));
     constexpr uint32_t kQBytes = HC * D * sizeof(T);
     const uint64_t pol = l2_policy_evict_first();
-    Producer prod;
+    Producer<G> prod;
     prod.cur.init(pa, lo, hi, seq, base);
     const long long n_tiles = (hi - lo) * kSub;
     int sub = 0, phys = -1, seg = 0;
@@ -432,7 +435,7 @@ __device__ void produce_tiles(const GqaParams &p, const PlanArgs &pa, long long 
             if (lane == 0) s_gmask[s] = gm;
         }
         if (lane == 0)
-            issue_tile<D, TK, kTileTok>(p, prod.cur, phys, sub,
+            issue_tile<D, TK, kTileTok, G>(p, prod.cur, phys, sub,
                                        stage_base + (size_t)s * kStageBytes, &full_bar[s],
                                        pol);
         if (++sub == kSub) {
@@ -761,7 +764,7 @@ gqa_split_kernel(const GqaParams p) {
     if ((int)blockIdx.x >= P) return;
     const long long lo = cta_bound(blockIdx.x, W, P);
     const long long hi = cta_bound(blockIdx.x + 1, W, P);
-    SegmentWalker walk;
+    SegmentWalkerT<G> walk;
     walk.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
 
     // ------------------------------------------------------------ producer
@@ -786,7 +789,7 @@ gqa_split_kernel(const GqaParams p) {
             }
             // The epilogue of every segment, while the compute warps go on
             // with the next one.
-            SegmentWalker ew;
+            SegmentWalkerT<G> ew;
             ew.init(pa, lo, hi, plan_sh->seq, plan_sh->base);
             for (int es = 0; !ew.done(); ++es) {
                 const int len = ew.seg_len();
@@ -1045,7 +1048,7 @@ gqa_split_kernel(const GqaParams p) {
         }
         if (!ok) break;
 
-        SegmentWalker next = walk;
+        SegmentWalkerT<G> next = walk;
         next.advance(len);
 
         // ---- stash this warp's state for the epilogue warps

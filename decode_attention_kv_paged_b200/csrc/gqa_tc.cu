@@ -158,7 +158,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint64_t pol = l2_policy_evict_first();
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
-            TileCursor cur;
+            TileCursorT<G> cur;
             cur.init(pa, lo, hi, first_seq, first_base);
             int tile = 0, seg = 0;
             while (!cur.done()) {
@@ -244,7 +244,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (warp == 1) {
                 constexpr uint32_t idesc_s = umma_idesc_bf16(kTcM, 64, 0, 0);
                 const uint32_t q_base = smem_u32(sQ);
-                TileCursor cs;
+                TileCursorT<G> cs;
                 cs.init(pa, lo, hi, first_seq, first_base);
                 int seg_s = 0;
                 for (int n = 0; n < n_tiles; ++n) {
@@ -274,7 +274,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             } else {
                 constexpr uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, 0, 1);
                 const uint32_t p_base = smem_u32(sP);
-                TileCursor cv;
+                TileCursorT<G> cv;
                 cv.init(pa, lo, hi, first_seq, first_base);
                 int seg_v = 0;
                 for (int i = 0; i < n_tiles; ++i) {
@@ -321,7 +321,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
         unsigned char *prow0 = sP + (lane < 16 ? row : 0) * 128;
         auto all = [](bool v) { return __all_sync(0xffffffffu, v); };
-        TileCursor cur;
+        TileCursorT<G> cur;
         cur.init(pa, lo, hi, first_seq, first_base);
         float m_run = kNegInf, l_run = 0.f;
         for (int i = 0; i < n_tiles; ++i) {

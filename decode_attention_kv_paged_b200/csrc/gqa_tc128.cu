@@ -157,7 +157,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const uint64_t pol = l2_policy_evict_first();
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
-            TileCursor cur;
+            TileCursorT<G> cur;
             cur.init(pa, lo, hi, first_seq, first_base);
             int tile = 0;
             constexpr int kRing = F8 ? C::kRaw : C::kStages;   // the ring this thread fills
@@ -252,7 +252,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             if (warp == 1) {
                 constexpr uint32_t idesc_s =
                     F8 ? umma_idesc_f16(128, 64, 0, 0) : umma_idesc_bf16(128, 64, 0, 0);
-                TileCursor cs;
+                TileCursorT<G> cs;
                 cs.init(pa, lo, hi, first_seq, first_base);
                 int seg_s = 0;
                 for (int n = 0; n < n_tiles; ++n) {
@@ -280,7 +280,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             } else {
                 constexpr uint32_t idesc_pv =
                     F8 ? umma_idesc_f16(128, D, 0, 1) : umma_idesc_bf16(128, D, 0, 1);
-                TileCursor cv;
+                TileCursorT<G> cv;
                 cv.init(pa, lo, hi, first_seq, first_base);
                 int seg_v = 0;
                 for (int i = 0; i < n_tiles; ++i) {
@@ -395,7 +395,7 @@ gqa_tc128_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             for (int c = 0; c < 4; ++c) tmem_st32(trow + C::kTmemP + 32 * c, z);
         }
 
-        TileCursor cur;
+        TileCursorT<G> cur;
         cur.init(pa, lo, hi, first_seq, first_base);
         float m_run = kNegInf, l_run = 0.f;
         int q_seg = 0;

@@ -221,12 +221,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             const uint64_t pol = l2_policy_evict_first();
             constexpr uint32_t kElem = F8 ? 1 : 2;     // bytes per cached value
             tma_prefetch_map(&tm_c);
-            TileCursor cur;
+            TileCursorT<false> cur;
             cur.init(pa, lo, hi, first_seq, first_base);
             // Rank 0 also pulls whole blocks (all 576 columns, contiguous)
             // into L2 kMlaPrefetch tiles ahead, so the ring's loads of both
             // CTAs are served from L2 rather than waiting on HBM.
-            TileCursor pf;
+            TileCursorT<false> pf;
             pf.init(pa, lo, hi, first_seq, first_base);
             auto prefetch_next = [&]() {
                 if (rank != 0 || pf.done()) return;
@@ -316,7 +316,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             if (warp == 1) {
                 constexpr uint32_t idesc_s =
                     F8 ? umma_idesc_f16(128, 64, 0, 0) : umma_idesc_bf16(128, 64, 0, 0);
-                TileCursor cs;
+                TileCursorT<false> cs;
                 cs.init(pa, lo, hi, first_seq, first_base);
                 int seg_s = 0;
                 for (int n = 0; n < n_tiles; ++n) {
@@ -345,7 +345,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
                 constexpr uint32_t idesc_pv =
                     F8 ? umma_idesc_f16(128, 256, 0, 1) : umma_idesc_bf16(128, 256, 0, 1);
                 const uint32_t p_base = smem_u32(sP);
-                TileCursor cv;
+                TileCursorT<false> cv;
                 cv.init(pa, lo, hi, first_seq, first_base);
                 int seg_v = 0;
                 for (int i = 0; i < n_tiles; ++i) {
@@ -474,7 +474,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
             mbar_arrive_warp(&bars->q_full);
             return true;
         };
-        TileCursor cur, nxt;
+        TileCursorT<false> cur, nxt;
         cur.init(pa, lo, hi, first_seq, first_base);
         nxt.init(pa, lo, hi, first_seq, first_base);
         int q_seg = 0, n_seg = 0;

@@ -244,6 +244,9 @@ __device__ __forceinline__ unsigned long long global_mask_thread(const Visibilit
 // of global positions) followed by a run starting at logical block
 // *first_block; visible block v is logical block first_block + v -
 // sink_blks for v >= sink_blks, else v (sink) or global_block(v) (set G).
+// G = false compiles out the explicit-global-set code (callers that never
+// see a set: it must not bloat their per-tile loops).
+template <bool G = true>
 __device__ __forceinline__ int visible_blocks(int T, const Visibility &v, int max_blocks,
                                               int *first_block, int *sink_blks, bool *bad,
                                               int b = 0) {
@@ -259,7 +262,7 @@ __device__ __forceinline__ int visible_blocks(int T, const Visibility &v, int ma
     }
     *bad = false;
     const int w1 = (T - 1) / kBlockSize + 1;             // one past the last block
-    if (v.n_g > 0) {
+    if (G && v.n_g > 0) {
         if (v.ring > 0 && window_lo(v, T) > 0 && global_query(v, b, T)) {
             *bad = true;                                  // history left the ring
             return 0;
@@ -438,8 +441,10 @@ __device__ __noinline__ static void plan_locate(const PlanArgs &a, int target_ct
 }
 
 // Walks the segments of one CTA's block range.  A segment is the part of one
-// unit's visible blocks that lies in the range.
-struct SegmentWalker {
+// unit's visible blocks that lies in the range.  G: the call may carry an
+// explicit global set (G = false compiles that code out).
+template <bool G = true>
+struct SegmentWalkerT {
     // fixed
     const int32_t *seq_lens;
     Visibility vis;
@@ -452,19 +457,19 @@ struct SegmentWalker {
     __device__ void load_seq() {
         bool bad;
         T = seq_lens[b];
-        nb = visible_blocks(T, vis, max_blocks, &first_blk, &sink_blks, &bad, b);
-        lo = vis.n_g > 0 ? seq_window_lo(vis, b, T) : window_lo(vis, T);
+        nb = visible_blocks<G>(T, vis, max_blocks, &first_blk, &sink_blks, &bad, b);
+        lo = (G && vis.n_g > 0) ? seq_window_lo(vis, b, T) : window_lo(vis, T);
     }
 
     // Logical block of visible block v of the current sequence.
     __device__ int logical(int v) const {
         if (v >= sink_blks) return first_blk + (v - sink_blks);
-        return vis.n_g > 0 ? global_block(vis, b, v) : v;
+        return (G && vis.n_g > 0) ? global_block(vis, b, v) : v;
     }
 
     // Table slot of visible block v of the current sequence.
     __device__ int slot(int v) const {
-        if (v < sink_blks && vis.n_g > 0 && vis.ring > 0) return global_slot(vis, b, v);
+        if (G && v < sink_blks && vis.n_g > 0 && vis.ring > 0) return global_slot(vis, b, v);
         return table_slot(vis, logical(v));
     }
 
@@ -504,5 +509,6 @@ struct SegmentWalker {
         }
     }
 };
+using SegmentWalker = SegmentWalkerT<true>;
 
 }  // namespace attn
