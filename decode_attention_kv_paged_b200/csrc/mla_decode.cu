@@ -41,7 +41,7 @@
 //     wait is bounded; TMEM is always freed; the final cluster handshake is a
 //     bounded mbarrier exchange.
 // Each (sequence, cluster) segment writes an fp32 partial (O/l and log2-sum-
-// exp) that the combine kernel reduces in cluster order.
+// exp) that a combine kernel reduces in cluster order.
 //
 // FP8 latent cache (template flag F8): rows stored as OCP E4M3 codes with one
 // fp32 scale per row (value = code value x scale).  The TMA loads each tile's
@@ -164,6 +164,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
     const int cluster = (int)cluster_id_x();
     const int nbox = rank == 0 ? 4 : 5;          // 64-column boxes this CTA owns
     const int col0 = rank == 0 ? 0 : 256;
+
+    // Programmatic dependent launch: the launch overlaps the previous kernel;
+    // every input is read after the wait.  The combine may be scheduled as
+    // soon as SMs free up (it waits for this grid to finish).
+    pdl_wait_primary();
+    pdl_launch_dependents();
 
     // ---- plan (both CTAs of the cluster compute the same range)
     PlanArgs pa{p.seq_lens, p.B, 1, Visibility{0, 0, 0}, p.max_blocks, p.num_clusters};
@@ -730,6 +736,133 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_c, const MlaParams p) {
 // -------------------------------------------------------------- host side
 namespace {
 
+// ---- combine of the per-cluster partials, for shapes with few partials per
+// sequence (many sequences): z[b, h] = sum_s 2^(lse_s - L) O_s /
+// sum_s 2^(lse_s - L) over the partials of sequence b, one per cluster whose
+// tile range meets it, in cluster order (fixed, deterministic).  A partial
+// with lse = -inf has weight zero.  One CTA makes 8 heads x 512 columns:
+// warp w computes head w's weights once (shared memory), then every thread
+// accumulates four float4 of output over the partials, so each CTA's set-up
+// round trips (sequence length, prefix, log-sum-exps) are paid for 4096
+// outputs.  The host picks it when sequences expect few partials; a ragged
+// sequence that spans more than kMlaCombMaxW clusters still combines
+// correctly (its further weights are recomputed from the log-sum-exps).
+// Shapes with many partials per sequence use the generic combine, which
+// spreads one output over several threads.
+constexpr int kMlaCombThreads = 256;
+constexpr int kMlaCombHeads = 8;                 // heads per CTA
+constexpr int kMlaCombMaxW = 128;                // weights per head held in shared memory
+constexpr int kMlaCombExpected = 8;              // host: expected partials per sequence
+constexpr int kMlaCombVec = kMlaCombHeads * kMlaDc / 4 / kMlaCombThreads;   // float4 per thread
+
+struct MlaCombineParams {
+    const int32_t *seq_lens;
+    const long long *ws_prefix;
+    const float *ws_o;      // [slots][128][512]
+    const float *ws_lse;    // [slots][128]
+    __nv_bfloat16 *out;     // [B][128][512]
+    int B, max_blocks, num_clusters;
+};
+
+__global__ void __launch_bounds__(kMlaCombThreads)
+mla_combine_kernel(const MlaCombineParams p) {
+    __shared__ float s_w[kMlaCombHeads][kMlaCombMaxW];
+    __shared__ float s_max[kMlaCombHeads], s_inv[kMlaCombHeads];
+    __shared__ long long s_first;
+    __shared__ int s_n;
+    pdl_wait_primary();                           // the partials are the decode's output
+    constexpr int kParts = kMlaH / kMlaCombHeads;
+    const int b = blockIdx.x / kParts;
+    const int h0 = (blockIdx.x % kParts) * kMlaCombHeads;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        int fb, sb;
+        bool bad;
+        const int nb = visible_blocks<false>(p.seq_lens[b], Visibility{0, 0, 0}, p.max_blocks,
+                                             &fb, &sb, &bad, b);
+        int n = 0;
+        long long first = 0;
+        if (nb > 0) {
+            const long long W = p.ws_prefix[p.B];
+            const int P = working_ctas(W, p.num_clusters);
+            const long long s_u = p.ws_prefix[b];
+            const int c0 = cta_of(s_u, W, P);
+            const int c1 = cta_of(s_u + nb - 1, W, P);
+            n = c1 - c0 + 1;
+            first = (long long)b + c0;
+        }
+        s_n = n;
+        s_first = first;
+    }
+    __syncthreads();
+    const int n = s_n;
+    const long long s0 = s_first;
+    // Weights of head h0 + warp over the n partials (lane-strided).
+    const float *lse = p.ws_lse + (size_t)s0 * kMlaH + h0;    // [partial][head]
+    if (warp < kMlaCombHeads) {
+        float L = kNegInf;
+        for (int i = lane; i < n; i += 32) L = fmaxf(L, lse[(size_t)i * kMlaH + warp]);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, m));
+        float den = 0.f;
+        for (int i = lane; i < n; i += 32) {
+            const float w = L == kNegInf ? 0.f : exp2f(lse[(size_t)i * kMlaH + warp] - L);
+            if (i < kMlaCombMaxW) s_w[warp][i] = w;
+            den += w;
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
+        if (lane == 0) {
+            s_max[warp] = L;
+            s_inv[warp] = den > 0.f ? 1.f / den : 0.f;
+        }
+    }
+    __syncthreads();
+    float4 acc[kMlaCombVec];
+#pragma unroll
+    for (int k = 0; k < kMlaCombVec; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *src = p.ws_o + ((size_t)s0 * kMlaH + h0) * kMlaDc;
+    for (int i = 0; i < n; ++i) {
+        const float *pi = src + (size_t)i * kMlaH * kMlaDc;
+        float4 v[kMlaCombVec];
+#pragma unroll
+        for (int k = 0; k < kMlaCombVec; ++k)
+            v[k] = *reinterpret_cast<const float4 *>(pi + 4 * (tid + k * kMlaCombThreads));
+#pragma unroll
+        for (int k = 0; k < kMlaCombVec; ++k) {
+            const int hh = (tid + k * kMlaCombThreads) / (kMlaDc / 4);
+            const float w = i < kMlaCombMaxW ? s_w[hh][i]
+                            : s_max[hh] == kNegInf
+                                ? 0.f
+                                : exp2f(lse[(size_t)i * kMlaH + hh] - s_max[hh]);
+            acc[k].x = fmaf(w, v[k].x, acc[k].x);
+            acc[k].y = fmaf(w, v[k].y, acc[k].y);
+            acc[k].z = fmaf(w, v[k].z, acc[k].z);
+            acc[k].w = fmaf(w, v[k].w, acc[k].w);
+        }
+    }
+    __nv_bfloat16 *out = p.out + ((size_t)b * kMlaH + h0) * kMlaDc;
+    const bool vec = (reinterpret_cast<uintptr_t>(out) & 7) == 0;
+#pragma unroll
+    for (int k = 0; k < kMlaCombVec; ++k) {
+        const int q = tid + k * kMlaCombThreads;
+        const float inv = s_inv[q / (kMlaDc / 4)];
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[k].x * inv, acc[k].y * inv);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[k].z * inv, acc[k].w * inv);
+        if (vec) {
+            uint2 u;
+            u.x = *reinterpret_cast<const uint32_t *>(&lo);
+            u.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(out + 4 * q) = u;
+        } else {
+            out[4 * q] = lo.x;
+            out[4 * q + 1] = lo.y;
+            out[4 * q + 2] = hi.x;
+            out[4 * q + 3] = hi.y;
+        }
+    }
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave,
@@ -816,13 +949,15 @@ int mla_launch(const MlaParams &mp, const CUtensorMap &tc, int clusters, cudaStr
     cfg.blockDim = dim3(F8 ? kMlaThreadsF8 : kMlaThreads);
     cfg.dynamicSmemBytes = MlaCfg<F8>::kSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (ev_start) cudaEventRecord(ev_start, stream);
     if (cudaLaunchKernelEx(&cfg, mla_decode_kernel<F8>, tc, mp) != cudaSuccess)
         return ATTN_ERR_CUDA;
@@ -879,6 +1014,32 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
              : mla_launch<false>(mp, tc, clusters, stream, ev_start, ev_stop);
     if (rc) return rc;
 
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // Few expected partials per sequence and enough sequences to fill the
+    // SMs: the 8-head combine; else the generic one.
+    if (clusters / B + 1 <= kMlaCombExpected &&
+        (long long)B * (kMlaH / kMlaCombHeads) >= num_sms) {
+        MlaCombineParams mc{};
+        mc.seq_lens = seq_lens;
+        mc.ws_prefix = mp.ws_prefix;
+        mc.ws_o = mp.ws_o;
+        mc.ws_lse = mp.ws_lse;
+        mc.out = static_cast<__nv_bfloat16 *>(out);
+        mc.B = B;
+        mc.max_blocks = max_blocks;
+        mc.num_clusters = clusters;
+        cfg.gridDim = dim3(B * (kMlaH / kMlaCombHeads));
+        cfg.blockDim = dim3(kMlaCombThreads);
+        return cudaLaunchKernelEx(&cfg, mla_combine_kernel, mc) == cudaSuccess ? ATTN_OK
+                                                                             : ATTN_ERR_CUDA;
+    }
     CombineParams cp{};
     cp.seq_lens = seq_lens;
     cp.ws_prefix = mp.ws_prefix;
@@ -898,8 +1059,10 @@ int mla_decode_entry(const void *q_latent, const void *q_rope, const void *laten
     cp.copies = 1;
     cp.lanes = combine_lanes(clusters / B + 1);
     cp.blocks_per_unit = combine_blocks_per_unit(kMlaH, kMlaDc, cp.lanes);
-    combine_kernel<__nv_bfloat16><<<B * cp.blocks_per_unit, kCombineThreads, 0, stream>>>(cp);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    cfg.gridDim = dim3(B * cp.blocks_per_unit);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<__nv_bfloat16>, cp) == cudaSuccess
+               ? ATTN_OK
+               : ATTN_ERR_CUDA;
 }
 
 }  // namespace attn
