@@ -12,7 +12,10 @@
 // Design (B200):
 //   * One CTA per SM over the split-KV partition (plan.cuh).  Warp 0 issues
 //     2-D TMA loads (128-byte swizzle) of each 64-token K and V tile of the
-//     paged cache into a multi-stage ring and of the unit's query rows; one
+//     paged cache into two rings and of the unit's query rows: a K slot is
+//     released by its S product, a V slot only after the softmax and the P V
+//     product, so the V ring is the deeper one (at d = 256 the fixed buffers
+//     leave room for five 32 KiB slots: two K, three V); one
 //     thread of warp 1 issues the S MMAs and one of warp 2 the P V MMAs as
 //     their inputs become ready; warps 4-7 run the softmax and the epilogue.
 //   * S: M = 64 query rows, N = 64 tokens, K = d, both operands in shared
@@ -51,34 +54,38 @@ template <int D>
 struct TcCfg {
     static constexpr int kBoxes = D / 64;
     static constexpr int kQBytes = kBoxes * kTcBox;
-    static constexpr int kStageBytes = 2 * kBoxes * kTcBox;     // K then V
+    static constexpr int kSlotBytes = kBoxes * kTcBox;          // one K or V tile
     // P is double-buffered (hi and lo halves each): the softmax of tile i + 1
     // writes while the P V of tile i reads.
     static constexpr int kPBytes = 4 * kTcPBytes;
     static constexpr int kFixed = kQBytes + kPBytes + 1024 /*bars*/ + 1024 /*align*/;
-    static constexpr int kStagesRaw = (227 * 1024 - kFixed) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+    static constexpr int kSlots = (227 * 1024 - kFixed) / kSlotBytes;
+    static constexpr int kKHalf = kSlots / 2 < 2 ? 2 : kSlots / 2;
+    static constexpr int kKStages = kKHalf > 6 ? 6 : kKHalf;
+    static constexpr int kVStages = kSlots - kKStages > 6 ? 6 : kSlots - kKStages;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffC = kOffQ + kQBytes;
-    static constexpr int kOffP = kOffC + kStages * kStageBytes;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kKStages * kSlotBytes;
+    static constexpr int kOffP = kOffV + kVStages * kSlotBytes;
     static constexpr int kOffBar = kOffP + kPBytes;
     static constexpr int kSmem = kOffBar + 1024 + 1024;
     static constexpr uint32_t kTmemO = 0, kTmemS = D;            // S buffers at D, D + 64
     static constexpr uint32_t kTmemCols = D + 128 <= 256 ? 256 : 512;
-    static_assert(kStages >= 2, "at least two stages");
+    static_assert(kKStages >= 2 && kVStages >= 2, "at least two stages per ring");
     static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 struct TcBars {
     uint64_t q_full, q_empty;
-    uint64_t c_full[6], c_empty[6];
+    uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
     uint64_t s_full[2], s_free[2];
     // One P-ready and one P V-done barrier per P buffer: the softmax can
     // finish two tiles before the MMA thread tests the first, which a single
     // barrier could not tell apart.
     uint64_t p_full[2], pv_done[2], o_free, mma_final;
-    // Per stage: global positions among the staged block's keys below the
-    // window (bit t: key 64 * block + t), written before the stage is armed.
+    // Per V slot (held until the tile's P V, so past the softmax that reads
+    // it): global positions among the staged block's keys below the window
+    // (bit t: key 64 * block + t), written before the slot is armed.
     unsigned long long gmask[6];
     uint32_t tmem_base;
     int abort;
@@ -99,7 +106,8 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     unsigned char *sQ = smem + C::kOffQ;
-    unsigned char *sC = smem + C::kOffC;
+    unsigned char *sK = smem + C::kOffK;
+    unsigned char *sV = smem + C::kOffV;
     unsigned char *sP = smem + C::kOffP;
     TcBars *bars = reinterpret_cast<TcBars *>(smem + C::kOffBar);
     volatile int *abort_flag = &bars->abort;
@@ -129,9 +137,13 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) {
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&bars->c_full[s], 1);
-            mbar_init(&bars->c_empty[s], 1);
+        for (int s = 0; s < C::kKStages; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+        }
+        for (int s = 0; s < C::kVStages; ++s) {
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
@@ -160,7 +172,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tma_prefetch_map(&tm_v);
             TileCursorT<G> cur;
             cur.init(pa, lo, hi, first_seq, first_base);
-            int tile = 0, seg = 0;
+            int tile = 0, seg = 0, n_k = 0, n_v = 0;   // tiles; K and V loads issued
             while (!cur.done()) {
                 const int kvh = cur.w.unit / p.n_hc, hc = cur.w.unit % p.n_hc;
                 if (cur.t == 0) {
@@ -175,10 +187,11 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                         &bars->q_full, pol);
                     ++seg;
                 }
-                const int st = tile % C::kStages;
-                if (tile >= C::kStages &&
-                    !mbar_wait(&bars->c_empty[st], (uint32_t)(((tile - C::kStages) / C::kStages) & 1),
-                               p.timeout_ns, p.err, abort_flag))
+                const int ks = tile % C::kKStages, vs = tile % C::kVStages;
+                if (tile >= C::kKStages &&
+                    !mbar_wait(&bars->k_empty[ks],
+                               (uint32_t)(((tile - C::kKStages) / C::kKStages) & 1), p.timeout_ns,
+                               p.err, abort_flag))
                     break;
                 int phys = p.block_table[(size_t)cur.w.b * p.max_blocks +
                                          cur.table_slot_of_tile()];
@@ -187,23 +200,35 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     phys = p.num_blocks;                 // wholly out of bounds: zero fill
                 }
                 const int row = (phys * p.H_kv + kvh) * 64;
-                unsigned char *dst = sC + st * C::kStageBytes;
+                mbar_arrive_expect_tx(&bars->k_full[ks], C::kSlotBytes);
+                for (int j = 0; j < C::kBoxes; ++j)
+                    tma_load_2d(sK + ks * C::kSlotBytes + j * kTcBox, &tm_k, 64 * j, row,
+                                &bars->k_full[ks], pol);
+                n_k = tile + 1;
+                if (tile >= C::kVStages &&
+                    !mbar_wait(&bars->v_empty[vs],
+                               (uint32_t)(((tile - C::kVStages) / C::kVStages) & 1), p.timeout_ns,
+                               p.err, abort_flag))
+                    break;
                 if constexpr (G) {
                     const int blk = cur.logical_block();
-                    bars->gmask[st] = blk * 64 < cur.w.lo
+                    bars->gmask[vs] = blk * 64 < cur.w.lo
                                           ? global_mask_thread(p.vis, cur.w.b, blk) : 0ull;
                 }
-                mbar_arrive_expect_tx(&bars->c_full[st], C::kStageBytes);
-                for (int j = 0; j < C::kBoxes; ++j) {
-                    tma_load_2d(dst + j * kTcBox, &tm_k, 64 * j, row, &bars->c_full[st], pol);
-                    tma_load_2d(dst + (C::kBoxes + j) * kTcBox, &tm_v, 64 * j, row,
-                                &bars->c_full[st], pol);
-                }
+                mbar_arrive_expect_tx(&bars->v_full[vs], C::kSlotBytes);
+                for (int j = 0; j < C::kBoxes; ++j)
+                    tma_load_2d(sV + vs * C::kSlotBytes + j * kTcBox, &tm_v, 64 * j, row,
+                                &bars->v_full[vs], pol);
+                n_v = tile + 1;
                 cur.next();
                 ++tile;
             }
-            for (int t = tile - C::kStages < 0 ? 0 : tile - C::kStages; t < tile; ++t)
-                mbar_wait(&bars->c_full[t % C::kStages], (uint32_t)((t / C::kStages) & 1),
+            // Every issued load must have landed before the CTA exits.
+            for (int t = n_k - C::kKStages < 0 ? 0 : n_k - C::kKStages; t < n_k; ++t)
+                mbar_wait(&bars->k_full[t % C::kKStages], (uint32_t)((t / C::kKStages) & 1),
+                          p.timeout_ns, p.err, nullptr);
+            for (int t = n_v - C::kVStages < 0 ? 0 : n_v - C::kVStages; t < n_v; ++t)
+                mbar_wait(&bars->v_full[t % C::kVStages], (uint32_t)((t / C::kVStages) & 1),
                           p.timeout_ns, p.err, nullptr);
             if (seg > 0)
                 mbar_wait(&bars->q_full, (uint32_t)((seg - 1) & 1), p.timeout_ns, p.err, nullptr);
@@ -213,12 +238,12 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ============================================================ MMA
         // Two issuing threads: lane 0 of warp 1 issues S(n) = Q K(n)^T for
         // every tile in order, lane 0 of warp 2 issues O += P(i) V(i).  Each
-        // chain waits only on its own inputs (S on the staged tile and a free
-        // S buffer, P V on the softmax's P), so the two streams of MMAs
-        // overlap instead of queueing behind one thread.  A stage is released
-        // by the commit after P V(i): S(i) has completed by then, since the
-        // softmax read it before producing P(i).  Barriers are polled (a
-        // sleeping wait wakes up too late for these chains).
+        // chain waits only on its own inputs (S on the staged K tile and a
+        // free S buffer, P V on the softmax's P and the staged V tile), so the
+        // two streams of MMAs overlap instead of queueing behind one thread.
+        // A K slot is released by the commit after S(n), a V slot by the
+        // commit after P V(i).  Barriers are polled (a sleeping wait wakes up
+        // too late for these chains).
         if (lane == 0) {
             auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
                 unsigned long long t0 = 0;
@@ -240,7 +265,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             };
-            const uint32_t c_base = smem_u32(sC);
+            const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
             if (warp == 1) {
                 constexpr uint32_t idesc_s = umma_idesc_bf16(kTcM, 64, 0, 0);
                 const uint32_t q_base = smem_u32(sQ);
@@ -251,13 +276,13 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // S(n) into S buffer n % 2, once the softmax of tile
                     // n - 2 has read it.
                     const bool first = cs.t == 0, last = cs.t == cs.len - 1;
-                    const int st = n % C::kStages, sb = n & 1;
+                    const int ks = n % C::kKStages, sb = n & 1;
                     if (first && !wait(&bars->q_full, (uint32_t)(seg_s & 1))) break;
-                    if (!wait(&bars->c_full[st], (uint32_t)((n / C::kStages) & 1))) break;
+                    if (!wait(&bars->k_full[ks], (uint32_t)((n / C::kKStages) & 1))) break;
                     if (n >= 2 && !wait(&bars->s_free[sb], (uint32_t)(((n - 2) >> 1) & 1)))
                         break;
                     tc_fence_after();
-                    const uint32_t kst = c_base + st * C::kStageBytes;
+                    const uint32_t kst = k_base + ks * C::kSlotBytes;
                     for (int j = 0; j < C::kBoxes; ++j)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -267,6 +292,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             umma_bf16(tmem + C::kTmemS + 64 * sb, a, b, idesc_s, (j | k) != 0);
                         }
                     umma_commit(&bars->s_full[sb]);
+                    umma_commit(&bars->k_empty[ks]);       // K(n) read once S(n) completes
                     if (last) umma_commit(&bars->q_empty);
                     if (first) ++seg_s;
                     cs.next();
@@ -286,8 +312,9 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (first && seg_v > 0 && !wait(&bars->o_free, (uint32_t)((seg_v - 1) & 1)))
                         break;
                     tc_fence_after();
-                    const int st = i % C::kStages;
-                    const uint32_t vst = c_base + st * C::kStageBytes + C::kBoxes * kTcBox;
+                    const int vs = i % C::kVStages;
+                    if (!wait(&bars->v_full[vs], (uint32_t)((i / C::kVStages) & 1))) break;
+                    const uint32_t vst = v_base + vs * C::kSlotBytes;
                     const uint32_t pb = p_base + (i & 1) * 2 * kTcPBytes;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -297,7 +324,7 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         umma_bf16(tmem + C::kTmemO, a_hi, b, idesc_pv, !(first && k == 0));
                         umma_bf16(tmem + C::kTmemO, a_lo, b, idesc_pv, 1);
                     }
-                    umma_commit(&bars->c_empty[st]);
+                    umma_commit(&bars->v_empty[vs]);
                     umma_commit(&bars->pv_done[i & 1]);
                     if (first) ++seg_v;
                     cv.next();
@@ -333,14 +360,14 @@ gqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // Global positions among this block's keys below the window.
             unsigned long long gmask = 0ull;
             if (G && blk * 64 < lo_tok) {
-                // The stage of tile i is still armed for it (it is refilled only
-                // after this tile's P V), so this wait returns at once and orders
-                // the producer's mask before the read.
-                const int st = i % C::kStages;
-                if (!all(mbar_wait(&bars->c_full[st], (uint32_t)((i / C::kStages) & 1),
+                // The V slot of tile i stays armed for it (it is refilled only
+                // after this tile's P V), so this wait orders the producer's
+                // mask before the read.
+                const int vs = i % C::kVStages;
+                if (!all(mbar_wait(&bars->v_full[vs], (uint32_t)((i / C::kVStages) & 1),
                                    p.timeout_ns, p.err, abort_flag)))
                     break;
-                gmask = bars->gmask[st];
+                gmask = bars->gmask[vs];
             }
             const int sb = i & 1;
             if (!all(mbar_wait(&bars->s_full[sb], (uint32_t)((i >> 1) & 1), p.timeout_ns, p.err,
