@@ -47,6 +47,42 @@ def test_mla_cluster_count_invariance(lib, clusters):
     assert_parity(got, ref, torch.bfloat16, f"{clusters} clusters")
 
 
+def test_mla_many_sequences_ragged_match_oracle(lib):
+    """Enough sequences that the 8-head combine merges the cluster partials
+    (few partials per sequence): ragged lengths, empty sequences, one-token
+    and block-edge lengths; every sequence against the oracle."""
+    lens = [0, 1, 64, 65, 700, 3000, 5, 128, 129, 2048, 0, 63, 1000, 17, 640, 4096]
+    x = make_mla_inputs(MLAConfig("mla_many", B=len(lens), seq_lens=lens, seed=31))
+    got = run_gpu(lib, x).float().cpu().numpy()
+    ref = oracle_mla_sequences(x, [b for b, T in enumerate(lens) if T > 0])
+    for b, T in enumerate(lens):
+        if T == 0:
+            assert np.all(got[b] == 0), f"empty sequence {b}"
+        else:
+            assert_parity(got[b], ref[b], torch.bfloat16, f"mla many b={b} T={T}")
+
+
+def test_mla_combine_sequence_spanning_many_clusters(lib):
+    """20 sequences over 140 clusters, one holding 95 % of the tiles: it
+    spans more clusters than the 8-head combine keeps weights for in shared
+    memory (its further weights are recomputed from the log-sum-exps)."""
+    lens = [20000] + [64] * 18 + [0]
+    x = make_mla_inputs(MLAConfig("mla_span", B=len(lens), seq_lens=lens, seed=41))
+    tiles = [(T + BLOCK_SIZE - 1) // BLOCK_SIZE for T in lens]
+    W, P = sum(tiles), 140
+    last_cluster = (tiles[0] - 1) * P // W           # cluster of the long sequence's last tile
+    assert last_cluster + 1 > 128                    # the case this test is for
+    lib.set_num_ctas(P)
+    try:
+        got = run_gpu(lib, x).float().cpu().numpy()
+    finally:
+        lib.set_num_ctas(0)
+    ref = oracle_mla_sequences(x, [0, 1, 18])
+    for b, r in ref.items():
+        assert_parity(got[b], r, torch.bfloat16, f"mla span b={b}")
+    assert np.all(got[19] == 0)
+
+
 def test_mla_empty_sequence_gives_zero_row(lib):
     x = make_mla_inputs(MLAConfig("mla_empty", B=3, seq_lens=[0, 100, 0], seed=5))
     got = run_gpu(lib, x).float().cpu().numpy()
