@@ -246,7 +246,7 @@ def test_window_brute_force_membership():
 
 
 def test_window_at_least_T_equals_full_causal():
-    """A window w >= T drops nothing (BASELINE pin (d); HEADS §3)."""
+    """A window w >= T drops nothing: it reduces to full causal attention (HEADS §3)."""
     rng = np.random.default_rng(9)
     q, K, V = _rand_problem(rng, 2, 4, 2, 200, 16)
     kc, vc, table = _paged_from_dense(K, V, perm_seed=1)
